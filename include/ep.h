@@ -1,0 +1,220 @@
+/*
+ * ep.h -- C ABI of the B200 (sm_100a) expert-parallel dispatch / combine library.
+ *
+ * The library moves MoE tokens between R expert-parallel ranks that live as
+ * R slabs of ONE GPU's memory ("emulated ranks"): rank r owns token rows
+ * x[r], routing topk_idx[r] / topk_weights[r], output rows out[r], and the
+ * experts [r*E_local, (r+1)*E_local) with E_local = num_experts / num_ranks.
+ * Sending a row to rank d is a store into d's receive slab; there is no peer
+ * access and no collective.
+ *
+ * Operations and where they are defined:
+ *   ep_layout   -- Buffer.get_dispatch_layout of the NeMo AutoModel page
+ *                  "nemo_automodel.components.moe.uccl_ep.buffer"
+ *                  (num_tokens_per_rank, is_token_in_rank,
+ *                  num_tokens_per_expert), plus the communication handle that
+ *                  Buffer.dispatch returns and Buffer.low_latency_combine
+ *                  consumes (here: pair_row, expert_rank_offset, recv_count).
+ *   ep_dispatch -- Buffer.low_latency_dispatch with use_fp8=False on the same
+ *                  page: bf16 rows into per-local-expert receive slabs
+ *                  [num_local_experts, num_ranks * num_max_dispatch_tokens_per_rank,
+ *                  hidden]; only some slab rows are valid.
+ *   ep_combine  -- Buffer.low_latency_combine on the same page: reduce WITH
+ *                  weights back to [num_tokens, hidden] bf16, -1 indices
+ *                  supported; the active-rank mask is re-checked as in the
+ *                  ai-dynamo/nixl PR "nixl_ep: Optimize low-latency NVLink
+ *                  path" (combine active rank mask optimization).
+ *   ep_reroute  -- load computation, placement planning and routing expansion
+ *                  of the GitDiagram page "dots-infra/ultraep architecture"
+ *                  (GPU operations), with the placement rule "add one replica
+ *                  at a time to the expert with the largest load/replicas,
+ *                  ties to the lowest id".
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, except
+ *     where noted.  The library never allocates, frees or synchronises: each
+ *     call validates its arguments on the host, enqueues kernels on `stream`
+ *     (a cudaStream_t, NULL = legacy default stream) and returns.
+ *   - Arrays are dense, C-contiguous (row-major) with the shapes given below.
+ *     bf16 tensors are passed as uint16_t bit patterns.  R = num_ranks,
+ *     T = num_tokens (tokens per rank, = num_max_dispatch_tokens_per_rank),
+ *     k = num_topk, E = num_experts, H = hidden, CAP = R*T (slab rows per
+ *     expert).
+ *   - topk_idx is int32 (the index width the nixl PR made the default);
+ *     -1 means "no selection".  A pair (r,t,j) is LIVE when
+ *     0 <= e = topk_idx[r,t,j] < E, active[r] != 0 and active[e/E_local] != 0:
+ *     a masked rank neither sends nor receives.
+ *   - Data errors never trap.  Kernels OR bits into *status (int32, device,
+ *     zeroed by the caller): EP_STATUS_BAD_EXPERT (an id outside [-1, E);
+ *     the pair is dropped), EP_STATUS_OVERFLOW (an expert received more than
+ *     CAP rows; rows >= CAP are neither written nor read), EP_STATUS_TIMEOUT
+ *     (a bounded wait gave up; outputs are incomplete).
+ *   - Return value: EP_OK, or a negative EP_ERR_* code for an argument the
+ *     host rejected (nothing was enqueued) or a launch the CUDA runtime
+ *     refused.  ep_strerror() names every code.
+ *   - Calls that share output buffers must be ordered by the caller (same
+ *     stream, or events); calls on disjoint buffers may run concurrently.
+ */
+#ifndef EP_B200_EP_H
+#define EP_B200_EP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host-side return codes. */
+enum {
+    EP_OK = 0,
+    EP_ERR_INVALID = -1,      /* null/misaligned pointer, bad shape, workspace too small */
+    EP_ERR_UNSUPPORTED = -2,  /* shape outside the limits below */
+    EP_ERR_CUDA = -3          /* the CUDA runtime refused a launch or query */
+};
+
+/* Device status bits (OR-ed into *status). */
+enum {
+    EP_STATUS_BAD_EXPERT = 1,
+    EP_STATUS_OVERFLOW = 2,
+    EP_STATUS_TIMEOUT = 8
+};
+
+/* Limits checked on the host (EP_ERR_UNSUPPORTED beyond them). */
+enum {
+    EP_MAX_RANKS = 64,        /* is_token_in_rank is built from a 64-bit rank set */
+    EP_MAX_TOPK = 32,         /* one lane per slot */
+    EP_MAX_EXPERTS = 8192     /* per-warp shared-memory histograms */
+};
+
+/* Problem shape.  E % R == 0, H % 8 == 0 (rows move as 16-byte vectors),
+ * 1 <= k <= min(E, EP_MAX_TOPK), R*T*k < 2^31.  T may be 0. */
+typedef struct ep_dims {
+    int32_t num_ranks;    /* R */
+    int32_t num_tokens;   /* T, tokens per rank */
+    int32_t num_topk;     /* k */
+    int32_t num_experts;  /* E, physical experts over all ranks */
+    int32_t hidden;       /* H, bf16 elements per token row */
+} ep_dims_t;
+
+/* Launch tuning (cf. Buffer.get_dispatch_config / get_combine_config and
+ * num_sms on the NeMo page).  A zero field means "choose automatically". */
+typedef struct ep_cfg {
+    int32_t max_ctas;     /* cap on CTAs of the row-moving kernels */
+    int32_t threads;      /* threads per CTA where the kernel allows a choice */
+    int32_t stages;       /* shared-memory pipeline depth of dispatch / combine */
+} ep_cfg_t;
+
+/* Human-readable name of an EP_OK / EP_ERR_* code (static storage). */
+const char *ep_strerror(int code);
+
+/* Library version string (static storage). */
+const char *ep_version(void);
+
+/* Bytes of device workspace ep_layout needs for `d` (0 only if R*T == 0). */
+size_t ep_layout_workspace_bytes(ep_dims_t d);
+
+/*
+ * ep_layout -- per-expert / per-rank histogram, prefix sums and stable rows.
+ *
+ * in:
+ *   topk_idx              int32 [R,T,k]
+ *   active                uint8 [R]       active-rank mask at dispatch time
+ *   workspace             >= ep_layout_workspace_bytes(d) bytes, 16-byte aligned,
+ *                         scratch owned by the caller; contents on entry are
+ *                         ignored, on return are undefined
+ * out (every element written):
+ *   num_tokens_per_expert int32 [R,E]     live pairs of source rank r on expert e
+ *   num_tokens_per_rank   int32 [R,R]     tokens of r with >= 1 live pair on rank d
+ *   is_token_in_rank      uint8 [R,T,R]   0/1
+ *   recv_count            int32 [E]       rows expert e receives (valid rows are
+ *                                         [0, min(recv_count[e], CAP)))
+ *   expert_rank_offset    int32 [E,R]     first row of source rank r inside expert e
+ *                                         = sum over r' < r of num_tokens_per_expert[r'][e]
+ *   pair_row              int32 [R,T,k]   slab row of each live pair, -1 if not live
+ * The row of a live pair is its position among expert e's live pairs taken in
+ * (source rank, token, slot) order, so each expert's rows are ordered by
+ * (src_rank, token) and the result is unique (bit-exact, deterministic).
+ */
+int ep_layout(ep_dims_t d, const int32_t *topk_idx, const uint8_t *active,
+              void *workspace, size_t workspace_bytes,
+              int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
+              uint8_t *is_token_in_rank, int32_t *recv_count,
+              int32_t *expert_rank_offset, int32_t *pair_row,
+              int32_t *status, ep_cfg_t cfg, void *stream);
+
+/*
+ * ep_dispatch -- scatter token rows into the experts' receive slabs.
+ *
+ * in:
+ *   x          bf16 [R,T,H]     16-byte aligned
+ *   topk_idx   int32 [R,T,k]
+ *   pair_row   int32 [R,T,k]    from ep_layout on the same topk_idx / active
+ * out:
+ *   recv_x     bf16 [E,CAP,H]   16-byte aligned; rank d's low-latency slab
+ *                               [E_local, CAP, H] is recv_x[d*E_local : (d+1)*E_local].
+ *                               Row pair_row[r,t,j] of expert topk_idx[r,t,j]
+ *                               receives x[r,t,:] bit for bit; other rows are
+ *                               left untouched.
+ *   src_info   int32 [E,CAP,2]  (src_rank, src_token) of every written row;
+ *                               other rows untouched.
+ * Each token row is read from HBM once however many experts it goes to.
+ */
+int ep_dispatch(ep_dims_t d, const uint16_t *x, const int32_t *topk_idx,
+                const int32_t *pair_row, uint16_t *recv_x, int32_t *src_info,
+                int32_t *status, ep_cfg_t cfg, void *stream);
+
+/*
+ * ep_combine -- top-k weighted gather-reduce back to the source ranks.
+ *
+ * in:
+ *   y            bf16 [E,CAP,H]  16-byte aligned expert outputs (rows as laid out
+ *                                by ep_dispatch; may be recv_x itself, zero copy)
+ *   topk_idx     int32 [R,T,k]
+ *   topk_weights float [R,T,k]
+ *   pair_row     int32 [R,T,k]   from ep_layout
+ *   active       uint8 [R]       mask at combine time (may differ from dispatch)
+ * out:
+ *   out          bf16 [R,T,H]    16-byte aligned, every element written:
+ *     out[r,t,:] = bf16_rne( sum over j = 0..k-1, in that order, of
+ *                  w[r,t,j] * y[e][pair_row[r,t,j]][:] )   (float32 accumulate)
+ *     taking only slots with pair_row >= 0, pair_row < CAP, e in range and
+ *     active[e/E_local]; rows of a source rank with active[r] == 0 are zeros.
+ */
+int ep_combine(ep_dims_t d, const uint16_t *y, const int32_t *topk_idx,
+               const float *topk_weights, const int32_t *pair_row,
+               const uint8_t *active, uint16_t *out,
+               int32_t *status, ep_cfg_t cfg, void *stream);
+
+/* Bytes of device workspace ep_reroute needs. */
+size_t ep_reroute_workspace_bytes(int32_t num_ranks, int32_t num_tokens, int32_t num_topk,
+                                  int32_t num_logical);
+
+/*
+ * ep_reroute -- logical expert load, greedy replica placement, routing expansion.
+ *
+ * in:
+ *   topk_idx_logical int32 [R,T,k]   logical ids in [0, num_logical), or -1
+ *   workspace        >= ep_reroute_workspace_bytes(...) bytes, 16-byte aligned
+ * out:
+ *   load           int32 [num_logical]      (token, slot) pairs per logical expert
+ *   num_replicas   int32 [num_logical]      starts at 1; num_extra times, +1 for the
+ *                                           expert with the largest load/replicas
+ *                                           (exact integer compare, ties -> lowest id)
+ *   phys_base      int32 [num_logical + 1]  exclusive prefix sum of num_replicas
+ *   topk_idx_phys  int32 [R,T,k]            phys_base[e] + ((r*T + t) mod num_replicas[e]),
+ *                                           -1 where the logical id is -1 or out of range
+ * num_logical + num_extra physical experts result; ep_layout / ep_dispatch /
+ * ep_combine then run with num_experts = num_logical + num_extra.
+ */
+int ep_reroute(int32_t num_ranks, int32_t num_tokens, int32_t num_topk,
+               int32_t num_logical, int32_t num_extra,
+               const int32_t *topk_idx_logical, void *workspace, size_t workspace_bytes,
+               int32_t *load, int32_t *num_replicas, int32_t *phys_base,
+               int32_t *topk_idx_phys, int32_t *status, ep_cfg_t cfg, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_B200_EP_H */

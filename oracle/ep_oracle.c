@@ -1,0 +1,269 @@
+/*
+ * ep_oracle.c -- plain, single-threaded CPU oracle for expert-parallel
+ * dispatch / combine and replica routing expansion.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package's smoke check
+ * and the benchmark's CPU-baseline leg may load this library.  It shares no
+ * code, header, table or helper with the CUDA path: every function below is
+ * the plain definition of one step, written as loops in the order the
+ * definition states, with no blocking, fusion or reordering.  Build with
+ * plain gcc (no -ffast-math, -ffp-contract=off) so the float64 arithmetic is
+ * IEEE round-to-nearest in program order.
+ *
+ * Sources (web pages; cited by title and section):
+ *  [P1] NeMo AutoModel API docs, "nemo_automodel.components.moe.uccl_ep.buffer":
+ *       Buffer.get_dispatch_layout, Buffer.dispatch, Buffer.low_latency_dispatch,
+ *       Buffer.low_latency_combine, Buffer.get_next_low_latency_combine_buffer.
+ *  [P3] GitDiagram, "dots-infra/ultraep architecture": GPU operations
+ *       (load computation, placement planning, routing expansion).
+ *  [P4] ai-dynamo/nixl PR "nixl_ep: Optimize low-latency NVLink path":
+ *       active rank mask in combine; 32-bit topk index width.
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *  - a pair (r,t,j) is live iff 0 <= e < E, active[r] and active[e / E_local];
+ *    e == -1 means "no selection" ([P1] get_dispatch_layout), any other
+ *    out-of-range id is counted as an error (status bit 1) and dropped;
+ *  - rows inside an expert's receive slab are compact: the row of a live pair
+ *    is its position in that expert's list of live pairs enumerated in
+ *    (src_rank, token, slot) order, so valid rows are [0, recv_count[e]);
+ *  - the slab holds num_ranks * num_tokens rows per expert ([P1]
+ *    low_latency_dispatch shape); a pair whose row is past that capacity is
+ *    counted as an overflow (status bit 2) and neither sent nor reduced;
+ *  - combine is the weighted reduce of [P1] low_latency_combine, re-checking
+ *    the active mask given at combine time ([P4]); rows of an inactive source
+ *    rank come out as zeros; weights are not renormalised;
+ *  - replica planning starts every logical expert at one replica and adds the
+ *    extra replicas one at a time to the expert with the largest
+ *    load/replicas (exact integer comparison, ties to the lowest id); replica
+ *    i of logical expert e is physical expert phys_base[e] + i; a pair goes to
+ *    replica (r*T + t) mod n_rep[e].
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_BAD_EXPERT 1
+#define ORACLE_OVERFLOW   2
+
+/* bfloat16 bit pattern -> double.  A bf16 value is the upper half of the
+ * float32 with the same sign, exponent and leading 7 mantissa bits. */
+static double bf16_to_double(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int pair_is_live(int e, int r, int E, int E_local, const uint8_t *active) {
+    if (e < 0 || e >= E) return 0;
+    if (!active[r]) return 0;
+    if (!active[e / E_local]) return 0;
+    return 1;
+}
+
+/*
+ * Layout ([P1] Buffer.get_dispatch_layout) plus the handle that dispatch and
+ * combine share ([P1] Buffer.dispatch "handle", Buffer.low_latency_combine
+ * "handle").  Enumerates (r, t, j) in lexicographic order and appends every
+ * live pair to its expert's list.
+ *
+ * outputs:
+ *   num_tokens_per_expert [R,E]  live pairs of source rank r routed to e
+ *   num_tokens_per_rank   [R,R]  tokens of r with >= 1 live pair on rank d
+ *   is_token_in_rank      [R,T,R]
+ *   recv_count            [E]    length of list[e]
+ *   expert_rank_offset    [E,R]  first index in list[e] whose source rank >= r
+ *   pair_row              [R,T,k] position in list[e], -1 if not live
+ *   src_list              [sum(recv_count), 2] (r, t) of list entries,
+ *                                 expert-major; may be NULL
+ *   list_base             [E+1]  start of list[e] in src_list
+ * returns the status bits (1: bad expert id, 2: row past capacity).
+ */
+int oracle_layout(int R, int T, int k, int E, const int32_t *topk_idx, const uint8_t *active,
+                  int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
+                  uint8_t *is_token_in_rank, int32_t *recv_count, int32_t *expert_rank_offset,
+                  int32_t *pair_row, int32_t *src_list, int64_t *list_base) {
+    int status = 0;
+    const int E_local = E / R;
+    const int64_t capacity = (int64_t)R * T;
+
+    memset(num_tokens_per_expert, 0, sizeof(int32_t) * (size_t)R * E);
+    memset(num_tokens_per_rank, 0, sizeof(int32_t) * (size_t)R * R);
+    memset(is_token_in_rank, 0, (size_t)R * T * R);
+    memset(recv_count, 0, sizeof(int32_t) * (size_t)E);
+
+    /* append every live pair to list[e]: its row is the list length so far */
+    for (int r = 0; r < R; r++) {
+        for (int t = 0; t < T; t++) {
+            for (int j = 0; j < k; j++) {
+                int64_t p = ((int64_t)r * T + t) * k + j;
+                int e = topk_idx[p];
+                if (e < -1 || e >= E) status |= ORACLE_BAD_EXPERT;
+                if (!pair_is_live(e, r, E, E_local, active)) {
+                    pair_row[p] = -1;
+                    continue;
+                }
+                pair_row[p] = recv_count[e];
+                recv_count[e] += 1;
+                num_tokens_per_expert[(int64_t)r * E + e] += 1;
+                is_token_in_rank[((int64_t)r * T + t) * R + e / E_local] = 1;
+            }
+        }
+    }
+    for (int e = 0; e < E; e++)
+        if (recv_count[e] > capacity) status |= ORACLE_OVERFLOW;
+
+    /* a token counts once per destination rank */
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < T; t++)
+            for (int d = 0; d < R; d++)
+                num_tokens_per_rank[(int64_t)r * R + d] += is_token_in_rank[((int64_t)r * T + t) * R + d];
+
+    /* materialise the lists: entry pair_row of list[e] is (r, t) */
+    list_base[0] = 0;
+    for (int e = 0; e < E; e++) list_base[e + 1] = list_base[e] + recv_count[e];
+    int32_t *list = src_list;
+    int32_t *own = NULL;
+    if (list == NULL) {
+        own = (int32_t *)malloc(sizeof(int32_t) * 2 * (size_t)(list_base[E] > 0 ? list_base[E] : 1));
+        list = own;
+    }
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < T; t++)
+            for (int j = 0; j < k; j++) {
+                int64_t p = ((int64_t)r * T + t) * k + j;
+                if (pair_row[p] < 0) continue;
+                int e = topk_idx[p];
+                int64_t at = list_base[e] + pair_row[p];
+                list[2 * at + 0] = r;
+                list[2 * at + 1] = t;
+            }
+
+    /* offset of source rank r inside list[e]: first entry with src rank >= r */
+    for (int e = 0; e < E; e++) {
+        for (int r = 0; r < R; r++) {
+            int32_t pos = recv_count[e];
+            for (int32_t i = 0; i < recv_count[e]; i++) {
+                if (list[2 * (list_base[e] + i)] >= r) { pos = i; break; }
+            }
+            expert_rank_offset[(int64_t)e * R + r] = pos;
+        }
+    }
+    free(own);
+    return status;
+}
+
+/*
+ * Dispatch ([P1] Buffer.low_latency_dispatch with use_fp8=False): every live
+ * pair's token row is copied, bit for bit, into its expert's list position.
+ * Only list entries are materialised (packed, expert-major at list_base[e]),
+ * never the empty tail of the receive slab.  Rows past the slab capacity are
+ * not sent.
+ *   x       [R,T,H] bf16 bits
+ *   packed  [list_base[E], H] bf16 bits (rows past capacity left untouched)
+ */
+int oracle_dispatch(int R, int T, int k, int E, int H, const uint16_t *x, const int32_t *topk_idx,
+                    const int32_t *pair_row, const int64_t *list_base, uint16_t *packed) {
+    int status = 0;
+    const int64_t capacity = (int64_t)R * T;
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < T; t++)
+            for (int j = 0; j < k; j++) {
+                int64_t p = ((int64_t)r * T + t) * k + j;
+                int32_t row = pair_row[p];
+                if (row < 0) continue;
+                if (row >= capacity) { status |= ORACLE_OVERFLOW; continue; }
+                int e = topk_idx[p];
+                if (e < 0 || e >= E) continue;
+                const uint16_t *src = x + ((int64_t)r * T + t) * H;
+                uint16_t *dst = packed + (list_base[e] + row) * H;
+                for (int h = 0; h < H; h++) dst[h] = src[h];
+            }
+    return status;
+}
+
+/*
+ * Combine ([P1] Buffer.low_latency_combine, "reduce with weights"; active
+ * mask per [P4]) for a list of tokens.  For token (r, t):
+ *   out[h] = sum over slots j whose pair is live under active_now and whose
+ *            row is inside the capacity of  w[r,t,j] * y[e][row][h]
+ * accumulated in float64.  Rows of an inactive source rank are 0.
+ *   y        bf16 bits; row (e, row) lives at y + (y_row_base[e] + row) * H
+ *   tokens   [n_tokens, 2] (r, t) pairs, or NULL for every (r, t) in order
+ *   out      float64 [n_tokens, H]
+ */
+int oracle_combine(int R, int T, int k, int E, int H, const uint16_t *y, const int64_t *y_row_base,
+                   const int32_t *topk_idx, const float *topk_weights, const int32_t *pair_row,
+                   const uint8_t *active_now, const int32_t *tokens, int64_t n_tokens, double *out) {
+    int status = 0;
+    const int E_local = E / R;
+    const int64_t capacity = (int64_t)R * T;
+    if (tokens == NULL) n_tokens = (int64_t)R * T;
+    for (int64_t i = 0; i < n_tokens; i++) {
+        int r = tokens ? tokens[2 * i] : (int)(i / T);
+        int t = tokens ? tokens[2 * i + 1] : (int)(i % T);
+        double *o = out + i * H;
+        for (int h = 0; h < H; h++) o[h] = 0.0;
+        if (!active_now[r]) continue;
+        for (int j = 0; j < k; j++) {
+            int64_t p = ((int64_t)r * T + t) * k + j;
+            int32_t row = pair_row[p];
+            int e = topk_idx[p];
+            if (row < 0) continue;
+            if (e < 0 || e >= E) continue;
+            if (!active_now[e / E_local]) continue;
+            if (row >= capacity) { status |= ORACLE_OVERFLOW; continue; }
+            double w = (double)topk_weights[p];
+            const uint16_t *yr = y + (y_row_base[e] + row) * H;
+            for (int h = 0; h < H; h++) o[h] += w * bf16_to_double(yr[h]);
+        }
+    }
+    return status;
+}
+
+/*
+ * Load computation, placement planning and routing expansion ([P3] GPU
+ * operations: load_compute, placement, reroute).
+ *   load        [E_log]   (token, slot) pairs routed to each logical expert
+ *   n_rep       [E_log]   replicas per logical expert (sum = E_log + n_extra)
+ *   phys_base   [E_log+1] exclusive prefix sum of n_rep
+ *   topk_phys   [R,T,k]   physical id, -1 where the logical id is -1 or bad
+ */
+int oracle_reroute(int R, int T, int k, int E_log, int n_extra, const int32_t *topk_logical,
+                   int32_t *load, int32_t *n_rep, int32_t *phys_base, int32_t *topk_phys) {
+    int status = 0;
+    const int64_t n_pairs = (int64_t)R * T * k;
+
+    for (int e = 0; e < E_log; e++) load[e] = 0;
+    for (int64_t p = 0; p < n_pairs; p++) {
+        int e = topk_logical[p];
+        if (e >= 0 && e < E_log) load[e] += 1;
+        else if (e != -1) status |= ORACLE_BAD_EXPERT;
+    }
+
+    for (int e = 0; e < E_log; e++) n_rep[e] = 1;
+    for (int step = 0; step < n_extra; step++) {
+        int best = 0;
+        for (int e = 1; e < E_log; e++) {
+            /* load[e]/n_rep[e] > load[best]/n_rep[best], compared exactly */
+            int64_t lhs = (int64_t)load[e] * n_rep[best];
+            int64_t rhs = (int64_t)load[best] * n_rep[e];
+            if (lhs > rhs) best = e;
+        }
+        n_rep[best] += 1;
+    }
+
+    phys_base[0] = 0;
+    for (int e = 0; e < E_log; e++) phys_base[e + 1] = phys_base[e] + n_rep[e];
+
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < T; t++)
+            for (int j = 0; j < k; j++) {
+                int64_t p = ((int64_t)r * T + t) * k + j;
+                int e = topk_logical[p];
+                if (e < 0 || e >= E_log) { topk_phys[p] = -1; continue; }
+                int64_t global_token = (int64_t)r * T + t;
+                topk_phys[p] = phys_base[e] + (int32_t)(global_token % n_rep[e]);
+            }
+    return status;
+}

@@ -1,0 +1,374 @@
+"""Pins that tie the CPU oracle to something other than itself.
+
+Every ``pin_*`` function takes a loaded oracle library and raises
+``AssertionError`` when the oracle disagrees with:
+
+* hand-worked examples (``tests/golden/*.json``), derived on paper from the
+  definitions on the pages;
+* brute force through a library routine (a stable ``numpy.lexsort`` of the
+  live pairs, ``numpy.bincount``), which shares no loop with the oracle;
+* invariants the definitions imply (counts sum to the live pairs, offsets are
+  prefix sums, every live pair lands exactly once, ...);
+* closed-form special cases of combine (one-hot weights return the token,
+  scaling the weights scales the result, ...);
+* exhaustive search (greedy replica placement reaches the min-max optimum).
+
+The same functions run against deliberately broken copies of the oracle in
+``test_oracle_mutants.py`` to show that a plausible slip fails at least one.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+
+import oracle
+from combine_get_dispatch_histogram_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------- brute force
+
+def brute_layout(topk_idx, active, E):
+    """Layout via a stable lexsort of the live pairs (independent of the oracle's loop)."""
+    topk_idx = np.asarray(topk_idx, np.int64)
+    active = np.asarray(active, bool)
+    R, T, k = topk_idx.shape
+    El = E // R
+    rr, tt, jj = np.meshgrid(np.arange(R), np.arange(T), np.arange(k), indexing="ij")
+    e = topk_idx
+    valid = (e >= 0) & (e < E)
+    dst = np.where(valid, e // El, 0)
+    live = valid & active[rr] & active[dst]
+    flat = np.flatnonzero(live.ravel())
+    ee = e.ravel()[flat]
+    order = np.lexsort((jj.ravel()[flat], tt.ravel()[flat], rr.ravel()[flat], ee))
+    se = ee[order]
+    pos = np.arange(len(order)) - np.searchsorted(se, se, side="left")
+    pair_row = np.full(R * T * k, -1, np.int64)
+    pair_row[flat[order]] = pos
+    recv_count = np.bincount(ee, minlength=E)
+    C = np.zeros((R, E), np.int64)
+    np.add.at(C, (rr.ravel()[flat], ee), 1)
+    offs = np.concatenate([np.zeros((1, E), np.int64), np.cumsum(C, axis=0)[:-1]], axis=0).T
+    itr = np.zeros((R, T, R), np.int64)
+    itr[rr.ravel()[flat], tt.ravel()[flat], dst.ravel()[flat]] = 1
+    src = np.stack([rr.ravel()[flat][order], tt.ravel()[flat][order]], axis=1)
+    return dict(pair_row=pair_row.reshape(R, T, k), recv_count=recv_count, num_tokens_per_expert=C,
+                expert_rank_offset=offs, is_token_in_rank=itr, num_tokens_per_rank=itr.sum(axis=1),
+                src_list=src, live=live)
+
+
+def _random_case(rng, R=None, El=None, k=None, T=None, p_none=0.15, p_mask=0.3, dup=False):
+    R = R or int(rng.integers(1, 5))
+    El = El or int(rng.integers(1, 5))
+    E = R * El
+    k = k or int(rng.integers(1, min(E, 4) + 1))
+    T = T or int(rng.integers(1, 17))
+    if dup:
+        idx = rng.integers(0, E, size=(R, T, k))
+    else:
+        idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k)
+    idx = np.where(rng.random((R, T, k)) < p_none, -1, idx).astype(np.int32)
+    active = np.ones(R, np.uint8)
+    if R > 1 and rng.random() < p_mask:
+        active[rng.integers(0, R)] = 0
+    return idx, active, E
+
+
+def _check_layout_equal(lay, ref, tag=""):
+    for key in ("pair_row", "recv_count", "num_tokens_per_expert", "expert_rank_offset",
+                "is_token_in_rank", "num_tokens_per_rank", "src_list"):
+        a = np.asarray(lay[key], np.int64)
+        b = np.asarray(ref[key], np.int64)
+        assert a.shape == b.shape and np.array_equal(a, b), f"{tag} {key} differs"
+
+
+# ----------------------------------------------------------------------------- layout pins
+
+def pin_layout_golden(lib):
+    g = _golden("layout_tiny.json")
+    idx = np.array(g["topk_idx"], np.int32)
+    for case in g["cases"]:
+        lay = oracle.layout(idx, np.array(case["active"], np.uint8), g["E"], lib=lib)
+        for key in ("pair_row", "recv_count", "num_tokens_per_expert", "is_token_in_rank",
+                    "num_tokens_per_rank", "expert_rank_offset"):
+            assert np.array_equal(np.asarray(lay[key]), np.array(case[key])), f"golden {key}"
+        for e, lst in enumerate(case["src_lists"]):
+            a, b = lay.list_base[e], lay.list_base[e + 1]
+            got = lay.src_list[a:b].tolist()
+            assert got == lst, f"golden src list of expert {e}: {got} != {lst}"
+        assert lay.status == 0
+
+
+def pin_layout_bruteforce(lib):
+    rng = np.random.default_rng(1234)
+    for it in range(300):
+        idx, active, E = _random_case(rng, dup=(it % 5 == 0))
+        lay = oracle.layout(idx, active, E, lib=lib)
+        _check_layout_equal(lay, brute_layout(idx, active, E), f"case {it}")
+
+
+def pin_layout_invariants(lib):
+    """Decode-shaped routing: sums, offsets, capacity, token counts."""
+    w = inputs.decode()
+    inp = inputs.make_inputs(w, tokens=False)
+    for active in (inp.active, np.array([1, 1, 1, 1, 1, 0, 1, 1], np.uint8)):
+        lay = oracle.layout(inp.topk_idx, active, w.num_experts, lib=lib)
+        R, T, k, E = w.num_ranks, w.num_tokens, w.num_topk, w.num_experts
+        El = E // R
+        live = brute_layout(inp.topk_idx, active, E)["live"]
+        L = int(live.sum())
+        assert int(lay.recv_count.sum()) == L
+        assert np.array_equal(lay.num_tokens_per_expert.sum(axis=1), live.reshape(R, -1).sum(axis=1))
+        if active.all():
+            assert int(lay.recv_count.sum()) == R * T * k       # counts sum to T*k per rank
+            assert np.all(lay.num_tokens_per_expert.sum(axis=1) == T * k)
+        off = lay.expert_rank_offset
+        assert np.all(np.diff(off, axis=1) >= 0)
+        assert np.array_equal(off[:, -1] + lay.num_tokens_per_expert[-1], lay.recv_count)
+        assert np.array_equal(np.diff(off, axis=1), lay.num_tokens_per_expert[:-1].T)
+        assert np.array_equal(lay.num_tokens_per_rank, lay.is_token_in_rank.sum(axis=1))
+        assert np.all(lay.recv_count <= R * T)
+        # a masked rank neither sends nor receives
+        for d in np.flatnonzero(active == 0):
+            assert lay.recv_count[d * El:(d + 1) * El].sum() == 0
+            assert lay.num_tokens_per_rank[d].sum() == 0 and lay.num_tokens_per_rank[:, d].sum() == 0
+        # rows of one expert are the distinct values 0..recv_count-1
+        pr = lay.pair_row.ravel()
+        ee = inp.topk_idx.ravel()
+        for e in range(0, E, 17):
+            rows = np.sort(pr[(ee == e) & (pr >= 0)])
+            assert np.array_equal(rows, np.arange(lay.recv_count[e]))
+
+
+def pin_layout_status(lib):
+    idx = np.array([[[0, 9], [-1, 1]], [[-2, 3], [2, 3]]], np.int32)     # 9 and -2 are bad ids
+    lay = oracle.layout(idx, np.ones(2, np.uint8), 4, lib=lib)
+    assert lay.status & oracle.BAD_EXPERT
+    assert lay.pair_row[0, 0, 1] == -1 and lay.pair_row[1, 0, 0] == -1
+    # duplicates: every token picks expert 0 twice -> 2*R*T rows > capacity R*T
+    R, T, k = 2, 3, 2
+    idx = np.zeros((R, T, k), np.int32)
+    lay = oracle.layout(idx, np.ones(R, np.uint8), 2, lib=lib)
+    assert lay.status & oracle.OVERFLOW
+    assert lay.recv_count[0] == R * T * k
+    assert np.array_equal(np.sort(lay.pair_row.ravel()), np.arange(R * T * k))
+
+
+# ----------------------------------------------------------------------------- dispatch pins
+
+def pin_dispatch_golden(lib):
+    g = _golden("layout_tiny.json")
+    idx = np.array(g["topk_idx"], np.int32)
+    R, T, E, H = g["R"], g["T"], g["E"], 8
+    x = np.arange(R * T * H, dtype=np.uint16).reshape(R, T, H) * 3 + 7
+    for case in g["cases"]:
+        lay = oracle.layout(idx, np.array(case["active"], np.uint8), E, lib=lib)
+        packed, st = oracle.dispatch(x, idx, lay, lib=lib)
+        assert st == 0
+        want = [x[r, t] for lst in case["src_lists"] for (r, t) in lst]
+        want = np.array(want, np.uint16).reshape(-1, H)
+        assert np.array_equal(packed, want), "golden dispatch rows"
+
+
+def pin_dispatch_bijection(lib):
+    rng = np.random.default_rng(99)
+    for it in range(120):
+        idx, active, E = _random_case(rng, dup=(it % 4 == 0))
+        R, T, k = idx.shape
+        H = 8 * int(rng.integers(1, 4))
+        x = rng.integers(0, 1 << 16, size=(R, T, H), dtype=np.uint16)
+        lay = oracle.layout(idx, active, E, lib=lib)
+        packed, _ = oracle.dispatch(x, idx, lay, lib=lib)
+        ref = brute_layout(idx, active, E)
+        live = ref["live"]
+        # the multiset of (src_rank, src_token, expert) over rows equals the live pairs
+        got = sorted((int(r), int(t), e) for e in range(E)
+                     for (r, t) in lay.src_list[lay.list_base[e]:lay.list_base[e + 1]])
+        rr, tt, jj = np.nonzero(live)
+        want = sorted((int(r), int(t), int(idx[r, t, j])) for r, t, j in zip(rr, tt, jj))
+        assert got == want, f"case {it}: dispatched pairs are not the live pairs"
+        cap = R * T
+        for e in range(E):
+            a, b = lay.list_base[e], lay.list_base[e + 1]
+            src = lay.src_list[a:b]
+            keys = src[:, 0].astype(np.int64) * T + src[:, 1]
+            assert np.all(np.diff(keys) >= 0), "rows of an expert not ordered by (src_rank, token)"
+            for i in range(min(b - a, cap)):
+                r, t = src[i]
+                assert np.array_equal(packed[a + i], x[r, t]), "payload row differs from its source"
+
+
+# ----------------------------------------------------------------------------- combine pins
+
+def _slab_row_base(E, cap):
+    return np.arange(E, dtype=np.int64) * cap
+
+
+def pin_combine_golden(lib):
+    g = _golden("layout_tiny.json")
+    c = _golden("combine_tiny.json")
+    idx = np.array(g["topk_idx"], np.int32)
+    R, T, E, H = g["R"], g["T"], g["E"], c["H"]
+    cap = R * T
+    lay = oracle.layout(idx, np.ones(R, np.uint8), E, lib=lib)
+    vals = np.array([[[8 * e + row + h / 4 for h in range(H)] for row in range(cap)] for e in range(E)],
+                    np.float32)
+    y = (vals.view(np.uint32) >> 16).astype(np.uint16)        # exact: values fit bf16
+    assert np.array_equal(oracle.bf16_bits_to_f64(y), vals.astype(np.float64))
+    w = np.array(c["topk_weights"], np.float32)
+    for case in c["cases"]:
+        out, _ = oracle.combine(y, _slab_row_base(E, cap), idx, w, lay.pair_row,
+                                np.array(case["active_now"], np.uint8), E, lib=lib)
+        want = np.array(case["out"], np.float64)
+        # 0.3 and 0.7 never meet a live row, every other weight is a dyadic rational
+        assert np.array_equal(out, want), f"golden combine {case['active_now']}"
+
+
+def _identity_case(rng, R, El, k, T, H):
+    E = R * El
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k).astype(np.int32)
+    x = inputs.bf16_tokens(rng, R * T, H).reshape(R, T, H)
+    return idx, x, E
+
+
+def pin_combine_special_cases(lib):
+    rng = np.random.default_rng(7)
+    R, El, k, T, H = 3, 3, 4, 10, 24
+    idx, x, E = _identity_case(rng, R, El, k, T, H)
+    act = np.ones(R, np.uint8)
+    lay = oracle.layout(idx, act, E, lib=lib)
+    packed, _ = oracle.dispatch(x, idx, lay, lib=lib)
+    base = lay.list_base[:-1]
+    xf = oracle.bf16_bits_to_f64(x)
+    # one-hot weights on a random slot return the token exactly
+    hot = rng.integers(0, k, size=(R, T))
+    w = np.zeros((R, T, k), np.float32)
+    w[np.arange(R)[:, None], np.arange(T)[None, :], hot] = 1.0
+    out, _ = oracle.combine(packed, base, idx, w, lay.pair_row, act, E, lib=lib)
+    assert np.array_equal(out, xf), "one-hot combine != token"
+    # k = 1, weight 1: identity
+    lay1 = oracle.layout(idx[:, :, :1].copy(), act, E, lib=lib)
+    p1, _ = oracle.dispatch(x, idx[:, :, :1].copy(), lay1, lib=lib)
+    out1, _ = oracle.combine(p1, lay1.list_base[:-1], idx[:, :, :1].copy(), np.ones((R, T, 1), np.float32),
+                             lay1.pair_row, act, E, lib=lib)
+    assert np.array_equal(out1, xf), "k=1 combine != token"
+    # softmax weights with identity experts return the token within the weights' rounding
+    ws = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+    outs, _ = oracle.combine(packed, base, idx, ws, lay.pair_row, act, E, lib=lib)
+    wsum = ws.astype(np.float64).sum(axis=2, keepdims=True)
+    assert np.all(np.abs(wsum - 1) < 1e-6)
+    assert np.allclose(outs, xf * wsum, rtol=1e-12, atol=0), "identity experts do not return w_sum * x"
+    assert np.all(np.abs(outs - xf) <= 2e-6 * np.abs(xf) + 1e-300)
+    # scaling the weights by 2 scales the result exactly
+    out2, _ = oracle.combine(packed, base, idx, 2 * ws, lay.pair_row, act, E, lib=lib)
+    assert np.array_equal(out2, 2 * outs)
+    # additivity over slots: the full reduce equals the ordered sum of one-slot reduces
+    y = inputs.bf16_tokens(rng, packed.shape[0], H)
+    full, _ = oracle.combine(y, base, idx, ws, lay.pair_row, act, E, lib=lib)
+    acc = np.zeros_like(full)
+    for j in range(k):
+        wj = np.zeros_like(ws)
+        wj[:, :, j] = ws[:, :, j]
+        part, _ = oracle.combine(y, base, idx, wj, lay.pair_row, act, E, lib=lib)
+        acc = acc + part
+    assert np.array_equal(full, acc), "combine is not the slot-ordered sum of its terms"
+    # each one-slot term is w * y[row of that slot]
+    for j in range(k):
+        wj = np.zeros_like(ws)
+        wj[:, :, j] = ws[:, :, j]
+        part, _ = oracle.combine(y, base, idx, wj, lay.pair_row, act, E, lib=lib)
+        e = idx[:, :, j]
+        rows = base[e] + lay.pair_row[:, :, j]
+        want = ws[:, :, j, None].astype(np.float64) * oracle.bf16_bits_to_f64(y[rows])
+        assert np.array_equal(part, want), f"slot {j} term is not w * y[e][row]"
+
+
+def pin_combine_mask(lib):
+    rng = np.random.default_rng(11)
+    R, El, k, T, H = 4, 2, 3, 9, 16
+    idx, x, E = _identity_case(rng, R, El, k, T, H)
+    all_on = np.ones(R, np.uint8)
+    lay = oracle.layout(idx, all_on, E, lib=lib)
+    y = inputs.bf16_tokens(rng, int(lay.list_base[-1]), H)
+    base = lay.list_base[:-1]
+    ws = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+    full, _ = oracle.combine(y, base, idx, ws, lay.pair_row, all_on, E, lib=lib)
+    for d in range(R):
+        now = all_on.copy()
+        now[d] = 0
+        got, _ = oracle.combine(y, base, idx, ws, lay.pair_row, now, E, lib=lib)
+        assert np.all(got[d] == 0), "inactive source rank must come out as zeros"
+        # dropping rank d's experts equals zeroing the weights of those slots
+        wz = ws.copy()
+        wz[(idx // El) == d] = 0
+        ref, _ = oracle.combine(y, base, idx, wz, lay.pair_row, all_on, E, lib=lib)
+        ref[d] = 0
+        assert np.array_equal(got, ref), "mask flip must drop exactly the masked experts' terms"
+    assert np.any(full != 0)
+
+
+# ----------------------------------------------------------------------------- reroute pins
+
+def pin_reroute_golden(lib):
+    g = _golden("reroute_tiny.json")
+    for case in g["cases"]:
+        idx = np.array(case["topk_idx"], np.int32)
+        res = oracle.reroute(idx, case["E_logical"], case["num_extra"], lib=lib)
+        for key in ("load", "num_replicas", "phys_base", "topk_idx_phys"):
+            assert np.array_equal(res[key], np.array(case[key])), f"golden reroute {key}"
+
+
+def _min_max_ratio(load, extra):
+    best = None
+    E = len(load)
+    for alloc in itertools.product(range(extra + 1), repeat=E):
+        if sum(alloc) != extra:
+            continue
+        m = max(Fraction(int(load[e]), 1 + alloc[e]) for e in range(E))
+        best = m if best is None or m < best else best
+    return best
+
+
+def pin_reroute_invariants(lib):
+    rng = np.random.default_rng(5)
+    for it in range(60):
+        E = int(rng.integers(1, 5))
+        extra = int(rng.integers(0, 5))
+        R, T, k = int(rng.integers(1, 3)), int(rng.integers(1, 7)), int(rng.integers(1, E + 1))
+        idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k)
+        skew = rng.random() < 0.5
+        if skew:
+            idx = np.where(rng.random((R, T, k)) < 0.6, 0, idx)
+        idx = np.where(rng.random((R, T, k)) < 0.1, -1, idx).astype(np.int32)
+        res = oracle.reroute(idx, E, extra, lib=lib)
+        load = np.bincount(idx[idx >= 0], minlength=E)
+        assert np.array_equal(res["load"], load)
+        n = res["num_replicas"]
+        assert n.sum() == E + extra and n.min() >= 1
+        assert np.array_equal(res["phys_base"], np.concatenate([[0], np.cumsum(n)]))
+        got = max(Fraction(int(load[e]), int(n[e])) for e in range(E))
+        assert got == _min_max_ratio(load, extra), "greedy placement is not min-max optimal"
+        phys = res["topk_idx_phys"]
+        assert np.array_equal(phys < 0, idx < 0)
+        pc = np.bincount(phys[phys >= 0], minlength=E + extra)
+        for e in range(E):
+            b = res["phys_base"]
+            assert pc[b[e]:b[e + 1]].sum() == load[e]
+            # round-robin over replicas: replica loads differ by at most the token multiplicity
+            assert np.all((phys[idx == e] >= b[e]) & (phys[idx == e] < b[e + 1]))
+
+
+ALL_PINS = [pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
+            pin_dispatch_golden, pin_dispatch_bijection, pin_combine_golden,
+            pin_combine_special_cases, pin_combine_mask, pin_reroute_golden, pin_reroute_invariants]

@@ -1,0 +1,72 @@
+"""Plant plausible mistakes in a copy of the oracle and check the pins catch each one.
+
+Every mutant is a one-line textual change to a temporary copy of
+``oracle/ep_oracle.c`` (the real oracle is never modified), built with gcc on
+the CPU.  A mutant that no pin rejects would mean the oracle's parity rests on
+that line alone.
+"""
+import os
+import shutil
+
+import pytest
+
+import oracle
+import oracle_pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ep_oracle.c")
+
+MUTANTS = {
+    # layout
+    "dst_rank_modulo": ("if (!active[e / E_local]) return 0;", "if (!active[e % E_local]) return 0;"),
+    "no_src_mask": ("if (!active[r]) return 0;", ""),
+    "no_dst_mask": ("if (!active[e / E_local]) return 0;", ""),
+    "token_in_rank_index": ("* R + e / E_local] = 1;", "* R + e % R] = 1;"),
+    "offset_strict": ("if (list[2 * (list_base[e] + i)] >= r)", "if (list[2 * (list_base[e] + i)] > r)"),
+    "row_one_based": ("pair_row[p] = recv_count[e];\n                recv_count[e] += 1;",
+                      "recv_count[e] += 1;\n                pair_row[p] = recv_count[e] - (e > 0);"),
+    "per_expert_count_wrong_rank": ("num_tokens_per_expert[(int64_t)r * E + e] += 1;",
+                                    "num_tokens_per_expert[(int64_t)(R - 1 - r) * E + e] += 1;"),
+    "bad_id_not_flagged": ("if (e < -1 || e >= E) status |= ORACLE_BAD_EXPERT;", ""),
+    # dispatch
+    "dispatch_src_transposed": ("const uint16_t *src = x + ((int64_t)r * T + t) * H;",
+                                "const uint16_t *src = x + ((int64_t)t * R + r) * H;"),
+    "dispatch_drop_last_elem": ("for (int h = 0; h < H; h++) dst[h] = src[h];",
+                                "for (int h = 0; h < H - 1; h++) dst[h] = src[h];"),
+    # combine
+    "combine_no_weight": ("o[h] += w * bf16_to_double(yr[h]);", "o[h] += bf16_to_double(yr[h]);"),
+    "combine_weight_reversed": ("double w = (double)topk_weights[p];",
+                                "double w = (double)topk_weights[p - j + (k - 1 - j)];"),
+    "combine_src_not_zeroed": ("if (!active_now[r]) continue;", ""),
+    "combine_no_mask_recheck": ("if (!active_now[e / E_local]) continue;", ""),
+    "combine_wrong_row_base": ("const uint16_t *yr = y + (y_row_base[e] + row) * H;",
+                               "const uint16_t *yr = y + (y_row_base[e] + row) * H + (row > 0);"),
+    "combine_negative_sign": ("o[h] += w * bf16_to_double(yr[h]);", "o[h] -= w * bf16_to_double(yr[h]);"),
+    # reroute
+    "reroute_tie_highest": ("if (lhs > rhs) best = e;", "if (lhs >= rhs) best = e;"),
+    "reroute_local_token": ("topk_phys[p] = phys_base[e] + (int32_t)(global_token % n_rep[e]);",
+                            "topk_phys[p] = phys_base[e] + (int32_t)(t % n_rep[e]);"),
+    "reroute_ratio_inverted": ("int64_t lhs = (int64_t)load[e] * n_rep[best];",
+                               "int64_t lhs = (int64_t)load[e] * n_rep[e];"),
+    "reroute_base_inclusive": ("phys_base[e + 1] = phys_base[e] + n_rep[e];",
+                               "phys_base[e + 1] = phys_base[e] + n_rep[e] - (e == 0);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    find, repl = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(find) >= 1, f"mutation site for {name} not found"
+    mutated = src.replace(find, repl, 1)
+    path = tmp_path / "ep_oracle_mutant.c"
+    path.write_text(mutated)
+    so = str(tmp_path / "libmutant.so")
+    oracle.build(force=True, src=str(path), out=so, werror=False)
+    lib = oracle.load(so)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(lib)
+        except Exception as exc:  # AssertionError, or an index error from garbage output
+            caught.append((pin.__name__, type(exc).__name__))
+    assert caught, f"mutant {name} passed every pin"
