@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""Benchmark: expert-parallel layout -> dispatch -> combine on B200, one JSON line.
+
+A step is one pass of the whole hot path over one batch: ``ep_layout``,
+``ep_dispatch`` and ``ep_combine`` (plus ``ep_reroute`` first for the replica
+workload) through the C ABI, on inputs already resident in HBM.  The default
+workload is the prefill shape (R=8 emulated ranks, E=256 experts, top-8 with
+Zipf(1.2) popularity, T=4096 tokens per rank, hidden 7168): its receive slab
+is 120 GB, far larger than L2, so no flush is needed between steps.
+
+Reported:
+  value        effective HBM GB/s of the whole step: the algorithmic bytes of
+               dispatch + combine (one read of every live token row plus one
+               write per live pair, and the mirror image for combine) divided
+               by the step time, summed over ranks and divided by the slowest
+               rank's time;
+  dispatch/combine/layout microseconds per call, from CUDA events recorded on
+               the launching stream around every call in the timed region;
+  roofline     the dominant kernel's achieved GB/s against the measured copy
+               bandwidth of this GPU type (MEASURED_PEAKS.json);
+  e2e          the same metric with host buffers: every step copies its inputs
+               from pinned host memory and reads the output back;
+  cpu_baseline the plain single-threaded CPU oracle on a bounded sample of the
+               same workload (rank 0, one GPU only).
+
+``--impl reference`` times that CPU oracle alone as the reference arm.
+Multi-GPU (torchrun): every rank runs an independent replica (the emulated
+EP world lives inside one GPU); NCCL only carries the barrier and the max of
+the per-rank times.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from combine_get_dispatch_histogram_b200 import inputs  # noqa: E402
+
+METRIC = "dispatch & combine µs/call and effective HBM GB/s (fraction of ~8 TB/s)"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = {"dispatch_kernel": "ep_dispatch.cu", "combine_kernel": "ep_combine.cu"}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_hbm_gbs():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_sha(fname: str) -> str:
+    path = os.path.join(ROOT, "combine_get_dispatch_histogram_b200", "csrc", fname)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+    except Exception:
+        return None
+    if rec.get("source_sha") != source_sha(KERNEL_SOURCES[kernel]):
+        return None
+    per = rec.get("per_workload", {}).get(workload)
+    return None if per is None else int(per)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ep_bench_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu_index), "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                        rows.append(parts)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(float(r[2]) for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def algorithmic_bytes(H: int, tokens_sent: int, live_pairs: int, tokens_out: int):
+    row = 2 * H
+    return row * (tokens_sent + live_pairs), row * (live_pairs + tokens_out)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from combine_get_dispatch_histogram_b200 import ep
+
+    ep.load_library()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = inputs.named(args.workload)
+    inp = inputs.make_inputs(w)
+    R, T, k, H = w.num_ranks, w.num_tokens, w.num_topk, w.hidden
+    E = w.num_physical
+    cap = R * T
+    reroute = w.num_extra > 0
+
+    slab_bytes = E * cap * H * 2
+    free, _ = torch.cuda.mem_get_info(dev)
+    if free < slab_bytes + (4 << 30):
+        raise SystemExit(f"workload {w.name} needs {slab_bytes / 1e9:.1f} GB for the receive slab; "
+                         f"{free / 1e9:.1f} GB free")
+
+    # device-resident inputs and preallocated outputs (the library allocates nothing)
+    idx_log = torch.from_numpy(inp.topk_idx).to(dev)
+    wts = torch.from_numpy(inp.topk_weights).to(dev)
+    act = torch.from_numpy(inp.active).to(dev)
+    x = torch.from_numpy(inp.x.view(np.int16)).to(dev).view(torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    recv_x = torch.empty((E, cap, H), dtype=torch.bfloat16, device=dev)
+    src_info = torch.empty((E, cap, 2), dtype=torch.int32, device=dev)
+    out = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
+    lay_ws = torch.empty(max(16, ep.ep_layout_workspace_bytes(R, T, k, E, H)), dtype=torch.uint8, device=dev)
+    rr_ws = rr_out = None
+    if reroute:
+        rr_ws = torch.empty(max(16, ep.ep_reroute_workspace_bytes(R, T, k, w.num_experts)), dtype=torch.uint8,
+                            device=dev)
+        rr_out = dict(load=torch.empty(w.num_experts, dtype=torch.int32, device=dev),
+                      num_replicas=torch.empty(w.num_experts, dtype=torch.int32, device=dev),
+                      phys_base=torch.empty(w.num_experts + 1, dtype=torch.int32, device=dev),
+                      topk_idx_phys=torch.empty((R, T, k), dtype=torch.int32, device=dev))
+    lay = ep.DispatchLayout(torch.empty((R, E), dtype=torch.int32, device=dev),
+                            torch.empty((R, R), dtype=torch.int32, device=dev),
+                            torch.empty((R, T, R), dtype=torch.uint8, device=dev),
+                            torch.empty((E,), dtype=torch.int32, device=dev),
+                            torch.empty((E, R), dtype=torch.int32, device=dev),
+                            torch.empty((R, T, k), dtype=torch.int32, device=dev), status)
+    stream = torch.cuda.Stream(dev)
+    n_ev = 4
+    launches_per_step = 5 + (2 if reroute else 0)
+
+    def step(events=None):
+        def mark(i):
+            if events is not None:
+                events[i].record(stream)
+        mark(0)
+        idx = idx_log
+        if reroute:
+            ep.ep_reroute(idx_log, w.num_experts, w.num_extra, workspace=rr_ws, out=rr_out, status=status,
+                          stream=stream)
+            idx = rr_out["topk_idx_phys"]
+        ep.ep_layout(idx, act, E, hidden=H, workspace=lay_ws, out=lay, status=status, stream=stream)
+        mark(1)
+        ep.ep_dispatch(x, idx, lay.pair_row, E, recv_x=recv_x, src_info=src_info, status=status, stream=stream)
+        mark(2)
+        ep.ep_combine(recv_x, idx, wts, lay.pair_row, act, out=out, status=status, stream=stream)
+        mark(3)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    if int(status.item()) != 0:
+        raise SystemExit(f"device status {int(status.item())} after warm-up")
+    live_pairs = int(lay.recv_count.sum().item())
+    tokens_sent = int(lay.is_token_in_rank.view(R * T, R).amax(dim=1).sum().item())
+    tokens_out = R * T
+    d_bytes, c_bytes = algorithmic_bytes(H, tokens_sent, live_pairs, tokens_out)
+
+    # ---------------------------------------------------------------- timed region (device resident)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(gpu_index_of(local_rank))
+    with sampler, torch.cuda.stream(stream):
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(events[i])
+        t_end.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    total_ms = t_start.elapsed_time(t_end)
+    lay_ms = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
+    dis_ms = sum(e[1].elapsed_time(e[2]) for e in events) / args.steps
+    com_ms = sum(e[2].elapsed_time(e[3]) for e in events) / args.steps
+    if int(status.item()) != 0:
+        raise SystemExit(f"device status {int(status.item())} after the timed steps")
+
+    # ---------------------------------------------------------------- e2e: host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        h_idx = torch.from_numpy(inp.topk_idx).pin_memory()
+        h_w = torch.from_numpy(inp.topk_weights).pin_memory()
+        h_act = torch.from_numpy(inp.active).pin_memory()
+        h_x = torch.from_numpy(inp.x.view(np.int16)).pin_memory()
+        h_out = torch.empty((R, T, H), dtype=torch.int16).pin_memory()
+        h2d = h_idx.numel() * 4 + h_w.numel() * 4 + h_act.numel() + h_x.numel() * 2
+        d2h = h_out.numel() * 2
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.e2e_steps):
+                idx_log.copy_(h_idx, non_blocking=True)
+                wts.copy_(h_w, non_blocking=True)
+                act.copy_(h_act, non_blocking=True)
+                x.view(torch.int16).copy_(h_x, non_blocking=True)
+                step()
+                h_out.copy_(out.view(torch.int16), non_blocking=True)
+            e1.record(stream)
+            stream.synchronize()
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        e2e = dict(ms=e2e_ms, h2d=h2d, d2h=d2h)
+        assert np.array_equal(h_out.numpy(), out.view(torch.int16).cpu().numpy())
+
+    # ---------------------------------------------------------------- reduce over ranks
+    vals = torch.tensor([total_ms, lay_ms, dis_ms, com_ms, e2e["ms"] if e2e else 0.0], dtype=torch.float64,
+                        device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, lay_ms, dis_ms, com_ms, e2e_ms = vals.tolist()
+    ms_per_step = total_ms / args.steps
+    step_bytes = d_bytes + c_bytes
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    dis_gbs = d_bytes / (dis_ms * 1e-3) / 1e9
+    com_gbs = c_bytes / (com_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_gbs()
+    dom = ("dispatch_kernel", d_bytes, dis_ms) if dis_ms >= com_ms else ("combine_kernel", c_bytes, com_ms)
+    achieved = dom[1] / (dom[2] * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name} " + " ".join(f"{k_}={v}" for k_, v in w.describe().items()),
+                   **w.describe(), "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
+                   "emulated_ep_ranks": R,
+                   "l2": "no flush: inputs larger than L2 (x %.0f MB, receive slab %.1f GB)"
+                         % (R * T * H * 2 / 1e6, slab_bytes / 1e9)},
+        "dispatch_us": round(dis_ms * 1e3, 2),
+        "combine_us": round(com_ms * 1e3, 2),
+        "layout_us": round(lay_ms * 1e3, 2),
+        "dispatch_gbs": round(dis_gbs, 1),
+        "combine_gbs": round(com_gbs, 1),
+        "dispatch_frac_of_8tbs": round(dis_gbs / NOMINAL_HBM_GBS, 4),
+        "combine_frac_of_8tbs": round(com_gbs / NOMINAL_HBM_GBS, 4),
+        "bytes_per_direction": d_bytes,
+        "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": round(achieved, 1), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(dom[0], w.name),
+                     "algorithmic_bytes": dom[1]},
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if e2e is not None:
+        line["e2e"] = {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": round(e2e_ms, 3)}
+    clk = sampler.summary()
+    if clk is not None:
+        line["clocks"] = clk
+    return line
+
+
+def gpu_index_of(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            return int(vis.split(",")[local_rank])
+        except Exception:
+            pass
+    return local_rank
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+
+def oracle_sample(w: inputs.Workload, sample_tokens: int):
+    """Time the CPU oracle on the first `sample_tokens` tokens of every rank of the workload."""
+    import oracle
+
+    inp = inputs.make_inputs(w)
+    Ts = min(sample_tokens, w.num_tokens)
+    idx = np.ascontiguousarray(inp.topk_idx[:, :Ts])
+    x = np.ascontiguousarray(inp.x[:, :Ts])
+    wts = np.ascontiguousarray(inp.topk_weights[:, :Ts])
+    E, H, R = w.num_physical, w.hidden, w.num_ranks
+    t0 = time.perf_counter()
+    if w.num_extra:
+        idx = oracle.reroute(idx, w.num_experts, w.num_extra)["topk_idx_phys"]
+    ref = oracle.layout(idx, inp.active, E)
+    packed, _ = oracle.dispatch(x, idx, ref)
+    oracle.combine(packed, ref.list_base[:-1], idx, wts, ref.pair_row, inp.active, E)
+    secs = time.perf_counter() - t0
+    live = int(ref.recv_count.sum())
+    sent = int(ref.is_token_in_rank.reshape(R * Ts, R).max(axis=1).sum())
+    d_b, c_b = algorithmic_bytes(H, sent, live, R * Ts)
+    return dict(value=round((d_b + c_b) / secs / 1e9, 3), unit="GB/s", cores=1, kind="oracle",
+                sample=f"first {Ts} of {w.num_tokens} tokens of each of the {R} ranks "
+                       f"(reroute + layout + dispatch + combine, single-threaded C, float64 combine)",
+                seconds=round(secs, 3))
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return None
+
+
+def run_reference(args, world):
+    w = inputs.named(args.workload)
+    samples = []
+    for _ in range(args.warmup):
+        oracle_sample(w, args.cpu_sample_tokens)
+    for _ in range(args.steps):
+        samples.append(oracle_sample(w, args.cpu_sample_tokens))
+    secs = sum(s["seconds"] for s in samples) / len(samples)
+    value = statistics.median(s["value"] for s in samples)
+    base = dict(samples[0])
+    base["value"] = value
+    base["host_cores"] = os.cpu_count()
+    base["cpu_model"] = cpu_model()
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(secs * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name} " + " ".join(f"{k_}={v}" for k_, v in w.describe().items()),
+                   **w.describe(), "parallelism": "cpu-oracle"},
+        "cpu_baseline": base,
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill",
+                    help="prefill | decode | replica | tiny | sweep_T<n>[_mask5]")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=512,
+                    help="tokens per rank in the CPU oracle's timed sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, world)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            cb = oracle_sample(inputs.named(args.workload), args.cpu_sample_tokens)
+            cb["host_cores"] = os.cpu_count()
+            cb["cpu_model"] = cpu_model()
+            line["cpu_baseline"] = cb
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

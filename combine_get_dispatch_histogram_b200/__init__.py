@@ -1,0 +1,19 @@
+"""B200 (sm_100a) expert-parallel token dispatch / combine.
+
+The compute path is the C-ABI library ``libep.so`` (hand-written CUDA in
+``csrc/``, declared in ``include/ep.h``); :mod:`.ep` is its thin Python
+binding and :mod:`.inputs` draws seeded synthetic workloads.
+"""
+from .ep import (  # noqa: F401
+    DispatchLayout,
+    EPError,
+    ep_combine,
+    ep_dispatch,
+    ep_layout,
+    ep_layout_workspace_bytes,
+    ep_reroute,
+    ep_reroute_workspace_bytes,
+    ep_strerror,
+    ep_version,
+    load_library,
+)

@@ -1,0 +1,210 @@
+// ep_dispatch.cu -- token dispatch on sm_100a: every token row is read from HBM
+// once and written to each expert slab row its live pairs name.
+//
+// Defines Buffer.low_latency_dispatch (use_fp8=False) of the NeMo AutoModel
+// page "nemo_automodel.components.moe.uccl_ep.buffer": bf16 rows into the
+// per-local-expert receive slabs [num_local_experts,
+// num_ranks * num_max_dispatch_tokens_per_rank, hidden], of which only some
+// rows are valid.  The emulated ranks' slabs are consecutive slices of one
+// [E, R*T, H] allocation.
+//
+// Design.  A persistent grid of single-warp CTAs walks "units" (a token row,
+// or a piece of it when a row is longer than one pipeline stage), unit
+// u = blockIdx.x + i * gridDim.x.  Each CTA runs an S-stage shared-memory
+// ring driven by the Tensor Memory Accelerator's bulk (non-tensor) copies:
+//   - lane 0 issues one cp.async.bulk global->shared load of the row piece,
+//     completing on the stage's mbarrier (skipped when no pair is live);
+//   - after the stage's mbarrier flips, lane j (< k) issues one
+//     cp.async.bulk shared->global store of the staged piece to its slab row
+//     and writes the row's (src_rank, src_token);
+//   - a stage is refilled once the stores that read it have finished reading
+//     shared memory (cp.async.bulk.wait_group.read), one iteration later so
+//     the wait is normally already satisfied.
+// No thread touches the payload: HBM traffic is one read of each live token
+// plus one write per live pair, issued by the copy engine.  The routing of
+// the unit being refilled is prefetched one iteration ahead into registers
+// and parked in shared memory for the consumer.
+#include <algorithm>
+#include <cstdint>
+
+#include "ep.h"
+#include "ep_device.cuh"
+#include "ep_host.h"
+
+namespace ep {
+namespace {
+
+constexpr uint32_t kDispatchPieceMax = 16384;  // largest row piece staged at once
+constexpr int kDispatchMaxStages = 16;
+
+struct DispatchArgs {
+    const uint8_t* x;
+    const int32_t* topk_idx;
+    const int32_t* pair_row;
+    uint8_t* recv_x;
+    int32_t* src_info;
+    int32_t* status;
+    int T, k, E;
+    int64_t row_bytes;
+    int64_t cap;
+    int n_pieces;
+    uint32_t piece_bytes;
+    uint32_t stage_bytes;
+    int stages;
+    int64_t n_units;
+};
+
+struct UnitMeta {
+    int e;
+    int row;
+};
+
+__device__ __forceinline__ UnitMeta load_meta(const DispatchArgs& a, int64_t unit, int lane) {
+    UnitMeta m{-1, -1};
+    if (lane < a.k) {
+        const int64_t p = (unit / a.n_pieces) * a.k + lane;
+        m.e = __ldg(a.topk_idx + p);
+        m.row = __ldg(a.pair_row + p);
+    }
+    return m;
+}
+
+__device__ __forceinline__ uint32_t piece_size(const DispatchArgs& a, int q) {
+    return q + 1 < a.n_pieces ? a.piece_bytes : uint32_t(a.row_bytes - int64_t(q) * a.piece_bytes);
+}
+
+__global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x;
+    const int S = a.stages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(S) * a.stage_bytes);
+    int2* meta = reinterpret_cast<int2*>(full + S);  // [S][32] (e, row) of the staged unit
+
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(smem_u32(full + s), 1);
+        mbar_init_fence();
+    }
+    __syncwarp();
+
+    const int64_t first = blockIdx.x, step = gridDim.x;
+    const int64_t my_n = first < a.n_units ? (a.n_units - 1 - first) / step + 1 : 0;
+    const uint64_t pol_load = policy_evict_first();
+    const uint64_t pol_store = policy_evict_first();
+
+    // Stage unit i: park its routing in shared memory and start the row load.
+    auto issue = [&](int64_t i, UnitMeta m) {
+        const int s = int(i % S);
+        const int64_t u = first + i * step;
+        const int q = int(u % a.n_pieces);
+        const bool valid_row = m.row >= 0 && m.row < a.cap;
+        const bool live = valid_row && m.e >= 0 && m.e < a.E;
+        meta[s * 32 + lane] = make_int2(live ? m.e : -1, m.row);
+        if (q == 0) {
+            if (m.row >= a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
+            if (valid_row && !live) flag_status(a.status, EP_STATUS_BAD_EXPERT);
+        }
+        const bool any = __ballot_sync(0xffffffffu, live) != 0u;
+        __syncwarp();
+        if (lane == 0) {
+            const uint32_t bar = smem_u32(full + s);
+            if (any) {
+                const uint32_t bytes = piece_size(a, q);
+                mbar_arrive_expect_tx(bar, bytes);
+                const uint8_t* src = a.x + (u / a.n_pieces) * a.row_bytes + int64_t(q) * a.piece_bytes;
+                bulk_load(smem_u32(smem + size_t(s) * a.stage_bytes), src, bytes, bar, pol_load);
+            } else {
+                mbar_arrive(bar);
+            }
+        }
+    };
+
+    const int64_t prologue = my_n < S ? my_n : S;
+    for (int64_t i = 0; i < prologue; ++i) issue(i, load_meta(a, first + i * step, lane));
+    UnitMeta next{-1, -1};  // routing of the next unit to refill: unit S, if this CTA has one
+    if (int64_t(S) < my_n) next = load_meta(a, first + int64_t(S) * step, lane);
+
+    for (int64_t i = 0; i < my_n; ++i) {
+        const int s = int(i % S);
+        const uint32_t parity = uint32_t((i / S) & 1);
+        const int64_t u = first + i * step;
+        const int q = int(u % a.n_pieces);
+        const bool landed = __all_sync(0xffffffffu, mbar_wait(smem_u32(full + s), parity));
+        if (!landed) {
+            if (lane == 0) flag_status(a.status, EP_STATUS_TIMEOUT);
+            break;
+        }
+        const int2 m = meta[s * 32 + lane];
+        if (m.x >= 0) {
+            const int64_t tok = u / a.n_pieces;
+            const int64_t slab_row = int64_t(m.x) * a.cap + m.y;
+            bulk_store(a.recv_x + slab_row * a.row_bytes + int64_t(q) * a.piece_bytes,
+                       smem_u32(smem + size_t(s) * a.stage_bytes), piece_size(a, q), pol_store);
+            if (q == 0) {
+                const int src_rank = int(tok / a.T);
+                reinterpret_cast<int2*>(a.src_info)[slab_row] = make_int2(src_rank, int(tok - int64_t(src_rank) * a.T));
+            }
+        }
+        bulk_commit();
+        // refill the stage of unit i-1 with unit i-1+S once its stores have read it
+        const int64_t refill = i - 1 + S;
+        if (i >= 1 && refill < my_n) {
+            bulk_wait_read<1>();
+            __syncwarp();
+            const UnitMeta cur = next;
+            if (refill + 1 < my_n) next = load_meta(a, first + (refill + 1) * step, lane);
+            issue(refill, cur);
+        }
+    }
+    bulk_wait<0>();
+}
+
+}  // namespace
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" int ep_dispatch(ep_dims_t d, const uint16_t* x, const int32_t* topk_idx, const int32_t* pair_row,
+                           uint16_t* recv_x, int32_t* src_info, int32_t* status, ep_cfg_t cfg, void* stream) {
+    int rc = check_dims(d);
+    if (rc != EP_OK) return rc;
+    const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
+    if (RT == 0 || d.hidden == 0) return EP_OK;
+    if (!x || !topk_idx || !pair_row || !recv_x || !src_info) return EP_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(recv_x) || (reinterpret_cast<uintptr_t>(src_info) & 7u)) return EP_ERR_INVALID;
+
+    DispatchArgs a;
+    a.x = reinterpret_cast<const uint8_t*>(x);
+    a.topk_idx = topk_idx;
+    a.pair_row = pair_row;
+    a.recv_x = reinterpret_cast<uint8_t*>(recv_x);
+    a.src_info = src_info;
+    a.status = status;
+    a.T = d.num_tokens;
+    a.k = d.num_topk;
+    a.E = d.num_experts;
+    a.row_bytes = int64_t(d.hidden) * 2;
+    a.cap = RT;
+    a.n_pieces = int(ceil_div(a.row_bytes, kDispatchPieceMax));
+    a.piece_bytes = uint32_t(round_up16(size_t(ceil_div(a.row_bytes, a.n_pieces))));
+    if (int64_t(a.n_pieces - 1) * a.piece_bytes >= a.row_bytes) return EP_ERR_UNSUPPORTED;
+    a.stage_bytes = uint32_t((a.piece_bytes + 127) & ~127u);
+    a.n_units = RT * a.n_pieces;
+
+    const int sms = sm_count();
+    if (sms <= 0) return EP_ERR_CUDA;
+    const int ctas_per_sm = 2;
+    const int budget = std::max(1, max_smem_optin() / ctas_per_sm - 1024);
+    int stages = cfg.stages > 0 ? cfg.stages : int(budget / (a.stage_bytes + 8 + 256));
+    stages = std::max(2, std::min(kDispatchMaxStages, stages));
+    a.stages = stages;
+    const size_t smem = size_t(stages) * (a.stage_bytes + 8 + 256);
+    if (smem > size_t(max_smem_optin())) return EP_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+        return EP_ERR_CUDA;
+    int64_t grid = int64_t(sms) * ctas_per_sm;
+    if (cfg.max_ctas > 0) grid = std::min<int64_t>(grid, cfg.max_ctas);
+    grid = std::min<int64_t>(grid, a.n_units);
+    dispatch_kernel<<<unsigned(grid), 32, smem, static_cast<cudaStream_t>(stream)>>>(a);
+    return launch_result();
+}

@@ -1,0 +1,294 @@
+"""Python binding of the sm_100a C-ABI library ``libep.so`` (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: it checks dtypes / devices / shapes, allocates missing
+outputs with PyTorch (the library itself never allocates), passes raw device
+pointers and the current CUDA stream, and raises :class:`EPError` on a
+non-zero return code.  There is no fallback: if ``libep.so`` is missing or no
+GPU is present, the call fails loudly.
+
+Tensor conventions (R ranks, T tokens per rank, k slots, E experts, H hidden,
+CAP = R*T slab rows per expert) follow ``include/ep.h``.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libep.so")
+
+EP_OK = 0
+EP_ERR_INVALID = -1
+EP_ERR_UNSUPPORTED = -2
+EP_ERR_CUDA = -3
+EP_STATUS_BAD_EXPERT = 1
+EP_STATUS_OVERFLOW = 2
+EP_STATUS_TIMEOUT = 8
+
+_lib = None
+
+
+class EPError(RuntimeError):
+    def __init__(self, func: str, code: int, msg: str):
+        super().__init__(f"{func} failed with {code}: {msg}")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("num_ranks", ctypes.c_int32), ("num_tokens", ctypes.c_int32), ("num_topk", ctypes.c_int32),
+                ("num_experts", ctypes.c_int32), ("hidden", ctypes.c_int32)]
+
+
+class Cfg(ctypes.Structure):
+    _fields_ = [("max_ctas", ctypes.c_int32), ("threads", ctypes.c_int32), ("stages", ctypes.c_int32)]
+
+
+def load_library(path: str = LIB_PATH):
+    """Load ``libep.so`` (built by ``combine_get_dispatch_histogram_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library {path} is missing: build it with "
+                           "`python -m combine_get_dispatch_histogram_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    lib.ep_strerror.argtypes = [ctypes.c_int]
+    lib.ep_strerror.restype = ctypes.c_char_p
+    lib.ep_version.argtypes = []
+    lib.ep_version.restype = ctypes.c_char_p
+    lib.ep_layout_workspace_bytes.argtypes = [Dims]
+    lib.ep_layout_workspace_bytes.restype = SZ
+    lib.ep_layout.argtypes = [Dims, P, P, P, SZ, P, P, P, P, P, P, P, Cfg, P]
+    lib.ep_layout.restype = ctypes.c_int
+    lib.ep_dispatch.argtypes = [Dims, P, P, P, P, P, P, Cfg, P]
+    lib.ep_dispatch.restype = ctypes.c_int
+    lib.ep_combine.argtypes = [Dims, P, P, P, P, P, P, P, Cfg, P]
+    lib.ep_combine.restype = ctypes.c_int
+    lib.ep_reroute_workspace_bytes.argtypes = [I32, I32, I32, I32]
+    lib.ep_reroute_workspace_bytes.restype = SZ
+    lib.ep_reroute.argtypes = [I32, I32, I32, I32, I32, P, P, SZ, P, P, P, P, P, Cfg, P]
+    lib.ep_reroute.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def ep_version() -> str:
+    return load_library().ep_version().decode()
+
+
+def ep_strerror(code: int) -> str:
+    return load_library().ep_strerror(code).decode()
+
+
+def _check(func: str, code: int):
+    if code != EP_OK:
+        raise EPError(func, code, ep_strerror(code))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    return t
+
+
+def _cfg(cfg) -> Cfg:
+    if cfg is None:
+        return Cfg(0, 0, 0)
+    if isinstance(cfg, Cfg):
+        return cfg
+    return Cfg(int(cfg.get("max_ctas", 0)), int(cfg.get("threads", 0)), int(cfg.get("stages", 0)))
+
+
+def _stream(device, stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _status(device, status):
+    if status is None:
+        return torch.zeros(1, dtype=torch.int32, device=device)
+    return _need(status, "status", torch.int32, device=device)
+
+
+@dataclasses.dataclass
+class DispatchLayout:
+    """Outputs of :func:`ep_layout`: the layout plus the dispatch / combine handle."""
+
+    num_tokens_per_expert: torch.Tensor  # int32 [R, E]
+    num_tokens_per_rank: torch.Tensor    # int32 [R, R]
+    is_token_in_rank: torch.Tensor       # uint8 [R, T, R]
+    recv_count: torch.Tensor             # int32 [E]
+    expert_rank_offset: torch.Tensor     # int32 [E, R]
+    pair_row: torch.Tensor               # int32 [R, T, k]
+    status: torch.Tensor                 # int32 [1]
+
+
+def ep_layout_workspace_bytes(num_ranks: int, num_tokens: int, num_topk: int, num_experts: int,
+                              hidden: int = 8) -> int:
+    return int(load_library().ep_layout_workspace_bytes(Dims(num_ranks, num_tokens, num_topk, num_experts,
+                                                             hidden)))
+
+
+def ep_layout(topk_idx: torch.Tensor, active: torch.Tensor, num_experts: int, *, hidden: int = 8,
+              workspace: Optional[torch.Tensor] = None, out: Optional[DispatchLayout] = None,
+              status: Optional[torch.Tensor] = None, cfg=None, stream=None) -> DispatchLayout:
+    """Histogram, prefix sums and stable slab rows (``ep_layout`` of ``include/ep.h``)."""
+    lib = load_library()
+    _need(topk_idx, "topk_idx", torch.int32)
+    if topk_idx.dim() != 3:
+        raise ValueError("topk_idx must be [R, T, k]")
+    R, T, k = topk_idx.shape
+    dev = topk_idx.device
+    E = int(num_experts)
+    _need(active, "active", torch.uint8, (R,), dev)
+    dims = Dims(R, T, k, E, hidden)
+    ws_bytes = int(lib.ep_layout_workspace_bytes(dims))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, device=dev)
+    if out is None:
+        out = DispatchLayout(
+            torch.empty((R, E), dtype=torch.int32, device=dev), torch.empty((R, R), dtype=torch.int32, device=dev),
+            torch.empty((R, T, R), dtype=torch.uint8, device=dev), torch.empty((E,), dtype=torch.int32, device=dev),
+            torch.empty((E, R), dtype=torch.int32, device=dev), torch.empty((R, T, k), dtype=torch.int32, device=dev),
+            _status(dev, status))
+    else:
+        _need(out.num_tokens_per_expert, "num_tokens_per_expert", torch.int32, (R, E), dev)
+        _need(out.num_tokens_per_rank, "num_tokens_per_rank", torch.int32, (R, R), dev)
+        _need(out.is_token_in_rank, "is_token_in_rank", torch.uint8, (R, T, R), dev)
+        _need(out.recv_count, "recv_count", torch.int32, (E,), dev)
+        _need(out.expert_rank_offset, "expert_rank_offset", torch.int32, (E, R), dev)
+        _need(out.pair_row, "pair_row", torch.int32, (R, T, k), dev)
+        if status is not None:
+            out.status = _need(status, "status", torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.ep_layout(dims, _ptr(topk_idx), _ptr(active), _ptr(workspace), workspace.numel(),
+                           _ptr(out.num_tokens_per_expert), _ptr(out.num_tokens_per_rank),
+                           _ptr(out.is_token_in_rank), _ptr(out.recv_count), _ptr(out.expert_rank_offset),
+                           _ptr(out.pair_row), _ptr(out.status), _cfg(cfg), _stream(dev, stream))
+    _check("ep_layout", rc)
+    return out
+
+
+def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, pair_row: torch.Tensor, num_experts: int, *,
+                recv_x: Optional[torch.Tensor] = None, src_info: Optional[torch.Tensor] = None,
+                status: Optional[torch.Tensor] = None, cfg=None, stream=None):
+    """Scatter token rows into the [E, R*T, H] receive slabs (``ep_dispatch``).
+
+    Returns ``(recv_x, src_info, status)``; rows past ``recv_count`` are untouched.
+    """
+    lib = load_library()
+    _need(x, "x", torch.bfloat16)
+    if x.dim() != 3:
+        raise ValueError("x must be [R, T, H]")
+    R, T, H = x.shape
+    dev = x.device
+    _need(topk_idx, "topk_idx", torch.int32, device=dev)
+    if topk_idx.dim() != 3 or tuple(topk_idx.shape[:2]) != (R, T):
+        raise ValueError("topk_idx must be [R, T, k]")
+    k = topk_idx.shape[2]
+    _need(pair_row, "pair_row", torch.int32, (R, T, k), dev)
+    E = int(num_experts)
+    cap = R * T
+    if recv_x is None:
+        recv_x = torch.empty((E, cap, H), dtype=torch.bfloat16, device=dev)
+    if src_info is None:
+        src_info = torch.empty((E, cap, 2), dtype=torch.int32, device=dev)
+    _need(recv_x, "recv_x", torch.bfloat16, (E, cap, H), dev)
+    _need(src_info, "src_info", torch.int32, (E, cap, 2), dev)
+    status = _status(dev, status)
+    with torch.cuda.device(dev):
+        rc = lib.ep_dispatch(Dims(R, T, k, E, H), _ptr(x), _ptr(topk_idx), _ptr(pair_row), _ptr(recv_x),
+                             _ptr(src_info), _ptr(status), _cfg(cfg), _stream(dev, stream))
+    _check("ep_dispatch", rc)
+    return recv_x, src_info, status
+
+
+def ep_combine(y: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor, pair_row: torch.Tensor,
+               active: torch.Tensor, *, out: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+               cfg=None, stream=None):
+    """Weighted top-k gather-reduce back to [R, T, H] bf16 (``ep_combine``). Returns ``(out, status)``."""
+    lib = load_library()
+    _need(y, "y", torch.bfloat16)
+    if y.dim() != 3:
+        raise ValueError("y must be [E, R*T, H]")
+    E, cap, H = y.shape
+    dev = y.device
+    _need(topk_idx, "topk_idx", torch.int32, device=dev)
+    if topk_idx.dim() != 3:
+        raise ValueError("topk_idx must be [R, T, k]")
+    R, T, k = topk_idx.shape
+    if cap != R * T:
+        raise ValueError(f"y has {cap} rows per expert, expected R*T = {R * T}")
+    _need(topk_weights, "topk_weights", torch.float32, (R, T, k), dev)
+    _need(pair_row, "pair_row", torch.int32, (R, T, k), dev)
+    _need(active, "active", torch.uint8, (R,), dev)
+    if out is None:
+        out = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (R, T, H), dev)
+    status = _status(dev, status)
+    with torch.cuda.device(dev):
+        rc = lib.ep_combine(Dims(R, T, k, E, H), _ptr(y), _ptr(topk_idx), _ptr(topk_weights), _ptr(pair_row),
+                            _ptr(active), _ptr(out), _ptr(status), _cfg(cfg), _stream(dev, stream))
+    _check("ep_combine", rc)
+    return out, status
+
+
+def ep_reroute_workspace_bytes(num_ranks: int, num_tokens: int, num_topk: int, num_logical: int) -> int:
+    return int(load_library().ep_reroute_workspace_bytes(num_ranks, num_tokens, num_topk, num_logical))
+
+
+def ep_reroute(topk_idx_logical: torch.Tensor, num_logical: int, num_extra: int, *,
+               workspace: Optional[torch.Tensor] = None, out: Optional[dict] = None,
+               status: Optional[torch.Tensor] = None, cfg=None, stream=None) -> dict:
+    """Logical load, greedy replicas and physical routing (``ep_reroute``).
+
+    Returns a dict with ``load``, ``num_replicas``, ``phys_base``, ``topk_idx_phys``, ``status``.
+    """
+    lib = load_library()
+    _need(topk_idx_logical, "topk_idx_logical", torch.int32)
+    if topk_idx_logical.dim() != 3:
+        raise ValueError("topk_idx_logical must be [R, T, k]")
+    R, T, k = topk_idx_logical.shape
+    dev = topk_idx_logical.device
+    L = int(num_logical)
+    ws_bytes = int(lib.ep_reroute_workspace_bytes(R, T, k, L))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, device=dev)
+    if out is None:
+        out = dict(load=torch.empty(L, dtype=torch.int32, device=dev),
+                   num_replicas=torch.empty(L, dtype=torch.int32, device=dev),
+                   phys_base=torch.empty(L + 1, dtype=torch.int32, device=dev),
+                   topk_idx_phys=torch.empty((R, T, k), dtype=torch.int32, device=dev))
+    _need(out["load"], "load", torch.int32, (L,), dev)
+    _need(out["num_replicas"], "num_replicas", torch.int32, (L,), dev)
+    _need(out["phys_base"], "phys_base", torch.int32, (L + 1,), dev)
+    _need(out["topk_idx_phys"], "topk_idx_phys", torch.int32, (R, T, k), dev)
+    out["status"] = _status(dev, status)
+    with torch.cuda.device(dev):
+        rc = lib.ep_reroute(R, T, k, L, int(num_extra), _ptr(topk_idx_logical), _ptr(workspace), workspace.numel(),
+                            _ptr(out["load"]), _ptr(out["num_replicas"]), _ptr(out["phys_base"]),
+                            _ptr(out["topk_idx_phys"]), _ptr(out["status"]), _cfg(cfg), _stream(dev, stream))
+    _check("ep_reroute", rc)
+    return out

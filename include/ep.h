@@ -61,6 +61,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define EP_API __attribute__((visibility("default")))
+#else
+#define EP_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -106,13 +112,13 @@ typedef struct ep_cfg {
 } ep_cfg_t;
 
 /* Human-readable name of an EP_OK / EP_ERR_* code (static storage). */
-const char *ep_strerror(int code);
+EP_API const char *ep_strerror(int code);
 
 /* Library version string (static storage). */
-const char *ep_version(void);
+EP_API const char *ep_version(void);
 
 /* Bytes of device workspace ep_layout needs for `d` (0 only if R*T == 0). */
-size_t ep_layout_workspace_bytes(ep_dims_t d);
+EP_API size_t ep_layout_workspace_bytes(ep_dims_t d);
 
 /*
  * ep_layout -- per-expert / per-rank histogram, prefix sums and stable rows.
@@ -136,7 +142,7 @@ size_t ep_layout_workspace_bytes(ep_dims_t d);
  * (source rank, token, slot) order, so each expert's rows are ordered by
  * (src_rank, token) and the result is unique (bit-exact, deterministic).
  */
-int ep_layout(ep_dims_t d, const int32_t *topk_idx, const uint8_t *active,
+EP_API int ep_layout(ep_dims_t d, const int32_t *topk_idx, const uint8_t *active,
               void *workspace, size_t workspace_bytes,
               int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
               uint8_t *is_token_in_rank, int32_t *recv_count,
@@ -160,7 +166,7 @@ int ep_layout(ep_dims_t d, const int32_t *topk_idx, const uint8_t *active,
  *                               other rows untouched.
  * Each token row is read from HBM once however many experts it goes to.
  */
-int ep_dispatch(ep_dims_t d, const uint16_t *x, const int32_t *topk_idx,
+EP_API int ep_dispatch(ep_dims_t d, const uint16_t *x, const int32_t *topk_idx,
                 const int32_t *pair_row, uint16_t *recv_x, int32_t *src_info,
                 int32_t *status, ep_cfg_t cfg, void *stream);
 
@@ -181,13 +187,13 @@ int ep_dispatch(ep_dims_t d, const uint16_t *x, const int32_t *topk_idx,
  *     taking only slots with pair_row >= 0, pair_row < CAP, e in range and
  *     active[e/E_local]; rows of a source rank with active[r] == 0 are zeros.
  */
-int ep_combine(ep_dims_t d, const uint16_t *y, const int32_t *topk_idx,
+EP_API int ep_combine(ep_dims_t d, const uint16_t *y, const int32_t *topk_idx,
                const float *topk_weights, const int32_t *pair_row,
                const uint8_t *active, uint16_t *out,
                int32_t *status, ep_cfg_t cfg, void *stream);
 
 /* Bytes of device workspace ep_reroute needs. */
-size_t ep_reroute_workspace_bytes(int32_t num_ranks, int32_t num_tokens, int32_t num_topk,
+EP_API size_t ep_reroute_workspace_bytes(int32_t num_ranks, int32_t num_tokens, int32_t num_topk,
                                   int32_t num_logical);
 
 /*
@@ -207,7 +213,7 @@ size_t ep_reroute_workspace_bytes(int32_t num_ranks, int32_t num_tokens, int32_t
  * num_logical + num_extra physical experts result; ep_layout / ep_dispatch /
  * ep_combine then run with num_experts = num_logical + num_extra.
  */
-int ep_reroute(int32_t num_ranks, int32_t num_tokens, int32_t num_topk,
+EP_API int ep_reroute(int32_t num_ranks, int32_t num_tokens, int32_t num_topk,
                int32_t num_logical, int32_t num_extra,
                const int32_t *topk_idx_logical, void *workspace, size_t workspace_bytes,
                int32_t *load, int32_t *num_replicas, int32_t *phys_base,

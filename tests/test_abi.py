@@ -1,0 +1,88 @@
+"""CPU checks of the C ABI: the library builds, loads and exports every declared entry point.
+
+Only host-side calls run here (error names, workspace sizes, argument
+validation that rejects before touching a device); nothing is launched.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from combine_get_dispatch_histogram_b200 import build, ep
+
+    build.build()
+    return ep.load_library()
+
+
+def declared_symbols():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^EP_API\s+[\w\s\*]+?\**\b(ep_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_header_declares_the_entry_points():
+    names = set(declared_symbols())
+    for want in ("ep_layout", "ep_dispatch", "ep_combine", "ep_reroute", "ep_layout_workspace_bytes",
+                 "ep_reroute_workspace_bytes", "ep_strerror", "ep_version"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_error_names_and_version(lib):
+    from combine_get_dispatch_histogram_b200 import ep
+
+    for code in (ep.EP_OK, ep.EP_ERR_INVALID, ep.EP_ERR_UNSUPPORTED, ep.EP_ERR_CUDA):
+        assert ep.ep_strerror(code) and ep.ep_strerror(code) != "unknown error code"
+    assert "sm_100a" in ep.ep_version()
+
+
+def test_workspace_sizes(lib):
+    from combine_get_dispatch_histogram_b200 import ep
+
+    # 8 ranks x 4096 tokens: 1024 chunks of 32 tokens, E + R ints each
+    assert ep.ep_layout_workspace_bytes(8, 4096, 8, 256, 7168) == 1024 * 256 * 4 + 1024 * 8 * 4
+    assert ep.ep_layout_workspace_bytes(2, 0, 2, 8, 256) == 0
+    assert ep.ep_layout_workspace_bytes(3, 4, 2, 8, 256) == 0        # E % R != 0 is invalid
+    assert ep.ep_reroute_workspace_bytes(8, 2048, 6, 64) % 16 == 0
+
+
+def test_host_validation_rejects_without_launching(lib):
+    from combine_get_dispatch_histogram_b200 import ep
+
+    cfg = ep.Cfg(0, 0, 0)
+    bad_dims = [ep.Dims(3, 4, 2, 8, 256),      # E not a multiple of R
+                ep.Dims(2, 4, 9, 8, 256),      # k > E
+                ep.Dims(2, 4, 2, 8, 12),       # H not a multiple of 8
+                ep.Dims(0, 4, 2, 8, 256)]
+    for d in bad_dims:
+        assert lib.ep_layout(d, None, None, None, 0, None, None, None, None, None, None, None, cfg, None) \
+            == ep.EP_ERR_INVALID
+        assert lib.ep_dispatch(d, None, None, None, None, None, None, cfg, None) == ep.EP_ERR_INVALID
+        assert lib.ep_combine(d, None, None, None, None, None, None, None, cfg, None) == ep.EP_ERR_INVALID
+    big = ep.Dims(128, 4, 2, 128, 256)           # more ranks than the rank-set width
+    assert lib.ep_layout(big, None, None, None, 0, None, None, None, None, None, None, None, cfg, None) \
+        == ep.EP_ERR_UNSUPPORTED
+    good = ep.Dims(2, 4, 2, 8, 256)
+    # null outputs are rejected before any device work
+    assert lib.ep_layout(good, None, None, None, 0, None, None, None, None, None, None, None, cfg, None) \
+        == ep.EP_ERR_INVALID
+    assert lib.ep_dispatch(good, None, None, None, None, None, None, cfg, None) == ep.EP_ERR_INVALID
+    # misaligned token pointer
+    fake = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1008)
+    assert lib.ep_dispatch(good, odd, fake, fake, fake, fake, fake, cfg, None) == ep.EP_ERR_INVALID
+    assert lib.ep_reroute(1, 4, 2, 0, 1, None, None, 0, None, None, None, None, None, cfg, None) \
+        == ep.EP_ERR_INVALID

@@ -1,0 +1,296 @@
+"""GPU parity: the sm_100a path through the C ABI against the CPU oracle.
+
+Layout, handle, src_info and payload must be bit-exact; combine (bf16) must
+satisfy |gpu - oracle| <= 1e-2 + 1e-2 |oracle| with the oracle accumulating in
+float64.  Every input is drawn by ``combine_get_dispatch_histogram_b200.inputs``.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_get_dispatch_histogram_b200 import ep, inputs
+from gpu_util import (bf16_dev, bf16_host, check_close, check_dispatch, check_layout, dev, f32_dev, i32_dev,
+                      run_path, u8_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _free_memory():
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def _oracle_all(inp, E, active_combine=None):
+    ref = oracle.layout(inp.topk_idx, inp.active, E)
+    packed, _ = oracle.dispatch(inp.x, inp.topk_idx, ref)
+    act_c = inp.active if active_combine is None else active_combine
+    want, _ = oracle.combine(packed, ref.list_base[:-1], inp.topk_idx, inp.topk_weights, ref.pair_row, act_c, E)
+    return ref, packed, want
+
+
+def _check_all(res, ref, packed, want, tag):
+    check_layout(res["lay"], ref, tag)
+    check_dispatch(res["recv_x"], res["src_info"], ref, packed, tag)
+    check_close(bf16_host(res["out"]), want, tag)
+    assert res["status"] == ref.status, f"{tag} status {res['status']} != {ref.status}"
+
+
+WORKLOADS = ["tiny", "decode"] + [f"sweep_T{t}" for t in inputs.SWEEP_TOKENS] + \
+            [f"sweep_T{t}_mask5" for t in inputs.SWEEP_TOKENS]
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_pipeline_matches_oracle(name):
+    w = inputs.named(name)
+    inp = inputs.make_inputs(w)
+    ref, packed, want = _oracle_all(inp, w.num_experts)
+    res = run_path(inp, w.num_experts, w.hidden)
+    _check_all(res, ref, packed, want, name)
+    if w.inactive:
+        # the masked rank neither sends nor receives
+        El = w.num_experts // w.num_ranks
+        for d in w.inactive:
+            assert int(res["lay"].recv_count[d * El:(d + 1) * El].sum()) == 0
+            assert bool((res["out"][d] == 0).all())
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "sweep_T64_mask5"])
+def test_combine_on_independent_expert_outputs(name):
+    """Combine of a seeded random slab (not the dispatched rows) against the oracle."""
+    w = inputs.named(name)
+    inp = inputs.make_inputs(w)
+    E, cap, H = w.num_experts, w.num_ranks * w.num_tokens, w.hidden
+    ref = oracle.layout(inp.topk_idx, inp.active, E)
+    rng = np.random.default_rng(2024)
+    y = inputs.random_slab(rng, E, cap, H)
+    want, _ = oracle.combine(y, np.arange(E, dtype=np.int64) * cap, inp.topk_idx, inp.topk_weights,
+                             ref.pair_row, inp.active, E)
+    out, st = ep.ep_combine(bf16_dev(y), i32_dev(inp.topk_idx), f32_dev(inp.topk_weights),
+                            i32_dev(ref.pair_row), u8_dev(inp.active))
+    torch.cuda.synchronize()
+    check_close(bf16_host(out), want, name)
+    assert int(st.item()) == 0
+
+
+@pytest.mark.parametrize("flip", [(5,), (0, 3), ()])
+def test_mask_changed_between_dispatch_and_combine(flip):
+    w = inputs.decode()
+    inp = inputs.make_inputs(w)
+    now = inp.active.copy()
+    for r in flip:
+        now[r] = 0
+    ref, packed, want = _oracle_all(inp, w.num_experts, active_combine=now)
+    res = run_path(inp, w.num_experts, w.hidden, active_combine=now)
+    _check_all(res, ref, packed, want, f"flip{flip}")
+
+
+def test_replica_workload_full_size():
+    """Reroute (64 logical -> 80 physical experts) then layout / dispatch / combine."""
+    w = inputs.replica()
+    inp = inputs.make_inputs(w)
+    rr = ep.ep_reroute(i32_dev(inp.topk_idx), w.num_experts, w.num_extra)
+    torch.cuda.synchronize()
+    rref = oracle.reroute(inp.topk_idx, w.num_experts, w.num_extra)
+    for key in ("load", "num_replicas", "phys_base", "topk_idx_phys"):
+        assert np.array_equal(rr[key].cpu().numpy(), rref[key]), key
+    assert int(rr["status"].item()) == 0
+    E = w.num_physical
+    phys = inputs.Inputs(rref["topk_idx_phys"], inp.topk_weights, inp.x, inp.active)
+    ref = oracle.layout(phys.topk_idx, phys.active, E)
+    packed, _ = oracle.dispatch(phys.x, phys.topk_idx, ref)
+    rng = np.random.default_rng(3)
+    tokens = np.stack([rng.integers(0, w.num_ranks, 3000), rng.integers(0, w.num_tokens, 3000)], axis=1)
+    want, _ = oracle.combine(packed, ref.list_base[:-1], phys.topk_idx, phys.topk_weights, ref.pair_row,
+                             phys.active, E, tokens=tokens)
+    # the GPU runs on its own rerouted ids
+    idx = rr["topk_idx_phys"]
+    status = torch.zeros(1, dtype=torch.int32, device=dev())
+    lay = ep.ep_layout(idx, u8_dev(inp.active), E, hidden=w.hidden, status=status)
+    recv_x, src_info, _ = ep.ep_dispatch(bf16_dev(inp.x), idx, lay.pair_row, E, status=status)
+    out, _ = ep.ep_combine(recv_x, idx, f32_dev(inp.topk_weights), lay.pair_row, u8_dev(inp.active), status=status)
+    torch.cuda.synchronize()
+    check_layout(lay, ref, "replica")
+    check_dispatch(recv_x, src_info, ref, packed, "replica")
+    got = bf16_host(out)[tokens[:, 0], tokens[:, 1]]
+    check_close(got, want, "replica")
+    assert int(status.item()) == 0
+
+
+# ----------------------------------------------------------------------------- edge cases
+
+def _custom(R, T, k, E, H, idx, active=None, seed=0):
+    rng = np.random.default_rng(seed)
+    w = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+    x = inputs.bf16_tokens(rng, R * T, H).reshape(R, T, H)
+    act = np.ones(R, np.uint8) if active is None else np.asarray(active, np.uint8)
+    return inputs.Inputs(np.ascontiguousarray(idx, dtype=np.int32), w, x, act)
+
+
+def _uniform_idx(rng, R, T, k, E):
+    return np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k)
+
+
+EDGE = {
+    "k1": dict(R=4, T=40, k=1, E=8, H=64),
+    "T1": dict(R=8, T=1, k=8, E=256, H=7168),
+    "R1": dict(R=1, T=70, k=3, E=5, H=64),
+    "E_equals_R": dict(R=4, T=33, k=2, E=4, H=128),
+    "H8": dict(R=2, T=37, k=2, E=8, H=8),
+    "ragged_H": dict(R=2, T=19, k=4, E=8, H=7176),
+    "wide_H": dict(R=2, T=9, k=3, E=4, H=20000),
+    "k32": dict(R=2, T=35, k=32, E=64, H=256),
+    "many_experts": dict(R=4, T=50, k=6, E=4096, H=64),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_edge_shapes(name):
+    c = EDGE[name]
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    idx = _uniform_idx(rng, c["R"], c["T"], c["k"], c["E"])
+    inp = _custom(c["R"], c["T"], c["k"], c["E"], c["H"], idx)
+    ref, packed, want = _oracle_all(inp, c["E"])
+    _check_all(run_path(inp, c["E"], c["H"]), ref, packed, want, name)
+
+
+def test_all_none_selected():
+    R, T, k, E, H = 3, 20, 2, 6, 64
+    inp = _custom(R, T, k, E, H, np.full((R, T, k), -1))
+    ref, packed, want = _oracle_all(inp, E)
+    res = run_path(inp, E, H)
+    _check_all(res, ref, packed, want, "all -1")
+    assert bool((res["out"] == 0).all())
+
+
+def test_every_token_to_one_expert():
+    """Expert 0 receives every token of every rank: recv_count == CAP exactly."""
+    R, T, k, E, H = 4, 64, 4, 16, 256
+    rng = np.random.default_rng(8)
+    idx = np.stack([np.concatenate([[0], 1 + rng.permutation(E - 1)[:k - 1]]) for _ in range(R * T)])
+    idx = idx.reshape(R, T, k)
+    inp = _custom(R, T, k, E, H, idx)
+    ref, packed, want = _oracle_all(inp, E)
+    assert ref.recv_count[0] == R * T
+    _check_all(run_path(inp, E, H), ref, packed, want, "one expert")
+
+
+def test_duplicate_slots_overflow_is_flagged():
+    """A token naming the same expert in every slot overflows the slab: flagged, never written past CAP."""
+    R, T, k, E, H = 2, 16, 3, 4, 64
+    inp = _custom(R, T, k, E, H, np.zeros((R, T, k), np.int32))
+    ref, packed, want = _oracle_all(inp, E)
+    assert ref.status & oracle.OVERFLOW
+    res = run_path(inp, E, H)
+    _check_all(res, ref, packed, want, "overflow")
+    assert res["status"] & ep.EP_STATUS_OVERFLOW
+
+
+def test_bad_expert_ids_are_flagged_not_trapped():
+    R, T, k, E, H = 2, 24, 3, 8, 64
+    rng = np.random.default_rng(9)
+    idx = _uniform_idx(rng, R, T, k, E)
+    idx[0, 3, 1] = 8
+    idx[1, 5, 0] = -7
+    idx[1, 6, 2] = 1 << 20
+    inp = _custom(R, T, k, E, H, idx)
+    ref, packed, want = _oracle_all(inp, E)
+    assert ref.status & oracle.BAD_EXPERT
+    res = run_path(inp, E, H)
+    _check_all(res, ref, packed, want, "bad ids")
+    assert res["status"] & ep.EP_STATUS_BAD_EXPERT
+
+
+def test_all_ranks_masked():
+    R, T, k, E, H = 4, 32, 2, 8, 64
+    rng = np.random.default_rng(10)
+    inp = _custom(R, T, k, E, H, _uniform_idx(rng, R, T, k, E), active=np.zeros(R))
+    ref, packed, want = _oracle_all(inp, E)
+    res = run_path(inp, E, H)
+    _check_all(res, ref, packed, want, "all masked")
+    assert int(res["lay"].recv_count.sum()) == 0 and bool((res["out"] == 0).all())
+
+
+def test_empty_token_batch():
+    R, T, k, E, H = 2, 0, 2, 8, 64
+    idx = torch.zeros((R, T, k), dtype=torch.int32, device=dev())
+    act = torch.ones(R, dtype=torch.uint8, device=dev())
+    lay = ep.ep_layout(idx, act, E, hidden=H)
+    x = torch.zeros((R, T, H), dtype=torch.bfloat16, device=dev())
+    recv_x, src_info, _ = ep.ep_dispatch(x, idx, lay.pair_row, E)
+    out, st = ep.ep_combine(recv_x, idx, torch.zeros((R, T, k), device=dev()), lay.pair_row, act)
+    torch.cuda.synchronize()
+    assert int(lay.recv_count.abs().sum()) == 0 and int(lay.num_tokens_per_expert.abs().sum()) == 0
+    assert int(lay.num_tokens_per_rank.abs().sum()) == 0 and int(lay.expert_rank_offset.abs().sum()) == 0
+    assert out.numel() == 0 and int(st.item()) == 0
+
+
+def test_invalid_hidden_raises():
+    R, T, k, E = 2, 4, 2, 8
+    idx = torch.zeros((R, T, k), dtype=torch.int32, device=dev())
+    pr = torch.full((R, T, k), -1, dtype=torch.int32, device=dev())
+    x = torch.zeros((R, T, 12), dtype=torch.bfloat16, device=dev())
+    with pytest.raises(ep.EPError) as ei:
+        ep.ep_dispatch(x, idx, pr, E)
+    assert ei.value.code == ep.EP_ERR_INVALID
+
+
+@pytest.mark.parametrize("cfg", [dict(stages=2), dict(max_ctas=1), dict(max_ctas=3, stages=3),
+                                 dict(threads=64), dict(max_ctas=1, stages=2, threads=96)])
+def test_launch_configs(cfg):
+    """Ring wrap-around and tiny grids: a single CTA walks every unit through 2 stages."""
+    w = inputs.sweep(32, masked=True)
+    inp = inputs.make_inputs(w)
+    ref, packed, want = _oracle_all(inp, w.num_experts)
+    _check_all(run_path(inp, w.num_experts, w.hidden, cfg=cfg), ref, packed, want, str(cfg))
+
+
+def test_deterministic_and_idempotent():
+    w = inputs.decode()
+    inp = inputs.make_inputs(w)
+    a = run_path(inp, w.num_experts, w.hidden)
+    b = run_path(inp, w.num_experts, w.hidden)
+    for key in ("pair_row", "recv_count", "expert_rank_offset", "num_tokens_per_expert"):
+        assert torch.equal(getattr(a["lay"], key), getattr(b["lay"], key))
+    assert torch.equal(a["out"].view(torch.int16), b["out"].view(torch.int16))
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_fuzz_small(seed):
+    rng = np.random.default_rng(1000 + seed)
+    R = int(rng.integers(1, 9))
+    El = int(rng.integers(1, 9))
+    E = R * El
+    k = int(rng.integers(1, min(E, 8) + 1))
+    T = int(rng.integers(1, 100))
+    H = int(rng.choice([8, 64, 256, 1032, 7168]))
+    idx = _uniform_idx(rng, R, T, k, E)
+    idx = np.where(rng.random(idx.shape) < 0.1, -1, idx)
+    active = (rng.random(R) > 0.2).astype(np.uint8)
+    inp = _custom(R, T, k, E, H, idx, active=active, seed=seed)
+    now = active.copy()
+    if R > 1 and rng.random() < 0.5:
+        now[rng.integers(0, R)] ^= 1
+    ref, packed, want = _oracle_all(inp, E, active_combine=now)
+    res = run_path(inp, E, H, active_combine=now)
+    _check_all(res, ref, packed, want, f"fuzz{seed}")
+
+
+def test_reroute_small_cases():
+    rng = np.random.default_rng(77)
+    for it in range(20):
+        E = int(rng.integers(1, 70))
+        extra = int(rng.integers(0, 40))
+        R, T = int(rng.integers(1, 5)), int(rng.integers(1, 300))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        idx = inputs.zipf_topk(rng, R * T, E, k, 1.3).reshape(R, T, k)
+        idx = np.where(rng.random(idx.shape) < 0.05, -1, idx).astype(np.int32)
+        rr = ep.ep_reroute(i32_dev(idx), E, extra)
+        torch.cuda.synchronize()
+        rref = oracle.reroute(idx, E, extra)
+        for key in ("load", "num_replicas", "phys_base", "topk_idx_phys"):
+            assert np.array_equal(rr[key].cpu().numpy(), rref[key]), (it, key)
