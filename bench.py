@@ -346,11 +346,11 @@ def gpu_index_of(local_rank: int) -> int:
 
 # ----------------------------------------------------------------------------- CPU oracle arm
 
-def oracle_sample(w: inputs.Workload, sample_tokens: int):
+def oracle_sample(w: inputs.Workload, sample_tokens: int, inp=None):
     """Time the CPU oracle on the first `sample_tokens` tokens of every rank of the workload."""
     import oracle
 
-    inp = inputs.make_inputs(w)
+    inp = inp if inp is not None else inputs.make_inputs(w)
     Ts = min(sample_tokens, w.num_tokens)
     idx = np.ascontiguousarray(inp.topk_idx[:, :Ts])
     x = np.ascontiguousarray(inp.x[:, :Ts])
@@ -385,11 +385,12 @@ def cpu_model():
 
 def run_reference(args, world):
     w = inputs.named(args.workload)
+    inp = inputs.make_inputs(w)
     samples = []
     for _ in range(args.warmup):
-        oracle_sample(w, args.cpu_sample_tokens)
+        oracle_sample(w, args.cpu_sample_tokens, inp)
     for _ in range(args.steps):
-        samples.append(oracle_sample(w, args.cpu_sample_tokens))
+        samples.append(oracle_sample(w, args.cpu_sample_tokens, inp))
     secs = sum(s["seconds"] for s in samples) / len(samples)
     value = statistics.median(s["value"] for s in samples)
     base = dict(samples[0])
@@ -428,7 +429,7 @@ def main():
     ap.add_argument("--workload", default="prefill",
                     help="prefill | decode | replica | tiny | sweep_T<n>[_mask5]")
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--cpu-sample-tokens", type=int, default=512,
+    ap.add_argument("--cpu-sample-tokens", type=int, default=1024,
                     help="tokens per rank in the CPU oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

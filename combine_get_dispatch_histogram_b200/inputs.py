@@ -106,8 +106,14 @@ def replica(num_tokens: int = 2048) -> Workload:
                     num_tokens, 6, 64, 4096, routing="zipf", zipf_s=1.5, num_extra=16)
 
 
+def small_slab() -> Workload:
+    """Decode-like routing with a 1.9 GB slab: the size used for detailed hardware-counter captures."""
+    return Workload("small_slab", 8, 512, 8, 32, 7168)
+
+
 def named(name: str) -> Workload:
-    table = {"tiny": tiny(), "decode": decode(), "prefill": prefill(), "replica": replica()}
+    table = {"tiny": tiny(), "decode": decode(), "prefill": prefill(), "replica": replica(),
+             "small_slab": small_slab()}
     if name in table:
         return table[name]
     if name.startswith("sweep_T"):
