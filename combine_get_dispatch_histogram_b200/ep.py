@@ -292,3 +292,41 @@ def ep_reroute(topk_idx_logical: torch.Tensor, num_logical: int, num_extra: int,
                             _ptr(out["topk_idx_phys"]), _ptr(out["status"]), _cfg(cfg), _stream(dev, stream))
     _check("ep_reroute", rc)
     return out
+
+
+def ep_layout_noalloc(topk_idx: torch.Tensor, active: torch.Tensor, num_experts: int, *, hidden: int = 8,
+                      out: Optional[DispatchLayout] = None, status: Optional[torch.Tensor] = None, cfg=None,
+                      stream=None) -> DispatchLayout:
+    """``ep_layout`` without a workspace argument (``ep_layout_noalloc`` of ``include/ep.h``).
+
+    For callers that cannot allocate device scratch: the library keeps a fixed
+    4 MiB scratch array per GPU.  Calls on one GPU share that array, so calls
+    that could overlap on the GPU must be ordered (same stream or events).
+    Outputs are allocated here only when ``out`` is not given.
+    """
+    lib = load_library()
+    if not getattr(lib.ep_layout_noalloc, "_ep_bound", False):
+        P = ctypes.c_void_p
+        lib.ep_layout_noalloc.argtypes = [Dims, P, P, P, P, P, P, P, P, P, Cfg, P]
+        lib.ep_layout_noalloc.restype = ctypes.c_int
+        lib.ep_layout_noalloc._ep_bound = True
+    _need(topk_idx, "topk_idx", torch.int32)
+    if topk_idx.dim() != 3:
+        raise ValueError("topk_idx must be [R, T, k]")
+    R, T, k = topk_idx.shape
+    dev = topk_idx.device
+    E = int(num_experts)
+    _need(active, "active", torch.uint8, (R,), dev)
+    if out is None:
+        out = DispatchLayout(
+            torch.empty((R, E), dtype=torch.int32, device=dev), torch.empty((R, R), dtype=torch.int32, device=dev),
+            torch.empty((R, T, R), dtype=torch.uint8, device=dev), torch.empty((E,), dtype=torch.int32, device=dev),
+            torch.empty((E, R), dtype=torch.int32, device=dev), torch.empty((R, T, k), dtype=torch.int32, device=dev),
+            _status(dev, status))
+    with torch.cuda.device(dev):
+        rc = lib.ep_layout_noalloc(Dims(R, T, k, E, hidden), _ptr(topk_idx), _ptr(active),
+                                   _ptr(out.num_tokens_per_expert), _ptr(out.num_tokens_per_rank),
+                                   _ptr(out.is_token_in_rank), _ptr(out.recv_count), _ptr(out.expert_rank_offset),
+                                   _ptr(out.pair_row), _ptr(out.status), _cfg(cfg), _stream(dev, stream))
+    _check("ep_layout_noalloc", rc)
+    return out

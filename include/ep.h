@@ -149,6 +149,39 @@ EP_API int ep_layout(ep_dims_t d, const int32_t *topk_idx, const uint8_t *active
               int32_t *expert_rank_offset, int32_t *pair_row,
               int32_t *status, ep_cfg_t cfg, void *stream);
 
+/* Scratch that ep_layout_noalloc keeps inside the library: 4 MiB per GPU. */
+enum { EP_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024 };
+
+/*
+ * ep_layout_noalloc -- ep_layout for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot hand ep_layout a workspace: a C or C++ host with no framework
+ * allocator would need cudaMalloc, which synchronises the device and is ruled
+ * out on hot paths that run under a fixed, pre-reserved memory budget.
+ * Arguments, outputs and results are those of ep_layout without the
+ * workspace: the scratch is a fixed array of EP_LAYOUT_NOALLOC_SCRATCH_BYTES
+ * inside the library's device image, one per GPU that loads the library,
+ * held until the process exits.  Nothing is allocated at call time.
+ *   - Shapes whose ep_layout_workspace_bytes(d) exceeds
+ *     EP_LAYOUT_NOALLOC_SCRATCH_BYTES are rejected with EP_ERR_UNSUPPORTED
+ *     before anything is enqueued (prefill shape R=8, T=4096, E=256 needs
+ *     1.08 MB).
+ *   - The first call on a device looks up that device's scratch address
+ *     (cudaGetSymbolAddress with the device current) and caches it; make
+ *     that first call before any stream capture.  EP_ERR_CUDA if the lookup
+ *     fails.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents; nothing in it needs to start at zero.  Calls whose kernels
+ *     may overlap on the same GPU race on it: order them (one stream, or
+ *     events).
+ */
+EP_API int ep_layout_noalloc(ep_dims_t d, const int32_t *topk_idx, const uint8_t *active,
+              int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
+              uint8_t *is_token_in_rank, int32_t *recv_count,
+              int32_t *expert_rank_offset, int32_t *pair_row,
+              int32_t *status, ep_cfg_t cfg, void *stream);
+
 /*
  * ep_dispatch -- scatter token rows into the experts' receive slabs.
  *
