@@ -206,9 +206,11 @@ def run_ours(args, rank, world, local_rank):
             idx = rr_out["topk_idx_phys"]
         ep.ep_layout(idx, act, E, hidden=H, workspace=lay_ws, out=lay, status=status, stream=stream)
         mark(1)
-        ep.ep_dispatch(x, idx, lay.pair_row, E, recv_x=recv_x, src_info=src_info, status=status, stream=stream)
+        ep.ep_dispatch(x, idx, lay.pair_row, E, recv_x=recv_x, src_info=src_info, status=status, stream=stream,
+                       cfg=args.dispatch_cfg)
         mark(2)
-        ep.ep_combine(recv_x, idx, wts, lay.pair_row, act, out=out, status=status, stream=stream)
+        ep.ep_combine(recv_x, idx, wts, lay.pair_row, act, out=out, status=status, stream=stream,
+                      cfg=args.combine_cfg)
         mark(3)
 
     with torch.cuda.stream(stream):
@@ -324,6 +326,8 @@ def run_ours(args, rank, world, local_rank):
                      "algorithmic_bytes": dom[1]},
         "gpu_launches": launches_per_step * args.steps,
     }
+    if args.dispatch_cfg or args.combine_cfg:
+        line["launch_cfg"] = {"dispatch": args.dispatch_cfg, "combine": args.combine_cfg}
     if e2e is not None:
         line["e2e"] = {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
@@ -420,6 +424,16 @@ def run_reference(args, world):
 
 # ----------------------------------------------------------------------------- main
 
+def parse_cfg(text: str) -> dict:
+    cfg = {}
+    for part in filter(None, text.split(",")):
+        key, val = part.split("=")
+        if key not in ("max_ctas", "threads", "stages", "variant"):
+            raise argparse.ArgumentTypeError(f"unknown launch-config key {key}")
+        cfg[key] = int(val)
+    return cfg
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -432,6 +446,10 @@ def main():
     ap.add_argument("--cpu-sample-tokens", type=int, default=1024,
                     help="tokens per rank in the CPU oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dispatch-cfg", type=parse_cfg, default=None,
+                    help="launch config of ep_dispatch, e.g. max_ctas=296,stages=7")
+    ap.add_argument("--combine-cfg", type=parse_cfg, default=None,
+                    help="launch config of ep_combine, e.g. stages=8,threads=256")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

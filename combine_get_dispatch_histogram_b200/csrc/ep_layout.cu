@@ -18,11 +18,14 @@
 //                atomics are needed).  It also builds each token's destination
 //                rank set (is_token_in_rank) and the chunk's per-rank token
 //                counts.
-//   2. scan   -- one lane per expert sums the chunk histograms of each source
-//                rank (num_tokens_per_expert), scans them over ranks
+//   2. scan   -- one lane per expert (32 experts per CTA, 32 warps splitting
+//                each rank's chunks into segments) sums the chunk histograms of
+//                each source rank (num_tokens_per_expert), scans them over ranks
 //                (expert_rank_offset, recv_count) and turns every chunk count
 //                into the chunk's first row (an exclusive scan over chunks in
-//                (rank, chunk) order), in place in the workspace.
+//                (rank, chunk) order), in place in the workspace; one warp per
+//                (source, destination) rank pair reduces the chunk token counts
+//                (num_tokens_per_rank).
 //   3. rank   -- the warp walks its chunk again in (token, slot) order, 32
 //                pairs at a time; a pair's row is the chunk base of its expert
 //                + the warp's running count + its rank among equal experts to
@@ -39,6 +42,7 @@ namespace ep {
 namespace {
 
 constexpr int kChunkTokens = 32;
+constexpr int kBatch = 8;  // 32-pair steps whose loads are issued together
 constexpr int kActiveSlots = 64;  // shared-memory copy of the active mask (EP_MAX_RANKS)
 
 struct LayoutArgs {
@@ -82,14 +86,23 @@ __global__ void layout_count_kernel(LayoutArgs a) {
     const int np = nt * a.k;
 
     bool bad = false;
-    for (int p0 = 0; p0 < np; p0 += 32) {
-        const int p = p0 + lane;
-        const int e = p < np ? __ldg(base + p) : -1;
-        bad |= (e < -1 || e >= a.E);
-        const bool live = pair_live(e, a.E, a.E_local, src_ok, act);
-        const uint32_t m = __match_any_sync(0xffffffffu, live ? e : -1);
-        if (live && lane == __ffs(m) - 1) h[e] += __popc(m);
-        __syncwarp();
+    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+        int ev[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            ev[u] = p < np ? __ldg(base + p) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            if (p0 + u * 32 >= np) break;
+            const int e = ev[u];
+            bad |= (e < -1 || e >= a.E);
+            const bool live = pair_live(e, a.E, a.E_local, src_ok, act);
+            const uint32_t m = __match_any_sync(0xffffffffu, live ? e : -1);
+            if (live && lane == __ffs(m) - 1) h[e] += __popc(m);
+            __syncwarp();
+        }
     }
 
     // destination-rank set of each token (lane <-> token)
@@ -114,57 +127,85 @@ __global__ void layout_count_kernel(LayoutArgs a) {
     for (int e = lane; e < a.E; e += 32) out[e] = h[e];
 }
 
-__global__ void layout_scan_kernel(LayoutArgs a) {
+// One CTA per 32 experts (lane <-> expert).  Each rank's chunk range is cut
+// into `segs` segments and every warp takes (rank, segment) items, so each
+// lane walks only a few chunks; warp 0 then scans the segment totals in
+// (rank, segment) order.  Separately, one warp per (source, destination) rank
+// pair sums the per-chunk token counts.
+__global__ void __launch_bounds__(1024) layout_scan_kernel(LayoutArgs a, int segs) {
     extern __shared__ int32_t smem[];
-    const int SW = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int32_t* per_rank = smem;             // [R][32] live pairs of rank r on this lane's expert
-    int32_t* rank_first = smem + a.R * 32;  // [R][32] first row of rank r
+    const int NW = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int items = a.R * segs;
+    int32_t* seg_sum = smem;                // [items][32]
+    int32_t* seg_first = smem + items * 32;  // [items][32]
     const int e = blockIdx.x * 32 + lane;
     const bool ok = e < a.E;
     const int C = a.chunks_per_rank;
+    const int seg_len = (C + segs - 1) / segs;
 
-    for (int r = warp; r < a.R; r += SW) {
+    // tokens per (source, destination) rank: warp-parallel sums over chunks
+    const int RR = a.R * a.R;
+    for (int pr = blockIdx.x * NW + warp; pr < RR; pr += gridDim.x * NW) {
+        const int r = pr / a.R, d = pr - r * a.R;
+        const int32_t* col = a.chunk_tpr + int64_t(r) * C * a.R + d;
+        int32_t s = 0;
+        for (int c = lane; c < C; c += 32) s += col[int64_t(c) * a.R];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) a.num_tokens_per_rank[pr] = s;
+    }
+
+    for (int it = warp; it < items; it += NW) {
+        const int r = it / segs, sg = it - r * segs;
+        const int c0 = sg * seg_len, c1 = min(C, c0 + seg_len);
         int32_t s = 0;
         if (ok) {
             const int32_t* col = a.chunk_hist + int64_t(r) * C * a.E + e;
 #pragma unroll 8
-            for (int c = 0; c < C; ++c) s += col[int64_t(c) * a.E];
-            a.num_tokens_per_expert[int64_t(r) * a.E + e] = s;
+            for (int c = c0; c < c1; ++c) s += col[int64_t(c) * a.E];
         }
-        per_rank[r * 32 + lane] = s;
+        seg_sum[it * 32 + lane] = s;
     }
     __syncthreads();
     if (warp == 0) {
-        int32_t off = 0;
+        int32_t run = 0;
         for (int r = 0; r < a.R; ++r) {
-            rank_first[r * 32 + lane] = off;
-            if (ok) a.expert_rank_offset[int64_t(e) * a.R + r] = off;
-            off += per_rank[r * 32 + lane];
+            const int32_t rank_first = run;
+            if (ok) a.expert_rank_offset[int64_t(e) * a.R + r] = rank_first;
+            for (int sg = 0; sg < segs; ++sg) {
+                seg_first[(r * segs + sg) * 32 + lane] = run;
+                run += seg_sum[(r * segs + sg) * 32 + lane];
+            }
+            if (ok) a.num_tokens_per_expert[int64_t(r) * a.E + e] = run - rank_first;
         }
         if (ok) {
-            a.recv_count[e] = off;
-            if (off > a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
+            a.recv_count[e] = run;
+            if (run > a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
         }
     }
     __syncthreads();
-    for (int r = warp; r < a.R; r += SW) {
-        if (!ok) continue;
-        int32_t run = rank_first[r * 32 + lane];
+    if (!ok) return;
+    for (int it = warp; it < items; it += NW) {
+        const int r = it / segs, sg = it - r * segs;
+        const int c0 = sg * seg_len, c1 = min(C, c0 + seg_len);
+        int32_t run = seg_first[it * 32 + lane];
         int32_t* col = a.chunk_hist + int64_t(r) * C * a.E + e;
-        for (int c = 0; c < C; ++c) {
+        int c = c0;
+        for (; c + 8 <= c1; c += 8) {
+            int32_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = col[int64_t(c + u) * a.E];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                col[int64_t(c + u) * a.E] = run;
+                run += v[u];
+            }
+        }
+        for (; c < c1; ++c) {
             const int32_t v = col[int64_t(c) * a.E];
             col[int64_t(c) * a.E] = run;
             run += v;
         }
-    }
-    // tokens per (source, destination) rank: sum of the chunk counts
-    const int RR = a.R * a.R;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < RR; i += gridDim.x * blockDim.x) {
-        const int r = i / a.R, d = i - r * a.R;
-        int32_t s = 0;
-        const int32_t* col = a.chunk_tpr + int64_t(r) * C * a.R + d;
-        for (int c = 0; c < C; ++c) s += col[int64_t(c) * a.R];
-        a.num_tokens_per_rank[i] = s;
     }
 }
 
@@ -191,16 +232,26 @@ __global__ void layout_rank_kernel(LayoutArgs a) {
     const int np = nt * a.k;
     const uint32_t below = lanemask_lt();
 
-    for (int p0 = 0; p0 < np; p0 += 32) {
-        const int p = p0 + lane;
-        const int e = p < np ? __ldg(base + p) : -1;
-        const bool live = pair_live(e, a.E, a.E_local, src_ok, act);
-        const uint32_t m = __match_any_sync(0xffffffffu, live ? e : -1);
-        const int32_t b = live ? next_row[e] : 0;
-        __syncwarp();
-        if (live && lane == __ffs(m) - 1) next_row[e] = b + __popc(m);
-        __syncwarp();
-        if (p < np) rows[p] = live ? b + __popc(m & below) : -1;
+    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+        int ev[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            ev[u] = p < np ? __ldg(base + p) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            if (p0 + u * 32 >= np) break;
+            const int e = ev[u];
+            const bool live = pair_live(e, a.E, a.E_local, src_ok, act);
+            const uint32_t m = __match_any_sync(0xffffffffu, live ? e : -1);
+            const int32_t b = live ? next_row[e] : 0;
+            __syncwarp();
+            if (live && lane == __ffs(m) - 1) next_row[e] = b + __popc(m);
+            __syncwarp();
+            if (p < np) rows[p] = live ? b + __popc(m & below) : -1;
+        }
     }
 }
 
@@ -279,9 +330,11 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     }
     const int chunk_blocks = int(ceil_div(a.G, W));
     if (a.G > 0) layout_count_kernel<<<chunk_blocks, 32 * W, chunk_smem, s>>>(a);
-    const int SW = std::min(d.num_ranks, 8);
-    const size_t scan_smem = size_t(2) * d.num_ranks * 32 * 4;
-    layout_scan_kernel<<<int(ceil_div(d.num_experts, 32)), 32 * SW, scan_smem, s>>>(a);
+    // scan: 32 warps per CTA; segments so that ranks x segments covers the warps
+    const int scan_warps = 32;
+    const int segs = std::max(1, std::min(a.chunks_per_rank, scan_warps / std::max(1, std::min(d.num_ranks, scan_warps))));
+    const size_t scan_smem = size_t(2) * d.num_ranks * segs * 32 * 4;
+    layout_scan_kernel<<<int(ceil_div(d.num_experts, 32)), 32 * scan_warps, scan_smem, s>>>(a, segs);
     if (a.G > 0) layout_rank_kernel<<<chunk_blocks, 32 * W, chunk_smem, s>>>(a);
     return launch_result();
 }

@@ -29,6 +29,9 @@ EP_ERR_CUDA = -3
 EP_STATUS_BAD_EXPERT = 1
 EP_STATUS_OVERFLOW = 2
 EP_STATUS_TIMEOUT = 8
+EP_VARIANT_AUTO = 0
+EP_VARIANT_BULK = 1
+EP_VARIANT_VECTOR = 2
 
 _lib = None
 
@@ -45,7 +48,8 @@ class Dims(ctypes.Structure):
 
 
 class Cfg(ctypes.Structure):
-    _fields_ = [("max_ctas", ctypes.c_int32), ("threads", ctypes.c_int32), ("stages", ctypes.c_int32)]
+    _fields_ = [("max_ctas", ctypes.c_int32), ("threads", ctypes.c_int32), ("stages", ctypes.c_int32),
+                ("variant", ctypes.c_int32)]
 
 
 def load_library(path: str = LIB_PATH):
@@ -113,10 +117,11 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None, device=Non
 
 def _cfg(cfg) -> Cfg:
     if cfg is None:
-        return Cfg(0, 0, 0)
+        return Cfg(0, 0, 0, 0)
     if isinstance(cfg, Cfg):
         return cfg
-    return Cfg(int(cfg.get("max_ctas", 0)), int(cfg.get("threads", 0)), int(cfg.get("stages", 0)))
+    return Cfg(int(cfg.get("max_ctas", 0)), int(cfg.get("threads", 0)), int(cfg.get("stages", 0)),
+               int(cfg.get("variant", 0)))
 
 
 def _stream(device, stream) -> ctypes.c_void_p:

@@ -106,10 +106,19 @@ typedef struct ep_dims {
 /* Launch tuning (cf. Buffer.get_dispatch_config / get_combine_config and
  * num_sms on the NeMo page).  A zero field means "choose automatically". */
 typedef struct ep_cfg {
-    int32_t max_ctas;     /* cap on CTAs of the row-moving kernels */
+    int32_t max_ctas;     /* CTAs of the row-moving kernels (dispatch: the grid, default
+                             2 per SM; combine: a cap, default 1 per SM) */
     int32_t threads;      /* threads per CTA where the kernel allows a choice */
     int32_t stages;       /* shared-memory pipeline depth of dispatch / combine */
+    int32_t variant;      /* dispatch / combine data path: EP_VARIANT_* */
 } ep_cfg_t;
+
+/* Data paths of ep_dispatch / ep_combine (ep_cfg_t.variant). */
+enum {
+    EP_VARIANT_AUTO = 0,      /* the faster path for the shape, as measured on B200 */
+    EP_VARIANT_BULK = 1,      /* rows staged in shared memory by bulk async copies */
+    EP_VARIANT_VECTOR = 2     /* rows moved through registers as 16-byte vectors */
+};
 
 /* Human-readable name of an EP_OK / EP_ERR_* code (static storage). */
 EP_API const char *ep_strerror(int code);

@@ -62,7 +62,7 @@ def test_workspace_sizes(lib):
 def test_host_validation_rejects_without_launching(lib):
     from combine_get_dispatch_histogram_b200 import ep
 
-    cfg = ep.Cfg(0, 0, 0)
+    cfg = ep.Cfg(0, 0, 0, 0)
     bad_dims = [ep.Dims(3, 4, 2, 8, 256),      # E not a multiple of R
                 ep.Dims(2, 4, 9, 8, 256),      # k > E
                 ep.Dims(2, 4, 2, 8, 12),       # H not a multiple of 8

@@ -239,8 +239,11 @@ def test_invalid_hidden_raises():
     assert ei.value.code == ep.EP_ERR_INVALID
 
 
-@pytest.mark.parametrize("cfg", [dict(stages=2), dict(max_ctas=1), dict(max_ctas=3, stages=3),
-                                 dict(threads=64), dict(max_ctas=1, stages=2, threads=96)])
+@pytest.mark.parametrize("cfg", [dict(variant=1, stages=2), dict(variant=1, max_ctas=1),
+                                 dict(variant=1, max_ctas=3, stages=3), dict(variant=1, threads=64),
+                                 dict(variant=1, max_ctas=1, stages=2, threads=96),
+                                 dict(variant=2), dict(variant=2, threads=1), dict(variant=2, threads=2),
+                                 dict(variant=2, max_ctas=1), dict(variant=2, max_ctas=5, threads=1)])
 def test_launch_configs(cfg):
     """Ring wrap-around and tiny grids: a single CTA walks every unit through 2 stages."""
     w = inputs.sweep(32, masked=True)
@@ -294,3 +297,36 @@ def test_reroute_small_cases():
         rref = oracle.reroute(idx, E, extra)
         for key in ("load", "num_replicas", "phys_base", "topk_idx_phys"):
             assert np.array_equal(rr[key].cpu().numpy(), rref[key]), (it, key)
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("name", ["tiny", "decode", "sweep_T16_mask5", "sweep_T512"])
+def test_variants_match_oracle(name, variant):
+    w = inputs.named(name)
+    inp = inputs.make_inputs(w)
+    ref, packed, want = _oracle_all(inp, w.num_experts)
+    _check_all(run_path(inp, w.num_experts, w.hidden, cfg=dict(variant=variant)), ref, packed, want,
+               f"{name} variant {variant}")
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("name", ["k1", "H8", "ragged_H", "wide_H", "R1"])
+def test_variants_edge_shapes(name, variant):
+    c = EDGE[name]
+    rng = np.random.default_rng(zlib.crc32(name.encode()) + variant)
+    idx = _uniform_idx(rng, c["R"], c["T"], c["k"], c["E"])
+    idx = np.where(rng.random(idx.shape) < 0.1, -1, idx)
+    inp = _custom(c["R"], c["T"], c["k"], c["E"], c["H"], idx, active=np.r_[np.ones(c["R"] - 1), 0] if c["R"] > 1
+                  else None)
+    ref, packed, want = _oracle_all(inp, c["E"])
+    _check_all(run_path(inp, c["E"], c["H"], cfg=dict(variant=variant)), ref, packed, want, f"{name} v{variant}")
+
+
+def test_vector_variant_rejects_wide_topk():
+    R, T, k, E, H = 2, 4, 9, 16, 64
+    idx = torch.zeros((R, T, k), dtype=torch.int32, device=dev())
+    pr = torch.full((R, T, k), -1, dtype=torch.int32, device=dev())
+    x = torch.zeros((R, T, H), dtype=torch.bfloat16, device=dev())
+    with pytest.raises(ep.EPError) as ei:
+        ep.ep_dispatch(x, idx, pr, E, cfg=dict(variant=2))
+    assert ei.value.code == ep.EP_ERR_UNSUPPORTED

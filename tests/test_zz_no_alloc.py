@@ -57,7 +57,7 @@ def test_noalloc_layout_equals_workspace_layout_on_two_calls_in_a_row():
                 ctypes.c_void_p(got.num_tokens_per_rank.data_ptr()),
                 ctypes.c_void_p(got.is_token_in_rank.data_ptr()), ctypes.c_void_p(got.recv_count.data_ptr()),
                 ctypes.c_void_p(got.expert_rank_offset.data_ptr()), ctypes.c_void_p(got.pair_row.data_ptr()),
-                ctypes.c_void_p(got.status.data_ptr()), ep.Cfg(0, 0, 0), ctypes.c_void_p(stream.cuda_stream))
+                ctypes.c_void_p(got.status.data_ptr()), ep.Cfg(0, 0, 0, 0), ctypes.c_void_p(stream.cuda_stream))
         assert rc == ep.EP_OK, ep.ep_strerror(rc)
         torch.cuda.synchronize()
         for key in KEYS:
@@ -71,5 +71,5 @@ def test_noalloc_layout_rejects_shapes_beyond_its_scratch():
     d = ep.Dims(8, 65536, 8, 256, 7168)
     assert ep.ep_layout_workspace_bytes(8, 65536, 8, 256, 7168) > 4 * 1024 * 1024
     fake = ctypes.c_void_p(16)
-    rc = fn(d, fake, fake, fake, fake, fake, fake, fake, fake, fake, ep.Cfg(0, 0, 0), None)
+    rc = fn(d, fake, fake, fake, fake, fake, fake, fake, fake, fake, ep.Cfg(0, 0, 0, 0), None)
     assert rc == ep.EP_ERR_UNSUPPORTED
