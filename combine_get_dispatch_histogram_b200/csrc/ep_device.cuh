@@ -125,6 +125,20 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     return m;
 }
 
+// Lanes (among `live`) whose key equals this lane's, found with one ballot per
+// key bit (vote instructions) instead of __match_any_sync, whose throughput is
+// low when many warps of an SM use it at once.  Keys compare on bits
+// [0, nbits); lanes outside `live` never appear in the result.
+__device__ __forceinline__ uint32_t match_key(uint32_t key, int nbits, uint32_t live) {
+    uint32_t m = live;
+    for (int b = 0; b < nbits; ++b) {
+        const uint32_t bit = (key >> b) & 1u;
+        const uint32_t bal = __ballot_sync(0xffffffffu, bit);
+        m &= bit ? bal : ~bal;
+    }
+    return m;
+}
+
 // 16-byte load of data read once: bypass L1, ask L2 to fetch the surrounding 256 bytes.
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     uint4 v;

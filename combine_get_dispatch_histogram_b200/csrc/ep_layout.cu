@@ -8,28 +8,37 @@
 // among its expert's live pairs in (source rank, token, slot) order: a stable
 // counting sort keyed by expert.
 //
-// Work decomposition.  The R*T*k pairs are cut into CHUNKS of 32 tokens of one
-// source rank (chunk g = r * chunks_per_rank + c), and every chunk is owned by
-// one warp in two passes:
-//   1. count  -- the warp builds a private shared-memory histogram of its
-//                chunk; lanes holding the same expert are merged with
-//                __match_any_sync so one leader adds the group's popcount
-//                (a warp-aggregated update; the histogram is warp-private so no
-//                atomics are needed).  It also builds each token's destination
-//                rank set (is_token_in_rank) and the chunk's per-rank token
-//                counts.
-//   2. scan   -- one lane per expert (32 experts per CTA, 32 warps splitting
-//                each rank's chunks into segments) sums the chunk histograms of
-//                each source rank (num_tokens_per_expert), scans them over ranks
-//                (expert_rank_offset, recv_count) and turns every chunk count
-//                into the chunk's first row (an exclusive scan over chunks in
-//                (rank, chunk) order), in place in the workspace; one warp per
-//                (source, destination) rank pair reduces the chunk token counts
-//                (num_tokens_per_rank).
-//   3. rank   -- the warp walks its chunk again in (token, slot) order, 32
-//                pairs at a time; a pair's row is the chunk base of its expert
-//                + the warp's running count + its rank among equal experts to
-//                its left in the same 32 (popc of the match mask below it).
+// Two paths compute the same result (ep_cfg_t.variant selects one; AUTO picks
+// by size).  Both sort with the same two ideas: lanes holding the same expert
+// are merged (a match mask built from one warp ballot per expert-id bit) so
+// one leader updates the group's count (a warp-aggregated update), and a
+// pair's row inside a run of 32 consecutive
+// pairs is its running count plus its rank among equal experts to its left
+// (popc of the match mask below it).  Destination ranks come from a shared
+// table rank_of[e] (-1 when that rank is masked), so no pair test divides.
+//
+// Single-CTA path (EP_LAYOUT_SINGLE_CTA; R <= 32, E <= 1024, <= 32768 pairs;
+// AUTO up to 4096 pairs): one 1024-thread CTA, one launch, no workspace.  Each rank's tokens are split
+// among 32/R warps in (rank, token) order; every warp builds a private
+// histogram of its part, the CTA scans them over warps per expert (which also
+// yields expert_rank_offset, num_tokens_per_expert, recv_count), and every
+// warp then walks its part again assigning rows.
+//
+// Chunked path (EP_LAYOUT_CHUNKED; any shape): each rank's tokens are cut into
+// C contiguous chunks (chunk g = r*C + c, ordered like the sort key; about a
+// hundred chunks in all) over three launches:
+//   1. count -- one CTA per chunk builds the chunk's expert histogram with
+//               warp-aggregated shared atomics, each token's destination-rank
+//               set (is_token_in_rank) and the chunk's per-destination token
+//               counts, into the workspace;
+//   2. scan  -- one CTA per 32 experts (lane <-> expert, warps <-> runs of
+//               chunks, values held in registers) turns every chunk count into
+//               the chunk's first row (exclusive scan over (rank, chunk)), in
+//               place, and writes expert_rank_offset, num_tokens_per_expert,
+//               recv_count; warps also reduce num_tokens_per_rank;
+//   3. rank  -- one CTA per chunk splits it among its warps, counts each
+//               warp's part into a warp-private histogram, scans those over
+//               warps on top of the chunk's first rows, and assigns rows.
 // Every step is deterministic: rows are unique and identical run to run.
 #include <algorithm>
 #include <cstdint>
@@ -41,14 +50,24 @@
 namespace ep {
 namespace {
 
-constexpr int kChunkTokens = 32;
-constexpr int kBatch = 8;  // 32-pair steps whose loads are issued together
-constexpr int kActiveSlots = 64;  // shared-memory copy of the active mask (EP_MAX_RANKS)
+constexpr int kTargetChunks = 32;    // chunks over all ranks at least
+constexpr int kPairsPerChunk = 2048;  // aim for this many pairs per chunk
+constexpr int kMaxChunks = 148;       // G <= kMaxChunks + R - 1 <= 32 * kScanRowsPerWarp
+constexpr int kScanWarps = 32;
+constexpr int kScanRowsPerWarp = 8;
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallMaxPairs = 32768;
+constexpr int kSmallAutoPairs = 4096;  // AUTO takes the single-CTA path up to here (B200 measurement)
+constexpr int kSmallMaxExperts = 1024;
+constexpr int kSmallMaxRanks = 32;
+constexpr int kMaxWarps = 16;
+constexpr int kBatch = 8;           // 32-pair steps whose loads are issued together
+constexpr int kActiveSlots = 64;    // shared copy of the active mask (EP_MAX_RANKS)
 
 struct LayoutArgs {
     const int32_t* topk_idx;
     const uint8_t* active;
-    int32_t* chunk_hist;  // workspace [G][E]: counts, then first rows
+    int32_t* chunk_hist;  // workspace [G][E]
     int32_t* chunk_tpr;   // workspace [G][R]: tokens of the chunk per destination rank
     int32_t* num_tokens_per_expert;
     int32_t* num_tokens_per_rank;
@@ -58,32 +77,185 @@ struct LayoutArgs {
     int32_t* pair_row;
     int32_t* status;
     int R, T, k, E, E_local;
-    int chunks_per_rank, G;
+    int key_bits;      // bits that tell experts apart: ceil(log2(E))
+    int C, G;          // chunks per rank, chunks
+    int chunk_tokens;  // tokens per chunk (the last chunk of a rank may be shorter)
     int64_t cap;
 };
 
-__device__ __forceinline__ bool pair_live(int e, int E, int E_local, bool src_ok, const int32_t* act) {
-    return e >= 0 && e < E && src_ok && act[e / E_local] != 0;
+struct ChunkGeom {
+    int r, t0, t1;
+};
+
+__device__ __forceinline__ ChunkGeom chunk_of(const LayoutArgs& a, int g) {
+    ChunkGeom c;
+    c.r = g / a.C;
+    c.t0 = min(a.T, (g - c.r * a.C) * a.chunk_tokens);
+    c.t1 = min(a.T, c.t0 + a.chunk_tokens);
+    return c;
 }
 
-__global__ void layout_count_kernel(LayoutArgs a) {
+// act[] <- active mask, rank_of[e] <- destination rank of e, or -1 if it is masked.
+__device__ __forceinline__ void load_tables(const LayoutArgs& a, int32_t* act, int32_t* rank_of) {
+    for (int i = threadIdx.x; i < a.R; i += blockDim.x) act[i] = a.active[i];
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        const int d = e / a.E_local;
+        rank_of[e] = a.active[d] ? d : -1;
+    }
+}
+
+__device__ __forceinline__ bool pair_live(int e, int E, bool src_ok, const int32_t* rank_of) {
+    return src_ok && e >= 0 && e < E && rank_of[e] >= 0;
+}
+
+__global__ void __launch_bounds__(32 * kMaxWarps) layout_count_kernel(LayoutArgs a) {
     extern __shared__ int32_t smem[];
     int32_t* act = smem;
-    const int W = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i < a.R; i += blockDim.x) act[i] = a.active[i];
+    int32_t* tpr = smem + kActiveSlots;
+    int32_t* rank_of = smem + 2 * kActiveSlots;
+    int32_t* hist = rank_of + a.E;
+    load_tables(a, act, rank_of);
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) hist[e] = 0;
+    for (int d = threadIdx.x; d < a.R; d += blockDim.x) tpr[d] = 0;
     __syncthreads();
-    const int g = blockIdx.x * W + warp;
-    if (g >= a.G) return;
-    int32_t* h = smem + kActiveSlots + warp * a.E;
-    for (int e = lane; e < a.E; e += 32) h[e] = 0;
-    __syncwarp();
 
-    const int r = g / a.chunks_per_rank;
-    const int t0 = (g - r * a.chunks_per_rank) * kChunkTokens;
-    const int nt = min(kChunkTokens, a.T - t0);
-    const bool src_ok = act[r] != 0;
-    const int32_t* base = a.topk_idx + (int64_t(r) * a.T + t0) * a.k;
-    const int np = nt * a.k;
+    const ChunkGeom cg = chunk_of(a, blockIdx.x);
+    const bool src_ok = act[cg.r] != 0;
+    const int64_t pbase = (int64_t(cg.r) * a.T + cg.t0) * a.k;
+    const int32_t* base = a.topk_idx + pbase;
+    const int np = (cg.t1 - cg.t0) * a.k;
+
+    bool bad = false;
+    const int stride = blockDim.x * kBatch;
+    for (int p0 = (threadIdx.x & ~31) * kBatch; p0 < np; p0 += stride) {
+        int ev[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + (threadIdx.x & 31);
+            ev[u] = p < np ? __ldg(base + p) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int e = ev[u];
+            bad |= (e < -1 || e >= a.E);
+            const bool live = pair_live(e, a.E, src_ok, rank_of);
+            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
+            if (live && (threadIdx.x & 31) == __ffs(m) - 1) atomicAdd(hist + e, __popc(m));
+        }
+    }
+
+    // destination-rank set of each token (thread <-> token)
+    const int lane = threadIdx.x & 31;
+    for (int t0 = cg.t0 + (threadIdx.x & ~31); t0 < cg.t1; t0 += blockDim.x) {
+        const int t = t0 + lane;
+        uint64_t ranks = 0;
+        if (t < cg.t1) {
+            const int32_t* tb = a.topk_idx + (int64_t(cg.r) * a.T + t) * a.k;
+            for (int j = 0; j < a.k; ++j) {
+                const int e = __ldg(tb + j);
+                if (pair_live(e, a.E, src_ok, rank_of)) ranks |= 1ull << rank_of[e];
+            }
+            uint8_t* itr = a.is_token_in_rank + (int64_t(cg.r) * a.T + t) * a.R;
+            for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
+        }
+        for (int d = 0; d < a.R; ++d) {
+            const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
+            if (lane == 0 && n) atomicAdd(tpr + d, n);
+        }
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
+    int32_t* out = a.chunk_hist + int64_t(blockIdx.x) * a.E;
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) out[e] = hist[e];
+    for (int d = threadIdx.x; d < a.R; d += blockDim.x) a.chunk_tpr[int64_t(blockIdx.x) * a.R + d] = tpr[d];
+}
+
+// One CTA per 32 experts; warp w holds chunk rows [w*rpw, (w+1)*rpw) in registers.
+__global__ void __launch_bounds__(32 * kScanWarps) layout_scan_kernel(LayoutArgs a) {
+    __shared__ int32_t seg[kScanWarps][32];
+    __shared__ int32_t total[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 32 + lane;
+    const bool ok = e < a.E;
+    const int rpw = (a.G + kScanWarps - 1) / kScanWarps;
+    const int g0 = warp * rpw;
+    int32_t v[kScanRowsPerWarp];
+    int32_t s = 0;
+#pragma unroll
+    for (int i = 0; i < kScanRowsPerWarp; ++i) {
+        const int g = g0 + i;
+        v[i] = (ok && i < rpw && g < a.G) ? a.chunk_hist[int64_t(g) * a.E + e] : 0;
+        s += v[i];
+    }
+    seg[warp][lane] = s;
+    __syncthreads();
+    if (warp == 0) {
+        int32_t run = 0;
+        for (int w = 0; w < kScanWarps; ++w) {
+            const int32_t t = seg[w][lane];
+            seg[w][lane] = run;
+            run += t;
+        }
+        total[lane] = run;
+        if (ok) {
+            a.recv_count[e] = run;
+            if (run > a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
+        }
+    }
+    __syncthreads();
+    int32_t run = seg[warp][lane];
+#pragma unroll
+    for (int i = 0; i < kScanRowsPerWarp; ++i) {
+        const int g = g0 + i;
+        if (ok && i < rpw && g < a.G) a.chunk_hist[int64_t(g) * a.E + e] = run;
+        run += v[i];
+    }
+    __syncthreads();
+    if (ok) {
+        for (int r = warp; r < a.R; r += kScanWarps) {
+            const int32_t off = a.chunk_hist[int64_t(r) * a.C * a.E + e];
+            const int32_t next = r + 1 < a.R ? a.chunk_hist[int64_t(r + 1) * a.C * a.E + e] : total[lane];
+            a.expert_rank_offset[int64_t(e) * a.R + r] = off;
+            a.num_tokens_per_expert[int64_t(r) * a.E + e] = next - off;
+        }
+    }
+    const int RR = a.R * a.R;
+    for (int pr = blockIdx.x * kScanWarps + warp; pr < RR; pr += gridDim.x * kScanWarps) {
+        const int r = pr / a.R, d = pr - r * a.R;
+        const int32_t* col = a.chunk_tpr + int64_t(r) * a.C * a.R + d;
+        int32_t t = 0;
+        for (int c = lane; c < a.C; c += 32) t += col[int64_t(c) * a.R];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+        if (lane == 0) a.num_tokens_per_rank[pr] = t;
+    }
+}
+
+// Single CTA: the whole layout in one launch (small problems).
+__global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(LayoutArgs a) {
+    extern __shared__ int32_t smem[];
+    constexpr int NW = kSmallThreads / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int32_t* act = smem;
+    int32_t* tpr = smem + kActiveSlots;                        // [R][R]
+    int32_t* rank_of = tpr + kSmallMaxRanks * kSmallMaxRanks;   // [E]
+    int32_t* whist = rank_of + a.E;                            // [NW][E]
+    load_tables(a, act, rank_of);
+    for (int i = threadIdx.x; i < NW * a.E; i += blockDim.x) whist[i] = 0;
+    for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) tpr[i] = 0;
+    __syncthreads();
+
+    // warps per rank and this warp's token range (in (rank, token) order)
+    const int wpr = NW / a.R;  // R <= 32
+    const int r = warp / wpr, part = warp - r * wpr;
+    const bool has_rank = r < a.R;
+    const int tw = (a.T + wpr - 1) / wpr;
+    const int wt0 = has_rank ? min(a.T, part * tw) : 0, wt1 = has_rank ? min(a.T, wt0 + tw) : 0;
+    const bool src_ok = has_rank && act[r] != 0;
+    const int64_t pbase = has_rank ? (int64_t(r) * a.T + wt0) * a.k : 0;
+    const int32_t* base = a.topk_idx + pbase;
+    int32_t* rows = a.pair_row + pbase;
+    const int np = (wt1 - wt0) * a.k;
+    int32_t* mine = whist + warp * a.E;
 
     bool bad = false;
     for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
@@ -95,143 +267,54 @@ __global__ void layout_count_kernel(LayoutArgs a) {
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
-            if (p0 + u * 32 >= np) break;
             const int e = ev[u];
             bad |= (e < -1 || e >= a.E);
-            const bool live = pair_live(e, a.E, a.E_local, src_ok, act);
-            const uint32_t m = __match_any_sync(0xffffffffu, live ? e : -1);
-            if (live && lane == __ffs(m) - 1) h[e] += __popc(m);
+            const bool live = pair_live(e, a.E, src_ok, rank_of);
+            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
+            if (live && lane == __ffs(m) - 1) mine[e] += __popc(m);
             __syncwarp();
         }
     }
-
-    // destination-rank set of each token (lane <-> token)
-    uint64_t ranks = 0;
-    if (lane < nt) {
-        const int32_t* tb = base + lane * a.k;
-        for (int j = 0; j < a.k; ++j) {
-            const int e = __ldg(tb + j);
-            if (pair_live(e, a.E, a.E_local, src_ok, act)) ranks |= 1ull << (e / a.E_local);
+    // destination-rank set of each token of this warp's part
+    for (int t0 = wt0; t0 < wt1; t0 += 32) {
+        const int t = t0 + lane;
+        uint64_t ranks = 0;
+        if (t < wt1) {
+            const int32_t* tb = a.topk_idx + (int64_t(r) * a.T + t) * a.k;
+            for (int j = 0; j < a.k; ++j) {
+                const int e = __ldg(tb + j);
+                if (pair_live(e, a.E, src_ok, rank_of)) ranks |= 1ull << rank_of[e];
+            }
+            uint8_t* itr = a.is_token_in_rank + (int64_t(r) * a.T + t) * a.R;
+            for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
         }
-        uint8_t* itr = a.is_token_in_rank + (int64_t(r) * a.T + t0 + lane) * a.R;
-        for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
-    }
-    int32_t* tpr = a.chunk_tpr + int64_t(g) * a.R;
-    for (int d = 0; d < a.R; ++d) {
-        const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
-        if (lane == 0) tpr[d] = n;
-    }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
-
-    int32_t* out = a.chunk_hist + int64_t(g) * a.E;
-    for (int e = lane; e < a.E; e += 32) out[e] = h[e];
-}
-
-// One CTA per 32 experts (lane <-> expert).  Each rank's chunk range is cut
-// into `segs` segments and every warp takes (rank, segment) items, so each
-// lane walks only a few chunks; warp 0 then scans the segment totals in
-// (rank, segment) order.  Separately, one warp per (source, destination) rank
-// pair sums the per-chunk token counts.
-__global__ void __launch_bounds__(1024) layout_scan_kernel(LayoutArgs a, int segs) {
-    extern __shared__ int32_t smem[];
-    const int NW = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int items = a.R * segs;
-    int32_t* seg_sum = smem;                // [items][32]
-    int32_t* seg_first = smem + items * 32;  // [items][32]
-    const int e = blockIdx.x * 32 + lane;
-    const bool ok = e < a.E;
-    const int C = a.chunks_per_rank;
-    const int seg_len = (C + segs - 1) / segs;
-
-    // tokens per (source, destination) rank: warp-parallel sums over chunks
-    const int RR = a.R * a.R;
-    for (int pr = blockIdx.x * NW + warp; pr < RR; pr += gridDim.x * NW) {
-        const int r = pr / a.R, d = pr - r * a.R;
-        const int32_t* col = a.chunk_tpr + int64_t(r) * C * a.R + d;
-        int32_t s = 0;
-        for (int c = lane; c < C; c += 32) s += col[int64_t(c) * a.R];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (lane == 0) a.num_tokens_per_rank[pr] = s;
-    }
-
-    for (int it = warp; it < items; it += NW) {
-        const int r = it / segs, sg = it - r * segs;
-        const int c0 = sg * seg_len, c1 = min(C, c0 + seg_len);
-        int32_t s = 0;
-        if (ok) {
-            const int32_t* col = a.chunk_hist + int64_t(r) * C * a.E + e;
-#pragma unroll 8
-            for (int c = c0; c < c1; ++c) s += col[int64_t(c) * a.E];
+        for (int d = 0; d < a.R; ++d) {
+            const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
+            if (lane == 0 && n) atomicAdd(tpr + r * a.R + d, n);
         }
-        seg_sum[it * 32 + lane] = s;
     }
-    __syncthreads();
-    if (warp == 0) {
+    if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
+
+    // scan the warp histograms per expert in warp order = (rank, part) order
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         int32_t run = 0;
-        for (int r = 0; r < a.R; ++r) {
+        for (int rr = 0; rr < a.R; ++rr) {
             const int32_t rank_first = run;
-            if (ok) a.expert_rank_offset[int64_t(e) * a.R + r] = rank_first;
-            for (int sg = 0; sg < segs; ++sg) {
-                seg_first[(r * segs + sg) * 32 + lane] = run;
-                run += seg_sum[(r * segs + sg) * 32 + lane];
+            a.expert_rank_offset[int64_t(e) * a.R + rr] = rank_first;
+            for (int w = rr * wpr; w < (rr + 1) * wpr; ++w) {
+                const int32_t c = whist[w * a.E + e];
+                whist[w * a.E + e] = run;
+                run += c;
             }
-            if (ok) a.num_tokens_per_expert[int64_t(r) * a.E + e] = run - rank_first;
+            a.num_tokens_per_expert[int64_t(rr) * a.E + e] = run - rank_first;
         }
-        if (ok) {
-            a.recv_count[e] = run;
-            if (run > a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
-        }
+        a.recv_count[e] = run;
+        if (run > a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
     }
+    for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) a.num_tokens_per_rank[i] = tpr[i];
     __syncthreads();
-    if (!ok) return;
-    for (int it = warp; it < items; it += NW) {
-        const int r = it / segs, sg = it - r * segs;
-        const int c0 = sg * seg_len, c1 = min(C, c0 + seg_len);
-        int32_t run = seg_first[it * 32 + lane];
-        int32_t* col = a.chunk_hist + int64_t(r) * C * a.E + e;
-        int c = c0;
-        for (; c + 8 <= c1; c += 8) {
-            int32_t v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = col[int64_t(c + u) * a.E];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                col[int64_t(c + u) * a.E] = run;
-                run += v[u];
-            }
-        }
-        for (; c < c1; ++c) {
-            const int32_t v = col[int64_t(c) * a.E];
-            col[int64_t(c) * a.E] = run;
-            run += v;
-        }
-    }
-}
 
-__global__ void layout_rank_kernel(LayoutArgs a) {
-    extern __shared__ int32_t smem[];
-    int32_t* act = smem;
-    const int W = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i < a.R; i += blockDim.x) act[i] = a.active[i];
-    __syncthreads();
-    const int g = blockIdx.x * W + warp;
-    if (g >= a.G) return;
-    int32_t* next_row = smem + kActiveSlots + warp * a.E;
-    const int32_t* first = a.chunk_hist + int64_t(g) * a.E;
-    for (int e = lane; e < a.E; e += 32) next_row[e] = first[e];
-    __syncwarp();
-
-    const int r = g / a.chunks_per_rank;
-    const int t0 = (g - r * a.chunks_per_rank) * kChunkTokens;
-    const int nt = min(kChunkTokens, a.T - t0);
-    const bool src_ok = act[r] != 0;
-    const int64_t pbase = (int64_t(r) * a.T + t0) * a.k;
-    const int32_t* base = a.topk_idx + pbase;
-    int32_t* rows = a.pair_row + pbase;
-    const int np = nt * a.k;
     const uint32_t below = lanemask_lt();
-
     for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
         int ev[kBatch];
 #pragma unroll
@@ -244,32 +327,118 @@ __global__ void layout_rank_kernel(LayoutArgs a) {
             const int p = p0 + u * 32 + lane;
             if (p0 + u * 32 >= np) break;
             const int e = ev[u];
-            const bool live = pair_live(e, a.E, a.E_local, src_ok, act);
-            const uint32_t m = __match_any_sync(0xffffffffu, live ? e : -1);
-            const int32_t b = live ? next_row[e] : 0;
+            const bool live = pair_live(e, a.E, src_ok, rank_of);
+            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
+            const int32_t b = live ? mine[e] : 0;
             __syncwarp();
-            if (live && lane == __ffs(m) - 1) next_row[e] = b + __popc(m);
+            if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
             __syncwarp();
             if (p < np) rows[p] = live ? b + __popc(m & below) : -1;
         }
     }
 }
 
-// Warps per CTA of the count / rank kernels: each warp holds an E-entry histogram.
-int chunk_warps(int E) {
-    const int per_warp = E * 4;
-    const int budget = 96 * 1024 - kActiveSlots * 4;
-    return std::max(1, std::min(8, budget / per_warp));
+__global__ void __launch_bounds__(32 * kMaxWarps) layout_rank_kernel(LayoutArgs a) {
+    extern __shared__ int32_t smem[];
+    const int W = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int32_t* act = smem;
+    int32_t* rank_of = smem + kActiveSlots;
+    int32_t* first = rank_of + a.E;   // [E] first row of this chunk, per expert
+    int32_t* whist = first + a.E;     // [W][E] per-warp counts, then per-warp first rows
+    load_tables(a, act, rank_of);
+    for (int i = threadIdx.x; i < W * a.E; i += blockDim.x) whist[i] = 0;
+    __syncthreads();
+
+    const int g = blockIdx.x;
+    const ChunkGeom cg = chunk_of(a, g);
+    const bool src_ok = act[cg.r] != 0;
+
+    // 1. first rows of this chunk (written by the scan)
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) first[e] = a.chunk_hist[int64_t(g) * a.E + e];
+    // per-warp counts of this chunk (warp w owns tokens [t0 + w*tw, t0 + (w+1)*tw))
+    const int tw = (cg.t1 - cg.t0 + W - 1) / W;
+    const int wt0 = min(cg.t1, cg.t0 + warp * tw), wt1 = min(cg.t1, wt0 + tw);
+    const int64_t pbase = (int64_t(cg.r) * a.T + wt0) * a.k;
+    const int32_t* base = a.topk_idx + pbase;
+    int32_t* rows = a.pair_row + pbase;
+    const int np = (wt1 - wt0) * a.k;
+    int32_t* mine = whist + warp * a.E;
+    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+        int ev[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            ev[u] = p < np ? __ldg(base + p) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int e = ev[u];
+            const bool live = pair_live(e, a.E, src_ok, rank_of);
+            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
+            if (live && lane == __ffs(m) - 1) mine[e] += __popc(m);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+
+    // 2. per-warp first rows: exclusive scan over warps, on top of the chunk's first rows
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        int32_t run = first[e];
+        for (int w = 0; w < W; ++w) {
+            const int32_t v = whist[w * a.E + e];
+            whist[w * a.E + e] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+
+    // 3. rows, in (token, slot) order within each warp's part
+    const uint32_t below = lanemask_lt();
+    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+        int ev[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            ev[u] = p < np ? __ldg(base + p) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            if (p0 + u * 32 >= np) break;
+            const int e = ev[u];
+            const bool live = pair_live(e, a.E, src_ok, rank_of);
+            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
+            const int32_t b = live ? mine[e] : 0;
+            __syncwarp();
+            if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
+            __syncwarp();
+            if (p < np) rows[p] = live ? b + __popc(m & below) : -1;
+        }
+    }
 }
 
-size_t layout_ws_hist_bytes(const ep_dims_t& d) {
-    const int64_t G = int64_t(d.num_ranks) * ceil_div(d.num_tokens, kChunkTokens);
-    return round_up16(size_t(G) * d.num_experts * 4);
+struct LayoutGeom {
+    int C, G, chunk_tokens, warps;
+};
+
+// Chunks per rank, tokens per chunk and warps per CTA for a shape.
+LayoutGeom layout_geom(const ep_dims_t& d) {
+    LayoutGeom lg;
+    const int64_t pairs = int64_t(d.num_ranks) * d.num_tokens * d.num_topk;
+    const int64_t target = std::min<int64_t>(kMaxChunks, std::max<int64_t>(kTargetChunks, ceil_div(pairs, kPairsPerChunk)));
+    int64_t C = std::max<int64_t>(1, ceil_div(target, d.num_ranks));
+    C = std::max<int64_t>(1, std::min<int64_t>(C, d.num_tokens));
+    lg.chunk_tokens = int(std::max<int64_t>(1, ceil_div(d.num_tokens, C)));
+    lg.C = int(std::max<int64_t>(1, ceil_div(std::max(d.num_tokens, 1), lg.chunk_tokens)));
+    lg.G = d.num_ranks * lg.C;
+    // warp-private histograms of the rank kernel: W * E ints within ~96 KB
+    const int64_t per_warp = int64_t(d.num_experts) * 4;
+    lg.warps = int(std::max<int64_t>(1, std::min<int64_t>(kMaxWarps, (96 * 1024) / per_warp)));
+    return lg;
 }
 
-size_t layout_ws_tpr_bytes(const ep_dims_t& d) {
-    const int64_t G = int64_t(d.num_ranks) * ceil_div(d.num_tokens, kChunkTokens);
-    return round_up16(size_t(G) * d.num_ranks * 4);
+size_t layout_ws_hist_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
+    return round_up16(size_t(lg.G) * d.num_experts * 4);
 }
 
 }  // namespace
@@ -279,14 +448,14 @@ using namespace ep;
 
 extern "C" size_t ep_layout_workspace_bytes(ep_dims_t d) {
     if (check_dims(d) != EP_OK) return 0;
-    return layout_ws_hist_bytes(d) + layout_ws_tpr_bytes(d);
+    const LayoutGeom lg = layout_geom(d);
+    return layout_ws_hist_bytes(d, lg) + round_up16(size_t(lg.G) * d.num_ranks * 4);
 }
 
 extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* active, void* workspace,
-                         size_t workspace_bytes, int32_t* num_tokens_per_expert,
-                         int32_t* num_tokens_per_rank, uint8_t* is_token_in_rank, int32_t* recv_count,
-                         int32_t* expert_rank_offset, int32_t* pair_row, int32_t* status, ep_cfg_t cfg,
-                         void* stream) {
+                         size_t workspace_bytes, int32_t* num_tokens_per_expert, int32_t* num_tokens_per_rank,
+                         uint8_t* is_token_in_rank, int32_t* recv_count, int32_t* expert_rank_offset,
+                         int32_t* pair_row, int32_t* status, ep_cfg_t cfg, void* stream) {
     (void)cfg;
     int rc = check_dims(d);
     if (rc != EP_OK) return rc;
@@ -295,13 +464,14 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
         return EP_ERR_INVALID;
     if (RT > 0 && (!topk_idx || !is_token_in_rank || !pair_row)) return EP_ERR_INVALID;
     const size_t need = ep_layout_workspace_bytes(d);
-    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return EP_ERR_INVALID;
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return EP_ERR_INVALID;
 
+    const LayoutGeom lg = layout_geom(d);
     LayoutArgs a;
     a.topk_idx = topk_idx;
     a.active = active;
     a.chunk_hist = static_cast<int32_t*>(workspace);
-    a.chunk_tpr = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + layout_ws_hist_bytes(d));
+    a.chunk_tpr = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + layout_ws_hist_bytes(d, lg));
     a.num_tokens_per_expert = num_tokens_per_expert;
     a.num_tokens_per_rank = num_tokens_per_rank;
     a.is_token_in_rank = is_token_in_rank;
@@ -314,27 +484,45 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     a.k = d.num_topk;
     a.E = d.num_experts;
     a.E_local = d.num_experts / d.num_ranks;
-    a.chunks_per_rank = int(ceil_div(d.num_tokens, kChunkTokens));
-    a.G = d.num_ranks * a.chunks_per_rank;
+    a.key_bits = 0;
+    while ((1 << a.key_bits) < d.num_experts) ++a.key_bits;
+    a.C = lg.C;
+    a.G = lg.G;
+    a.chunk_tokens = lg.chunk_tokens;
     a.cap = RT;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int W = chunk_warps(d.num_experts);
-    const size_t chunk_smem = size_t(kActiveSlots) * 4 + size_t(W) * d.num_experts * 4;
-    if (chunk_smem > 48 * 1024) {
-        if (cudaFuncSetAttribute(layout_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(chunk_smem)) != cudaSuccess ||
-            cudaFuncSetAttribute(layout_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(chunk_smem)) != cudaSuccess)
+    const int64_t pairs = int64_t(d.num_ranks) * d.num_tokens * d.num_topk;
+    const bool small_ok = d.num_ranks <= kSmallMaxRanks && d.num_experts <= kSmallMaxExperts &&
+                          pairs <= kSmallMaxPairs;
+    // one CTA beats three launches only while its warps' sequential walks stay short
+    const int path = cfg.variant != EP_VARIANT_AUTO ? cfg.variant
+                     : (small_ok && pairs <= kSmallAutoPairs ? EP_LAYOUT_SINGLE_CTA : EP_LAYOUT_CHUNKED);
+    if (path == EP_LAYOUT_SINGLE_CTA) {
+        if (!small_ok) return EP_ERR_UNSUPPORTED;
+        const size_t smem = size_t(kActiveSlots + kSmallMaxRanks * kSmallMaxRanks + d.num_experts +
+                                   (kSmallThreads / 32) * d.num_experts) * 4;
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(layout_single_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem)) != cudaSuccess)
             return EP_ERR_CUDA;
+        layout_single_cta_kernel<<<1, kSmallThreads, smem, s>>>(a);
+        return launch_result();
     }
-    const int chunk_blocks = int(ceil_div(a.G, W));
-    if (a.G > 0) layout_count_kernel<<<chunk_blocks, 32 * W, chunk_smem, s>>>(a);
-    // scan: 32 warps per CTA; segments so that ranks x segments covers the warps
-    const int scan_warps = 32;
-    const int segs = std::max(1, std::min(a.chunks_per_rank, scan_warps / std::max(1, std::min(d.num_ranks, scan_warps))));
-    const size_t scan_smem = size_t(2) * d.num_ranks * segs * 32 * 4;
-    layout_scan_kernel<<<int(ceil_div(d.num_experts, 32)), 32 * scan_warps, scan_smem, s>>>(a, segs);
-    if (a.G > 0) layout_rank_kernel<<<chunk_blocks, 32 * W, chunk_smem, s>>>(a);
+    if (path != EP_LAYOUT_CHUNKED) return EP_ERR_INVALID;
+    const int W = lg.warps;
+    const size_t count_smem = size_t(2 * kActiveSlots + 2 * d.num_experts) * 4;
+    const size_t rank_smem = size_t(kActiveSlots + 2 * d.num_experts + W * d.num_experts) * 4;
+    if (count_smem > 48 * 1024 &&
+        cudaFuncSetAttribute(layout_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(count_smem)) !=
+            cudaSuccess)
+        return EP_ERR_CUDA;
+    if (rank_smem > 48 * 1024 &&
+        cudaFuncSetAttribute(layout_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(rank_smem)) !=
+            cudaSuccess)
+        return EP_ERR_CUDA;
+    layout_count_kernel<<<lg.G, 32 * kMaxWarps, count_smem, s>>>(a);
+    layout_scan_kernel<<<int(ceil_div(d.num_experts, 32)), 32 * kScanWarps, 0, s>>>(a);
+    layout_rank_kernel<<<lg.G, 32 * W, rank_smem, s>>>(a);
     return launch_result();
 }

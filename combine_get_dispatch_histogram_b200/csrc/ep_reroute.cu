@@ -13,9 +13,10 @@
 //
 // Two launches:
 //   1. load   -- each CTA counts its slice of the routing into a shared
-//                histogram with warp-aggregated shared-memory atomics
-//                (__match_any_sync groups equal ids, one leader adds the
-//                group size) and writes it to the workspace;
+//                histogram with warp-aggregated shared-memory atomics (a
+//                match mask from one warp ballot per id bit groups equal ids,
+//                one leader adds the group size) and writes it to the
+//                workspace;
 //   2. expand -- every CTA sums the partial histograms, plans the replicas
 //                (one warp: per step, a lane-parallel argmax of load/replicas
 //                with shuffles) and rewrites its slice of the routing; CTA 0
@@ -43,6 +44,7 @@ struct RerouteArgs {
     int32_t* topk_phys;
     int32_t* status;
     int T, k, E_log, n_extra;
+    int key_bits;  // ceil(log2(E_log))
     int64_t n_pairs;
     int64_t per_block;  // pairs per CTA slice
 };
@@ -59,7 +61,7 @@ __global__ void __launch_bounds__(kRerouteThreads) reroute_load_kernel(RerouteAr
         const int e = p < hi ? __ldg(a.topk_logical + p) : -1;
         const bool ok = e >= 0 && e < a.E_log;
         bad |= (e < -1 || e >= a.E_log);
-        const uint32_t m = __match_any_sync(0xffffffffu, ok ? e : -1);
+        const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, ok));
         if (ok && (threadIdx.x & 31) == __ffs(m) - 1) atomicAdd(hist + e, __popc(m));
     }
     if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
@@ -181,6 +183,8 @@ extern "C" int ep_reroute(int32_t num_ranks, int32_t num_tokens, int32_t num_top
     a.k = num_topk;
     a.E_log = num_logical;
     a.n_extra = num_extra;
+    a.key_bits = 0;
+    while ((1 << a.key_bits) < num_logical) ++a.key_bits;
     a.n_pairs = n_pairs;
     a.per_block = std::max<int64_t>(1, ceil_div(n_pairs, blocks));
 

@@ -1,0 +1,110 @@
+"""Run one C-ABI operation on a named workload and print its CUDA-event time per call.
+
+    python -m combine_get_dispatch_histogram_b200.run_op --op layout --workload prefill --iters 20
+
+Allocates only what the chosen operation needs (``layout`` and ``reroute``
+never touch the receive slab), so single kernels can be timed or profiled on
+full-size routing without holding the 120 GB slab.  ``--graph`` captures the
+calls in a CUDA graph and times graph replays instead of stream launches.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import numpy as np
+import torch
+
+from . import ep, inputs
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--op", choices=["layout", "dispatch", "combine", "reroute", "step"], required=True)
+    ap.add_argument("--workload", default="prefill")
+    ap.add_argument("--iters", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--graph", action="store_true", help="time CUDA-graph replays of the calls")
+    ap.add_argument("--variant", type=int, default=0, help="ep_cfg_t.variant of dispatch / combine")
+    ap.add_argument("--layout-variant", type=int, default=0, help="ep_cfg_t.variant of layout")
+    args = ap.parse_args()
+
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    w = inputs.named(args.workload)
+    need_x = args.op in ("dispatch", "step")
+    inp = inputs.make_inputs(w, tokens=need_x or args.op == "combine")
+    R, T, k, H, E = w.num_ranks, w.num_tokens, w.num_topk, w.hidden, w.num_physical
+    cap = R * T
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    idx = torch.from_numpy(inp.topk_idx).to(dev)
+    act = torch.from_numpy(inp.active).to(dev)
+    cfg = dict(variant=args.variant)
+    stream = torch.cuda.Stream(dev)
+
+    if w.num_extra:
+        rr = ep.ep_reroute(idx, w.num_experts, w.num_extra, status=status)
+        torch.cuda.synchronize()
+        idx_phys = rr["topk_idx_phys"]
+    else:
+        idx_phys = idx
+    lay = ep.ep_layout(idx_phys, act, E, hidden=H, status=status)
+    ws = torch.empty(max(16, ep.ep_layout_workspace_bytes(R, T, k, E, H)), dtype=torch.uint8, device=dev)
+    calls = []
+    if args.op == "reroute":
+        rr_ws = torch.empty(max(16, ep.ep_reroute_workspace_bytes(R, T, k, w.num_experts)), dtype=torch.uint8,
+                            device=dev)
+        out = ep.ep_reroute(idx, w.num_experts, w.num_extra, status=status)
+        calls.append(lambda: ep.ep_reroute(idx, w.num_experts, w.num_extra, workspace=rr_ws, out=out,
+                                           status=status, stream=stream))
+    if args.op in ("layout", "step"):
+        calls.append(lambda: ep.ep_layout(idx_phys, act, E, hidden=H, workspace=ws, out=lay, status=status,
+                                          stream=stream, cfg=dict(variant=args.layout_variant)))
+    if args.op in ("dispatch", "combine", "step"):
+        recv_x = torch.empty((E, cap, H), dtype=torch.bfloat16, device=dev)
+        src_info = torch.empty((E, cap, 2), dtype=torch.int32, device=dev)
+        x = (torch.from_numpy(inp.x.view(np.int16)).to(dev).view(torch.bfloat16) if inp.x is not None else
+             torch.zeros((R, T, H), dtype=torch.bfloat16, device=dev))
+        ep.ep_dispatch(x, idx_phys, lay.pair_row, E, recv_x=recv_x, src_info=src_info, status=status)
+        wts = torch.from_numpy(inp.topk_weights).to(dev)
+        out = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
+        if args.op in ("dispatch", "step"):
+            calls.append(lambda: ep.ep_dispatch(x, idx_phys, lay.pair_row, E, recv_x=recv_x, src_info=src_info,
+                                                status=status, stream=stream, cfg=cfg))
+        if args.op in ("combine", "step"):
+            calls.append(lambda: ep.ep_combine(recv_x, idx_phys, wts, lay.pair_row, act, out=out, status=status,
+                                               stream=stream, cfg=cfg))
+    torch.cuda.synchronize()
+
+    def run_all():
+        for c in calls:
+            c()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            run_all()
+    stream.synchronize()
+    graph = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            run_all()
+        torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.iters):
+            if graph is not None:
+                graph.replay()
+            else:
+                run_all()
+        e1.record(stream)
+    stream.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / args.iters
+    print(json.dumps({"op": args.op, "workload": w.name, "us_per_call": round(us, 2), "graph": args.graph,
+                      "variant": args.variant, "layout_variant": args.layout_variant, "status": int(status.item())}))
+
+
+if __name__ == "__main__":
+    main()

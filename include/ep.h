@@ -113,6 +113,12 @@ typedef struct ep_cfg {
     int32_t variant;      /* dispatch / combine data path: EP_VARIANT_* */
 } ep_cfg_t;
 
+/* Paths of ep_layout (ep_cfg_t.variant; AUTO picks by size). */
+enum {
+    EP_LAYOUT_CHUNKED = 1,    /* three launches over chunks of each rank's tokens; any shape */
+    EP_LAYOUT_SINGLE_CTA = 2  /* one launch, one CTA; R <= 32, E <= 1024, R*T*k <= 32768 */
+};
+
 /* Data paths of ep_dispatch / ep_combine (ep_cfg_t.variant). */
 enum {
     EP_VARIANT_AUTO = 0,      /* the faster path for the shape, as measured on B200 */
@@ -126,7 +132,7 @@ EP_API const char *ep_strerror(int code);
 /* Library version string (static storage). */
 EP_API const char *ep_version(void);
 
-/* Bytes of device workspace ep_layout needs for `d` (0 only if R*T == 0). */
+/* Bytes of device workspace ep_layout needs for `d` (0 for an invalid shape). */
 EP_API size_t ep_layout_workspace_bytes(ep_dims_t d);
 
 /*

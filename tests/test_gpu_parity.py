@@ -330,3 +330,46 @@ def test_vector_variant_rejects_wide_topk():
     with pytest.raises(ep.EPError) as ei:
         ep.ep_dispatch(x, idx, pr, E, cfg=dict(variant=2))
     assert ei.value.code == ep.EP_ERR_UNSUPPORTED
+
+
+LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA = 1, 2
+
+
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA])
+@pytest.mark.parametrize("name", ["tiny", "decode", "sweep_T16_mask5", "sweep_T512", "sweep_T256_mask5"])
+def test_layout_paths_match_oracle(name, path):
+    w = inputs.named(name)
+    inp = inputs.make_inputs(w)
+    ref, packed, want = _oracle_all(inp, w.num_experts)
+    _check_all(run_path(inp, w.num_experts, w.hidden, layout_cfg=dict(variant=path)), ref, packed, want,
+               f"{name} layout path {path}")
+
+
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA])
+@pytest.mark.parametrize("name", ["k1", "T1", "R1", "E_equals_R", "k32", "many_experts"])
+def test_layout_paths_edge_shapes(name, path):
+    c = EDGE[name]
+    if path == LAYOUT_SINGLE_CTA and (c["E"] > 1024 or c["R"] > 32 or c["R"] * c["T"] * c["k"] > 32768):
+        pytest.skip("shape outside the single-CTA path's limits")
+    rng = np.random.default_rng(zlib.crc32(name.encode()) + 7)
+    idx = _uniform_idx(rng, c["R"], c["T"], c["k"], c["E"])
+    idx = np.where(rng.random(idx.shape) < 0.1, -1, idx)
+    act = np.ones(c["R"], np.uint8)
+    if c["R"] > 2:
+        act[1] = 0
+    inp = _custom(c["R"], c["T"], c["k"], c["E"], c["H"], idx, active=act)
+    ref, packed, want = _oracle_all(inp, c["E"])
+    _check_all(run_path(inp, c["E"], c["H"], layout_cfg=dict(variant=path)), ref, packed, want,
+               f"{name} layout path {path}")
+
+
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA])
+def test_layout_paths_overflow_and_bad_ids(path):
+    R, T, k, E, H = 2, 16, 3, 4, 64
+    idx = np.zeros((R, T, k), np.int32)
+    idx[1, 3, 2] = 77
+    inp = _custom(R, T, k, E, H, idx)
+    ref, packed, want = _oracle_all(inp, E)
+    res = run_path(inp, E, H, layout_cfg=dict(variant=path))
+    _check_all(res, ref, packed, want, f"overflow path {path}")
+    assert res["status"] & ep.EP_STATUS_OVERFLOW and res["status"] & ep.EP_STATUS_BAD_EXPERT

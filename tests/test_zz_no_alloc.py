@@ -67,9 +67,9 @@ def test_noalloc_layout_equals_workspace_layout_on_two_calls_in_a_row():
 
 def test_noalloc_layout_rejects_shapes_beyond_its_scratch():
     fn = _bind()
-    # 8 ranks x 65536 tokens x 256 experts needs 16384 chunks x 264 ints = 17.3 MB > 4 MiB
-    d = ep.Dims(8, 65536, 8, 256, 7168)
-    assert ep.ep_layout_workspace_bytes(8, 65536, 8, 256, 7168) > 4 * 1024 * 1024
+    # 64 ranks x 2048 tokens x top-8 over 8192 experts: 128 chunks x 8256 ints = 4.2 MB > 4 MiB
+    d = ep.Dims(64, 2048, 8, 8192, 7168)
+    assert ep.ep_layout_workspace_bytes(64, 2048, 8, 8192, 7168) > 4 * 1024 * 1024
     fake = ctypes.c_void_p(16)
     rc = fn(d, fake, fake, fake, fake, fake, fake, fake, fake, fake, ep.Cfg(0, 0, 0, 0), None)
     assert rc == ep.EP_ERR_UNSUPPORTED
