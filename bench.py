@@ -50,7 +50,17 @@ from combine_get_dispatch_histogram_b200 import inputs  # noqa: E402
 METRIC = "dispatch & combine µs/call and effective HBM GB/s (fraction of ~8 TB/s)"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = {"dispatch_kernel": "ep_dispatch.cu", "combine_kernel": "ep_combine.cu"}
+KERNEL_SOURCES = {"dispatch_kernel": "ep_dispatch.cu", "dispatch_vec_kernel": "ep_dispatch.cu",
+                  "combine_kernel": "ep_combine.cu", "combine_vec_kernel": "ep_combine.cu"}
+
+
+def kernel_names(args, k):
+    """Names of the dispatch / combine kernels the launch configuration selects."""
+    dv = (args.dispatch_cfg or {}).get("variant", 0)
+    cv = (args.combine_cfg or {}).get("variant", 0)
+    dispatch = "dispatch_vec_kernel" if dv == 2 else "dispatch_kernel"
+    combine = "combine_vec_kernel" if (cv == 2 or (cv == 0 and k <= 8)) else "combine_kernel"
+    return dispatch, combine
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -292,7 +302,8 @@ def run_ours(args, rank, world, local_rank):
     dis_gbs = d_bytes / (dis_ms * 1e-3) / 1e9
     com_gbs = c_bytes / (com_ms * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_gbs()
-    dom = ("dispatch_kernel", d_bytes, dis_ms) if dis_ms >= com_ms else ("combine_kernel", c_bytes, com_ms)
+    d_name, c_name = kernel_names(args, k)
+    dom = (d_name, d_bytes, dis_ms) if dis_ms >= com_ms else (c_name, c_bytes, com_ms)
     achieved = dom[1] / (dom[2] * 1e-3) / 1e9
     line = {
         "metric": METRIC,
