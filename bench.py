@@ -185,7 +185,7 @@ def run_ours(args, rank, world, local_rank):
     recv_x = torch.empty((E, cap, H), dtype=torch.bfloat16, device=dev)
     src_info = torch.empty((E, cap, 2), dtype=torch.int32, device=dev)
     out = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
-    lay_ws = torch.empty(max(16, ep.ep_layout_workspace_bytes(R, T, k, E, H)), dtype=torch.uint8, device=dev)
+    lay_ws = torch.zeros(max(16, ep.ep_layout_workspace_bytes(R, T, k, E, H)), dtype=torch.uint8, device=dev)
     rr_ws = rr_out = None
     if reroute:
         rr_ws = torch.empty(max(16, ep.ep_reroute_workspace_bytes(R, T, k, w.num_experts)), dtype=torch.uint8,

@@ -8,8 +8,8 @@
 // among its expert's live pairs in (source rank, token, slot) order: a stable
 // counting sort keyed by expert.
 //
-// Two paths compute the same result (ep_cfg_t.variant selects one; AUTO picks
-// by size).  Both sort with the same two ideas: lanes holding the same expert
+// Three paths compute the same result (ep_cfg_t.variant selects one; AUTO
+// takes the chunked path, measured fastest on B200).  Both sort with the same two ideas: lanes holding the same expert
 // are merged (a match mask built from one warp ballot per expert-id bit) so
 // one leader updates the group's count (a warp-aggregated update), and a
 // pair's row inside a run of 32 consecutive
@@ -57,18 +57,20 @@ constexpr int kScanWarps = 32;
 constexpr int kScanRowsPerWarp = 8;
 constexpr int kSmallThreads = 1024;
 constexpr int kSmallMaxPairs = 32768;
-constexpr int kSmallAutoPairs = 4096;  // AUTO takes the single-CTA path up to here (B200 measurement)
 constexpr int kSmallMaxExperts = 1024;
 constexpr int kSmallMaxRanks = 32;
 constexpr int kMaxWarps = 16;
 constexpr int kBatch = 8;           // 32-pair steps whose loads are issued together
 constexpr int kActiveSlots = 64;    // shared copy of the active mask (EP_MAX_RANKS)
+constexpr int kMaxFlags = 255;      // >= kMaxChunks + EP_MAX_RANKS - 1
+constexpr size_t kSyncBytes = size_t(1 + kMaxFlags) * 8;  // epoch + flags, at offset 0 of the workspace
 
 struct LayoutArgs {
     const int32_t* topk_idx;
     const uint8_t* active;
     int32_t* chunk_hist;  // workspace [G][E]
     int32_t* chunk_tpr;   // workspace [G][R]: tokens of the chunk per destination rank
+    uint64_t* sync;       // workspace prefix: epoch, then one barrier flag per chunk (fused path)
     int32_t* num_tokens_per_expert;
     int32_t* num_tokens_per_rank;
     uint8_t* is_token_in_rank;
@@ -417,6 +419,238 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_rank_kernel(LayoutArgs 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Fused path (EP_LAYOUT_FUSED): the chunked algorithm in ONE cooperative launch
+// (all G CTAs co-resident), with two grid barriers instead of kernel
+// boundaries.  A barrier is one flag per CTA in the workspace: a CTA publishes
+// the barrier's value with a release store and waits (bounded) until every
+// flag holds it.  Values come from an epoch word that CTA 0 advances at the
+// end of every call (also when a barrier gives up), so repeated calls (and
+// replays of a captured graph) never
+// see a stale flag as current.  Epoch and flags sit at fixed offsets at the
+// start of the workspace, which must be zero before its first use and is left
+// consistent by every call (older flags always hold older epochs).  Each warp keeps its part's histogram in shared
+// memory from the count phase to the rank phase.
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// All CTAs of the grid meet here.  False (and EP_STATUS_TIMEOUT) if the wait gave up.
+__device__ bool grid_barrier(uint64_t* flags, int G, uint64_t value, int32_t* status) {
+    __shared__ int passed;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        st_release_u64(flags + blockIdx.x, value);
+    }
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        bool ok = true;
+        const uint64_t t0 = global_timer_ns();
+        for (int b = 0; b < G && ok; b += 32) {
+            const int g = b + lane;
+            for (uint32_t it = 0;; ++it) {
+                bool here = true;
+                if (g < G) {
+                    const uint64_t v = ld_acquire_u64(flags + g);
+                    here = v == value || v == value + 1;  // value + 1: that CTA has already passed
+                }
+                if (__all_sync(0xffffffffu, here)) break;
+                // the give-up decision must be the same on every lane
+                if ((it & 63u) == 63u && __any_sync(0xffffffffu, global_timer_ns() - t0 > kWaitTimeoutNs)) {
+                    ok = false;
+                    break;
+                }
+            }
+            ok = __all_sync(0xffffffffu, ok);
+        }
+        if (lane == 0) passed = ok;
+    }
+    __syncthreads();
+    if (!passed && threadIdx.x == 0) flag_status(status, EP_STATUS_TIMEOUT);
+    return passed != 0;
+}
+
+__global__ void __launch_bounds__(32 * kMaxWarps) layout_fused_kernel(LayoutArgs a) {
+    extern __shared__ int32_t smem[];
+    __shared__ int32_t seg[kMaxWarps][32];
+    __shared__ int32_t col_total[32];
+    const int W = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int32_t* act = smem;
+    int32_t* tpr = smem + kActiveSlots;
+    int32_t* rank_of = smem + 2 * kActiveSlots;
+    int32_t* first = rank_of + a.E;
+    int32_t* whist = first + a.E;  // [W][E]
+    const uint64_t epoch = *reinterpret_cast<volatile uint64_t*>(a.sync);
+    uint64_t* flags = a.sync + 1;
+    const uint64_t bar0 = 2 * (epoch + 1), bar1 = bar0 + 1;
+    load_tables(a, act, rank_of);
+    for (int i = threadIdx.x; i < W * a.E; i += blockDim.x) whist[i] = 0;
+    for (int d = threadIdx.x; d < a.R; d += blockDim.x) tpr[d] = 0;
+    __syncthreads();
+
+    const int g = blockIdx.x;
+    const ChunkGeom cg = chunk_of(a, g);
+    const bool src_ok = act[cg.r] != 0;
+    const int tw = (cg.t1 - cg.t0 + W - 1) / W;
+    const int wt0 = min(cg.t1, cg.t0 + warp * tw), wt1 = min(cg.t1, wt0 + tw);
+    const int64_t pbase = (int64_t(cg.r) * a.T + wt0) * a.k;
+    const int32_t* base = a.topk_idx + pbase;
+    int32_t* rows = a.pair_row + pbase;
+    const int np = (wt1 - wt0) * a.k;
+    int32_t* mine = whist + warp * a.E;
+
+    // ---- phase A: per-warp histograms, token rank sets, chunk histogram
+    bool bad = false;
+    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+        int ev[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            ev[u] = p < np ? __ldg(base + p) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int e = ev[u];
+            bad |= (e < -1 || e >= a.E);
+            const bool live = pair_live(e, a.E, src_ok, rank_of);
+            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
+            if (live && lane == __ffs(m) - 1) mine[e] += __popc(m);
+            __syncwarp();
+        }
+    }
+    for (int t0 = wt0; t0 < wt1; t0 += 32) {
+        const int t = t0 + lane;
+        uint64_t ranks = 0;
+        if (t < wt1) {
+            const int32_t* tb = a.topk_idx + (int64_t(cg.r) * a.T + t) * a.k;
+            for (int j = 0; j < a.k; ++j) {
+                const int e = __ldg(tb + j);
+                if (pair_live(e, a.E, src_ok, rank_of)) ranks |= 1ull << rank_of[e];
+            }
+            uint8_t* itr = a.is_token_in_rank + (int64_t(cg.r) * a.T + t) * a.R;
+            for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
+        }
+        for (int d = 0; d < a.R; ++d) {
+            const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
+            if (lane == 0 && n) atomicAdd(tpr + d, n);
+        }
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        int32_t s = 0;
+        for (int w = 0; w < W; ++w) s += whist[w * a.E + e];
+        a.chunk_hist[int64_t(g) * a.E + e] = s;
+    }
+    for (int d = threadIdx.x; d < a.R; d += blockDim.x) a.chunk_tpr[int64_t(g) * a.R + d] = tpr[d];
+    if (!grid_barrier(flags, a.G, bar0, a.status)) {
+        if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned long long*>(a.sync), epoch + 1);
+        return;
+    }
+
+    // ---- phase B: columns of 32 experts scanned over the chunks (chunk counts -> first rows)
+    const int cols = (a.E + 31) / 32;
+    const int rpw = (a.G + W - 1) / W;
+    for (int col = g; col < cols; col += a.G) {
+        const int e = col * 32 + lane;
+        const bool ok = e < a.E;
+        const int g0 = warp * rpw, g1 = min(a.G, g0 + rpw);
+        int32_t s = 0;
+        if (ok)
+            for (int gg = g0; gg < g1; ++gg) s += a.chunk_hist[int64_t(gg) * a.E + e];
+        seg[warp][lane] = s;
+        __syncthreads();
+        if (warp == 0) {
+            int32_t run = 0;
+            for (int w = 0; w < W; ++w) {
+                const int32_t t = seg[w][lane];
+                seg[w][lane] = run;
+                run += t;
+            }
+            col_total[lane] = run;
+            if (ok) {
+                a.recv_count[e] = run;
+                if (run > a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
+            }
+        }
+        __syncthreads();
+        if (ok) {
+            int32_t run = seg[warp][lane];
+            for (int gg = g0; gg < g1; ++gg) {
+                int32_t* q = a.chunk_hist + int64_t(gg) * a.E + e;
+                const int32_t v = *q;
+                *q = run;
+                run += v;
+            }
+        }
+        __syncthreads();
+        if (ok) {
+            for (int r = warp; r < a.R; r += W) {
+                const int32_t off = a.chunk_hist[int64_t(r) * a.C * a.E + e];
+                const int32_t next = r + 1 < a.R ? a.chunk_hist[int64_t(r + 1) * a.C * a.E + e] : col_total[lane];
+                a.expert_rank_offset[int64_t(e) * a.R + r] = off;
+                a.num_tokens_per_expert[int64_t(r) * a.E + e] = next - off;
+            }
+        }
+        __syncthreads();
+    }
+    const int RR = a.R * a.R;
+    for (int pr = g * W + warp; pr < RR; pr += a.G * W) {
+        const int r = pr / a.R, d = pr - r * a.R;
+        const int32_t* colp = a.chunk_tpr + int64_t(r) * a.C * a.R + d;
+        int32_t t = 0;
+        for (int c = lane; c < a.C; c += 32) t += colp[int64_t(c) * a.R];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+        if (lane == 0) a.num_tokens_per_rank[pr] = t;
+    }
+    if (!grid_barrier(flags, a.G, bar1, a.status)) {
+        if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned long long*>(a.sync), epoch + 1);
+        return;
+    }
+
+    // ---- phase C: per-warp first rows, then rows
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        int32_t run = a.chunk_hist[int64_t(g) * a.E + e];
+        for (int w = 0; w < W; ++w) {
+            const int32_t v = whist[w * a.E + e];
+            whist[w * a.E + e] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    const uint32_t below = lanemask_lt();
+    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+        int ev[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            ev[u] = p < np ? __ldg(base + p) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            if (p0 + u * 32 >= np) break;
+            const int e = ev[u];
+            const bool live = pair_live(e, a.E, src_ok, rank_of);
+            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
+            const int32_t b = live ? mine[e] : 0;
+            __syncwarp();
+            if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
+            __syncwarp();
+            if (p < np) rows[p] = live ? b + __popc(m & below) : -1;
+        }
+    }
+    // every CTA read the epoch before the first barrier; advance it for the next call
+    if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned long long*>(a.sync), epoch + 1);
+}
+
 struct LayoutGeom {
     int C, G, chunk_tokens, warps;
 };
@@ -441,6 +675,32 @@ size_t layout_ws_hist_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
     return round_up16(size_t(lg.G) * d.num_experts * 4);
 }
 
+size_t layout_ws_tpr_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
+    return round_up16(size_t(lg.G) * d.num_ranks * 4);
+}
+
+// Largest grid of the fused kernel that can be co-resident on the current device (0 if none).
+int fused_capacity(int threads, size_t smem) {
+    static int cached[64][kMaxWarps + 1] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    int coop = 0;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) return 0;
+    int& c = cached[dev & 63][threads / 32];
+    if (c == 0) {
+        int per_sm = 0;
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(layout_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+                cudaSuccess)
+            return 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel, threads, smem) !=
+            cudaSuccess)
+            return 0;
+        c = per_sm * sm_count();
+    }
+    return c;
+}
+
 }  // namespace
 }  // namespace ep
 
@@ -449,7 +709,7 @@ using namespace ep;
 extern "C" size_t ep_layout_workspace_bytes(ep_dims_t d) {
     if (check_dims(d) != EP_OK) return 0;
     const LayoutGeom lg = layout_geom(d);
-    return layout_ws_hist_bytes(d, lg) + round_up16(size_t(lg.G) * d.num_ranks * 4);
+    return kSyncBytes + layout_ws_hist_bytes(d, lg) + layout_ws_tpr_bytes(d, lg);
 }
 
 extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* active, void* workspace,
@@ -470,8 +730,10 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     LayoutArgs a;
     a.topk_idx = topk_idx;
     a.active = active;
-    a.chunk_hist = static_cast<int32_t*>(workspace);
-    a.chunk_tpr = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + layout_ws_hist_bytes(d, lg));
+    char* ws = static_cast<char*>(workspace);
+    a.sync = reinterpret_cast<uint64_t*>(ws);
+    a.chunk_hist = reinterpret_cast<int32_t*>(ws + kSyncBytes);
+    a.chunk_tpr = reinterpret_cast<int32_t*>(ws + kSyncBytes + layout_ws_hist_bytes(d, lg));
     a.num_tokens_per_expert = num_tokens_per_expert;
     a.num_tokens_per_rank = num_tokens_per_rank;
     a.is_token_in_rank = is_token_in_rank;
@@ -495,9 +757,32 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     const int64_t pairs = int64_t(d.num_ranks) * d.num_tokens * d.num_topk;
     const bool small_ok = d.num_ranks <= kSmallMaxRanks && d.num_experts <= kSmallMaxExperts &&
                           pairs <= kSmallMaxPairs;
-    // one CTA beats three launches only while its warps' sequential walks stay short
-    const int path = cfg.variant != EP_VARIANT_AUTO ? cfg.variant
-                     : (small_ok && pairs <= kSmallAutoPairs ? EP_LAYOUT_SINGLE_CTA : EP_LAYOUT_CHUNKED);
+    const int W = lg.warps;
+    const size_t fused_smem = size_t(2 * kActiveSlots + 2 * d.num_experts + W * d.num_experts) * 4;
+    const bool fused_ok = lg.G <= kMaxFlags && lg.G <= fused_capacity(32 * W, fused_smem);
+    // AUTO: the chunked path.  On B200 its three launches (about 17 us per call in a graph)
+    // beat the fused one (about 19 us: cooperative launch plus two grid barriers).
+    int path = cfg.variant;
+    if (path == EP_VARIANT_AUTO) path = EP_LAYOUT_CHUNKED;
+    if (path == EP_LAYOUT_FUSED) {
+        if (!fused_ok) return EP_ERR_UNSUPPORTED;
+        void* args[] = {&a};
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(lg.G);
+        lc.blockDim = dim3(32 * W);
+        lc.dynamicSmemBytes = fused_smem;
+        lc.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 1;
+        if (cudaLaunchKernelExC(&lc, reinterpret_cast<const void*>(layout_fused_kernel), args) != cudaSuccess) {
+            cudaGetLastError();
+            return EP_ERR_CUDA;
+        }
+        return launch_result();
+    }
     if (path == EP_LAYOUT_SINGLE_CTA) {
         if (!small_ok) return EP_ERR_UNSUPPORTED;
         const size_t smem = size_t(kActiveSlots + kSmallMaxRanks * kSmallMaxRanks + d.num_experts +
@@ -510,7 +795,6 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
         return launch_result();
     }
     if (path != EP_LAYOUT_CHUNKED) return EP_ERR_INVALID;
-    const int W = lg.warps;
     const size_t count_smem = size_t(2 * kActiveSlots + 2 * d.num_experts) * 4;
     const size_t rank_smem = size_t(kActiveSlots + 2 * d.num_experts + W * d.num_experts) * 4;
     if (count_smem > 48 * 1024 &&

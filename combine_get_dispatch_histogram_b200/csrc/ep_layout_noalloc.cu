@@ -12,11 +12,14 @@
 //
 // The array is reserved on every GPU that loads the library and stays
 // reserved until the process exits.  All calls on one device share it and it
-// keeps whatever the last call left there; nothing in it has to start at zero,
-// because every scratch word the layout kernels read was written earlier in
-// the same call.  Two calls whose kernels overlap on the same GPU (different
-// streams without ordering between them) would overwrite each other's scratch,
-// so such calls must be ordered by the caller.
+// keeps whatever the last call left there.  Like ep_layout's workspace, it
+// must start zeroed (its first words carry the layout's barrier state from
+// call to call): a static device array is zero when the library is loaded, and
+// every call leaves that state ready for the next one, so nothing is cleared
+// per call; the rest is scratch that each call writes before reading.  Two
+// calls whose kernels overlap on the same GPU (different streams without
+// ordering between them) would overwrite each other's scratch, so such calls
+// must be ordered by the caller.
 #include <mutex>
 
 #include <cuda_runtime.h>

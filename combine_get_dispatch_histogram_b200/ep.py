@@ -157,7 +157,11 @@ def ep_layout_workspace_bytes(num_ranks: int, num_tokens: int, num_topk: int, nu
 def ep_layout(topk_idx: torch.Tensor, active: torch.Tensor, num_experts: int, *, hidden: int = 8,
               workspace: Optional[torch.Tensor] = None, out: Optional[DispatchLayout] = None,
               status: Optional[torch.Tensor] = None, cfg=None, stream=None) -> DispatchLayout:
-    """Histogram, prefix sums and stable slab rows (``ep_layout`` of ``include/ep.h``)."""
+    """Histogram, prefix sums and stable slab rows (``ep_layout`` of ``include/ep.h``).
+
+    A caller-provided ``workspace`` (uint8, ``ep_layout_workspace_bytes`` long) must be
+    zero-filled before its first use and reserved for ep_layout calls afterwards.
+    """
     lib = load_library()
     _need(topk_idx, "topk_idx", torch.int32)
     if topk_idx.dim() != 3:
@@ -169,7 +173,7 @@ def ep_layout(topk_idx: torch.Tensor, active: torch.Tensor, num_experts: int, *,
     dims = Dims(R, T, k, E, hidden)
     ws_bytes = int(lib.ep_layout_workspace_bytes(dims))
     if workspace is None:
-        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        workspace = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     _need(workspace, "workspace", torch.uint8, device=dev)
     if out is None:
         out = DispatchLayout(

@@ -49,7 +49,7 @@ def main():
     else:
         idx_phys = idx
     lay = ep.ep_layout(idx_phys, act, E, hidden=H, status=status)
-    ws = torch.empty(max(16, ep.ep_layout_workspace_bytes(R, T, k, E, H)), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(max(16, ep.ep_layout_workspace_bytes(R, T, k, E, H)), dtype=torch.uint8, device=dev)
     calls = []
     if args.op == "reroute":
         rr_ws = torch.empty(max(16, ep.ep_reroute_workspace_bytes(R, T, k, w.num_experts)), dtype=torch.uint8,

@@ -113,10 +113,13 @@ typedef struct ep_cfg {
     int32_t variant;      /* dispatch / combine data path: EP_VARIANT_* */
 } ep_cfg_t;
 
-/* Paths of ep_layout (ep_cfg_t.variant; AUTO picks by size). */
+/* Paths of ep_layout (ep_cfg_t.variant); they compute the same result.  AUTO
+ * takes CHUNKED, the fastest on B200 at every measured shape. */
 enum {
     EP_LAYOUT_CHUNKED = 1,    /* three launches over chunks of each rank's tokens; any shape */
-    EP_LAYOUT_SINGLE_CTA = 2  /* one launch, one CTA; R <= 32, E <= 1024, R*T*k <= 32768 */
+    EP_LAYOUT_SINGLE_CTA = 2, /* one launch, one CTA; R <= 32, E <= 1024, R*T*k <= 32768 */
+    EP_LAYOUT_FUSED = 3       /* one cooperative launch with two grid barriers; needs the
+                                 chunk grid to fit the device (else EP_ERR_UNSUPPORTED) */
 };
 
 /* Data paths of ep_dispatch / ep_combine (ep_cfg_t.variant). */
@@ -142,8 +145,12 @@ EP_API size_t ep_layout_workspace_bytes(ep_dims_t d);
  *   topk_idx              int32 [R,T,k]
  *   active                uint8 [R]       active-rank mask at dispatch time
  *   workspace             >= ep_layout_workspace_bytes(d) bytes, 16-byte aligned,
- *                         scratch owned by the caller; contents on entry are
- *                         ignored, on return are undefined
+ *                         owned by the caller.  Zero-fill it once before its first
+ *                         use (e.g. cudaMemset) and keep it for ep_layout calls
+ *                         only: its first 2 KiB carry barrier state from call to
+ *                         call (cf. Buffer.clean_low_latency_buffer on the NeMo
+ *                         page); the rest is scratch.  Calls sharing a workspace
+ *                         must be ordered on the GPU.
  * out (every element written):
  *   num_tokens_per_expert int32 [R,E]     live pairs of source rank r on expert e
  *   num_tokens_per_rank   int32 [R,R]     tokens of r with >= 1 live pair on rank d
@@ -187,9 +194,10 @@ enum { EP_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024 };
  *     that first call before any stream capture.  EP_ERR_CUDA if the lookup
  *     fails.
  *   - All calls on a device share the one array and it keeps the last call's
- *     contents; nothing in it needs to start at zero.  Calls whose kernels
- *     may overlap on the same GPU race on it: order them (one stream, or
- *     events).
+ *     contents.  It is zero when the library is loaded, as the layout's
+ *     barrier state requires, and every call leaves that state ready for the
+ *     next, so nothing is cleared per call.  Calls whose kernels may overlap
+ *     on the same GPU race on it: order them (one stream, or events).
  */
 EP_API int ep_layout_noalloc(ep_dims_t d, const int32_t *topk_idx, const uint8_t *active,
               int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,

@@ -332,10 +332,10 @@ def test_vector_variant_rejects_wide_topk():
     assert ei.value.code == ep.EP_ERR_UNSUPPORTED
 
 
-LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA = 1, 2
+LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED = 1, 2, 3
 
 
-@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA])
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED])
 @pytest.mark.parametrize("name", ["tiny", "decode", "sweep_T16_mask5", "sweep_T512", "sweep_T256_mask5"])
 def test_layout_paths_match_oracle(name, path):
     w = inputs.named(name)
@@ -345,7 +345,7 @@ def test_layout_paths_match_oracle(name, path):
                f"{name} layout path {path}")
 
 
-@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA])
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED])
 @pytest.mark.parametrize("name", ["k1", "T1", "R1", "E_equals_R", "k32", "many_experts"])
 def test_layout_paths_edge_shapes(name, path):
     c = EDGE[name]
@@ -363,7 +363,7 @@ def test_layout_paths_edge_shapes(name, path):
                f"{name} layout path {path}")
 
 
-@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA])
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED])
 def test_layout_paths_overflow_and_bad_ids(path):
     R, T, k, E, H = 2, 16, 3, 4, 64
     idx = np.zeros((R, T, k), np.int32)
@@ -373,3 +373,37 @@ def test_layout_paths_overflow_and_bad_ids(path):
     res = run_path(inp, E, H, layout_cfg=dict(variant=path))
     _check_all(res, ref, packed, want, f"overflow path {path}")
     assert res["status"] & ep.EP_STATUS_OVERFLOW and res["status"] & ep.EP_STATUS_BAD_EXPERT
+
+
+def test_fused_layout_repeated_calls_and_shape_changes_on_one_workspace():
+    """One workspace, many calls with different shapes and masks: barrier state never goes stale."""
+    ws = torch.zeros(ep.ep_layout_workspace_bytes(8, 4096, 8, 256, 7168) + 4096, dtype=torch.uint8, device=dev())
+    cases = [inputs.prefill(), inputs.decode(), inputs.sweep(16, masked=True), inputs.prefill(), inputs.sweep(512)]
+    for it, w in enumerate(cases * 2):
+        inp = inputs.make_inputs(w, tokens=False)
+        ref = oracle.layout(inp.topk_idx, inp.active, w.num_experts)
+        lay = ep.ep_layout(i32_dev(inp.topk_idx), u8_dev(inp.active), w.num_experts, hidden=w.hidden,
+                           workspace=ws, cfg=dict(variant=LAYOUT_FUSED))
+        torch.cuda.synchronize()
+        check_layout(lay, ref, f"call {it} {w.name}")
+        assert int(lay.status.item()) == 0
+
+
+def test_fused_layout_in_cuda_graph_replays():
+    w = inputs.decode()
+    inp = inputs.make_inputs(w, tokens=False)
+    ref = oracle.layout(inp.topk_idx, inp.active, w.num_experts)
+    idx, act = i32_dev(inp.topk_idx), u8_dev(inp.active)
+    ws = torch.zeros(ep.ep_layout_workspace_bytes(8, 128, 8, 256, 7168), dtype=torch.uint8, device=dev())
+    lay = ep.ep_layout(idx, act, w.num_experts, hidden=w.hidden, workspace=ws, cfg=dict(variant=LAYOUT_FUSED))
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        ep.ep_layout(idx, act, w.num_experts, hidden=w.hidden, workspace=ws, out=lay, stream=stream,
+                     cfg=dict(variant=LAYOUT_FUSED))
+    for _ in range(5):
+        lay.pair_row.fill_(-5)
+        g.replay()
+        torch.cuda.synchronize()
+        check_layout(lay, ref, "graph replay")
