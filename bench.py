@@ -202,26 +202,33 @@ def run_ours(args, rank, world, local_rank):
                             torch.empty((R, T, k), dtype=torch.int32, device=dev), status)
     stream = torch.cuda.Stream(dev)
     n_ev = 4
-    launches_per_step = 5 + (2 if reroute else 0)
+    launches_per_step = 5 + (2 if reroute else 0)  # layout 3, dispatch 1, combine 1 (+ reroute 2)
 
-    def step(events=None):
-        def mark(i):
-            if events is not None:
-                events[i].record(stream)
-        mark(0)
-        idx = idx_log
+    idx_phys = rr_out["topk_idx_phys"] if reroute else idx_log
+
+    def do_layout():
         if reroute:
             ep.ep_reroute(idx_log, w.num_experts, w.num_extra, workspace=rr_ws, out=rr_out, status=status,
                           stream=stream)
-            idx = rr_out["topk_idx_phys"]
-        ep.ep_layout(idx, act, E, hidden=H, workspace=lay_ws, out=lay, status=status, stream=stream)
-        mark(1)
-        ep.ep_dispatch(x, idx, lay.pair_row, E, recv_x=recv_x, src_info=src_info, status=status, stream=stream,
-                       cfg=args.dispatch_cfg)
-        mark(2)
-        ep.ep_combine(recv_x, idx, wts, lay.pair_row, act, out=out, status=status, stream=stream,
+        ep.ep_layout(idx_phys, act, E, hidden=H, workspace=lay_ws, out=lay, status=status, stream=stream)
+
+    def do_dispatch():
+        ep.ep_dispatch(x, idx_phys, lay.pair_row, E, recv_x=recv_x, src_info=src_info, status=status,
+                       stream=stream, cfg=args.dispatch_cfg)
+
+    def do_combine():
+        ep.ep_combine(recv_x, idx_phys, wts, lay.pair_row, act, out=out, status=status, stream=stream,
                       cfg=args.combine_cfg)
-        mark(3)
+
+    parts = (do_layout, do_dispatch, do_combine)
+
+    def step(events=None):
+        for i, part in enumerate(parts):
+            if events is not None:
+                events[i].record(stream)
+            part()
+        if events is not None:
+            events[len(parts)].record(stream)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -238,6 +245,21 @@ def run_ours(args, rank, world, local_rank):
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    graphs = None
+    if args.graph:
+        # one graph for the whole step, one per part (for the per-kernel split)
+        graphs = []
+        for fns in ([step],) + tuple((p,) for p in parts):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for fn in fns:
+                    fn()
+            graphs.append(g)
+        torch.cuda.synchronize(dev)
+        for g in graphs:
+            for _ in range(args.warmup):
+                g.replay()
+        torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier(device_ids=[local_rank])
     torch.cuda.synchronize(dev)
@@ -245,16 +267,32 @@ def run_ours(args, rank, world, local_rank):
     with sampler, torch.cuda.stream(stream):
         t_start.record(stream)
         for i in range(args.steps):
-            step(events[i])
+            if graphs is not None:
+                graphs[0].replay()
+            else:
+                step(events[i])
         t_end.record(stream)
         stream.synchronize()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier(device_ids=[local_rank])
     total_ms = t_start.elapsed_time(t_end)
-    lay_ms = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
-    dis_ms = sum(e[1].elapsed_time(e[2]) for e in events) / args.steps
-    com_ms = sum(e[2].elapsed_time(e[3]) for e in events) / args.steps
+    if graphs is None:
+        lay_ms = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
+        dis_ms = sum(e[1].elapsed_time(e[2]) for e in events) / args.steps
+        com_ms = sum(e[2].elapsed_time(e[3]) for e in events) / args.steps
+    else:
+        part_ms = []
+        for g in graphs[1:]:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(args.steps):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            part_ms.append(e0.elapsed_time(e1) / args.steps)
+        lay_ms, dis_ms, com_ms = part_ms
     if int(status.item()) != 0:
         raise SystemExit(f"device status {int(status.item())} after the timed steps")
 
@@ -337,6 +375,8 @@ def run_ours(args, rank, world, local_rank):
                      "algorithmic_bytes": dom[1]},
         "gpu_launches": launches_per_step * args.steps,
     }
+    if args.graph:
+        line["graph"] = True
     if args.dispatch_cfg or args.combine_cfg:
         line["launch_cfg"] = {"dispatch": args.dispatch_cfg, "combine": args.combine_cfg}
     if e2e is not None:
@@ -454,6 +494,8 @@ def main():
     ap.add_argument("--workload", default="prefill",
                     help="prefill | decode | replica | tiny | sweep_T<n>[_mask5]")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--graph", action="store_true",
+                    help="replay the step as a CUDA graph (per-kernel split from per-kernel graphs)")
     ap.add_argument("--cpu-sample-tokens", type=int, default=1024,
                     help="tokens per rank in the CPU oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
