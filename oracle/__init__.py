@@ -33,7 +33,7 @@ def build(force: bool = False, src: str = _SRC, out: str = _LIB, werror: bool = 
     """Compile the oracle with plain gcc (IEEE float64, no contraction, one thread)."""
     if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
         cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
-               "-fno-fast-math", "-Wall", "-Wextra"] + (["-Werror"] if werror else []) + [src, "-o", out + ".tmp"]
+               "-fno-fast-math", "-Wall", "-Wextra"] + (["-Werror"] if werror else []) + [src, "-o", out + ".tmp", "-lm"]
         subprocess.check_call(cmd)
         os.replace(out + ".tmp", out)
     return out
@@ -61,6 +61,14 @@ def _bind(lib):
     lib.oracle_combine.restype = I
     lib.oracle_reroute.argtypes = [I, I, I, I, I, P, P, P, P, P]
     lib.oracle_reroute.restype = I
+    lib.oracle_e4m3_from_float.argtypes = [ctypes.c_float]
+    lib.oracle_e4m3_from_float.restype = ctypes.c_uint8
+    lib.oracle_fp8_quantize_row.argtypes = [P, I, I, P, P, P]
+    lib.oracle_fp8_quantize_row.restype = None
+    lib.oracle_dispatch_fp8.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P]
+    lib.oracle_dispatch_fp8.restype = I
+    lib.oracle_e4m3_array.argtypes = [P, ctypes.c_int64, P]
+    lib.oracle_e4m3_array.restype = None
     return lib
 
 
@@ -165,3 +173,41 @@ def reroute(topk_logical: np.ndarray, num_logical: int, num_extra: int, lib=None
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     """Exact widening of bf16 bit patterns (uint16) to float64."""
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def e4m3_codes(values: np.ndarray, lib=None) -> np.ndarray:
+    """float32 array -> e4m3 codes (uint8), element by element through the oracle's encoder."""
+    lib = lib or load()
+    v = np.ascontiguousarray(values, dtype=np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib.oracle_e4m3_array(_p(v), v.size, _p(out))
+    return out
+
+
+def fp8_quantize_row(x_row: np.ndarray, pow2: bool, lib=None):
+    """One bf16 row -> (codes [H], scales [H/128] float32, ue8m0 [H/128])."""
+    lib = lib or load()
+    x_row = np.ascontiguousarray(x_row, dtype=np.uint16)
+    H = x_row.shape[0]
+    codes = np.zeros(H, np.uint8)
+    scales = np.zeros(H // 128, np.float32)
+    ue = np.zeros(H // 128, np.uint8)
+    lib.oracle_fp8_quantize_row(_p(x_row), H, int(pow2), _p(codes), _p(scales), _p(ue))
+    return codes, scales, ue
+
+
+def dispatch_fp8(x: np.ndarray, topk_idx: np.ndarray, lay: Layout, pow2: bool, lib=None):
+    """Packed FP8 rows in list order: (codes [L, H], scales [L, H/128], ue8m0 [L, H/128], status)."""
+    lib = lib or load()
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    R, T, H = x.shape
+    k = topk_idx.shape[2]
+    E = lay.recv_count.shape[0]
+    L = int(lay.list_base[-1])
+    codes = np.zeros((L, H), np.uint8)
+    scales = np.zeros((L, H // 128), np.float32)
+    ue = np.zeros((L, H // 128), np.uint8)
+    status = lib.oracle_dispatch_fp8(R, T, k, E, H, int(pow2), _p(x), _p(np.ascontiguousarray(topk_idx, np.int32)),
+                                     _p(lay.pair_row), _p(lay.list_base), _p(codes) if L else None,
+                                     _p(scales) if L else None, _p(ue) if L else None)
+    return codes, scales, ue, int(status)

@@ -38,12 +38,14 @@
  *    i of logical expert e is physical expert phys_base[e] + i; a pair goes to
  *    replica (r*T + t) mod n_rep[e].
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
 #define ORACLE_BAD_EXPERT 1
 #define ORACLE_OVERFLOW   2
+
 
 /* bfloat16 bit pattern -> double.  A bf16 value is the upper half of the
  * float32 with the same sign, exponent and leading 7 mantissa bits. */
@@ -266,4 +268,123 @@ int oracle_reroute(int R, int T, int k, int E_log, int n_extra, const int32_t *t
                 topk_phys[p] = phys_base[e] + (int32_t)(global_token % n_rep[e]);
             }
     return status;
+}
+
+/*
+ * FP8 dispatch ([P1] Buffer.low_latency_dispatch, use_fp8=True): each token row
+ * is cast to float8 e4m3 with one scale per 128 channels; round_scale makes the
+ * scales powers of two; use_ue8m0 stores them as UE8M0 (biased exponent bytes),
+ * four per int32.  The pages name the format but not the arithmetic; the
+ * reading used here (also in the design notes):
+ *   amax  = max |x| over the group (bf16 values, exact in float32)
+ *   scale = 1 if amax == 0, else amax / 448 in float32 (448 = largest e4m3)
+ *   with round_scale: scale = 2^e, e = ceil(log2(amax / 448)) clamped to
+ *                     [-127, 127] (1 when amax == 0); UE8M0 byte = e + 127
+ *   code  = e4m3(x / scale), the division in float32, round to nearest even,
+ *           saturating at +-448.
+ */
+
+/* float32 -> float8 e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits, no infinities, 0x7F/0xFF = NaN): round to nearest, ties to even;
+ * magnitudes at or beyond 448 (and infinities) saturate to 448; NaN -> NaN. */
+uint8_t oracle_e4m3_from_float(float v) {
+    uint32_t bits;
+    memcpy(&bits, &v, sizeof bits);
+    const uint8_t sign = (uint8_t)((bits >> 24) & 0x80u);
+    if (v != v) return (uint8_t)(sign | 0x7Fu);
+    const double a = fabs((double)v);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7Eu);
+    if (a == 0.0) return sign;
+    /* binade exponent of a (a = m * 2^e, 1 <= m < 2); values below 2^-6 are
+     * subnormal and share the quantum 2^-9 of the smallest binade */
+    int e;
+    frexp(a, &e);
+    e -= 1;
+    if (e < -6) e = -6;
+    const double quantum = ldexp(1.0, e - 3);
+    const double val = rint(a / quantum) * quantum; /* rint: nearest, ties to even */
+    if (val == 0.0) return sign;
+    if (val < ldexp(1.0, -6)) return (uint8_t)(sign | (uint8_t)(val / ldexp(1.0, -9)));
+    int ve;
+    const double m = frexp(val, &ve); /* val = m * 2^ve, 0.5 <= m < 1 */
+    const int mant = (int)((m * 2.0 - 1.0) * 8.0);
+    return (uint8_t)(sign | (uint8_t)((ve - 1 + 7) << 3) | (uint8_t)mant);
+}
+
+/* Scale of one 128-channel group (see above); *ue8m0 gets the byte when
+ * pow2 is set. */
+static float group_scale(const uint16_t *x, int n, int pow2, uint8_t *ue8m0) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; i++) {
+        uint32_t u = ((uint32_t)x[i]) << 16;
+        float f;
+        memcpy(&f, &u, sizeof f);
+        if (f < 0) f = -f;
+        if (f > amax) amax = f;
+    }
+    if (!pow2) {
+        if (ue8m0) *ue8m0 = 127;
+        return amax == 0.0f ? 1.0f : amax / 448.0f;
+    }
+    int e = 0;
+    if (amax != 0.0f) {
+        const float s = amax / 448.0f;
+        /* smallest e with 2^e >= s: s = m * 2^f with 0.5 <= m < 1, so e = f unless m == 0.5 */
+        int f;
+        const double m = frexp((double)s, &f);
+        e = m == 0.5 ? f - 1 : f;
+        if (e < -127) e = -127;
+        if (e > 127) e = 127;
+    }
+    if (ue8m0) *ue8m0 = (uint8_t)(e + 127);
+    return (float)ldexp(1.0, e);
+}
+
+/* Quantise one row of H channels: codes[H], scales[H/128] (float32), and the
+ * UE8M0 bytes ue8m0[H/128] when pow2 is set (may be NULL). */
+void oracle_fp8_quantize_row(const uint16_t *x, int H, int pow2, uint8_t *codes, float *scales,
+                             uint8_t *ue8m0) {
+    for (int g = 0; g < H / 128; g++) {
+        const uint16_t *xg = x + g * 128;
+        const float scale = group_scale(xg, 128, pow2, ue8m0 ? ue8m0 + g : NULL);
+        scales[g] = scale;
+        for (int i = 0; i < 128; i++) {
+            uint32_t u = ((uint32_t)xg[i]) << 16;
+            float f;
+            memcpy(&f, &u, sizeof f);
+            const float q = f / scale;
+            codes[g * 128 + i] = oracle_e4m3_from_float(q);
+        }
+    }
+}
+
+/* FP8 dispatch of every live pair, packed in list order like oracle_dispatch:
+ *   codes  [list_base[E], H]      e4m3 codes
+ *   scales [list_base[E], H/128]  float32 scales (row-major here)
+ *   ue8m0  [list_base[E], H/128]  UE8M0 bytes (pow2 only; may be NULL) */
+int oracle_dispatch_fp8(int R, int T, int k, int E, int H, int pow2, const uint16_t *x,
+                        const int32_t *topk_idx, const int32_t *pair_row, const int64_t *list_base,
+                        uint8_t *codes, float *scales, uint8_t *ue8m0) {
+    int status = 0;
+    const int64_t capacity = (int64_t)R * T;
+    const int G = H / 128;
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < T; t++)
+            for (int j = 0; j < k; j++) {
+                int64_t p = ((int64_t)r * T + t) * k + j;
+                int32_t row = pair_row[p];
+                if (row < 0) continue;
+                if (row >= capacity) { status |= ORACLE_OVERFLOW; continue; }
+                int e = topk_idx[p];
+                if (e < 0 || e >= E) continue;
+                const int64_t at = list_base[e] + row;
+                oracle_fp8_quantize_row(x + ((int64_t)r * T + t) * H, H, pow2, codes + at * H, scales + at * G,
+                                        ue8m0 ? ue8m0 + at * G : NULL);
+            }
+    return status;
+}
+
+/* e4m3 encoding of an array (element by element). */
+void oracle_e4m3_array(const float *v, int64_t n, uint8_t *out) {
+    for (int64_t i = 0; i < n; i++) out[i] = oracle_e4m3_from_float(v[i]);
 }

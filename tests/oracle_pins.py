@@ -369,6 +369,53 @@ def pin_reroute_invariants(lib):
             assert np.all((phys[idx == e] >= b[e]) & (phys[idx == e] < b[e + 1]))
 
 
-ALL_PINS = [pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
+# ----------------------------------------------------------------------------- fp8 pins
+
+def pin_fp8_golden(lib):
+    g = _golden("fp8_tiny.json")
+    x = np.zeros(g["H"], np.float32)
+    for i, v in g["nonzero"]:
+        x[i] = v
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    codes, scales, _ = oracle.fp8_quantize_row(bits, False, lib=lib)
+    assert all(codes[i] == c for i, c in g["plain"]["codes"]) and np.count_nonzero(codes) == 6
+    assert scales[0] == g["plain"]["scale0"]
+    codes, scales, ue = oracle.fp8_quantize_row(bits, True, lib=lib)
+    assert all(codes[i] == c for i, c in g["pow2"]["codes"])
+    assert scales.tolist() == g["pow2"]["scales"] and ue.tolist() == g["pow2"]["ue8m0"]
+
+
+def pin_e4m3_against_torch(lib):
+    import torch
+
+    rng = np.random.default_rng(21)
+    v = (rng.standard_normal(400_000) * rng.choice([1e-3, 1.0, 50.0], 400_000)).astype(np.float32)
+    v = v[np.abs(v) < 464]
+    want = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_codes(v, lib=lib), want), "e4m3 encoder differs from torch"
+    # saturating cast: finite overflow and infinities clamp to +-448 (0x7E / 0xFE), NaN stays NaN
+    special = np.array([464.0, 500.0, 1e30, np.inf, -600.0, -np.inf, np.nan], np.float32)
+    assert oracle.e4m3_codes(special, lib=lib).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F]
+
+
+def pin_fp8_dequant_error(lib):
+    import torch
+
+    rng = np.random.default_rng(22)
+    for pow2 in (False, True):
+        bits = inputs.bf16_tokens(rng, 1, 512)[0]
+        xv = oracle.bf16_bits_to_f64(bits).reshape(-1, 128)
+        codes, scales, ue = oracle.fp8_quantize_row(bits, pow2, lib=lib)
+        deq = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy().reshape(-1, 128)
+        deq = deq * scales.astype(np.float64)[:, None]
+        assert np.all(np.abs(deq - xv) <= np.abs(xv) * 2.0 ** -4 + scales[:, None] * 2.0 ** -10)
+        amax = np.abs(xv).max(axis=1)
+        assert np.all(scales >= (amax / 448) * (1 - 1e-6))
+        if pow2:
+            assert np.all(scales / 2 < amax / 448)
+            assert np.array_equal(ue.astype(np.int64) - 127, np.log2(scales).astype(np.int64))
+
+
+ALL_PINS = [pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
             pin_dispatch_golden, pin_dispatch_bijection, pin_combine_golden,
             pin_combine_special_cases, pin_combine_mask, pin_reroute_golden, pin_reroute_invariants]

@@ -41,6 +41,14 @@ MUTANTS = {
     "combine_wrong_row_base": ("const uint16_t *yr = y + (y_row_base[e] + row) * H;",
                                "const uint16_t *yr = y + (y_row_base[e] + row) * H + (row > 0);"),
     "combine_negative_sign": ("o[h] += w * bf16_to_double(yr[h]);", "o[h] -= w * bf16_to_double(yr[h]);"),
+    # fp8 cast
+    "fp8_wrong_max": ("return amax == 0.0f ? 1.0f : amax / 448.0f;", "return amax == 0.0f ? 1.0f : amax / 240.0f;"),
+    "e4m3_truncates": ("const double val = rint(a / quantum) * quantum;",
+                       "const double val = floor(a / quantum) * quantum;"),
+    "e4m3_exponent_bias": ("((ve - 1 + 7) << 3)", "((ve - 1 + 8) << 3)"),
+    "ue8m0_bias": ("if (ue8m0) *ue8m0 = (uint8_t)(e + 127);", "if (ue8m0) *ue8m0 = (uint8_t)(e + 128);"),
+    "pow2_floor": ("e = m == 0.5 ? f - 1 : f;", "e = f - 1;"),
+    "fp8_no_saturation": ("if (a >= 448.0) return (uint8_t)(sign | 0x7Eu);", "if (a >= 480.0) return (uint8_t)(sign | 0x7Fu);"),
     # reroute
     "reroute_tie_highest": ("if (lhs > rhs) best = e;", "if (lhs >= rhs) best = e;"),
     "reroute_local_token": ("topk_phys[p] = phys_base[e] + (int32_t)(global_token % n_rep[e]);",
