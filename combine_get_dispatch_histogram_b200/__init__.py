@@ -9,6 +9,7 @@ from .ep import (  # noqa: F401
     EPError,
     ep_combine,
     ep_dispatch,
+    ep_dispatch_fp8,
     ep_layout,
     ep_layout_workspace_bytes,
     ep_reroute,

@@ -31,6 +31,8 @@
 #include <algorithm>
 #include <cstdint>
 
+#include <cuda_fp8.h>
+
 #include "ep.h"
 #include "ep_device.cuh"
 #include "ep_host.h"
@@ -255,10 +257,258 @@ int launch_dispatch_vec(const DispatchArgs& a, const ep_cfg_t& cfg, int sms, cud
     return launch_result();
 }
 
+// ---------------------------------------------------------------------------
+// FP8 dispatch (ep_dispatch_fp8): the vector path with a per-128-channel e4m3
+// cast.  A unit is a token x 512 channels (four scale groups); each lane holds
+// 2 x 8 channels, so a half-warp holds exactly one group and its amax is a
+// shuffle-max over 16 lanes.  The cast is computed once per token row and the
+// codes (8 bytes per lane and half) and scales are stored to every live row.
+struct DispatchFp8Args {
+    const uint8_t* x;
+    const int32_t* topk_idx;
+    const int32_t* pair_row;
+    uint8_t* codes;
+    uint8_t* scales;       // column-major [E][words][cap]
+    uint32_t* tok_scales;  // workspace [n_tok][words]: fp32 scales, or UE8M0 words
+    const int32_t* recv_count;
+    int32_t* src_info;
+    int32_t* status;
+    int T, k, E, H, groups;
+    int words;             // scale words per row: H/128 (fp32) or H/512 (UE8M0)
+    int64_t cap;
+    int64_t n_tok;
+};
+
+template <int FMT>
+__device__ __forceinline__ float fp8_group_scale(float amax, uint32_t* ue8m0) {
+    if (FMT == EP_FP8_SCALE_F32) {
+        *ue8m0 = 127u;
+        return amax == 0.0f ? 1.0f : amax / 448.0f;
+    }
+    int e = 0;
+    if (amax != 0.0f) {
+        int f;
+        const float m = frexpf(amax / 448.0f, &f);  // amax/448 = m * 2^f, 0.5 <= m < 1
+        e = m == 0.5f ? f - 1 : f;                   // smallest e with 2^e >= amax/448
+        e = max(-127, min(127, e));
+    }
+    *ue8m0 = uint32_t(e + 127);
+    return ldexpf(1.0f, e);
+}
+
+// codes of x / scale.  A power-of-two scale divides exactly as a multiplication by
+// its reciprocal (also a power of two, exact), so those formats multiply.
+template <int FMT>
+__device__ __forceinline__ uint2 fp8_cast8(const float* f, float scale) {
+    float q[8];
+    if (FMT == EP_FP8_SCALE_F32) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = f[i] / scale;
+    } else {
+        const float inv = 1.0f / scale;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = f[i] * inv;
+    }
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const __nv_fp8x2_storage_t lo =
+            __nv_cvt_float2_to_fp8x2(make_float2(q[4 * h], q[4 * h + 1]), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi =
+            __nv_cvt_float2_to_fp8x2(make_float2(q[4 * h + 2], q[4 * h + 3]), __NV_SATFINITE, __NV_E4M3);
+        w[h] = uint32_t(lo) | (uint32_t(hi) << 16);
+    }
+    return make_uint2(w[0], w[1]);
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(256) dispatch_fp8_kernel(DispatchFp8Args a) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+    const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int nvec = a.H >> 3;
+    constexpr int kPieceVec = 64;  // 512 channels
+    const int np = (nvec + kPieceVec - 1) / kPieceVec;
+    const int64_t n_units = a.n_tok * np;
+    const int64_t q = n_units / warps, rem = n_units % warps;
+    const int64_t u0 = gw * q + (gw < rem ? gw : rem);
+    const int64_t u1 = u0 + q + (gw < rem ? 1 : 0);
+
+    int64_t cur_tok = -1;
+    uint32_t mask = 0;
+    int my_e = -1, my_row = -1;
+    for (int64_t u = u0; u < u1; ++u) {
+        const int64_t tok = u / np;
+        const int pc = int(u - tok * np);
+        if (tok != cur_tok) {
+            cur_tok = tok;
+            int e = -1, row = -1;
+            if (lane < a.k) {
+                const int64_t p = tok * a.k + lane;
+                e = __ldg(a.topk_idx + p);
+                row = __ldg(a.pair_row + p);
+            }
+            const bool valid_row = row >= 0 && row < a.cap;
+            const bool live = valid_row && e >= 0 && e < a.E;
+            if (lane < a.k && pc == 0) {
+                if (row >= a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
+                if (valid_row && !live) flag_status(a.status, EP_STATUS_BAD_EXPERT);
+                if (live) {
+                    const int src_rank = int(tok / a.T);
+                    reinterpret_cast<int2*>(a.src_info)[int64_t(e) * a.cap + row] =
+                        make_int2(src_rank, int(tok - int64_t(src_rank) * a.T));
+                }
+            }
+            mask = __ballot_sync(0xffffffffu, live);
+            my_e = live ? e : -1;
+            my_row = row;
+        }
+        if (mask == 0u) continue;
+        const uint8_t* src = a.x + tok * int64_t(a.H) * 2;
+        uint2 code[2];
+        uint32_t ue[2] = {127u, 127u};
+        float scale[2] = {1.f, 1.f};
+        bool valid[2];
+#pragma unroll
+        for (int uu = 0; uu < 2; ++uu) {
+            const int v = pc * kPieceVec + uu * 32 + lane;
+            valid[uu] = v < nvec;  // a half-warp is one whole 128-channel group: valid for all 16 or none
+            float f[8];
+            float amax = 0.f;
+            if (valid[uu]) {
+                const uint4 raw = ld_stream_v4(src + int64_t(v) * 16);
+                const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    f[2 * i] = __uint_as_float(wds[i] << 16);
+                    f[2 * i + 1] = __uint_as_float(wds[i] & 0xffff0000u);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+            }
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            scale[uu] = fp8_group_scale<FMT>(amax, &ue[uu]);
+            if (valid[uu]) code[uu] = fp8_cast8<FMT>(f, scale[uu]);
+        }
+        // UE8M0: bytes of the piece's four groups (uu=0: lanes 0, 16; uu=1: lanes 0, 16) into one word
+        uint32_t ue_word = 0;
+        if (FMT == EP_FP8_SCALE_UE8M0) {
+            const uint32_t b1 = __shfl_sync(0xffffffffu, ue[0], 16);
+            const uint32_t b3 = __shfl_sync(0xffffffffu, ue[1], 16);
+            ue_word = ue[0] | (b1 << 8) | (ue[1] << 16) | (b3 << 24);
+        }
+        // the token's scales, once, row-major in the workspace
+        uint32_t* ts = a.tok_scales + tok * a.words;
+        if (FMT == EP_FP8_SCALE_UE8M0) {
+            if (lane == 0) ts[pc] = ue_word;
+        } else {
+#pragma unroll
+            for (int uu = 0; uu < 2; ++uu) {
+                const int v = pc * kPieceVec + uu * 32 + lane;
+                if (valid[uu] && (lane & 15) == 0) ts[v >> 4] = __float_as_uint(scale[uu]);  // 16 vectors per group
+            }
+        }
+        for (int j = 0; j < a.k; ++j) {
+            if (!((mask >> j) & 1u)) continue;
+            const int e = __shfl_sync(0xffffffffu, my_e, j);
+            const int row = __shfl_sync(0xffffffffu, my_row, j);
+            uint8_t* dst = a.codes + (int64_t(e) * a.cap + row) * a.H;
+#pragma unroll
+            for (int uu = 0; uu < 2; ++uu) {
+                const int v = pc * kPieceVec + uu * 32 + lane;
+                if (valid[uu]) *reinterpret_cast<uint2*>(dst + int64_t(v) * 8) = code[uu];
+            }
+        }
+    }
+}
+
+// Column-major scales: block (x, e) covers slab rows [x*256, x*256 + 256) of expert e;
+// a thread owns one valid row, finds its token in src_info and copies that
+// token's scale words, so for each word the block's stores are contiguous.
+__global__ void __launch_bounds__(256) fp8_scale_writer_kernel(DispatchFp8Args a) {
+    const int e = blockIdx.y;
+    const int64_t n = a.recv_count[e] < a.cap ? int64_t(a.recv_count[e]) : a.cap;
+    const int64_t row = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (int64_t(blockIdx.x) * blockDim.x >= n) return;
+    const bool ok = row < n;
+    const uint32_t* ts = nullptr;
+    bool ok_src = false;
+    if (ok) {
+        const int2 src = reinterpret_cast<const int2*>(a.src_info)[int64_t(e) * a.cap + row];
+        const int64_t tok = int64_t(src.x) * a.T + src.y;
+        // a recv_count that does not belong to this dispatch could point at a stale row
+        ok_src = src.y >= 0 && src.y < a.T && tok >= 0 && tok < a.n_tok;
+        if (ok_src) ts = a.tok_scales + tok * a.words;
+        else flag_status(a.status, EP_STATUS_BAD_EXPERT);
+    }
+    uint32_t* out = reinterpret_cast<uint32_t*>(a.scales) + int64_t(e) * a.words * a.cap + row;
+    for (int wd = 0; wd < a.words; ++wd)
+        if (ok_src) out[int64_t(wd) * a.cap] = ts[wd];
+}
+
 }  // namespace
 }  // namespace ep
 
 using namespace ep;
+
+extern "C" size_t ep_dispatch_fp8_workspace_bytes(ep_dims_t d, int32_t scale_format) {
+    if (check_dims(d) != EP_OK || d.hidden % 128 != 0) return 0;
+    const int words = scale_format == EP_FP8_SCALE_UE8M0 ? d.hidden / 512 : d.hidden / 128;
+    return round_up16(size_t(d.num_ranks) * d.num_tokens * words * 4);
+}
+
+extern "C" int ep_dispatch_fp8(ep_dims_t d, const uint16_t* x, const int32_t* topk_idx, const int32_t* pair_row,
+                               const int32_t* recv_count, int32_t scale_format, void* workspace,
+                               size_t workspace_bytes, uint8_t* recv_x, void* recv_scales, int32_t* src_info,
+                               int32_t* status, ep_cfg_t cfg, void* stream) {
+    int rc = check_dims(d);
+    if (rc != EP_OK) return rc;
+    if (scale_format != EP_FP8_SCALE_F32 && scale_format != EP_FP8_SCALE_POW2 && scale_format != EP_FP8_SCALE_UE8M0)
+        return EP_ERR_INVALID;
+    if (d.hidden % 128 != 0 || (scale_format == EP_FP8_SCALE_UE8M0 && d.hidden % 512 != 0)) return EP_ERR_INVALID;
+    const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
+    if (RT == 0) return EP_OK;
+    if (!x || !topk_idx || !pair_row || !recv_count || !recv_x || !recv_scales || !src_info) return EP_ERR_INVALID;
+    const size_t need = ep_dispatch_fp8_workspace_bytes(d, scale_format);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return EP_ERR_INVALID;
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(recv_x) & 7u) || (reinterpret_cast<uintptr_t>(recv_scales) & 3u) ||
+        (reinterpret_cast<uintptr_t>(src_info) & 7u))
+        return EP_ERR_INVALID;
+    DispatchFp8Args a;
+    a.x = reinterpret_cast<const uint8_t*>(x);
+    a.topk_idx = topk_idx;
+    a.pair_row = pair_row;
+    a.codes = recv_x;
+    a.scales = static_cast<uint8_t*>(recv_scales);
+    a.src_info = src_info;
+    a.status = status;
+    a.T = d.num_tokens;
+    a.k = d.num_topk;
+    a.E = d.num_experts;
+    a.H = d.hidden;
+    a.groups = d.hidden / 128;
+    a.words = scale_format == EP_FP8_SCALE_UE8M0 ? d.hidden / 512 : d.hidden / 128;
+    a.tok_scales = static_cast<uint32_t*>(workspace);
+    a.recv_count = recv_count;
+    a.cap = RT;
+    a.n_tok = RT;
+    const int sms = sm_count();
+    if (sms <= 0) return EP_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t units = RT * ceil_div(d.hidden / 8, 64);
+    int64_t grid = int64_t(sms) * 4;
+    if (cfg.max_ctas > 0) grid = cfg.max_ctas;
+    grid = std::max<int64_t>(1, std::min<int64_t>(grid, ceil_div(units, 8)));
+    switch (scale_format) {
+        case EP_FP8_SCALE_F32: dispatch_fp8_kernel<EP_FP8_SCALE_F32><<<unsigned(grid), 256, 0, st>>>(a); break;
+        case EP_FP8_SCALE_POW2: dispatch_fp8_kernel<EP_FP8_SCALE_POW2><<<unsigned(grid), 256, 0, st>>>(a); break;
+        default: dispatch_fp8_kernel<EP_FP8_SCALE_UE8M0><<<unsigned(grid), 256, 0, st>>>(a); break;
+    }
+    if (ceil_div(RT, 256) > 65535 * 256LL || d.num_experts > 65535) return EP_ERR_UNSUPPORTED;
+    fp8_scale_writer_kernel<<<dim3(unsigned(ceil_div(RT, 256)), unsigned(d.num_experts)), 256, 0, st>>>(a);
+    return launch_result();
+}
 
 extern "C" int ep_dispatch(ep_dims_t d, const uint16_t* x, const int32_t* topk_idx, const int32_t* pair_row,
                            uint16_t* recv_x, int32_t* src_info, int32_t* status, ep_cfg_t cfg, void* stream) {

@@ -30,6 +30,9 @@ EP_STATUS_BAD_EXPERT = 1
 EP_STATUS_OVERFLOW = 2
 EP_STATUS_TIMEOUT = 8
 EP_VARIANT_AUTO = 0
+EP_FP8_SCALE_F32 = 0
+EP_FP8_SCALE_POW2 = 1
+EP_FP8_SCALE_UE8M0 = 2
 EP_VARIANT_BULK = 1
 EP_VARIANT_VECTOR = 2
 
@@ -74,6 +77,10 @@ def load_library(path: str = LIB_PATH):
     lib.ep_dispatch.restype = ctypes.c_int
     lib.ep_combine.argtypes = [Dims, P, P, P, P, P, P, P, Cfg, P]
     lib.ep_combine.restype = ctypes.c_int
+    lib.ep_dispatch_fp8.argtypes = [Dims, P, P, P, P, I32, P, SZ, P, P, P, P, Cfg, P]
+    lib.ep_dispatch_fp8.restype = ctypes.c_int
+    lib.ep_dispatch_fp8_workspace_bytes.argtypes = [Dims, I32]
+    lib.ep_dispatch_fp8_workspace_bytes.restype = SZ
     lib.ep_reroute_workspace_bytes.argtypes = [I32, I32, I32, I32]
     lib.ep_reroute_workspace_bytes.restype = SZ
     lib.ep_reroute.argtypes = [I32, I32, I32, I32, I32, P, P, SZ, P, P, P, P, P, Cfg, P]
@@ -231,6 +238,65 @@ def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, pair_row: torch.Tensor,
                              _ptr(src_info), _ptr(status), _cfg(cfg), _stream(dev, stream))
     _check("ep_dispatch", rc)
     return recv_x, src_info, status
+
+
+def ep_dispatch_fp8(x: torch.Tensor, topk_idx: torch.Tensor, pair_row: torch.Tensor, recv_count: torch.Tensor,
+                    num_experts: int, scale_format: int = EP_FP8_SCALE_F32, *,
+                    workspace: Optional[torch.Tensor] = None, recv_x: Optional[torch.Tensor] = None,
+                    recv_scales: Optional[torch.Tensor] = None, src_info: Optional[torch.Tensor] = None,
+                    status: Optional[torch.Tensor] = None, cfg=None, stream=None):
+    """``ep_dispatch`` with an e4m3 payload and per-128-channel scales (``ep_dispatch_fp8``).
+
+    Returns ``(recv_x, recv_scales, src_info, status)``: ``recv_x`` is float8_e4m3fn
+    ``[E, R*T, H]``; ``recv_scales`` is the ``[E, R*T, H/128]`` float32 tensor (``[E, R*T, H/512]``
+    int32 for UE8M0) as a view whose last two dimensions are column-major, like the page's
+    low-latency dispatch.  Pass ``recv_scales`` as that storage, shaped ``[E, groups, R*T]``.
+    """
+    lib = load_library()
+    _need(x, "x", torch.bfloat16)
+    if x.dim() != 3:
+        raise ValueError("x must be [R, T, H]")
+    R, T, H = x.shape
+    dev = x.device
+    _need(topk_idx, "topk_idx", torch.int32, device=dev)
+    if topk_idx.dim() != 3 or tuple(topk_idx.shape[:2]) != (R, T):
+        raise ValueError("topk_idx must be [R, T, k]")
+    k = topk_idx.shape[2]
+    _need(pair_row, "pair_row", torch.int32, (R, T, k), dev)
+    E = int(num_experts)
+    _need(recv_count, "recv_count", torch.int32, (E,), dev)
+    cap = R * T
+    ue8m0 = scale_format == EP_FP8_SCALE_UE8M0
+    ws_bytes = int(lib.ep_dispatch_fp8_workspace_bytes(Dims(R, T, k, E, H), int(scale_format)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, device=dev)
+    groups = H // 512 if ue8m0 else H // 128
+    sdt = torch.int32 if ue8m0 else torch.float32
+    if recv_x is None:
+        recv_x = torch.empty((E, cap, H), dtype=torch.uint8, device=dev)
+    if recv_x.dtype == torch.float8_e4m3fn:
+        recv_x = recv_x.view(torch.uint8)
+    if recv_scales is None:
+        recv_scales = torch.empty((E, groups, cap), dtype=sdt, device=dev)
+    if src_info is None:
+        src_info = torch.empty((E, cap, 2), dtype=torch.int32, device=dev)
+    _need(recv_x, "recv_x", torch.uint8, (E, cap, H), dev)
+    _need(recv_scales, "recv_scales", sdt, (E, groups, cap), dev)
+    _need(src_info, "src_info", torch.int32, (E, cap, 2), dev)
+    status = _status(dev, status)
+    with torch.cuda.device(dev):
+        rc = lib.ep_dispatch_fp8(Dims(R, T, k, E, H), _ptr(x), _ptr(topk_idx), _ptr(pair_row), _ptr(recv_count),
+                                 int(scale_format), _ptr(workspace), workspace.numel(), _ptr(recv_x),
+                                 _ptr(recv_scales), _ptr(src_info), _ptr(status), _cfg(cfg), _stream(dev, stream))
+    _check("ep_dispatch_fp8", rc)
+    return recv_x.view(torch.float8_e4m3fn), recv_scales.transpose(1, 2), src_info, status
+
+
+def ep_dispatch_fp8_workspace_bytes(num_ranks: int, num_tokens: int, num_topk: int, num_experts: int, hidden: int,
+                                    scale_format: int = EP_FP8_SCALE_F32) -> int:
+    return int(load_library().ep_dispatch_fp8_workspace_bytes(Dims(num_ranks, num_tokens, num_topk, num_experts,
+                                                                   hidden), int(scale_format)))
 
 
 def ep_combine(y: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor, pair_row: torch.Tensor,

@@ -20,7 +20,9 @@ from . import ep, inputs
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("--op", choices=["layout", "dispatch", "combine", "reroute", "step"], required=True)
+    ap.add_argument("--op", choices=["layout", "dispatch", "dispatch_fp8", "combine", "reroute", "step"],
+                    required=True)
+    ap.add_argument("--scale-format", type=int, default=0, help="dispatch_fp8: 0 fp32, 1 power of two, 2 UE8M0")
     ap.add_argument("--workload", default="prefill")
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
@@ -32,7 +34,7 @@ def main():
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
     w = inputs.named(args.workload)
-    need_x = args.op in ("dispatch", "step")
+    need_x = args.op in ("dispatch", "dispatch_fp8", "step")
     inp = inputs.make_inputs(w, tokens=need_x or args.op == "combine")
     R, T, k, H, E = w.num_ranks, w.num_tokens, w.num_topk, w.hidden, w.num_physical
     cap = R * T
@@ -60,6 +62,18 @@ def main():
     if args.op in ("layout", "step"):
         calls.append(lambda: ep.ep_layout(idx_phys, act, E, hidden=H, workspace=ws, out=lay, status=status,
                                           stream=stream, cfg=dict(variant=args.layout_variant)))
+    if args.op == "dispatch_fp8":
+        x = torch.from_numpy(inp.x.view(np.int16)).to(dev).view(torch.bfloat16)
+        ue = args.scale_format == ep.EP_FP8_SCALE_UE8M0
+        codes = torch.empty((E, cap, H), dtype=torch.uint8, device=dev)
+        scales = torch.empty((E, H // (512 if ue else 128), cap), dtype=torch.int32 if ue else torch.float32,
+                             device=dev)
+        src_info = torch.empty((E, cap, 2), dtype=torch.int32, device=dev)
+        fp8_ws = torch.empty(max(16, ep.ep_dispatch_fp8_workspace_bytes(R, T, k, E, H, args.scale_format)),
+                             dtype=torch.uint8, device=dev)
+        calls.append(lambda: ep.ep_dispatch_fp8(x, idx_phys, lay.pair_row, lay.recv_count, E, args.scale_format,
+                                                workspace=fp8_ws, recv_x=codes, recv_scales=scales,
+                                                src_info=src_info, status=status, stream=stream, cfg=cfg))
     if args.op in ("dispatch", "combine", "step"):
         recv_x = torch.empty((E, cap, H), dtype=torch.bfloat16, device=dev)
         src_info = torch.empty((E, cap, 2), dtype=torch.int32, device=dev)
@@ -102,7 +116,17 @@ def main():
         e1.record(stream)
     stream.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / args.iters
+    live = int(lay.recv_count.sum().item())
+    sent = int(lay.is_token_in_rank.view(R * T, R).amax(dim=1).sum().item())
+    per_pair = {"dispatch": 2 * H, "combine": 2 * H,
+                "dispatch_fp8": H + (H // 512 if args.scale_format == ep.EP_FP8_SCALE_UE8M0 else H // 32)}
+    algo = None
+    if args.op in ("dispatch", "dispatch_fp8"):
+        algo = 2 * H * sent + per_pair[args.op] * live
+    elif args.op == "combine":
+        algo = 2 * H * (live + R * T)
     print(json.dumps({"op": args.op, "workload": w.name, "us_per_call": round(us, 2), "graph": args.graph,
+                      "algorithmic_bytes": algo, "gbs": round(algo / us / 1e3, 1) if algo else None,
                       "variant": args.variant, "layout_variant": args.layout_variant, "status": int(status.item())}))
 
 

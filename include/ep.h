@@ -226,6 +226,47 @@ EP_API int ep_dispatch(ep_dims_t d, const uint16_t *x, const int32_t *topk_idx,
                 const int32_t *pair_row, uint16_t *recv_x, int32_t *src_info,
                 int32_t *status, ep_cfg_t cfg, void *stream);
 
+/* Scale formats of ep_dispatch_fp8 (NeMo page, Buffer.low_latency_dispatch:
+ * use_fp8, round_scale, use_ue8m0). */
+enum {
+    EP_FP8_SCALE_F32 = 0,   /* float scale per 128 channels = amax / 448 (1 if amax == 0) */
+    EP_FP8_SCALE_POW2 = 1,  /* float scale 2^ceil(log2(amax / 448)), exponent clamped to [-127, 127] */
+    EP_FP8_SCALE_UE8M0 = 2  /* the POW2 scales as UE8M0 bytes (exponent + 127), four per int32 */
+};
+
+/*
+ * ep_dispatch_fp8 -- ep_dispatch with the payload cast to float8 e4m3.
+ *
+ * Buffer.low_latency_dispatch with use_fp8=True on the NeMo page: every live
+ * pair's token row arrives as e4m3 codes with one scale per 128 channels.
+ * Per group of 128 channels of a token row: amax = max |x|; scale per
+ * scale_format (above); code = e4m3(x / scale), the division in float32 and
+ * the cast rounding to nearest even, saturating at +-448.
+ * in:
+ *   x, topk_idx, pair_row   as for ep_dispatch; H % 128 == 0 (H % 512 == 0 for UE8M0)
+ *   recv_count   int32 [E]  from ep_layout (which slab rows are valid)
+ *   workspace    >= ep_dispatch_fp8_workspace_bytes(d, scale_format) bytes, 16-byte
+ *                aligned; scratch (contents ignored on entry, undefined on return)
+ * out:
+ *   recv_x       uint8 [E,CAP,H]   e4m3 codes of every written row (8-byte aligned)
+ *   recv_scales  EP_FP8_SCALE_F32 / _POW2: float [E, H/128, CAP];
+ *                EP_FP8_SCALE_UE8M0: int32 [E, H/512, CAP], byte j of word w is the
+ *                UE8M0 scale of channel group 4w+j.  This is the [E, CAP, groups]
+ *                tensor of the page stored column-major in its last two dimensions.
+ *   src_info     as for ep_dispatch
+ * Rows not written keep their contents.  Two launches: the cast (codes to every
+ * live row, each token's scales once to the workspace), then a scale writer that
+ * fills the column-major scale tensor with coalesced stores.
+ */
+EP_API int ep_dispatch_fp8(ep_dims_t d, const uint16_t *x, const int32_t *topk_idx,
+                           const int32_t *pair_row, const int32_t *recv_count,
+                           int32_t scale_format, void *workspace, size_t workspace_bytes,
+                           uint8_t *recv_x, void *recv_scales, int32_t *src_info,
+                           int32_t *status, ep_cfg_t cfg, void *stream);
+
+/* Bytes of scratch ep_dispatch_fp8 needs: each token's scales, row-major. */
+EP_API size_t ep_dispatch_fp8_workspace_bytes(ep_dims_t d, int32_t scale_format);
+
 /*
  * ep_combine -- top-k weighted gather-reduce back to the source ranks.
  *

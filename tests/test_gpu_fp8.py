@@ -1,0 +1,109 @@
+"""GPU parity of the FP8 dispatch (e4m3 codes, per-128-channel scales) against the CPU oracle.
+
+Codes and scales are integer decisions taken in float32 on both sides (same division, same
+round-to-nearest-even saturating cast), so they must be bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_get_dispatch_histogram_b200 import ep, inputs
+from gpu_util import bf16_dev, check_layout, dev, i32_dev, u8_dev
+
+pytestmark = pytest.mark.gpu
+
+FORMATS = [ep.EP_FP8_SCALE_F32, ep.EP_FP8_SCALE_POW2, ep.EP_FP8_SCALE_UE8M0]
+
+
+@pytest.fixture(autouse=True)
+def _free_memory():
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def run_fp8(inp, E, fmt):
+    idx = i32_dev(inp.topk_idx)
+    act = u8_dev(inp.active)
+    lay = ep.ep_layout(idx, act, E, hidden=inp.x.shape[2])
+    codes, scales, src, st = ep.ep_dispatch_fp8(bf16_dev(inp.x), idx, lay.pair_row, lay.recv_count, E, fmt,
+                                                status=lay.status)
+    torch.cuda.synchronize()
+    return lay, codes, scales, src, int(st.item())
+
+
+def check_fp8(inp, E, fmt, tag):
+    ref = oracle.layout(inp.topk_idx, inp.active, E)
+    pow2 = fmt != ep.EP_FP8_SCALE_F32
+    w_codes, w_scales, w_ue, _ = oracle.dispatch_fp8(inp.x, inp.topk_idx, ref, pow2)
+    lay, codes, scales, src, st = run_fp8(inp, E, fmt)
+    check_layout(lay, ref, tag)
+    assert st == ref.status
+    cap = codes.shape[1]
+    g_codes = codes.view(torch.uint8)
+    for e in range(E):
+        n = min(int(ref.recv_count[e]), cap)
+        if n == 0:
+            continue
+        a = int(ref.list_base[e])
+        assert np.array_equal(src[e, :n].cpu().numpy(), ref.src_list[a:a + n]), f"{tag} src_info {e}"
+        got = g_codes[e, :n].cpu().numpy()
+        want = w_codes[a:a + n]
+        if not np.array_equal(got, want):
+            bad = np.argwhere(got != want)[0]
+            raise AssertionError(f"{tag} codes of expert {e} row {bad[0]} ch {bad[1]}: "
+                                 f"{got[tuple(bad)]:#x} != {want[tuple(bad)]:#x}")
+        s = scales[e, :n].cpu().numpy()            # [n, groups] view of the column-major storage
+        if fmt == ep.EP_FP8_SCALE_UE8M0:
+            words = s.astype(np.int64) & 0xFFFFFFFF
+            bytes_ = np.stack([(words >> (8 * j)) & 0xFF for j in range(4)], axis=2).reshape(n, -1)
+            assert np.array_equal(bytes_, w_ue[a:a + n]), f"{tag} ue8m0 of expert {e}"
+        else:
+            assert np.array_equal(s.view(np.uint32), w_scales[a:a + n].view(np.uint32)), f"{tag} scales {e}"
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("name", ["decode", "sweep_T64_mask5", "replica_T256"])
+def test_fp8_dispatch_matches_oracle(name, fmt):
+    w = inputs.replica(256) if name == "replica_T256" else inputs.named(name)
+    inp = inputs.make_inputs(w)
+    if w.num_extra:
+        phys = oracle.reroute(inp.topk_idx, w.num_experts, w.num_extra)["topk_idx_phys"]
+        inp = inputs.Inputs(phys, inp.topk_weights, inp.x, inp.active)
+    check_fp8(inp, w.num_physical, fmt, f"{name} fmt {fmt}")
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("magnitude", [0.0, 1e-30, 1e-3, 1e3, 1e30])
+def test_fp8_dispatch_extreme_values(fmt, magnitude):
+    R, T, k, E, H = 2, 24, 3, 8, 1024
+    rng = np.random.default_rng(int(magnitude * 7) % 97 + fmt)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k).astype(np.int32)
+    x = (rng.standard_normal((R, T, H)) * magnitude).astype(np.float32)
+    x[0, 0, :128] = 0.0
+    x[1, 2, 256:384] = magnitude * 448.0
+    bits = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    w = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+    inp = inputs.Inputs(idx, w, bits, np.ones(R, np.uint8))
+    check_fp8(inp, E, fmt, f"magnitude {magnitude} fmt {fmt}")
+
+
+@pytest.mark.parametrize("fmt", [ep.EP_FP8_SCALE_F32, ep.EP_FP8_SCALE_POW2])
+def test_fp8_dispatch_small_hidden(fmt):
+    w = inputs.Workload("h128", 4, 40, 2, 8, 128)
+    inp = inputs.make_inputs(w)
+    check_fp8(inp, w.num_experts, fmt, f"H=128 fmt {fmt}")
+
+
+def test_fp8_dispatch_rejects_bad_hidden():
+    R, T, k, E = 2, 4, 2, 8
+    idx = torch.zeros((R, T, k), dtype=torch.int32, device=dev())
+    pr = torch.full((R, T, k), -1, dtype=torch.int32, device=dev())
+    rc = torch.zeros(E, dtype=torch.int32, device=dev())
+    x = torch.zeros((R, T, 256), dtype=torch.bfloat16, device=dev())
+    with pytest.raises(ep.EPError):
+        ep.ep_dispatch_fp8(x, idx, pr, rc, E, ep.EP_FP8_SCALE_UE8M0)  # 256 is not a multiple of 512
+    x = torch.zeros((R, T, 200), dtype=torch.bfloat16, device=dev())
+    with pytest.raises(ep.EPError):
+        ep.ep_dispatch_fp8(x, idx, pr, rc, E)                          # not a multiple of 128
