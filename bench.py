@@ -147,6 +147,37 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# ----------------------------------------------------------------------------- rank plumbing
+
+def rank_barrier(world: int, local_rank: int = 0):
+    """Barrier over all ranks (no-op on one rank); NCCL needs the rank's device."""
+    if world <= 1:
+        return
+    import torch.distributed as dist
+
+    if dist.get_backend() == "nccl":
+        dist.barrier(device_ids=[local_rank])
+    else:
+        dist.barrier()
+
+
+def reduce_over_ranks(values, world: int, device, op: str = "max"):
+    """Element-wise max (or sum) of a list of floats over all ranks."""
+    import torch
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return t.tolist()
+
+
+def whole_job_gbs(total_bytes: float, ms: float) -> float:
+    """GB/s of bytes moved by all ranks in the slowest rank's time."""
+    return total_bytes / (ms * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def algorithmic_bytes(H: int, tokens_sent: int, live_pairs: int, tokens_out: int):
@@ -260,8 +291,7 @@ def run_ours(args, rank, world, local_rank):
             for _ in range(args.warmup):
                 g.replay()
         torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier(device_ids=[local_rank])
+    rank_barrier(world, local_rank)
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(gpu_index_of(local_rank))
     with sampler, torch.cuda.stream(stream):
@@ -274,8 +304,7 @@ def run_ours(args, rank, world, local_rank):
         t_end.record(stream)
         stream.synchronize()
     torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier(device_ids=[local_rank])
+    rank_barrier(world, local_rank)
     total_ms = t_start.elapsed_time(t_end)
     if graphs is None:
         lay_ms = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
@@ -308,8 +337,7 @@ def run_ours(args, rank, world, local_rank):
         d2h = h_out.numel() * 2
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier(device_ids=[local_rank])
+        rank_barrier(world, local_rank)
         torch.cuda.synchronize(dev)
         with torch.cuda.stream(stream):
             e0.record(stream)
@@ -322,21 +350,18 @@ def run_ours(args, rank, world, local_rank):
                 h_out.copy_(out.view(torch.int16), non_blocking=True)
             e1.record(stream)
             stream.synchronize()
-        if world > 1:
-            dist.barrier(device_ids=[local_rank])
+        rank_barrier(world, local_rank)
         e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
         e2e = dict(ms=e2e_ms, h2d=h2d, d2h=d2h)
         assert np.array_equal(h_out.numpy(), out.view(torch.int16).cpu().numpy())
 
     # ---------------------------------------------------------------- reduce over ranks
-    vals = torch.tensor([total_ms, lay_ms, dis_ms, com_ms, e2e["ms"] if e2e else 0.0], dtype=torch.float64,
-                        device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, lay_ms, dis_ms, com_ms, e2e_ms = vals.tolist()
+    total_ms, lay_ms, dis_ms, com_ms, e2e_ms = reduce_over_ranks(
+        [total_ms, lay_ms, dis_ms, com_ms, e2e["ms"] if e2e else 0.0], world, dev, "max")
     ms_per_step = total_ms / args.steps
     step_bytes = d_bytes + c_bytes
-    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    (job_bytes,) = reduce_over_ranks([step_bytes], world, dev, "sum")
+    value = whole_job_gbs(job_bytes, ms_per_step)
     dis_gbs = d_bytes / (dis_ms * 1e-3) / 1e9
     com_gbs = c_bytes / (com_ms * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_gbs()
@@ -380,7 +405,7 @@ def run_ours(args, rank, world, local_rank):
     if args.dispatch_cfg or args.combine_cfg:
         line["launch_cfg"] = {"dispatch": args.dispatch_cfg, "combine": args.combine_cfg}
     if e2e is not None:
-        line["e2e"] = {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+        line["e2e"] = {"value": round(whole_job_gbs(job_bytes, e2e_ms), 1), "unit": "GB/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                        "ms_per_step": round(e2e_ms, 3)}
     clk = sampler.summary()

@@ -1,0 +1,68 @@
+"""Multi-rank plumbing of bench.py on CPU: gloo, world size 2 (the GPU path uses NCCL the same way)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench
+
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.rank_barrier(world)
+        mx = bench.reduce_over_ranks([1.0 + rank, 10.0 - rank, 3.5], world, "cpu", "max")
+        sm = bench.reduce_over_ranks([100.0 * (rank + 1)], world, "cpu", "sum")
+        out[rank] = (mx, sm)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_over_ranks_gloo_world2():
+    port = _free_port()
+    manager = mp.Manager()
+    out = manager.dict()
+    mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+    for rank in (0, 1):
+        mx, sm = out[rank]
+        assert mx == [2.0, 10.0, 3.5]          # max over ranks, element by element
+        assert sm == [300.0]                   # bytes of all ranks
+
+
+def test_whole_job_value():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    # two replicas moving 4 GB each in a slowest-rank step of 2 ms: 4 TB/s whole-job
+    assert bench.whole_job_gbs(8e9, 2.0) == pytest.approx(4000.0)
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", "--workload", "tiny",
+           "--cpu-sample-tokens", "16"]
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
