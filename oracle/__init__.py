@@ -69,6 +69,12 @@ def _bind(lib):
     lib.oracle_dispatch_fp8.restype = I
     lib.oracle_e4m3_array.argtypes = [P, ctypes.c_int64, P]
     lib.oracle_e4m3_array.restype = None
+    lib.oracle_normal_layout.argtypes = [I, I, I, I, P, P, I, I, P, P, P]
+    lib.oracle_normal_layout.restype = I
+    lib.oracle_normal_dispatch.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P]
+    lib.oracle_normal_dispatch.restype = I
+    lib.oracle_normal_combine.argtypes = [I, I, I, I, P, P, P, P]
+    lib.oracle_normal_combine.restype = I
     return lib
 
 
@@ -211,3 +217,48 @@ def dispatch_fp8(x: np.ndarray, topk_idx: np.ndarray, lay: Layout, pow2: bool, l
                                      _p(lay.pair_row), _p(lay.list_base), _p(codes) if L else None,
                                      _p(scales) if L else None, _p(ue) if L else None)
     return codes, scales, ue, int(status)
+
+
+def normal_layout(topk_idx, active, num_experts, alignment=1, capacity=None, lib=None) -> dict:
+    """Normal-mode receive rows: token_recv_row [R,T,R], recv_tokens [R], aligned per-expert counts [E]."""
+    lib = lib or load()
+    topk_idx = np.ascontiguousarray(topk_idx, np.int32)
+    R, T, k = topk_idx.shape
+    cap = R * T if capacity is None else int(capacity)
+    trr = np.zeros((R, T, R), np.int32)
+    rt = np.zeros(R, np.int32)
+    nre = np.zeros(int(num_experts), np.int32)
+    st = lib.oracle_normal_layout(R, T, k, int(num_experts), _p(topk_idx), _p(np.ascontiguousarray(active, np.uint8)),
+                                  int(alignment), cap, _p(trr), _p(rt), _p(nre))
+    return dict(token_recv_row=trr, recv_tokens=rt, num_recv_tokens_per_expert=nre, capacity=cap, status=int(st))
+
+
+def normal_dispatch(x, topk_idx, topk_weights, active, num_experts, nl: dict, lib=None) -> dict:
+    """Normal-mode receive buffers [R, capacity, ...] (rows past recv_tokens stay zero)."""
+    lib = lib or load()
+    x = np.ascontiguousarray(x, np.uint16)
+    R, T, H = x.shape
+    k = topk_idx.shape[2]
+    cap = nl["capacity"]
+    out = dict(recv_x=np.zeros((R, cap, H), np.uint16), recv_topk_idx=np.zeros((R, cap, k), np.int32),
+               recv_topk_weights=np.zeros((R, cap, k), np.float32), src_info=np.zeros((R, cap, 2), np.int32))
+    st = lib.oracle_normal_dispatch(R, T, k, int(num_experts), H, cap, _p(x),
+                                    _p(np.ascontiguousarray(topk_idx, np.int32)),
+                                    _p(np.ascontiguousarray(topk_weights, np.float32)),
+                                    _p(np.ascontiguousarray(active, np.uint8)), _p(nl["token_recv_row"]),
+                                    _p(out["recv_x"]), _p(out["recv_topk_idx"]), _p(out["recv_topk_weights"]),
+                                    _p(out["src_info"]))
+    out["status"] = int(st)
+    return out
+
+
+def normal_combine(y, token_recv_row, active_now, lib=None):
+    """Unweighted float64 sum of every returned row per source token: ([R, T, H], status)."""
+    lib = lib or load()
+    y = np.ascontiguousarray(y, np.uint16)
+    R, cap, H = y.shape
+    T = token_recv_row.shape[1]
+    out = np.zeros((R, T, H), np.float64)
+    st = lib.oracle_normal_combine(R, T, H, cap, _p(y), _p(np.ascontiguousarray(token_recv_row, np.int32)),
+                                   _p(np.ascontiguousarray(active_now, np.uint8)), _p(out))
+    return out, int(st)

@@ -388,3 +388,106 @@ int oracle_dispatch_fp8(int R, int T, int k, int E, int H, int pow2, const uint1
 void oracle_e4m3_array(const float *v, int64_t n, uint8_t *out) {
     for (int64_t i = 0; i < n; i++) out[i] = oracle_e4m3_from_float(v[i]);
 }
+
+/*
+ * Normal (high-throughput) mode ([P1] Buffer.dispatch and Buffer.combine):
+ * a token goes ONCE to every rank that one of its live pairs reaches
+ * (is_token_in_rank), and combine adds the returned rows WITHOUT weights.
+ * Readings (also in the design notes): rank d's received tokens are ordered
+ * by (source rank, token); a receive buffer holds `capacity` rows
+ * (num_worst_tokens), rows past it are counted as overflow and neither
+ * written nor read; recv_topk_idx holds the local expert id (e - d*E_local)
+ * of slots whose live expert is on rank d and -1 elsewhere, recv_topk_weights
+ * the slot's weight there and 0 elsewhere; the per-expert receive counts are
+ * the live pairs of each expert rounded up to a multiple of expert_alignment.
+ *   token_recv_row [R,T,R]  row of (r,t) in rank d's buffer, -1 if not sent
+ *   recv_tokens    [R]
+ *   num_recv_tokens_per_expert [E]
+ */
+int oracle_normal_layout(int R, int T, int k, int E, const int32_t *topk_idx, const uint8_t *active,
+                         int alignment, int capacity, int32_t *token_recv_row, int32_t *recv_tokens,
+                         int32_t *num_recv_tokens_per_expert) {
+    int status = 0;
+    const int E_local = E / R;
+    for (int d = 0; d < R; d++) recv_tokens[d] = 0;
+    for (int e = 0; e < E; e++) num_recv_tokens_per_expert[e] = 0;
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < T; t++) {
+            for (int d = 0; d < R; d++) {
+                int sent = 0;
+                for (int j = 0; j < k; j++) {
+                    int e = topk_idx[((int64_t)r * T + t) * k + j];
+                    if (pair_is_live(e, r, E, E_local, active) && e / E_local == d) sent = 1;
+                }
+                int64_t at = ((int64_t)r * T + t) * R + d;
+                if (sent) {
+                    token_recv_row[at] = recv_tokens[d];
+                    recv_tokens[d] += 1;
+                    if (token_recv_row[at] >= capacity) status |= ORACLE_OVERFLOW;
+                } else {
+                    token_recv_row[at] = -1;
+                }
+            }
+            for (int j = 0; j < k; j++) {
+                int e = topk_idx[((int64_t)r * T + t) * k + j];
+                if (e < -1 || e >= E) status |= ORACLE_BAD_EXPERT;
+                if (pair_is_live(e, r, E, E_local, active)) num_recv_tokens_per_expert[e] += 1;
+            }
+        }
+    for (int e = 0; e < E; e++) {
+        int n = num_recv_tokens_per_expert[e];
+        num_recv_tokens_per_expert[e] = ((n + alignment - 1) / alignment) * alignment;
+    }
+    return status;
+}
+
+/*   recv_x [R,capacity,H] bf16 bits, recv_topk_idx / recv_topk_weights [R,capacity,k],
+ *   src_info [R,capacity,2]; rows past recv_tokens[d] are left untouched. */
+int oracle_normal_dispatch(int R, int T, int k, int E, int H, int capacity, const uint16_t *x,
+                           const int32_t *topk_idx, const float *topk_weights, const uint8_t *active,
+                           const int32_t *token_recv_row, uint16_t *recv_x, int32_t *recv_topk_idx,
+                           float *recv_topk_weights, int32_t *src_info) {
+    int status = 0;
+    const int E_local = E / R;
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < T; t++)
+            for (int d = 0; d < R; d++) {
+                int32_t row = token_recv_row[((int64_t)r * T + t) * R + d];
+                if (row < 0) continue;
+                if (row >= capacity) { status |= ORACLE_OVERFLOW; continue; }
+                int64_t dst = (int64_t)d * capacity + row;
+                for (int h = 0; h < H; h++) recv_x[dst * H + h] = x[((int64_t)r * T + t) * H + h];
+                for (int j = 0; j < k; j++) {
+                    int64_t p = ((int64_t)r * T + t) * k + j;
+                    int e = topk_idx[p];
+                    int here = pair_is_live(e, r, E, E_local, active) && e / E_local == d;
+                    recv_topk_idx[dst * k + j] = here ? e - d * E_local : -1;
+                    recv_topk_weights[dst * k + j] = here ? topk_weights[p] : 0.0f;
+                }
+                src_info[2 * dst] = r;
+                src_info[2 * dst + 1] = t;
+            }
+    return status;
+}
+
+/* out [R,T,H] float64: for (r,t), the sum over ranks d in order of y[d][row]
+ * for every row the token was sent to, skipping ranks masked in active_now;
+ * zero rows for a masked source rank. */
+int oracle_normal_combine(int R, int T, int H, int capacity, const uint16_t *y, const int32_t *token_recv_row,
+                          const uint8_t *active_now, double *out) {
+    int status = 0;
+    for (int r = 0; r < R; r++)
+        for (int t = 0; t < T; t++) {
+            double *o = out + ((int64_t)r * T + t) * H;
+            for (int h = 0; h < H; h++) o[h] = 0.0;
+            if (!active_now[r]) continue;
+            for (int d = 0; d < R; d++) {
+                int32_t row = token_recv_row[((int64_t)r * T + t) * R + d];
+                if (row < 0 || !active_now[d]) continue;
+                if (row >= capacity) { status |= ORACLE_OVERFLOW; continue; }
+                const uint16_t *yr = y + ((int64_t)d * capacity + row) * H;
+                for (int h = 0; h < H; h++) o[h] += bf16_to_double(yr[h]);
+            }
+        }
+    return status;
+}

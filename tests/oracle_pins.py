@@ -416,6 +416,83 @@ def pin_fp8_dequant_error(lib):
             assert np.array_equal(ue.astype(np.int64) - 127, np.log2(scales).astype(np.int64))
 
 
-ALL_PINS = [pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
+# ----------------------------------------------------------------------------- normal-mode pins
+
+def pin_normal_golden(lib):
+    g = _golden("layout_tiny.json")
+    n = _golden("normal_tiny.json")
+    idx = np.array(g["topk_idx"], np.int32)
+    R, T, E, H = g["R"], g["T"], g["E"], 8
+    x = (np.arange(R * T * H, dtype=np.float32).reshape(R, T, H) / 8 + 1)
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)           # small multiples of 1/8: exact in bf16
+    w = np.arange(1, R * T * 2 + 1, dtype=np.float32).reshape(R, T, 2) / 16
+    for case in n["cases"]:
+        act = np.array(case["active"], np.uint8)
+        for align, counts in case["num_recv_tokens_per_expert"].items():
+            nl = oracle.normal_layout(idx, act, E, alignment=int(align), lib=lib)
+            assert nl["num_recv_tokens_per_expert"].tolist() == counts, f"aligned counts {align}"
+        nl = oracle.normal_layout(idx, act, E, lib=lib)
+        assert nl["token_recv_row"].tolist() == case["token_recv_row"]
+        assert nl["recv_tokens"].tolist() == case["recv_tokens"]
+        nd = oracle.normal_dispatch(xb, idx, w, act, E, nl, lib=lib)
+        for d in range(R):
+            rows = case["recv_topk_idx"][d]
+            assert nd["recv_topk_idx"][d, :len(rows)].tolist() == rows, f"recv_topk_idx of rank {d}"
+        out, _ = oracle.normal_combine(nd["recv_x"], nl["token_recv_row"], act, lib=lib)
+        mult = np.array(case["combine_multiplier"], np.float64)[:, :, None]
+        assert np.array_equal(out, mult * oracle.bf16_bits_to_f64(xb)), "unweighted combine"
+
+
+def pin_normal_bruteforce(lib):
+    rng = np.random.default_rng(31)
+    for it in range(150):
+        idx, active, E = _random_case(rng, dup=(it % 6 == 0))
+        R, T, k = idx.shape
+        nl = oracle.normal_layout(idx, active, E, lib=lib)
+        itr = brute_layout(idx, active, E)["is_token_in_rank"]        # [R, T, R] from the lexsort model
+        for d in range(R):
+            sent = np.flatnonzero(itr[:, :, d].ravel())               # (r, t) flattened, in order
+            want = np.full(R * T, -1)
+            want[sent] = np.arange(len(sent))
+            assert np.array_equal(nl["token_recv_row"][:, :, d].ravel(), want), f"case {it} rank {d}"
+            assert nl["recv_tokens"][d] == len(sent)
+        live = brute_layout(idx, active, E)["live"]
+        cnt = np.bincount(idx[live], minlength=E)
+        for a in (1, 2, 5):
+            got = oracle.normal_layout(idx, active, E, alignment=a, lib=lib)["num_recv_tokens_per_expert"]
+            assert np.array_equal(got, -(-cnt // a) * a)
+
+
+def pin_normal_dispatch_combine(lib):
+    rng = np.random.default_rng(32)
+    for it in range(40):
+        idx, active, E = _random_case(rng)
+        R, T, k = idx.shape
+        El = E // R
+        H = 8 * int(rng.integers(1, 3))
+        x = inputs.bf16_tokens(rng, R * T, H).reshape(R, T, H)
+        w = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+        nl = oracle.normal_layout(idx, active, E, lib=lib)
+        nd = oracle.normal_dispatch(x, idx, w, active, E, nl, lib=lib)
+        live = brute_layout(idx, active, E)["live"]
+        for d in range(R):
+            n = nl["recv_tokens"][d]
+            src = nd["src_info"][d, :n]
+            assert np.array_equal(nd["recv_x"][d, :n], x[src[:, 0], src[:, 1]])
+            keys = src[:, 0] * T + src[:, 1]
+            assert np.all(np.diff(keys) > 0), "received tokens not in (rank, token) order"
+            for i, (r, t) in enumerate(src):
+                here = live[r, t] & (idx[r, t] // El == d)
+                assert np.array_equal(nd["recv_topk_idx"][d, i], np.where(here, idx[r, t] - d * El, -1))
+                assert np.array_equal(nd["recv_topk_weights"][d, i], np.where(here, w[r, t], 0))
+        # identity experts: the unweighted combine returns (#ranks reached) * x, exactly
+        out, _ = oracle.normal_combine(nd["recv_x"], nl["token_recv_row"], active, lib=lib)
+        reach = (nl["token_recv_row"] >= 0).sum(axis=2)[:, :, None]
+        want = reach * oracle.bf16_bits_to_f64(x)
+        want[active == 0] = 0
+        assert np.array_equal(out, want)
+
+
+ALL_PINS = [pin_normal_golden, pin_normal_bruteforce, pin_normal_dispatch_combine, pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
             pin_dispatch_golden, pin_dispatch_bijection, pin_combine_golden,
             pin_combine_special_cases, pin_combine_mask, pin_reroute_golden, pin_reroute_invariants]

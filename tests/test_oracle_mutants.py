@@ -49,6 +49,15 @@ MUTANTS = {
     "ue8m0_bias": ("if (ue8m0) *ue8m0 = (uint8_t)(e + 127);", "if (ue8m0) *ue8m0 = (uint8_t)(e + 128);"),
     "pow2_floor": ("e = m == 0.5 ? f - 1 : f;", "e = f - 1;"),
     "fp8_no_saturation": ("if (a >= 448.0) return (uint8_t)(sign | 0x7Eu);", "if (a >= 480.0) return (uint8_t)(sign | 0x7Fu);"),
+    # normal mode
+    "normal_global_expert_id": ("recv_topk_idx[dst * k + j] = here ? e - d * E_local : -1;",
+                                "recv_topk_idx[dst * k + j] = here ? e : -1;"),
+    "normal_weighted_combine": ("for (int h = 0; h < H; h++) o[h] += bf16_to_double(yr[h]);",
+                                "for (int h = 0; h < H; h++) o[h] += 0.5 * bf16_to_double(yr[h]);"),
+    "normal_alignment_floor": ("num_recv_tokens_per_expert[e] = ((n + alignment - 1) / alignment) * alignment;",
+                               "num_recv_tokens_per_expert[e] = (n / alignment) * alignment;"),
+    "normal_sent_any_rank": ("if (pair_is_live(e, r, E, E_local, active) && e / E_local == d) sent = 1;",
+                             "if (pair_is_live(e, r, E, E_local, active)) sent = 1;"),
     # reroute
     "reroute_tie_highest": ("if (lhs > rhs) best = e;", "if (lhs >= rhs) best = e;"),
     "reroute_local_token": ("topk_phys[p] = phys_base[e] + (int32_t)(global_token % n_rep[e]);",
