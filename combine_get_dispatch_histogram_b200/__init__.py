@@ -12,6 +12,9 @@ from .ep import (  # noqa: F401
     ep_dispatch_fp8,
     ep_layout,
     ep_layout_workspace_bytes,
+    ep_normal_combine,
+    ep_normal_dispatch,
+    ep_normal_layout,
     ep_reroute,
     ep_reroute_workspace_bytes,
     ep_strerror,

@@ -103,17 +103,21 @@ struct SlotMeta {
     float w;
 };
 
+// Slot `lane` of a token: its slab (expert; in normal mode the destination rank
+// itself), slab row and weight (1 in normal mode: the sum is unweighted).
+template <bool NORMAL>
 __device__ __forceinline__ SlotMeta load_slot(const CombineArgs& a, int64_t tok, int lane) {
     SlotMeta m{-1, -1, 0.f};
     if (lane < a.k) {
         const int64_t p = tok * a.k + lane;
-        m.e = __ldg(a.topk_idx + p);
+        m.e = NORMAL ? lane : __ldg(a.topk_idx + p);
         m.row = __ldg(a.pair_row + p);
-        m.w = __ldg(a.w + p);
+        m.w = NORMAL ? 1.0f : __ldg(a.w + p);
     }
     return m;
 }
 
+template <bool NORMAL>
 __global__ void combine_kernel(CombineArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int S = a.stages;
@@ -145,11 +149,11 @@ __global__ void combine_kernel(CombineArgs a) {
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         const uint64_t pol = policy_evict_first();
-        SlotMeta nxt = my_tok > 0 ? load_slot(a, tok0, lane) : SlotMeta{-1, -1, 0.f};
+        SlotMeta nxt = my_tok > 0 ? load_slot<NORMAL>(a, tok0, lane) : SlotMeta{-1, -1, 0.f};
         for (int64_t t = 0; t < my_tok; ++t) {
             const int64_t tok = tok0 + t;
             const SlotMeta cur = nxt;
-            if (t + 1 < my_tok) nxt = load_slot(a, tok + 1, lane);  // prefetch the next token's routing
+            if (t + 1 < my_tok) nxt = load_slot<NORMAL>(a, tok + 1, lane);  // prefetch the next token's routing
             const int r = int(tok / a.T);
             const bool in_range = cur.e >= 0 && cur.e < a.E;
             const bool live = lane < a.k && cur.row >= 0 && cur.row < a.cap && in_range && act[r] != 0 &&
@@ -232,7 +236,7 @@ __global__ void combine_kernel(CombineArgs a) {
 // order and stores its U result vectors.
 constexpr int kVecKMax = 8;
 
-template <int U>
+template <int U, bool NORMAL>
 __global__ void __launch_bounds__(256) combine_vec_kernel(CombineArgs a) {
     __shared__ int32_t act[kActiveSlots];
     for (int i = threadIdx.x; i < a.R; i += blockDim.x) act[i] = a.active[i];
@@ -261,10 +265,10 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(CombineArgs a) {
             int e = -1, row = -1;
             float w = 0.f;
             if (lane < a.k) {
-                const int64_t p = tok * a.k + lane;
-                e = __ldg(a.topk_idx + p);
-                row = __ldg(a.pair_row + p);
-                w = __ldg(a.w + p);
+                const SlotMeta m = load_slot<NORMAL>(a, tok, lane);
+                e = m.e;
+                row = m.row;
+                w = m.w;
             }
             const bool in_range = e >= 0 && e < a.E;
             const bool live = lane < a.k && row >= 0 && row < a.cap && in_range && act[r] != 0 &&
@@ -307,20 +311,63 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(CombineArgs a) {
     }
 }
 
-template <int U>
+template <int U, bool NORMAL>
 int launch_combine_vec(const CombineArgs& a, const ep_cfg_t& cfg, int sms, cudaStream_t stream) {
     static int per_sm[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     int& occ = per_sm[dev & 63];
     if (occ == 0 &&
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, combine_vec_kernel<U>, 256, 0) != cudaSuccess)
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, combine_vec_kernel<U, NORMAL>, 256, 0) != cudaSuccess)
         return EP_ERR_CUDA;
     int64_t grid = int64_t(sms) * std::max(1, occ);
     if (cfg.max_ctas > 0) grid = std::min<int64_t>(grid, cfg.max_ctas);
     const int64_t warps_needed = ceil_div(int64_t(a.R) * a.T * ceil_div(a.row_bytes >> 4, 32 * U), 1);
     grid = std::max<int64_t>(1, std::min<int64_t>(grid, ceil_div(warps_needed, 8)));
-    combine_vec_kernel<U><<<unsigned(grid), 256, 0, stream>>>(a);
+    combine_vec_kernel<U, NORMAL><<<unsigned(grid), 256, 0, stream>>>(a);
+    return launch_result();
+}
+
+// Vector or bulk path for a filled CombineArgs (a.k slots per token).
+template <bool NORMAL>
+int run_combine(CombineArgs& a, const ep_cfg_t& cfg, int variant, cudaStream_t stream) {
+    if (variant == EP_VARIANT_VECTOR) {
+        const int sms = sm_count();
+        if (sms <= 0) return EP_ERR_CUDA;
+        // cfg.threads selects the columns per lane and unit (1 or 2; 2 measured faster on B200)
+        return cfg.threads == 1 ? launch_combine_vec<1, NORMAL>(a, cfg, sms, stream)
+                                : launch_combine_vec<2, NORMAL>(a, cfg, sms, stream);
+    }
+    const uint32_t piece_max =
+        std::max<uint32_t>(16, std::min<uint32_t>(kCombinePieceMax, (kCombineStageMax / a.k) & ~15u));
+    a.n_pieces = int(ceil_div(a.row_bytes, piece_max));
+    a.piece_bytes = uint32_t(round_up16(size_t(ceil_div(a.row_bytes, a.n_pieces))));
+    if (int64_t(a.n_pieces - 1) * a.piece_bytes >= a.row_bytes) return EP_ERR_UNSUPPORTED;
+    a.slot_bytes = a.piece_bytes;
+    a.stage_bytes = uint32_t(a.k) * a.slot_bytes;
+    a.n_units = int64_t(a.R) * a.T * a.n_pieces;
+
+    const int sms = sm_count();
+    if (sms <= 0) return EP_ERR_CUDA;
+    const size_t fixed = size_t(kActiveSlots) * 4 + 1024;
+    const size_t per_stage = size_t(a.stage_bytes) + sizeof(StageHeader) + 16;
+    const size_t budget = size_t(max_smem_optin()) - fixed;
+    int stages = cfg.stages > 0 ? cfg.stages : int(budget / per_stage);
+    stages = std::max(2, std::min(kCombineMaxStages, stages));
+    a.stages = stages;
+    const size_t smem = size_t(stages) * per_stage + size_t(kActiveSlots) * 4;
+    if (smem > size_t(max_smem_optin())) return EP_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(combine_kernel<NORMAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+        return EP_ERR_CUDA;
+
+    const int nvec = int(a.piece_bytes / 16);
+    int consumer_warps = cfg.threads > 0 ? std::max(1, cfg.threads / 32 - 1) : (nvec + 31) / 32;
+    consumer_warps = std::max(1, std::min(15, consumer_warps));
+    int64_t grid = sms;
+    if (cfg.max_ctas > 0) grid = std::min<int64_t>(grid, cfg.max_ctas);
+    grid = std::min<int64_t>(grid, int64_t(a.R) * a.T);
+    combine_kernel<NORMAL><<<unsigned(grid), 32 * (1 + consumer_warps), smem, stream>>>(a);
     return launch_result();
 }
 
@@ -359,42 +406,40 @@ extern "C" int ep_combine(ep_dims_t d, const uint16_t* y, const int32_t* topk_id
     a.E_local = d.num_experts / d.num_ranks;
     a.row_bytes = int64_t(d.hidden) * 2;
     a.cap = RT;
-    if (variant == EP_VARIANT_VECTOR) {
-        const int sms = sm_count();
-        if (sms <= 0) return EP_ERR_CUDA;
-        cudaStream_t st = static_cast<cudaStream_t>(stream);
-        // cfg.threads selects the columns per lane and unit (1 or 2; 2 measured faster on B200)
-        return cfg.threads == 1 ? launch_combine_vec<1>(a, cfg, sms, st) : launch_combine_vec<2>(a, cfg, sms, st);
-    }
-    const uint32_t piece_max =
-        std::max<uint32_t>(16, std::min<uint32_t>(kCombinePieceMax, (kCombineStageMax / d.num_topk) & ~15u));
-    a.n_pieces = int(ceil_div(a.row_bytes, piece_max));
-    a.piece_bytes = uint32_t(round_up16(size_t(ceil_div(a.row_bytes, a.n_pieces))));
-    if (int64_t(a.n_pieces - 1) * a.piece_bytes >= a.row_bytes) return EP_ERR_UNSUPPORTED;
-    a.slot_bytes = a.piece_bytes;
-    a.stage_bytes = uint32_t(d.num_topk) * a.slot_bytes;
-    a.n_units = RT * a.n_pieces;
+    return run_combine<false>(a, cfg, variant, static_cast<cudaStream_t>(stream));
+}
 
-    const int sms = sm_count();
-    if (sms <= 0) return EP_ERR_CUDA;
-    const size_t fixed = size_t(kActiveSlots) * 4 + 1024;
-    const size_t per_stage = size_t(a.stage_bytes) + sizeof(StageHeader) + 16;
-    const size_t budget = size_t(max_smem_optin()) - fixed;
-    int stages = cfg.stages > 0 ? cfg.stages : int(budget / per_stage);
-    stages = std::max(2, std::min(kCombineMaxStages, stages));
-    a.stages = stages;
-    const size_t smem = size_t(stages) * per_stage + size_t(kActiveSlots) * 4;
-    if (smem > size_t(max_smem_optin())) return EP_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-        return EP_ERR_CUDA;
 
-    const int nvec = int(a.piece_bytes / 16);
-    int consumer_warps = cfg.threads > 0 ? std::max(1, cfg.threads / 32 - 1) : (nvec + 31) / 32;
-    consumer_warps = std::max(1, std::min(15, consumer_warps));
-    int64_t grid = sms;
-    if (cfg.max_ctas > 0) grid = std::min<int64_t>(grid, cfg.max_ctas);
-    grid = std::min<int64_t>(grid, RT);
-    combine_kernel<<<unsigned(grid), 32 * (1 + consumer_warps), smem, static_cast<cudaStream_t>(stream)>>>(a);
-    return launch_result();
+extern "C" int ep_normal_combine(ep_dims_t d, int32_t recv_capacity, const uint16_t* y,
+                                 const int32_t* token_recv_row, const uint8_t* active, uint16_t* out,
+                                 int32_t* status, ep_cfg_t cfg, void* stream) {
+    int rc = check_dims(d);
+    if (rc != EP_OK) return rc;
+    if (recv_capacity < 0) return EP_ERR_INVALID;
+    if (d.num_ranks > EP_MAX_NORMAL_RANKS) return EP_ERR_UNSUPPORTED;
+    const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
+    if (RT == 0) return EP_OK;
+    if (!token_recv_row || !active || !out || (recv_capacity > 0 && !y)) return EP_ERR_INVALID;
+    if ((y && !aligned16(y)) || !aligned16(out)) return EP_ERR_INVALID;
+    const int variant = cfg.variant != EP_VARIANT_AUTO ? cfg.variant
+                        : (d.num_ranks <= kVecKMax ? EP_VARIANT_VECTOR : EP_VARIANT_BULK);
+    if (variant != EP_VARIANT_BULK && variant != EP_VARIANT_VECTOR) return EP_ERR_INVALID;
+    if (variant == EP_VARIANT_VECTOR && d.num_ranks > kVecKMax) return EP_ERR_UNSUPPORTED;
+    // slots are the destination ranks: slab d of y is rank d's receive buffer
+    CombineArgs a;
+    a.y = reinterpret_cast<const uint8_t*>(y);
+    a.topk_idx = nullptr;
+    a.w = nullptr;
+    a.pair_row = token_recv_row;
+    a.active = active;
+    a.out = reinterpret_cast<uint8_t*>(out);
+    a.status = status;
+    a.R = d.num_ranks;
+    a.T = d.num_tokens;
+    a.k = d.num_ranks;
+    a.E = d.num_ranks;
+    a.E_local = 1;
+    a.row_bytes = int64_t(d.hidden) * 2;
+    a.cap = recv_capacity;
+    return run_combine<true>(a, cfg, variant, static_cast<cudaStream_t>(stream));
 }

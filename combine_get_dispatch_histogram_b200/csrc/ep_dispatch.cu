@@ -45,12 +45,19 @@ constexpr int kDispatchMaxStages = 16;
 
 struct DispatchArgs {
     const uint8_t* x;
-    const int32_t* topk_idx;
-    const int32_t* pair_row;
+    const int32_t* topk_idx;   // low-latency mode: slot experts; unused in normal mode
+    const int32_t* pair_row;   // low-latency mode: [R*T, k] rows; normal mode: token_recv_row [R*T, R]
     uint8_t* recv_x;
     int32_t* src_info;
     int32_t* status;
-    int T, k, E;
+    int T, k, E;               // lanes per token (k, or R in normal mode) and their slab count
+    // normal mode only: the token's slots, to fill recv_topk_idx / recv_topk_weights
+    const int32_t* slot_idx;
+    const float* slot_w;
+    const uint8_t* active;
+    int32_t* recv_topk_idx;
+    float* recv_topk_weights;
+    int slots, slot_E, slot_E_local;
     int64_t row_bytes;
     int64_t cap;
     int n_pieces;
@@ -61,16 +68,28 @@ struct DispatchArgs {
 };
 
 struct UnitMeta {
-    int e;
+    int e;      // slab (expert; destination rank in normal mode)
     int row;
+    int se;     // normal mode: this lane's slot expert if live, else -1
+    float sw;   // normal mode: its weight
 };
 
+template <bool NORMAL>
 __device__ __forceinline__ UnitMeta load_meta(const DispatchArgs& a, int64_t unit, int lane) {
-    UnitMeta m{-1, -1};
+    UnitMeta m{-1, -1, -1, 0.f};
+    const int64_t tok = unit / a.n_pieces;
     if (lane < a.k) {
-        const int64_t p = (unit / a.n_pieces) * a.k + lane;
-        m.e = __ldg(a.topk_idx + p);
+        const int64_t p = tok * a.k + lane;
+        m.e = NORMAL ? lane : __ldg(a.topk_idx + p);
         m.row = __ldg(a.pair_row + p);
+    }
+    if (NORMAL && lane < a.slots) {
+        const int64_t p = tok * a.slots + lane;
+        const int e = __ldg(a.slot_idx + p);
+        const int r = int(tok / a.T);
+        const bool live = e >= 0 && e < a.slot_E && a.active[r] && a.active[e / a.slot_E_local];
+        m.se = live ? e : -1;
+        m.sw = __ldg(a.slot_w + p);
     }
     return m;
 }
@@ -79,12 +98,14 @@ __device__ __forceinline__ uint32_t piece_size(const DispatchArgs& a, int q) {
     return q + 1 < a.n_pieces ? a.piece_bytes : uint32_t(a.row_bytes - int64_t(q) * a.piece_bytes);
 }
 
+template <bool NORMAL>
 __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x;
     const int S = a.stages;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(S) * a.stage_bytes);
     int2* meta = reinterpret_cast<int2*>(full + S);  // [S][32] (e, row) of the staged unit
+    int2* slot = meta + S * 32;                       // [S][32] normal mode: (slot expert, weight bits)
 
     if (lane == 0) {
         for (int s = 0; s < S; ++s) mbar_init(smem_u32(full + s), 1);
@@ -105,6 +126,7 @@ __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
         const bool valid_row = m.row >= 0 && m.row < a.cap;
         const bool live = valid_row && m.e >= 0 && m.e < a.E;
         meta[s * 32 + lane] = make_int2(live ? m.e : -1, m.row);
+        if (NORMAL) slot[s * 32 + lane] = make_int2(m.se, __float_as_int(m.sw));
         if (q == 0) {
             if (m.row >= a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
             if (valid_row && !live) flag_status(a.status, EP_STATUS_BAD_EXPERT);
@@ -125,9 +147,9 @@ __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
     };
 
     const int64_t prologue = my_n < S ? my_n : S;
-    for (int64_t i = 0; i < prologue; ++i) issue(i, load_meta(a, first + i * step, lane));
-    UnitMeta next{-1, -1};  // routing of the next unit to refill: unit S, if this CTA has one
-    if (int64_t(S) < my_n) next = load_meta(a, first + int64_t(S) * step, lane);
+    for (int64_t i = 0; i < prologue; ++i) issue(i, load_meta<NORMAL>(a, first + i * step, lane));
+    UnitMeta next{-1, -1, -1, 0.f};  // routing of the next unit to refill: unit S, if this CTA has one
+    if (int64_t(S) < my_n) next = load_meta<NORMAL>(a, first + int64_t(S) * step, lane);
 
     for (int64_t i = 0; i < my_n; ++i) {
         const int s = int(i % S);
@@ -150,6 +172,22 @@ __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
                 reinterpret_cast<int2*>(a.src_info)[slab_row] = make_int2(src_rank, int(tok - int64_t(src_rank) * a.T));
             }
         }
+        if (NORMAL && q == 0) {
+            // the received token's slots, in rank d's local expert ids (-1 / 0 for other ranks' slots)
+            uint32_t dests = __ballot_sync(0xffffffffu, m.x >= 0);
+            const int2 sl = slot[s * 32 + lane];
+            while (dests) {
+                const int d = __ffs(dests) - 1;
+                dests &= dests - 1;
+                const int row = __shfl_sync(0xffffffffu, m.y, d);
+                if (lane < a.slots) {
+                    const bool here = sl.x >= 0 && sl.x / a.slot_E_local == d;
+                    const int64_t o = (int64_t(d) * a.cap + row) * a.slots + lane;
+                    a.recv_topk_idx[o] = here ? sl.x - d * a.slot_E_local : -1;
+                    a.recv_topk_weights[o] = here ? __int_as_float(sl.y) : 0.f;
+                }
+            }
+        }
         bulk_commit();
         // refill the stage of unit i-1 with unit i-1+S once its stores have read it
         const int64_t refill = i - 1 + S;
@@ -157,7 +195,7 @@ __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
             bulk_wait_read<1>();
             __syncwarp();
             const UnitMeta cur = next;
-            if (refill + 1 < my_n) next = load_meta(a, first + (refill + 1) * step, lane);
+            if (refill + 1 < my_n) next = load_meta<NORMAL>(a, first + (refill + 1) * step, lane);
             issue(refill, cur);
         }
     }
@@ -447,6 +485,22 @@ __global__ void __launch_bounds__(256) fp8_scale_writer_kernel(DispatchFp8Args a
         if (ok_src) out[int64_t(wd) * a.cap] = ts[wd];
 }
 
+// Stage count from the shared-memory budget, then the bulk-path launch.
+template <bool NORMAL>
+int launch_bulk_dispatch(DispatchArgs& a, const ep_cfg_t& cfg, int64_t grid, int budget, cudaStream_t stream) {
+    const size_t per_stage = size_t(a.stage_bytes) + 8 + 2 * 256;
+    int stages = cfg.stages > 0 ? cfg.stages : int(budget / per_stage);
+    stages = std::max(2, std::min(kDispatchMaxStages, stages));
+    a.stages = stages;
+    const size_t smem = size_t(stages) * per_stage;
+    if (smem > size_t(max_smem_optin())) return EP_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(dispatch_kernel<NORMAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+        return EP_ERR_CUDA;
+    dispatch_kernel<NORMAL><<<unsigned(grid), 32, smem, stream>>>(a);
+    return launch_result();
+}
+
 }  // namespace
 }  // namespace ep
 
@@ -535,6 +589,14 @@ extern "C" int ep_dispatch(ep_dims_t d, const uint16_t* x, const int32_t* topk_i
     a.E = d.num_experts;
     a.row_bytes = int64_t(d.hidden) * 2;
     a.cap = RT;
+    a.slot_idx = nullptr;
+    a.slot_w = nullptr;
+    a.active = nullptr;
+    a.recv_topk_idx = nullptr;
+    a.recv_topk_weights = nullptr;
+    a.slots = 0;
+    a.slot_E = 0;
+    a.slot_E_local = 1;
     a.n_pieces = int(ceil_div(a.row_bytes, kDispatchPieceMax));
     a.piece_bytes = uint32_t(round_up16(size_t(ceil_div(a.row_bytes, a.n_pieces))));
     if (int64_t(a.n_pieces - 1) * a.piece_bytes >= a.row_bytes) return EP_ERR_UNSUPPORTED;
@@ -556,14 +618,54 @@ extern "C" int ep_dispatch(ep_dims_t d, const uint16_t* x, const int32_t* topk_i
     grid = std::max<int64_t>(1, std::min<int64_t>(grid, a.n_units));
     const int ctas_per_sm = int(std::max<int64_t>(1, ceil_div(grid, sms)));
     const int budget = std::max(1, max_smem_optin() / ctas_per_sm - 1024);
-    int stages = cfg.stages > 0 ? cfg.stages : int(budget / (a.stage_bytes + 8 + 256));
-    stages = std::max(2, std::min(kDispatchMaxStages, stages));
-    a.stages = stages;
-    const size_t smem = size_t(stages) * (a.stage_bytes + 8 + 256);
-    if (smem > size_t(max_smem_optin())) return EP_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(dispatch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-        return EP_ERR_CUDA;
-    dispatch_kernel<<<unsigned(grid), 32, smem, static_cast<cudaStream_t>(stream)>>>(a);
-    return launch_result();
+    return launch_bulk_dispatch<false>(a, cfg, grid, budget, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int ep_normal_dispatch(ep_dims_t d, int32_t recv_capacity, const uint16_t* x, const int32_t* topk_idx,
+                                  const float* topk_weights, const uint8_t* active, const int32_t* token_recv_row,
+                                  uint16_t* recv_x, int32_t* recv_topk_idx, float* recv_topk_weights,
+                                  int32_t* src_info, int32_t* status, ep_cfg_t cfg, void* stream) {
+    int rc = check_dims(d);
+    if (rc != EP_OK) return rc;
+    if (recv_capacity < 0) return EP_ERR_INVALID;
+    if (d.num_ranks > EP_MAX_NORMAL_RANKS) return EP_ERR_UNSUPPORTED;
+    const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
+    if (RT == 0) return EP_OK;
+    if (!x || !topk_idx || !topk_weights || !active || !token_recv_row) return EP_ERR_INVALID;
+    if (recv_capacity > 0 && (!recv_x || !recv_topk_idx || !recv_topk_weights || !src_info)) return EP_ERR_INVALID;
+    if (!aligned16(x) || (recv_x && !aligned16(recv_x)) || (reinterpret_cast<uintptr_t>(src_info) & 7u))
+        return EP_ERR_INVALID;
+    // lanes are the destination ranks: slab d of recv_x is rank d's receive buffer
+    DispatchArgs a;
+    a.x = reinterpret_cast<const uint8_t*>(x);
+    a.topk_idx = nullptr;
+    a.pair_row = token_recv_row;
+    a.recv_x = reinterpret_cast<uint8_t*>(recv_x);
+    a.src_info = src_info;
+    a.status = status;
+    a.T = d.num_tokens;
+    a.k = d.num_ranks;
+    a.E = d.num_ranks;
+    a.row_bytes = int64_t(d.hidden) * 2;
+    a.cap = recv_capacity;
+    a.slot_idx = topk_idx;
+    a.slot_w = topk_weights;
+    a.active = active;
+    a.recv_topk_idx = recv_topk_idx;
+    a.recv_topk_weights = recv_topk_weights;
+    a.slots = d.num_topk;
+    a.slot_E = d.num_experts;
+    a.slot_E_local = d.num_experts / d.num_ranks;
+    a.n_pieces = int(ceil_div(a.row_bytes, kDispatchPieceMax));
+    a.piece_bytes = uint32_t(round_up16(size_t(ceil_div(a.row_bytes, a.n_pieces))));
+    if (int64_t(a.n_pieces - 1) * a.piece_bytes >= a.row_bytes) return EP_ERR_UNSUPPORTED;
+    a.stage_bytes = uint32_t((a.piece_bytes + 127) & ~127u);
+    a.n_units = RT * a.n_pieces;
+    const int sms = sm_count();
+    if (sms <= 0) return EP_ERR_CUDA;
+    int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas) : int64_t(sms) * 2;
+    grid = std::max<int64_t>(1, std::min<int64_t>(grid, a.n_units));
+    const int ctas_per_sm = int(std::max<int64_t>(1, ceil_div(grid, sms)));
+    const int budget = std::max(1, max_smem_optin() / ctas_per_sm - 1024);
+    return launch_bulk_dispatch<true>(a, cfg, grid, budget, static_cast<cudaStream_t>(stream));
 }

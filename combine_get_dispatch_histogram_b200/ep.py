@@ -81,6 +81,12 @@ def load_library(path: str = LIB_PATH):
     lib.ep_dispatch_fp8.restype = ctypes.c_int
     lib.ep_dispatch_fp8_workspace_bytes.argtypes = [Dims, I32]
     lib.ep_dispatch_fp8_workspace_bytes.restype = SZ
+    lib.ep_normal_layout.argtypes = [Dims, I32, I32, P, P, P, P, P, P, P, Cfg, P]
+    lib.ep_normal_layout.restype = ctypes.c_int
+    lib.ep_normal_dispatch.argtypes = [Dims, I32, P, P, P, P, P, P, P, P, P, P, Cfg, P]
+    lib.ep_normal_dispatch.restype = ctypes.c_int
+    lib.ep_normal_combine.argtypes = [Dims, I32, P, P, P, P, P, Cfg, P]
+    lib.ep_normal_combine.restype = ctypes.c_int
     lib.ep_reroute_workspace_bytes.argtypes = [I32, I32, I32, I32]
     lib.ep_reroute_workspace_bytes.restype = SZ
     lib.ep_reroute.argtypes = [I32, I32, I32, I32, I32, P, P, SZ, P, P, P, P, P, Cfg, P]
@@ -405,3 +411,99 @@ def ep_layout_noalloc(topk_idx: torch.Tensor, active: torch.Tensor, num_experts:
                                    _ptr(out.pair_row), _ptr(out.status), _cfg(cfg), _stream(dev, stream))
     _check("ep_layout_noalloc", rc)
     return out
+
+
+# ----------------------------------------------------------------------------- normal (high-throughput) mode
+
+def ep_normal_layout(lay: DispatchLayout, num_experts: int, *, recv_capacity: Optional[int] = None,
+                     expert_alignment: int = 1, hidden: int = 8, out: Optional[dict] = None,
+                     status: Optional[torch.Tensor] = None, cfg=None, stream=None) -> dict:
+    """Receive rows of the normal mode from an ``ep_layout`` result (``ep_normal_layout``).
+
+    Returns ``token_recv_row`` [R, T, R], ``recv_tokens`` [R], ``num_recv_tokens_per_expert`` [E]
+    (rounded up to ``expert_alignment``), ``recv_capacity`` and ``status``.
+    """
+    lib = load_library()
+    itr = _need(lay.is_token_in_rank, "is_token_in_rank", torch.uint8)
+    R, T, _ = itr.shape
+    dev = itr.device
+    E = int(num_experts)
+    cap = R * T if recv_capacity is None else int(recv_capacity)
+    if out is None:
+        out = dict(token_recv_row=torch.empty((R, T, R), dtype=torch.int32, device=dev),
+                   recv_tokens=torch.empty(R, dtype=torch.int32, device=dev),
+                   num_recv_tokens_per_expert=torch.empty(E, dtype=torch.int32, device=dev))
+    _need(out["token_recv_row"], "token_recv_row", torch.int32, (R, T, R), dev)
+    _need(out["recv_tokens"], "recv_tokens", torch.int32, (R,), dev)
+    _need(out["num_recv_tokens_per_expert"], "num_recv_tokens_per_expert", torch.int32, (E,), dev)
+    out["status"] = lay.status if status is None else _need(status, "status", torch.int32, device=dev)
+    out["recv_capacity"] = cap
+    k = lay.pair_row.shape[2]
+    with torch.cuda.device(dev):
+        rc = lib.ep_normal_layout(Dims(R, T, k, E, hidden), cap, int(expert_alignment), _ptr(itr),
+                                  _ptr(lay.num_tokens_per_rank), _ptr(lay.recv_count), _ptr(out["token_recv_row"]),
+                                  _ptr(out["recv_tokens"]), _ptr(out["num_recv_tokens_per_expert"]),
+                                  _ptr(out["status"]), _cfg(cfg), _stream(dev, stream))
+    _check("ep_normal_layout", rc)
+    return out
+
+
+def ep_normal_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor, active: torch.Tensor,
+                       nl: dict, num_experts: int, *, out: Optional[dict] = None,
+                       status: Optional[torch.Tensor] = None, cfg=None, stream=None) -> dict:
+    """Send each token row once per destination rank (``ep_normal_dispatch``).
+
+    Returns ``recv_x`` [R, cap, H], ``recv_topk_idx`` / ``recv_topk_weights`` [R, cap, k],
+    ``src_info`` [R, cap, 2] and ``status``; rows past ``recv_tokens`` are untouched.
+    """
+    lib = load_library()
+    _need(x, "x", torch.bfloat16)
+    R, T, H = x.shape
+    dev = x.device
+    _need(topk_idx, "topk_idx", torch.int32, device=dev)
+    k = topk_idx.shape[2]
+    _need(topk_weights, "topk_weights", torch.float32, (R, T, k), dev)
+    _need(active, "active", torch.uint8, (R,), dev)
+    trr = _need(nl["token_recv_row"], "token_recv_row", torch.int32, (R, T, R), dev)
+    cap = int(nl["recv_capacity"])
+    if out is None:
+        out = dict(recv_x=torch.empty((R, cap, H), dtype=torch.bfloat16, device=dev),
+                   recv_topk_idx=torch.empty((R, cap, k), dtype=torch.int32, device=dev),
+                   recv_topk_weights=torch.empty((R, cap, k), dtype=torch.float32, device=dev),
+                   src_info=torch.empty((R, cap, 2), dtype=torch.int32, device=dev))
+    _need(out["recv_x"], "recv_x", torch.bfloat16, (R, cap, H), dev)
+    _need(out["recv_topk_idx"], "recv_topk_idx", torch.int32, (R, cap, k), dev)
+    _need(out["recv_topk_weights"], "recv_topk_weights", torch.float32, (R, cap, k), dev)
+    _need(out["src_info"], "src_info", torch.int32, (R, cap, 2), dev)
+    out["status"] = _status(dev, status)
+    with torch.cuda.device(dev):
+        rc = lib.ep_normal_dispatch(Dims(R, T, k, int(num_experts), H), cap, _ptr(x), _ptr(topk_idx),
+                                    _ptr(topk_weights), _ptr(active), _ptr(trr), _ptr(out["recv_x"]),
+                                    _ptr(out["recv_topk_idx"]), _ptr(out["recv_topk_weights"]), _ptr(out["src_info"]),
+                                    _ptr(out["status"]), _cfg(cfg), _stream(dev, stream))
+    _check("ep_normal_dispatch", rc)
+    return out
+
+
+def ep_normal_combine(y: torch.Tensor, nl: dict, active: torch.Tensor, num_experts: int, num_topk: int, *,
+                      out: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None, cfg=None,
+                      stream=None):
+    """Unweighted sum of the rows returned from every rank a token reached (``ep_normal_combine``)."""
+    lib = load_library()
+    _need(y, "y", torch.bfloat16)
+    R, cap, H = y.shape
+    dev = y.device
+    trr = _need(nl["token_recv_row"], "token_recv_row", torch.int32)
+    T = trr.shape[1]
+    if tuple(trr.shape) != (R, T, R) or cap != int(nl["recv_capacity"]):
+        raise ValueError("y does not match the normal layout")
+    _need(active, "active", torch.uint8, (R,), dev)
+    if out is None:
+        out = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (R, T, H), dev)
+    status = _status(dev, status)
+    with torch.cuda.device(dev):
+        rc = lib.ep_normal_combine(Dims(R, T, int(num_topk), int(num_experts), H), cap, _ptr(y), _ptr(trr),
+                                   _ptr(active), _ptr(out), _ptr(status), _cfg(cfg), _stream(dev, stream))
+    _check("ep_normal_combine", rc)
+    return out, status

@@ -20,8 +20,8 @@ from . import ep, inputs
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("--op", choices=["layout", "dispatch", "dispatch_fp8", "combine", "reroute", "step"],
-                    required=True)
+    ap.add_argument("--op", choices=["layout", "dispatch", "dispatch_fp8", "combine", "reroute", "step",
+                                     "normal_layout", "normal_dispatch", "normal_combine"], required=True)
     ap.add_argument("--scale-format", type=int, default=0, help="dispatch_fp8: 0 fp32, 1 power of two, 2 UE8M0")
     ap.add_argument("--workload", default="prefill")
     ap.add_argument("--iters", type=int, default=20)
@@ -34,7 +34,7 @@ def main():
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
     w = inputs.named(args.workload)
-    need_x = args.op in ("dispatch", "dispatch_fp8", "step")
+    need_x = args.op in ("dispatch", "dispatch_fp8", "step") or args.op.startswith("normal_")
     inp = inputs.make_inputs(w, tokens=need_x or args.op == "combine")
     R, T, k, H, E = w.num_ranks, w.num_tokens, w.num_topk, w.hidden, w.num_physical
     cap = R * T
@@ -62,6 +62,20 @@ def main():
     if args.op in ("layout", "step"):
         calls.append(lambda: ep.ep_layout(idx_phys, act, E, hidden=H, workspace=ws, out=lay, status=status,
                                           stream=stream, cfg=dict(variant=args.layout_variant)))
+    if args.op.startswith("normal_"):
+        nl = ep.ep_normal_layout(lay, E, status=status)
+        x = torch.from_numpy(inp.x.view(np.int16)).to(dev).view(torch.bfloat16)
+        wts = torch.from_numpy(inp.topk_weights).to(dev)
+        nd = ep.ep_normal_dispatch(x, idx_phys, wts, act, nl, E, status=status)
+        nout = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
+        if args.op == "normal_layout":
+            calls.append(lambda: ep.ep_normal_layout(lay, E, out=nl, status=status, stream=stream))
+        elif args.op == "normal_dispatch":
+            calls.append(lambda: ep.ep_normal_dispatch(x, idx_phys, wts, act, nl, E, out=nd, status=status,
+                                                       stream=stream, cfg=cfg))
+        else:
+            calls.append(lambda: ep.ep_normal_combine(nd["recv_x"], nl, act, E, k, out=nout, status=status,
+                                                      stream=stream, cfg=cfg))
     if args.op == "dispatch_fp8":
         x = torch.from_numpy(inp.x.view(np.int16)).to(dev).view(torch.bfloat16)
         ue = args.scale_format == ep.EP_FP8_SCALE_UE8M0
@@ -121,7 +135,10 @@ def main():
     per_pair = {"dispatch": 2 * H, "combine": 2 * H,
                 "dispatch_fp8": H + (H // 512 if args.scale_format == ep.EP_FP8_SCALE_UE8M0 else H // 32)}
     algo = None
-    if args.op in ("dispatch", "dispatch_fp8"):
+    if args.op in ("normal_dispatch", "normal_combine"):
+        sends = int(nl["recv_tokens"].sum().item())     # (token, destination rank) rows
+        algo = 2 * H * (sent + sends) if args.op == "normal_dispatch" else 2 * H * (sends + R * T)
+    elif args.op in ("dispatch", "dispatch_fp8"):
         algo = 2 * H * sent + per_pair[args.op] * live
     elif args.op == "combine":
         algo = 2 * H * (live + R * T)

@@ -90,7 +90,8 @@ enum {
 enum {
     EP_MAX_RANKS = 64,        /* is_token_in_rank is built from a 64-bit rank set */
     EP_MAX_TOPK = 32,         /* one lane per slot */
-    EP_MAX_EXPERTS = 8192     /* per-warp shared-memory histograms */
+    EP_MAX_EXPERTS = 8192,    /* per-warp shared-memory histograms */
+    EP_MAX_NORMAL_RANKS = 32  /* normal mode: one lane per destination rank */
 };
 
 /* Problem shape.  E % R == 0, H % 8 == 0 (rows move as 16-byte vectors),
@@ -288,6 +289,58 @@ EP_API int ep_combine(ep_dims_t d, const uint16_t *y, const int32_t *topk_idx,
                const float *topk_weights, const int32_t *pair_row,
                const uint8_t *active, uint16_t *out,
                int32_t *status, ep_cfg_t cfg, void *stream);
+
+/*
+ * Normal (high-throughput) mode -- Buffer.dispatch / Buffer.combine of the NeMo
+ * page: a token goes ONCE to every rank it has a live expert on
+ * (is_token_in_rank) and combine adds the returned rows WITHOUT weights.
+ * Rank d's receive buffer holds recv_capacity rows (the page's
+ * num_worst_tokens; R*T can never overflow); its received tokens are ordered
+ * by (source rank, token).  R <= EP_MAX_NORMAL_RANKS.
+ *
+ * ep_normal_layout -- receive rows from ep_layout's outputs.
+ * in:  is_token_in_rank uint8 [R,T,R], num_tokens_per_rank int32 [R,R],
+ *      recv_count int32 [E] (all from ep_layout), expert_alignment >= 1
+ * out: token_recv_row int32 [R,T,R]  row of (r,t) in rank d's buffer, -1 if not sent
+ *      recv_tokens    int32 [R]      tokens rank d receives (rows >= recv_capacity are
+ *                                    flagged EP_STATUS_OVERFLOW and never written)
+ *      num_recv_tokens_per_expert int32 [E]  recv_count rounded up to a multiple of
+ *                                    expert_alignment (the page's per-expert list)
+ */
+EP_API int ep_normal_layout(ep_dims_t d, int32_t recv_capacity, int32_t expert_alignment,
+                            const uint8_t *is_token_in_rank, const int32_t *num_tokens_per_rank,
+                            const int32_t *recv_count, int32_t *token_recv_row,
+                            int32_t *recv_tokens, int32_t *num_recv_tokens_per_expert,
+                            int32_t *status, ep_cfg_t cfg, void *stream);
+
+/*
+ * ep_normal_dispatch -- send each token row once per destination rank.
+ * in:  x bf16 [R,T,H], topk_idx int32 [R,T,k], topk_weights float [R,T,k], active uint8 [R]
+ *      (the mask ep_layout used), token_recv_row from ep_normal_layout
+ * out (rows [0, min(recv_tokens[d], recv_capacity)) of every rank d; others untouched):
+ *      recv_x            bf16 [R, recv_capacity, H]
+ *      recv_topk_idx     int32 [R, recv_capacity, k]  local expert id (e - d*E_local) where the
+ *                                                     slot's live expert is on rank d, else -1
+ *      recv_topk_weights float [R, recv_capacity, k]  the slot's weight there, else 0
+ *      src_info          int32 [R, recv_capacity, 2]  (src_rank, src_token)
+ */
+EP_API int ep_normal_dispatch(ep_dims_t d, int32_t recv_capacity, const uint16_t *x,
+                              const int32_t *topk_idx, const float *topk_weights,
+                              const uint8_t *active, const int32_t *token_recv_row,
+                              uint16_t *recv_x, int32_t *recv_topk_idx, float *recv_topk_weights,
+                              int32_t *src_info, int32_t *status, ep_cfg_t cfg, void *stream);
+
+/*
+ * ep_normal_combine -- unweighted reduce of the returned rows.
+ * in:  y bf16 [R, recv_capacity, H] (rank d's processed received tokens), token_recv_row,
+ *      active uint8 [R] (mask at combine time)
+ * out: out bf16 [R,T,H]: out[r,t] = bf16_rne(sum over d = 0..R-1, in that order, of
+ *      y[d][token_recv_row[r,t,d]]) in float32, over rows >= 0 and < recv_capacity with
+ *      active[d]; zeros for a source rank with active[r] == 0.
+ */
+EP_API int ep_normal_combine(ep_dims_t d, int32_t recv_capacity, const uint16_t *y,
+                             const int32_t *token_recv_row, const uint8_t *active, uint16_t *out,
+                             int32_t *status, ep_cfg_t cfg, void *stream);
 
 /* Bytes of device workspace ep_reroute needs. */
 EP_API size_t ep_reroute_workspace_bytes(int32_t num_ranks, int32_t num_tokens, int32_t num_topk,

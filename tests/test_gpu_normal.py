@@ -1,0 +1,97 @@
+"""GPU parity of the normal (high-throughput) mode against the CPU oracle: receive rows, per-expert
+counts, received rows and their local top-k (bit-exact), and the unweighted combine (tolerance)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_get_dispatch_histogram_b200 import ep, inputs
+from gpu_util import bf16_dev, bf16_host, check_close, dev, f32_dev, i32_dev, u8_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _free_memory():
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def run_normal(inp, E, alignment=1, capacity=None, active_combine=None, cfg=None, y=None):
+    idx, act = i32_dev(inp.topk_idx), u8_dev(inp.active)
+    H = inp.x.shape[2]
+    lay = ep.ep_layout(idx, act, E, hidden=H)
+    nl = ep.ep_normal_layout(lay, E, recv_capacity=capacity, expert_alignment=alignment)
+    nd = ep.ep_normal_dispatch(bf16_dev(inp.x), idx, f32_dev(inp.topk_weights), act, nl, E, status=lay.status,
+                               cfg=cfg)
+    act_c = act if active_combine is None else u8_dev(active_combine)
+    out, _ = ep.ep_normal_combine(nd["recv_x"] if y is None else y, nl, act_c, E, idx.shape[2], status=lay.status,
+                                  cfg=cfg)
+    torch.cuda.synchronize()
+    return lay, nl, nd, out
+
+
+def check_normal(inp, E, tag, alignment=1, capacity=None, active_combine=None, cfg=None):
+    R, T, k = inp.topk_idx.shape
+    ref_nl = oracle.normal_layout(inp.topk_idx, inp.active, E, alignment=alignment, capacity=capacity)
+    ref_nd = oracle.normal_dispatch(inp.x, inp.topk_idx, inp.topk_weights, inp.active, E, ref_nl)
+    lay, nl, nd, out = run_normal(inp, E, alignment, capacity, active_combine, cfg)
+    assert np.array_equal(nl["token_recv_row"].cpu().numpy(), ref_nl["token_recv_row"]), f"{tag} token_recv_row"
+    assert np.array_equal(nl["recv_tokens"].cpu().numpy(), ref_nl["recv_tokens"]), f"{tag} recv_tokens"
+    assert np.array_equal(nl["num_recv_tokens_per_expert"].cpu().numpy(), ref_nl["num_recv_tokens_per_expert"])
+    cap = ref_nl["capacity"]
+    for d in range(R):
+        n = min(int(ref_nl["recv_tokens"][d]), cap)
+        assert np.array_equal(bf16_host(nd["recv_x"][d, :n]), ref_nd["recv_x"][d, :n]), f"{tag} recv_x {d}"
+        assert np.array_equal(nd["recv_topk_idx"][d, :n].cpu().numpy(), ref_nd["recv_topk_idx"][d, :n])
+        assert np.array_equal(nd["recv_topk_weights"][d, :n].cpu().numpy(), ref_nd["recv_topk_weights"][d, :n])
+        assert np.array_equal(nd["src_info"][d, :n].cpu().numpy(), ref_nd["src_info"][d, :n])
+    want, _ = oracle.normal_combine(ref_nd["recv_x"], ref_nl["token_recv_row"],
+                                    inp.active if active_combine is None else active_combine)
+    check_close(bf16_host(out), want, f"{tag} combine")
+    st = int(nd["status"].item()) | int(lay.status.item())
+    assert bool(st & ep.EP_STATUS_OVERFLOW) == bool(ref_nl["status"] & oracle.OVERFLOW)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "sweep_T16_mask5", "sweep_T512", "replica_T256"])
+def test_normal_mode_matches_oracle(name):
+    w = inputs.replica(256) if name == "replica_T256" else inputs.named(name)
+    inp = inputs.make_inputs(w)
+    if w.num_extra:
+        phys = oracle.reroute(inp.topk_idx, w.num_experts, w.num_extra)["topk_idx_phys"]
+        inp = inputs.Inputs(phys, inp.topk_weights, inp.x, inp.active)
+    check_normal(inp, w.num_physical, name)
+
+
+@pytest.mark.parametrize("alignment", [1, 4, 128])
+def test_normal_mode_expert_alignment(alignment):
+    w = inputs.decode()
+    check_normal(inputs.make_inputs(w), w.num_experts, f"align {alignment}", alignment=alignment)
+
+
+@pytest.mark.parametrize("capacity", [0, 50, 300])
+def test_normal_mode_worst_tokens_capacity(capacity):
+    """A receive buffer smaller than a rank's traffic: overflow is flagged, rows past it never written."""
+    w = inputs.sweep(64)
+    check_normal(inputs.make_inputs(w), w.num_experts, f"cap {capacity}", capacity=capacity)
+
+
+@pytest.mark.parametrize("cfg", [dict(variant=1), dict(variant=2), dict(variant=1, max_ctas=3, stages=2)])
+def test_normal_mode_paths_and_mask_flip(cfg):
+    w = inputs.sweep(32, masked=True)
+    inp = inputs.make_inputs(w)
+    now = inp.active.copy()
+    now[2] = 0
+    check_normal(inp, w.num_experts, f"cfg {cfg}", active_combine=now, cfg=cfg)
+
+
+def test_normal_mode_sixteen_ranks_bulk_combine():
+    R, T, k, E, H = 16, 40, 4, 64, 512
+    rng = np.random.default_rng(16)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k).astype(np.int32)
+    x = inputs.bf16_tokens(rng, R * T, H).reshape(R, T, H)
+    wts = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+    act = np.ones(R, np.uint8)
+    act[7] = 0
+    check_normal(inputs.Inputs(idx, wts, x, act), E, "R=16")
