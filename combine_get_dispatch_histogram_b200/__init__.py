@@ -15,6 +15,8 @@ from .ep import (  # noqa: F401
     ep_normal_combine,
     ep_normal_dispatch,
     ep_normal_layout,
+    ep_replica_grad_reduce,
+    ep_replica_weight_sync,
     ep_reroute,
     ep_reroute_workspace_bytes,
     ep_strerror,

@@ -87,6 +87,10 @@ def load_library(path: str = LIB_PATH):
     lib.ep_normal_dispatch.restype = ctypes.c_int
     lib.ep_normal_combine.argtypes = [Dims, I32, P, P, P, P, P, Cfg, P]
     lib.ep_normal_combine.restype = ctypes.c_int
+    lib.ep_replica_weight_sync.argtypes = [I32, I32, P, ctypes.c_int64, P, P, P, Cfg, P]
+    lib.ep_replica_weight_sync.restype = ctypes.c_int
+    lib.ep_replica_grad_reduce.argtypes = [I32, I32, P, ctypes.c_int64, P, P, P, Cfg, P]
+    lib.ep_replica_grad_reduce.restype = ctypes.c_int
     lib.ep_reroute_workspace_bytes.argtypes = [I32, I32, I32, I32]
     lib.ep_reroute_workspace_bytes.restype = SZ
     lib.ep_reroute.argtypes = [I32, I32, I32, I32, I32, P, P, SZ, P, P, P, P, P, Cfg, P]
@@ -507,3 +511,49 @@ def ep_normal_combine(y: torch.Tensor, nl: dict, active: torch.Tensor, num_exper
                                    _ptr(active), _ptr(out), _ptr(status), _cfg(cfg), _stream(dev, stream))
     _check("ep_normal_combine", rc)
     return out, status
+
+
+# ----------------------------------------------------------------------------- replica weights / gradients
+
+def ep_replica_weight_sync(master: torch.Tensor, phys_base: torch.Tensor, *, replicas: Optional[torch.Tensor] = None,
+                           status: Optional[torch.Tensor] = None, cfg=None, stream=None) -> torch.Tensor:
+    """Copy each logical expert's parameters to its replicas (``ep_replica_weight_sync``)."""
+    lib = load_library()
+    if not master.is_cuda or not master.is_contiguous():
+        raise ValueError("master must be a contiguous CUDA tensor")
+    dev = master.device
+    E_log = master.shape[0]
+    _need(phys_base, "phys_base", torch.int32, (E_log + 1,), dev)
+    E_phys = int(phys_base[-1].item()) if replicas is None else replicas.shape[0]
+    if replicas is None:
+        replicas = torch.empty((E_phys,) + tuple(master.shape[1:]), dtype=master.dtype, device=dev)
+    if replicas.dtype != master.dtype or tuple(replicas.shape[1:]) != tuple(master.shape[1:]) or \
+            not replicas.is_contiguous():
+        raise ValueError("replicas must be contiguous [E_phys, ...] like master")
+    nbytes = master[0].numel() * master.element_size() if E_log else 0
+    with torch.cuda.device(dev):
+        rc = lib.ep_replica_weight_sync(E_log, replicas.shape[0], _ptr(phys_base), nbytes, _ptr(master),
+                                        _ptr(replicas), _ptr(_status(dev, status)), _cfg(cfg), _stream(dev, stream))
+    _check("ep_replica_weight_sync", rc)
+    return replicas
+
+
+def ep_replica_grad_reduce(replica_grads: torch.Tensor, phys_base: torch.Tensor, *,
+                           master_grads: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                           cfg=None, stream=None) -> torch.Tensor:
+    """Sum each logical expert's replica gradients into its master gradient (``ep_replica_grad_reduce``)."""
+    lib = load_library()
+    _need(replica_grads, "replica_grads", torch.float32)
+    dev = replica_grads.device
+    E_log = phys_base.shape[0] - 1
+    _need(phys_base, "phys_base", torch.int32, (E_log + 1,), dev)
+    P = replica_grads[0].numel() if replica_grads.shape[0] else 0
+    if master_grads is None:
+        master_grads = torch.empty((E_log,) + tuple(replica_grads.shape[1:]), dtype=torch.float32, device=dev)
+    _need(master_grads, "master_grads", torch.float32, (E_log,) + tuple(replica_grads.shape[1:]), dev)
+    with torch.cuda.device(dev):
+        rc = lib.ep_replica_grad_reduce(E_log, replica_grads.shape[0], _ptr(phys_base), P, _ptr(replica_grads),
+                                        _ptr(master_grads), _ptr(_status(dev, status)), _cfg(cfg),
+                                        _stream(dev, stream))
+    _check("ep_replica_grad_reduce", rc)
+    return master_grads

@@ -21,7 +21,9 @@ from . import ep, inputs
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--op", choices=["layout", "dispatch", "dispatch_fp8", "combine", "reroute", "step",
-                                     "normal_layout", "normal_dispatch", "normal_combine"], required=True)
+                                     "normal_layout", "normal_dispatch", "normal_combine", "weight_sync",
+                                     "grad_reduce"], required=True)
+    ap.add_argument("--params", type=int, default=1 << 22, help="weight_sync / grad_reduce: float32 params per expert")
     ap.add_argument("--scale-format", type=int, default=0, help="dispatch_fp8: 0 fp32, 1 power of two, 2 UE8M0")
     ap.add_argument("--workload", default="prefill")
     ap.add_argument("--iters", type=int, default=20)
@@ -62,6 +64,18 @@ def main():
     if args.op in ("layout", "step"):
         calls.append(lambda: ep.ep_layout(idx_phys, act, E, hidden=H, workspace=ws, out=lay, status=status,
                                           stream=stream, cfg=dict(variant=args.layout_variant)))
+    if args.op in ("weight_sync", "grad_reduce"):
+        if not w.num_extra:
+            raise SystemExit("weight_sync / grad_reduce need a workload with replicas (e.g. replica)")
+        pb = rr["phys_base"]
+        n_phys = w.num_physical
+        master = torch.randn((w.num_experts, args.params), device=dev)
+        reps = torch.randn((n_phys, args.params), device=dev)
+        if args.op == "weight_sync":
+            calls.append(lambda: ep.ep_replica_weight_sync(master, pb, replicas=reps, status=status, stream=stream))
+        else:
+            calls.append(lambda: ep.ep_replica_grad_reduce(reps, pb, master_grads=master, status=status,
+                                                           stream=stream))
     if args.op.startswith("normal_"):
         nl = ep.ep_normal_layout(lay, E, status=status)
         x = torch.from_numpy(inp.x.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -135,7 +149,9 @@ def main():
     per_pair = {"dispatch": 2 * H, "combine": 2 * H,
                 "dispatch_fp8": H + (H // 512 if args.scale_format == ep.EP_FP8_SCALE_UE8M0 else H // 32)}
     algo = None
-    if args.op in ("normal_dispatch", "normal_combine"):
+    if args.op in ("weight_sync", "grad_reduce"):
+        algo = 4 * args.params * (w.num_experts + w.num_physical)
+    elif args.op in ("normal_dispatch", "normal_combine"):
         sends = int(nl["recv_tokens"].sum().item())     # (token, destination rank) rows
         algo = 2 * H * (sent + sends) if args.op == "normal_dispatch" else 2 * H * (sends + R * T)
     elif args.op in ("dispatch", "dispatch_fp8"):

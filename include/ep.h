@@ -369,6 +369,28 @@ EP_API int ep_reroute(int32_t num_ranks, int32_t num_tokens, int32_t num_topk,
                int32_t *load, int32_t *num_replicas, int32_t *phys_base,
                int32_t *topk_idx_phys, int32_t *status, ep_cfg_t cfg, void *stream);
 
+/*
+ * Replica weight sync and replica gradient reduction -- the GPU operations of
+ * the GitDiagram page "dots-infra/ultraep architecture" around routing
+ * expansion.  Replica i of logical expert e is physical expert phys_base[e] + i
+ * (phys_base int32 [num_logical + 1], device, from ep_reroute).
+ *
+ * ep_replica_weight_sync: replicas[phys_base[e] + i] = master[e] for every
+ *   replica, as raw bytes.  master [num_logical, param_bytes], replicas
+ *   [num_physical, param_bytes]; param_bytes % 16 == 0, 16-byte aligned.
+ * ep_replica_grad_reduce: master_grads[e][j] = sum over the replicas of e, in
+ *   replica order, of replica_grads[p][j], accumulated in float32.
+ *   replica_grads float [num_physical, num_params], master_grads float
+ *   [num_logical, num_params]; num_params % 4 == 0, 16-byte aligned.
+ */
+EP_API int ep_replica_weight_sync(int32_t num_logical, int32_t num_physical, const int32_t *phys_base,
+                                  int64_t param_bytes, const void *master, void *replicas,
+                                  int32_t *status, ep_cfg_t cfg, void *stream);
+
+EP_API int ep_replica_grad_reduce(int32_t num_logical, int32_t num_physical, const int32_t *phys_base,
+                                  int64_t num_params, const float *replica_grads, float *master_grads,
+                                  int32_t *status, ep_cfg_t cfg, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

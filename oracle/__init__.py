@@ -75,6 +75,10 @@ def _bind(lib):
     lib.oracle_normal_dispatch.restype = I
     lib.oracle_normal_combine.argtypes = [I, I, I, I, P, P, P, P]
     lib.oracle_normal_combine.restype = I
+    lib.oracle_replica_weight_sync.argtypes = [I, P, I64, P, P]
+    lib.oracle_replica_weight_sync.restype = None
+    lib.oracle_replica_grad_reduce.argtypes = [I, P, I64, P, P]
+    lib.oracle_replica_grad_reduce.restype = None
     return lib
 
 
@@ -262,3 +266,28 @@ def normal_combine(y, token_recv_row, active_now, lib=None):
     st = lib.oracle_normal_combine(R, T, H, cap, _p(y), _p(np.ascontiguousarray(token_recv_row, np.int32)),
                                    _p(np.ascontiguousarray(active_now, np.uint8)), _p(out))
     return out, int(st)
+
+
+def replica_weight_sync(master: np.ndarray, phys_base: np.ndarray, lib=None) -> np.ndarray:
+    """master [E_log, ...] -> replicas [E_phys, ...]: every replica of e holds e's bytes."""
+    lib = lib or load()
+    master = np.ascontiguousarray(master)
+    phys_base = np.ascontiguousarray(phys_base, np.int32)
+    E_log = master.shape[0]
+    nbytes = master[0].nbytes if E_log else 0
+    reps = np.zeros((int(phys_base[-1]),) + master.shape[1:], master.dtype)
+    lib.oracle_replica_weight_sync(E_log, _p(phys_base), nbytes, _p(master.view(np.uint8)),
+                                   _p(reps.view(np.uint8)) if reps.size else None)
+    return reps
+
+
+def replica_grad_reduce(replica_grads: np.ndarray, phys_base: np.ndarray, lib=None) -> np.ndarray:
+    """replica_grads [E_phys, P] float32 -> master [E_log, P] float64 (sum over each expert's replicas)."""
+    lib = lib or load()
+    g = np.ascontiguousarray(replica_grads, np.float32)
+    phys_base = np.ascontiguousarray(phys_base, np.int32)
+    E_log = phys_base.shape[0] - 1
+    P = g.shape[1]
+    out = np.zeros((E_log, P), np.float64)
+    lib.oracle_replica_grad_reduce(E_log, _p(phys_base), P, _p(g), _p(out))
+    return out

@@ -491,3 +491,30 @@ int oracle_normal_combine(int R, int T, int H, int capacity, const uint16_t *y, 
         }
     return status;
 }
+
+/*
+ * Replica weight sync and replica gradient reduction ([P3] GPU operations:
+ * "Replica weight sync" copies master expert weights to the replicas before
+ * expert compute; "Replica gradient reduction" sums the replicas' gradients
+ * into the master gradients in backward).  Replica i of logical expert e is
+ * physical expert phys_base[e] + i (the routing expansion's numbering).
+ */
+
+/* replicas[phys_base[e] + i] = master[e], bytes copied as they are. */
+void oracle_replica_weight_sync(int E_log, const int32_t *phys_base, int64_t param_bytes, const uint8_t *master,
+                                uint8_t *replicas) {
+    for (int e = 0; e < E_log; e++)
+        for (int32_t p = phys_base[e]; p < phys_base[e + 1]; p++)
+            for (int64_t b = 0; b < param_bytes; b++) replicas[(int64_t)p * param_bytes + b] = master[(int64_t)e * param_bytes + b];
+}
+
+/* master[e][i] = sum over replicas, in replica order, of replica_grads[p][i] (float64). */
+void oracle_replica_grad_reduce(int E_log, const int32_t *phys_base, int64_t num_params, const float *replica_grads,
+                                double *master) {
+    for (int e = 0; e < E_log; e++)
+        for (int64_t i = 0; i < num_params; i++) {
+            double acc = 0.0;
+            for (int32_t p = phys_base[e]; p < phys_base[e + 1]; p++) acc += (double)replica_grads[(int64_t)p * num_params + i];
+            master[(int64_t)e * num_params + i] = acc;
+        }
+}

@@ -493,6 +493,30 @@ def pin_normal_dispatch_combine(lib):
         assert np.array_equal(out, want)
 
 
-ALL_PINS = [pin_normal_golden, pin_normal_bruteforce, pin_normal_dispatch_combine, pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
+# ----------------------------------------------------------------------------- replica weights / gradients
+
+def pin_replica_sync_and_reduce(lib):
+    # hand-worked: loads [4,2,1,1] with 3 extra replicas -> n_rep [3,2,1,1], phys_base [0,3,5,6,7]
+    pb = np.array([0, 3, 5, 6, 7], np.int32)
+    master = np.array([[1.5, -2.0], [0.25, 8.0], [3.0, 3.0], [-1.0, 0.0]], np.float32)
+    reps = oracle.replica_weight_sync(master, pb, lib=lib)
+    assert reps.tolist() == [[1.5, -2.0]] * 3 + [[0.25, 8.0]] * 2 + [[3.0, 3.0], [-1.0, 0.0]]
+    # gradients of the replicas: the master gradient is their sum, replica by replica
+    g = np.array([[1, 2], [10, 20], [100, 200], [0.5, 0.25], [0.5, 0.75], [7, 8], [-3, -4]], np.float32)
+    assert oracle.replica_grad_reduce(g, pb, lib=lib).tolist() == [[111, 222], [1, 1], [7, 8], [-3, -4]]
+    # identical replica gradients sum to n_rep times the gradient (exact for these values)
+    rng = np.random.default_rng(41)
+    n_rep = rng.integers(1, 5, size=9)
+    pb = np.concatenate([[0], np.cumsum(n_rep)]).astype(np.int32)
+    base = np.round(rng.standard_normal((9, 33)) * 64) / 64
+    g = np.repeat(base, n_rep, axis=0).astype(np.float32)
+    assert np.array_equal(oracle.replica_grad_reduce(g, pb, lib=lib), n_rep[:, None] * base)
+    # weight sync then an all-ones "gradient": every replica row is a copy of its master row
+    m = rng.standard_normal((9, 5)).astype(np.float32)
+    r = oracle.replica_weight_sync(m, pb, lib=lib)
+    assert np.array_equal(r, np.repeat(m, n_rep, axis=0))
+
+
+ALL_PINS = [pin_replica_sync_and_reduce, pin_normal_golden, pin_normal_bruteforce, pin_normal_dispatch_combine, pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
             pin_dispatch_golden, pin_dispatch_bijection, pin_combine_golden,
             pin_combine_special_cases, pin_combine_mask, pin_reroute_golden, pin_reroute_invariants]

@@ -58,6 +58,11 @@ MUTANTS = {
                                "num_recv_tokens_per_expert[e] = (n / alignment) * alignment;"),
     "normal_sent_any_rank": ("if (pair_is_live(e, r, E, E_local, active) && e / E_local == d) sent = 1;",
                              "if (pair_is_live(e, r, E, E_local, active)) sent = 1;"),
+    # replica weights / gradients
+    "grad_reduce_skips_last_replica": ("for (int32_t p = phys_base[e]; p < phys_base[e + 1]; p++) acc +=",
+                                       "for (int32_t p = phys_base[e]; p < phys_base[e + 1] - 1; p++) acc +="),
+    "weight_sync_shifted": ("replicas[(int64_t)p * param_bytes + b] = master[(int64_t)e * param_bytes + b];",
+                            "replicas[(int64_t)p * param_bytes + b] = master[(int64_t)(p - phys_base[e]) * param_bytes + b];"),
     # reroute
     "reroute_tie_highest": ("if (lhs > rhs) best = e;", "if (lhs >= rhs) best = e;"),
     "reroute_local_token": ("topk_phys[p] = phys_base[e] + (int32_t)(global_token % n_rep[e]);",
