@@ -136,6 +136,8 @@ __global__ void combine_kernel(CombineArgs a) {
         }
         mbar_init_fence();
     }
+    pdl_wait();  // nothing upstream is read before this
+    // no early trigger: a streaming grid lets its dependent launch only as it exits
     for (int i = threadIdx.x; i < a.R; i += blockDim.x) act[i] = a.active[i];
     __syncthreads();
 
@@ -238,6 +240,8 @@ constexpr int kVecKMax = 8;
 
 template <int U, bool NORMAL>
 __global__ void __launch_bounds__(256) combine_vec_kernel(CombineArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    // no early trigger: a streaming grid lets its dependent launch only as it exits
     __shared__ int32_t act[kActiveSlots];
     for (int i = threadIdx.x; i < a.R; i += blockDim.x) act[i] = a.active[i];
     __syncthreads();
@@ -324,7 +328,8 @@ int launch_combine_vec(const CombineArgs& a, const ep_cfg_t& cfg, int sms, cudaS
     if (cfg.max_ctas > 0) grid = std::min<int64_t>(grid, cfg.max_ctas);
     const int64_t warps_needed = ceil_div(int64_t(a.R) * a.T * ceil_div(a.row_bytes >> 4, 32 * U), 1);
     grid = std::max<int64_t>(1, std::min<int64_t>(grid, ceil_div(warps_needed, 8)));
-    combine_vec_kernel<U, NORMAL><<<unsigned(grid), 256, 0, stream>>>(a);
+    if (launch_pdl(combine_vec_kernel<U, NORMAL>, dim3(unsigned(grid)), dim3(256), 0, stream, a) != cudaSuccess)
+        return EP_ERR_CUDA;
     return launch_result();
 }
 
@@ -367,7 +372,9 @@ int run_combine(CombineArgs& a, const ep_cfg_t& cfg, int variant, cudaStream_t s
     int64_t grid = sms;
     if (cfg.max_ctas > 0) grid = std::min<int64_t>(grid, cfg.max_ctas);
     grid = std::min<int64_t>(grid, int64_t(a.R) * a.T);
-    combine_kernel<NORMAL><<<unsigned(grid), 32 * (1 + consumer_warps), smem, stream>>>(a);
+    if (launch_pdl(combine_kernel<NORMAL>, dim3(unsigned(grid)), dim3(32 * (1 + consumer_warps)), smem, stream, a) !=
+        cudaSuccess)
+        return EP_ERR_CUDA;
     return launch_result();
 }
 

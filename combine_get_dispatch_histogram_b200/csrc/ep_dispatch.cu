@@ -112,6 +112,8 @@ __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
         mbar_init_fence();
     }
     __syncwarp();
+    pdl_wait();  // nothing upstream is read before this
+    // no early trigger: a streaming grid lets its dependent launch only as it exits
 
     const int64_t first = blockIdx.x, step = gridDim.x;
     const int64_t my_n = first < a.n_units ? (a.n_units - 1 - first) / step + 1 : 0;
@@ -213,6 +215,8 @@ constexpr int kVecKMax = 8;
 
 template <int U>
 __global__ void __launch_bounds__(256) dispatch_vec_kernel(DispatchArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    // no early trigger: a streaming grid lets its dependent launch only as it exits
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
     const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -291,16 +295,17 @@ int launch_dispatch_vec(const DispatchArgs& a, const ep_cfg_t& cfg, int sms, cud
     if (cfg.max_ctas > 0) grid = std::min<int64_t>(grid, cfg.max_ctas);
     const int64_t units = (a.n_units / a.n_pieces) * ceil_div(a.row_bytes >> 4, 32 * U);
     grid = std::max<int64_t>(1, std::min<int64_t>(grid, ceil_div(units, 8)));
-    dispatch_vec_kernel<U><<<unsigned(grid), 256, 0, stream>>>(a);
+    if (launch_pdl(dispatch_vec_kernel<U>, dim3(unsigned(grid)), dim3(256), 0, stream, a) != cudaSuccess)
+        return EP_ERR_CUDA;
     return launch_result();
 }
 
 // ---------------------------------------------------------------------------
 // FP8 dispatch (ep_dispatch_fp8): the vector path with a per-128-channel e4m3
-// cast.  A unit is a token x 512 channels (four scale groups); each lane holds
-// 2 x 8 channels, so a half-warp holds exactly one group and its amax is a
-// shuffle-max over 16 lanes.  The cast is computed once per token row and the
-// codes (8 bytes per lane and half) and scales are stored to every live row.
+// cast.  A unit is a token x 512 channels (four scale groups); lane l owns 16
+// contiguous channels, so 8 lanes hold one group and its amax is a
+// shuffle-max over 8 lanes.  The cast is computed once per token row and the
+// codes (16 bytes per lane) are stored to every live row.
 struct DispatchFp8Args {
     const uint8_t* x;
     const int32_t* topk_idx;
@@ -361,11 +366,13 @@ __device__ __forceinline__ uint2 fp8_cast8(const float* f, float scale) {
 
 template <int FMT>
 __global__ void __launch_bounds__(256) dispatch_fp8_kernel(DispatchFp8Args a) {
+    pdl_wait();  // nothing upstream is read before this
+    // no early trigger: a streaming grid lets its dependent launch only as it exits
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
     const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int nvec = a.H >> 3;
-    constexpr int kPieceVec = 64;  // 512 channels
+    const int nvec = a.H >> 3;     // 16-byte bf16 vectors per row
+    constexpr int kPieceVec = 64;  // 512 channels per unit; lane l owns channels [16l, 16l + 16)
     const int np = (nvec + kPieceVec - 1) / kPieceVec;
     const int64_t n_units = a.n_tok * np;
     const int64_t q = n_units / warps, rem = n_units % warps;
@@ -402,60 +409,53 @@ __global__ void __launch_bounds__(256) dispatch_fp8_kernel(DispatchFp8Args a) {
             my_row = row;
         }
         if (mask == 0u) continue;
+        // 8 lanes x 16 channels = one 128-channel scale group: valid for all 8 lanes or none
+        const int v = pc * kPieceVec + 2 * lane;
+        const bool valid = v < nvec;
         const uint8_t* src = a.x + tok * int64_t(a.H) * 2;
-        uint2 code[2];
-        uint32_t ue[2] = {127u, 127u};
-        float scale[2] = {1.f, 1.f};
-        bool valid[2];
+        float f[16];
+        float amax = 0.f;
+        if (valid) {
 #pragma unroll
-        for (int uu = 0; uu < 2; ++uu) {
-            const int v = pc * kPieceVec + uu * 32 + lane;
-            valid[uu] = v < nvec;  // a half-warp is one whole 128-channel group: valid for all 16 or none
-            float f[8];
-            float amax = 0.f;
-            if (valid[uu]) {
-                const uint4 raw = ld_stream_v4(src + int64_t(v) * 16);
+            for (int h = 0; h < 2; ++h) {
+                const uint4 raw = ld_stream_v4(src + int64_t(v + h) * 16);
                 const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    f[2 * i] = __uint_as_float(wds[i] << 16);
-                    f[2 * i + 1] = __uint_as_float(wds[i] & 0xffff0000u);
+                    f[8 * h + 2 * i] = __uint_as_float(wds[i] << 16);
+                    f[8 * h + 2 * i + 1] = __uint_as_float(wds[i] & 0xffff0000u);
                 }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
             }
 #pragma unroll
-            for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-            scale[uu] = fp8_group_scale<FMT>(amax, &ue[uu]);
-            if (valid[uu]) code[uu] = fp8_cast8<FMT>(f, scale[uu]);
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
         }
-        // UE8M0: bytes of the piece's four groups (uu=0: lanes 0, 16; uu=1: lanes 0, 16) into one word
-        uint32_t ue_word = 0;
-        if (FMT == EP_FP8_SCALE_UE8M0) {
-            const uint32_t b1 = __shfl_sync(0xffffffffu, ue[0], 16);
-            const uint32_t b3 = __shfl_sync(0xffffffffu, ue[1], 16);
-            ue_word = ue[0] | (b1 << 8) | (ue[1] << 16) | (b3 << 24);
+#pragma unroll
+        for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        uint32_t ue = 127u;
+        const float scale = fp8_group_scale<FMT>(amax, &ue);
+        uint4 code = make_uint4(0, 0, 0, 0);
+        if (valid) {
+            const uint2 lo = fp8_cast8<FMT>(f, scale);
+            const uint2 hi = fp8_cast8<FMT>(f + 8, scale);
+            code = make_uint4(lo.x, lo.y, hi.x, hi.y);
         }
-        // the token's scales, once, row-major in the workspace
+        // the token's scales, once, row-major in the workspace (group = lane / 8 within the piece)
         uint32_t* ts = a.tok_scales + tok * a.words;
         if (FMT == EP_FP8_SCALE_UE8M0) {
-            if (lane == 0) ts[pc] = ue_word;
-        } else {
-#pragma unroll
-            for (int uu = 0; uu < 2; ++uu) {
-                const int v = pc * kPieceVec + uu * 32 + lane;
-                if (valid[uu] && (lane & 15) == 0) ts[v >> 4] = __float_as_uint(scale[uu]);  // 16 vectors per group
-            }
+            const uint32_t b1 = __shfl_sync(0xffffffffu, ue, 8);
+            const uint32_t b2 = __shfl_sync(0xffffffffu, ue, 16);
+            const uint32_t b3 = __shfl_sync(0xffffffffu, ue, 24);
+            if (lane == 0) ts[pc] = ue | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        } else if (valid && (lane & 7) == 0) {
+            ts[v >> 4] = __float_as_uint(scale);  // 16 vectors per group
         }
         for (int j = 0; j < a.k; ++j) {
             if (!((mask >> j) & 1u)) continue;
             const int e = __shfl_sync(0xffffffffu, my_e, j);
             const int row = __shfl_sync(0xffffffffu, my_row, j);
-            uint8_t* dst = a.codes + (int64_t(e) * a.cap + row) * a.H;
-#pragma unroll
-            for (int uu = 0; uu < 2; ++uu) {
-                const int v = pc * kPieceVec + uu * 32 + lane;
-                if (valid[uu]) *reinterpret_cast<uint2*>(dst + int64_t(v) * 8) = code[uu];
+            if (valid) {
+                uint8_t* dst = a.codes + (int64_t(e) * a.cap + row) * a.H;
+                st_global_v4(dst + int64_t(v) * 8, code);
             }
         }
     }
@@ -465,6 +465,8 @@ __global__ void __launch_bounds__(256) dispatch_fp8_kernel(DispatchFp8Args a) {
 // a thread owns one valid row, finds its token in src_info and copies that
 // token's scale words, so for each word the block's stores are contiguous.
 __global__ void __launch_bounds__(256) fp8_scale_writer_kernel(DispatchFp8Args a) {
+    pdl_wait();  // nothing upstream is read before this
+    // no early trigger: a streaming grid lets its dependent launch only as it exits
     const int e = blockIdx.y;
     const int64_t n = a.recv_count[e] < a.cap ? int64_t(a.recv_count[e]) : a.cap;
     const int64_t row = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -497,7 +499,8 @@ int launch_bulk_dispatch(DispatchArgs& a, const ep_cfg_t& cfg, int64_t grid, int
     if (cudaFuncSetAttribute(dispatch_kernel<NORMAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
         cudaSuccess)
         return EP_ERR_CUDA;
-    dispatch_kernel<NORMAL><<<unsigned(grid), 32, smem, stream>>>(a);
+    if (launch_pdl(dispatch_kernel<NORMAL>, dim3(unsigned(grid)), dim3(32), smem, stream, a) != cudaSuccess)
+        return EP_ERR_CUDA;
     return launch_result();
 }
 
@@ -554,13 +557,17 @@ extern "C" int ep_dispatch_fp8(ep_dims_t d, const uint16_t* x, const int32_t* to
     int64_t grid = int64_t(sms) * 4;
     if (cfg.max_ctas > 0) grid = cfg.max_ctas;
     grid = std::max<int64_t>(1, std::min<int64_t>(grid, ceil_div(units, 8)));
+    cudaError_t lerr;
     switch (scale_format) {
-        case EP_FP8_SCALE_F32: dispatch_fp8_kernel<EP_FP8_SCALE_F32><<<unsigned(grid), 256, 0, st>>>(a); break;
-        case EP_FP8_SCALE_POW2: dispatch_fp8_kernel<EP_FP8_SCALE_POW2><<<unsigned(grid), 256, 0, st>>>(a); break;
-        default: dispatch_fp8_kernel<EP_FP8_SCALE_UE8M0><<<unsigned(grid), 256, 0, st>>>(a); break;
+        case EP_FP8_SCALE_F32: lerr = launch_pdl(dispatch_fp8_kernel<EP_FP8_SCALE_F32>, dim3(unsigned(grid)), dim3(256), 0, st, a); break;
+        case EP_FP8_SCALE_POW2: lerr = launch_pdl(dispatch_fp8_kernel<EP_FP8_SCALE_POW2>, dim3(unsigned(grid)), dim3(256), 0, st, a); break;
+        default: lerr = launch_pdl(dispatch_fp8_kernel<EP_FP8_SCALE_UE8M0>, dim3(unsigned(grid)), dim3(256), 0, st, a); break;
     }
+    if (lerr != cudaSuccess) return EP_ERR_CUDA;
     if (ceil_div(RT, 256) > 65535 * 256LL || d.num_experts > 65535) return EP_ERR_UNSUPPORTED;
-    fp8_scale_writer_kernel<<<dim3(unsigned(ceil_div(RT, 256)), unsigned(d.num_experts)), 256, 0, st>>>(a);
+    if (launch_pdl(fp8_scale_writer_kernel, dim3(unsigned(ceil_div(RT, 256)), unsigned(d.num_experts)), dim3(256), 0, st,
+                   a) != cudaSuccess)
+        return EP_ERR_CUDA;
     return launch_result();
 }
 

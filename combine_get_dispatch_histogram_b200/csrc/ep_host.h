@@ -30,6 +30,27 @@ inline int check_dims(const ep_dims_t& d) {
     return EP_OK;
 }
 
+// Launch with programmatic dependent launch: the kernel may be scheduled while
+// the previous kernel in the stream is finishing, and must call pdl_wait()
+// before reading anything produced upstream.  Overlaps launch latency and
+// prologues across the back-to-back kernels of a layout -> dispatch -> combine
+// step.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, kernel, args...);
+}
+
 // Streaming-multiprocessor count of the current device (cached per device).
 int sm_count();
 

@@ -111,6 +111,8 @@ __device__ __forceinline__ bool pair_live(int e, int E, bool src_ok, const int32
 }
 
 __global__ void __launch_bounds__(32 * kMaxWarps) layout_count_kernel(LayoutArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
     extern __shared__ int32_t smem[];
     int32_t* act = smem;
     int32_t* tpr = smem + kActiveSlots;
@@ -173,6 +175,8 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_count_kernel(LayoutArgs
 
 // One CTA per 32 experts; warp w holds chunk rows [w*rpw, (w+1)*rpw) in registers.
 __global__ void __launch_bounds__(32 * kScanWarps) layout_scan_kernel(LayoutArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
     __shared__ int32_t seg[kScanWarps][32];
     __shared__ int32_t total[32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -234,6 +238,8 @@ __global__ void __launch_bounds__(32 * kScanWarps) layout_scan_kernel(LayoutArgs
 
 // Single CTA: the whole layout in one launch (small problems).
 __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(LayoutArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
     extern __shared__ int32_t smem[];
     constexpr int NW = kSmallThreads / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -341,6 +347,8 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
 }
 
 __global__ void __launch_bounds__(32 * kMaxWarps) layout_rank_kernel(LayoutArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
     extern __shared__ int32_t smem[];
     const int W = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int32_t* act = smem;
@@ -478,6 +486,8 @@ __device__ bool grid_barrier(uint64_t* flags, int G, uint64_t value, int32_t* st
 }
 
 __global__ void __launch_bounds__(32 * kMaxWarps) layout_fused_kernel(LayoutArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
     extern __shared__ int32_t smem[];
     __shared__ int32_t seg[kMaxWarps][32];
     __shared__ int32_t col_total[32];
@@ -791,7 +801,8 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
             cudaFuncSetAttribute(layout_single_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(smem)) != cudaSuccess)
             return EP_ERR_CUDA;
-        layout_single_cta_kernel<<<1, kSmallThreads, smem, s>>>(a);
+        if (launch_pdl(layout_single_cta_kernel, dim3(1), dim3(kSmallThreads), smem, s, a) != cudaSuccess)
+            return EP_ERR_CUDA;
         return launch_result();
     }
     if (path != EP_LAYOUT_CHUNKED) return EP_ERR_INVALID;
@@ -805,8 +816,10 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
         cudaFuncSetAttribute(layout_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(rank_smem)) !=
             cudaSuccess)
         return EP_ERR_CUDA;
-    layout_count_kernel<<<lg.G, 32 * kMaxWarps, count_smem, s>>>(a);
-    layout_scan_kernel<<<int(ceil_div(d.num_experts, 32)), 32 * kScanWarps, 0, s>>>(a);
-    layout_rank_kernel<<<lg.G, 32 * W, rank_smem, s>>>(a);
+    if (launch_pdl(layout_count_kernel, dim3(lg.G), dim3(32 * kMaxWarps), count_smem, s, a) != cudaSuccess ||
+        launch_pdl(layout_scan_kernel, dim3(unsigned(ceil_div(d.num_experts, 32))), dim3(32 * kScanWarps), 0, s, a) !=
+            cudaSuccess ||
+        launch_pdl(layout_rank_kernel, dim3(lg.G), dim3(32 * W), rank_smem, s, a) != cudaSuccess)
+        return EP_ERR_CUDA;
     return launch_result();
 }

@@ -66,6 +66,8 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
 }
 
 __global__ void __launch_bounds__(kNormalThreads) normal_layout_kernel(NormalLayoutArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
     __shared__ int32_t first_row[EP_MAX_RANKS];
     __shared__ int32_t warp_sums[32];
     const int r = blockIdx.x;
@@ -137,6 +139,8 @@ extern "C" int ep_normal_layout(ep_dims_t d, int32_t recv_capacity, int32_t expe
     a.E = d.num_experts;
     a.alignment = expert_alignment;
     a.capacity = recv_capacity;
-    normal_layout_kernel<<<d.num_ranks, kNormalThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    if (launch_pdl(normal_layout_kernel, dim3(d.num_ranks), dim3(kNormalThreads), 0, static_cast<cudaStream_t>(stream),
+                   a) != cudaSuccess)
+        return EP_ERR_CUDA;
     return launch_result();
 }

@@ -27,6 +27,8 @@ constexpr int kVecPerThread = 4;
 __global__ void __launch_bounds__(kReplicaThreads)
     replica_weight_sync_kernel(const int32_t* phys_base, int32_t num_physical, int64_t nvec,
                                int32_t* status, const uint4* master, uint4* replicas) {
+    pdl_wait();  // nothing upstream is read before this
+    // no early trigger: a streaming grid lets its dependent launch only as it exits
     const int e = blockIdx.y;
     int32_t p0 = phys_base[e], p1 = phys_base[e + 1];
     if (p0 < 0 || p1 > num_physical || p0 > p1) {  // a malformed phys_base: touch nothing
@@ -52,6 +54,8 @@ __global__ void __launch_bounds__(kReplicaThreads)
 __global__ void __launch_bounds__(kReplicaThreads)
     replica_grad_reduce_kernel(const int32_t* phys_base, int32_t num_physical, int64_t nvec,
                                int32_t* status, const float4* grads, float4* master) {
+    pdl_wait();  // nothing upstream is read before this
+    // no early trigger: a streaming grid lets its dependent launch only as it exits
     const int e = blockIdx.y;
     int32_t p0 = phys_base[e], p1 = phys_base[e + 1];
     if (p0 < 0 || p1 > num_physical || p0 > p1) {  // a malformed phys_base: touch nothing
@@ -111,10 +115,10 @@ extern "C" int ep_replica_weight_sync(int32_t num_logical, int32_t num_physical,
     const int64_t nvec = param_bytes / 16;
     const int64_t blocks = ceil_div(nvec, int64_t(kReplicaThreads) * kVecPerThread);
     if (blocks > 0x7fffffff) return EP_ERR_UNSUPPORTED;
-    replica_weight_sync_kernel<<<dim3(unsigned(blocks), unsigned(num_logical)), kReplicaThreads, 0,
-                                 static_cast<cudaStream_t>(stream)>>>(phys_base, num_physical, nvec, status,
-                                                                       static_cast<const uint4*>(master),
-                                                                       static_cast<uint4*>(replicas));
+    if (launch_pdl(replica_weight_sync_kernel, dim3(unsigned(blocks), unsigned(num_logical)), dim3(kReplicaThreads), 0,
+                   static_cast<cudaStream_t>(stream), phys_base, num_physical, nvec, status,
+                   static_cast<const uint4*>(master), static_cast<uint4*>(replicas)) != cudaSuccess)
+        return EP_ERR_CUDA;
     return launch_result();
 }
 
@@ -128,9 +132,10 @@ extern "C" int ep_replica_grad_reduce(int32_t num_logical, int32_t num_physical,
     const int64_t nvec = num_params / 4;
     const int64_t blocks = ceil_div(nvec, int64_t(kReplicaThreads) * kVecPerThread);
     if (blocks > 0x7fffffff) return EP_ERR_UNSUPPORTED;
-    replica_grad_reduce_kernel<<<dim3(unsigned(blocks), unsigned(num_logical)), kReplicaThreads, 0,
-                                 static_cast<cudaStream_t>(stream)>>>(phys_base, num_physical, nvec, status,
-                                                                       reinterpret_cast<const float4*>(replica_grads),
-                                                                       reinterpret_cast<float4*>(master_grads));
+    if (launch_pdl(replica_grad_reduce_kernel, dim3(unsigned(blocks), unsigned(num_logical)), dim3(kReplicaThreads), 0,
+                   static_cast<cudaStream_t>(stream), phys_base, num_physical, nvec, status,
+                   reinterpret_cast<const float4*>(replica_grads), reinterpret_cast<float4*>(master_grads)) !=
+        cudaSuccess)
+        return EP_ERR_CUDA;
     return launch_result();
 }

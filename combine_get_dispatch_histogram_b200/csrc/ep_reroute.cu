@@ -50,6 +50,8 @@ struct RerouteArgs {
 };
 
 __global__ void __launch_bounds__(kRerouteThreads) reroute_load_kernel(RerouteArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
     extern __shared__ int32_t hist[];
     for (int e = threadIdx.x; e < a.E_log; e += blockDim.x) hist[e] = 0;
     __syncthreads();
@@ -76,6 +78,8 @@ __device__ __forceinline__ bool better(int32_t la, int32_t na, int ia, int32_t l
 }
 
 __global__ void __launch_bounds__(kRerouteThreads) reroute_expand_kernel(RerouteArgs a, int n_partials) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
     extern __shared__ int32_t sm[];
     int32_t* load = sm;                  // [E_log]
     int32_t* n_rep = sm + a.E_log;       // [E_log]
@@ -198,7 +202,8 @@ extern "C" int ep_reroute(int32_t num_ranks, int32_t num_tokens, int32_t num_top
                                  int(smem2)) != cudaSuccess)
             return EP_ERR_CUDA;
     }
-    reroute_load_kernel<<<blocks, kRerouteThreads, smem1, s>>>(a);
-    reroute_expand_kernel<<<blocks, kRerouteThreads, smem2, s>>>(a, blocks);
+    if (launch_pdl(reroute_load_kernel, dim3(blocks), dim3(kRerouteThreads), smem1, s, a) != cudaSuccess ||
+        launch_pdl(reroute_expand_kernel, dim3(blocks), dim3(kRerouteThreads), smem2, s, a, blocks) != cudaSuccess)
+        return EP_ERR_CUDA;
     return launch_result();
 }
