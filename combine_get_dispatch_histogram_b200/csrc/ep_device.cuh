@@ -91,6 +91,12 @@ __device__ __forceinline__ void bulk_store(void* dst, uint32_t src_smem, uint32_
                  : "memory");
 }
 
+// Order this thread's ordinary shared-memory writes before later bulk copies
+// (async proxy) that read the same bytes.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // All but the newest N bulk groups of this thread have finished READING shared memory.
@@ -134,6 +140,28 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // exit still saves the launch gap.
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- named barriers
+
+// Barrier `id` (1..15; 0 is __syncthreads) over the first arrivals of `count`
+// threads, a multiple of 32; every thread of each participating warp calls it.
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// named_bar_sync that also returns whether any participating thread passed true.
+__device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
+    uint32_t any;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(any)
+        : "r"(uint32_t(pred)), "r"(id), "r"(count)
+        : "memory");
+    return any != 0;
 }
 
 // ---------------------------------------------------------------- misc

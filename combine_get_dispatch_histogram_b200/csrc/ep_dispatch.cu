@@ -31,8 +31,6 @@
 #include <algorithm>
 #include <cstdint>
 
-#include <cuda_fp8.h>
-
 #include "ep.h"
 #include "ep_device.cuh"
 #include "ep_host.h"
@@ -300,193 +298,6 @@ int launch_dispatch_vec(const DispatchArgs& a, const ep_cfg_t& cfg, int sms, cud
     return launch_result();
 }
 
-// ---------------------------------------------------------------------------
-// FP8 dispatch (ep_dispatch_fp8): the vector path with a per-128-channel e4m3
-// cast.  A unit is a token x 512 channels (four scale groups); lane l owns 16
-// contiguous channels, so 8 lanes hold one group and its amax is a
-// shuffle-max over 8 lanes.  The cast is computed once per token row and the
-// codes (16 bytes per lane) are stored to every live row.
-struct DispatchFp8Args {
-    const uint8_t* x;
-    const int32_t* topk_idx;
-    const int32_t* pair_row;
-    uint8_t* codes;
-    uint8_t* scales;       // column-major [E][words][cap]
-    uint32_t* tok_scales;  // workspace [n_tok][words]: fp32 scales, or UE8M0 words
-    const int32_t* recv_count;
-    int32_t* src_info;
-    int32_t* status;
-    int T, k, E, H, groups;
-    int words;             // scale words per row: H/128 (fp32) or H/512 (UE8M0)
-    int64_t cap;
-    int64_t n_tok;
-};
-
-template <int FMT>
-__device__ __forceinline__ float fp8_group_scale(float amax, uint32_t* ue8m0) {
-    if (FMT == EP_FP8_SCALE_F32) {
-        *ue8m0 = 127u;
-        return amax == 0.0f ? 1.0f : amax / 448.0f;
-    }
-    int e = 0;
-    if (amax != 0.0f) {
-        int f;
-        const float m = frexpf(amax / 448.0f, &f);  // amax/448 = m * 2^f, 0.5 <= m < 1
-        e = m == 0.5f ? f - 1 : f;                   // smallest e with 2^e >= amax/448
-        e = max(-127, min(127, e));
-    }
-    *ue8m0 = uint32_t(e + 127);
-    return ldexpf(1.0f, e);
-}
-
-// codes of x / scale.  A power-of-two scale divides exactly as a multiplication by
-// its reciprocal (also a power of two, exact), so those formats multiply.
-template <int FMT>
-__device__ __forceinline__ uint2 fp8_cast8(const float* f, float scale) {
-    float q[8];
-    if (FMT == EP_FP8_SCALE_F32) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = f[i] / scale;
-    } else {
-        const float inv = 1.0f / scale;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = f[i] * inv;
-    }
-    uint32_t w[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const __nv_fp8x2_storage_t lo =
-            __nv_cvt_float2_to_fp8x2(make_float2(q[4 * h], q[4 * h + 1]), __NV_SATFINITE, __NV_E4M3);
-        const __nv_fp8x2_storage_t hi =
-            __nv_cvt_float2_to_fp8x2(make_float2(q[4 * h + 2], q[4 * h + 3]), __NV_SATFINITE, __NV_E4M3);
-        w[h] = uint32_t(lo) | (uint32_t(hi) << 16);
-    }
-    return make_uint2(w[0], w[1]);
-}
-
-template <int FMT>
-__global__ void __launch_bounds__(256) dispatch_fp8_kernel(DispatchFp8Args a) {
-    pdl_wait();  // nothing upstream is read before this
-    // no early trigger: a streaming grid lets its dependent launch only as it exits
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t(gridDim.x) * blockDim.x) >> 5;
-    const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int nvec = a.H >> 3;     // 16-byte bf16 vectors per row
-    constexpr int kPieceVec = 64;  // 512 channels per unit; lane l owns channels [16l, 16l + 16)
-    const int np = (nvec + kPieceVec - 1) / kPieceVec;
-    const int64_t n_units = a.n_tok * np;
-    const int64_t q = n_units / warps, rem = n_units % warps;
-    const int64_t u0 = gw * q + (gw < rem ? gw : rem);
-    const int64_t u1 = u0 + q + (gw < rem ? 1 : 0);
-
-    int64_t cur_tok = -1;
-    uint32_t mask = 0;
-    int my_e = -1, my_row = -1;
-    for (int64_t u = u0; u < u1; ++u) {
-        const int64_t tok = u / np;
-        const int pc = int(u - tok * np);
-        if (tok != cur_tok) {
-            cur_tok = tok;
-            int e = -1, row = -1;
-            if (lane < a.k) {
-                const int64_t p = tok * a.k + lane;
-                e = __ldg(a.topk_idx + p);
-                row = __ldg(a.pair_row + p);
-            }
-            const bool valid_row = row >= 0 && row < a.cap;
-            const bool live = valid_row && e >= 0 && e < a.E;
-            if (lane < a.k && pc == 0) {
-                if (row >= a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
-                if (valid_row && !live) flag_status(a.status, EP_STATUS_BAD_EXPERT);
-                if (live) {
-                    const int src_rank = int(tok / a.T);
-                    reinterpret_cast<int2*>(a.src_info)[int64_t(e) * a.cap + row] =
-                        make_int2(src_rank, int(tok - int64_t(src_rank) * a.T));
-                }
-            }
-            mask = __ballot_sync(0xffffffffu, live);
-            my_e = live ? e : -1;
-            my_row = row;
-        }
-        if (mask == 0u) continue;
-        // 8 lanes x 16 channels = one 128-channel scale group: valid for all 8 lanes or none
-        const int v = pc * kPieceVec + 2 * lane;
-        const bool valid = v < nvec;
-        const uint8_t* src = a.x + tok * int64_t(a.H) * 2;
-        float f[16];
-        float amax = 0.f;
-        if (valid) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint4 raw = ld_stream_v4(src + int64_t(v + h) * 16);
-                const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    f[8 * h + 2 * i] = __uint_as_float(wds[i] << 16);
-                    f[8 * h + 2 * i + 1] = __uint_as_float(wds[i] & 0xffff0000u);
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
-        }
-#pragma unroll
-        for (int off = 4; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        uint32_t ue = 127u;
-        const float scale = fp8_group_scale<FMT>(amax, &ue);
-        uint4 code = make_uint4(0, 0, 0, 0);
-        if (valid) {
-            const uint2 lo = fp8_cast8<FMT>(f, scale);
-            const uint2 hi = fp8_cast8<FMT>(f + 8, scale);
-            code = make_uint4(lo.x, lo.y, hi.x, hi.y);
-        }
-        // the token's scales, once, row-major in the workspace (group = lane / 8 within the piece)
-        uint32_t* ts = a.tok_scales + tok * a.words;
-        if (FMT == EP_FP8_SCALE_UE8M0) {
-            const uint32_t b1 = __shfl_sync(0xffffffffu, ue, 8);
-            const uint32_t b2 = __shfl_sync(0xffffffffu, ue, 16);
-            const uint32_t b3 = __shfl_sync(0xffffffffu, ue, 24);
-            if (lane == 0) ts[pc] = ue | (b1 << 8) | (b2 << 16) | (b3 << 24);
-        } else if (valid && (lane & 7) == 0) {
-            ts[v >> 4] = __float_as_uint(scale);  // 16 vectors per group
-        }
-        for (int j = 0; j < a.k; ++j) {
-            if (!((mask >> j) & 1u)) continue;
-            const int e = __shfl_sync(0xffffffffu, my_e, j);
-            const int row = __shfl_sync(0xffffffffu, my_row, j);
-            if (valid) {
-                uint8_t* dst = a.codes + (int64_t(e) * a.cap + row) * a.H;
-                st_global_v4(dst + int64_t(v) * 8, code);
-            }
-        }
-    }
-}
-
-// Column-major scales: block (x, e) covers slab rows [x*256, x*256 + 256) of expert e;
-// a thread owns one valid row, finds its token in src_info and copies that
-// token's scale words, so for each word the block's stores are contiguous.
-__global__ void __launch_bounds__(256) fp8_scale_writer_kernel(DispatchFp8Args a) {
-    pdl_wait();  // nothing upstream is read before this
-    // no early trigger: a streaming grid lets its dependent launch only as it exits
-    const int e = blockIdx.y;
-    const int64_t n = a.recv_count[e] < a.cap ? int64_t(a.recv_count[e]) : a.cap;
-    const int64_t row = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (int64_t(blockIdx.x) * blockDim.x >= n) return;
-    const bool ok = row < n;
-    const uint32_t* ts = nullptr;
-    bool ok_src = false;
-    if (ok) {
-        const int2 src = reinterpret_cast<const int2*>(a.src_info)[int64_t(e) * a.cap + row];
-        const int64_t tok = int64_t(src.x) * a.T + src.y;
-        // a recv_count that does not belong to this dispatch could point at a stale row
-        ok_src = src.y >= 0 && src.y < a.T && tok >= 0 && tok < a.n_tok;
-        if (ok_src) ts = a.tok_scales + tok * a.words;
-        else flag_status(a.status, EP_STATUS_BAD_EXPERT);
-    }
-    uint32_t* out = reinterpret_cast<uint32_t*>(a.scales) + int64_t(e) * a.words * a.cap + row;
-    for (int wd = 0; wd < a.words; ++wd)
-        if (ok_src) out[int64_t(wd) * a.cap] = ts[wd];
-}
-
 // Stage count from the shared-memory budget, then the bulk-path launch.
 template <bool NORMAL>
 int launch_bulk_dispatch(DispatchArgs& a, const ep_cfg_t& cfg, int64_t grid, int budget, cudaStream_t stream) {
@@ -508,68 +319,6 @@ int launch_bulk_dispatch(DispatchArgs& a, const ep_cfg_t& cfg, int64_t grid, int
 }  // namespace ep
 
 using namespace ep;
-
-extern "C" size_t ep_dispatch_fp8_workspace_bytes(ep_dims_t d, int32_t scale_format) {
-    if (check_dims(d) != EP_OK || d.hidden % 128 != 0) return 0;
-    const int words = scale_format == EP_FP8_SCALE_UE8M0 ? d.hidden / 512 : d.hidden / 128;
-    return round_up16(size_t(d.num_ranks) * d.num_tokens * words * 4);
-}
-
-extern "C" int ep_dispatch_fp8(ep_dims_t d, const uint16_t* x, const int32_t* topk_idx, const int32_t* pair_row,
-                               const int32_t* recv_count, int32_t scale_format, void* workspace,
-                               size_t workspace_bytes, uint8_t* recv_x, void* recv_scales, int32_t* src_info,
-                               int32_t* status, ep_cfg_t cfg, void* stream) {
-    int rc = check_dims(d);
-    if (rc != EP_OK) return rc;
-    if (scale_format != EP_FP8_SCALE_F32 && scale_format != EP_FP8_SCALE_POW2 && scale_format != EP_FP8_SCALE_UE8M0)
-        return EP_ERR_INVALID;
-    if (d.hidden % 128 != 0 || (scale_format == EP_FP8_SCALE_UE8M0 && d.hidden % 512 != 0)) return EP_ERR_INVALID;
-    const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
-    if (RT == 0) return EP_OK;
-    if (!x || !topk_idx || !pair_row || !recv_count || !recv_x || !recv_scales || !src_info) return EP_ERR_INVALID;
-    const size_t need = ep_dispatch_fp8_workspace_bytes(d, scale_format);
-    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return EP_ERR_INVALID;
-    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(recv_x) & 7u) || (reinterpret_cast<uintptr_t>(recv_scales) & 3u) ||
-        (reinterpret_cast<uintptr_t>(src_info) & 7u))
-        return EP_ERR_INVALID;
-    DispatchFp8Args a;
-    a.x = reinterpret_cast<const uint8_t*>(x);
-    a.topk_idx = topk_idx;
-    a.pair_row = pair_row;
-    a.codes = recv_x;
-    a.scales = static_cast<uint8_t*>(recv_scales);
-    a.src_info = src_info;
-    a.status = status;
-    a.T = d.num_tokens;
-    a.k = d.num_topk;
-    a.E = d.num_experts;
-    a.H = d.hidden;
-    a.groups = d.hidden / 128;
-    a.words = scale_format == EP_FP8_SCALE_UE8M0 ? d.hidden / 512 : d.hidden / 128;
-    a.tok_scales = static_cast<uint32_t*>(workspace);
-    a.recv_count = recv_count;
-    a.cap = RT;
-    a.n_tok = RT;
-    const int sms = sm_count();
-    if (sms <= 0) return EP_ERR_CUDA;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int64_t units = RT * ceil_div(d.hidden / 8, 64);
-    int64_t grid = int64_t(sms) * 4;
-    if (cfg.max_ctas > 0) grid = cfg.max_ctas;
-    grid = std::max<int64_t>(1, std::min<int64_t>(grid, ceil_div(units, 8)));
-    cudaError_t lerr;
-    switch (scale_format) {
-        case EP_FP8_SCALE_F32: lerr = launch_pdl(dispatch_fp8_kernel<EP_FP8_SCALE_F32>, dim3(unsigned(grid)), dim3(256), 0, st, a); break;
-        case EP_FP8_SCALE_POW2: lerr = launch_pdl(dispatch_fp8_kernel<EP_FP8_SCALE_POW2>, dim3(unsigned(grid)), dim3(256), 0, st, a); break;
-        default: lerr = launch_pdl(dispatch_fp8_kernel<EP_FP8_SCALE_UE8M0>, dim3(unsigned(grid)), dim3(256), 0, st, a); break;
-    }
-    if (lerr != cudaSuccess) return EP_ERR_CUDA;
-    if (ceil_div(RT, 256) > 65535 * 256LL || d.num_experts > 65535) return EP_ERR_UNSUPPORTED;
-    if (launch_pdl(fp8_scale_writer_kernel, dim3(unsigned(ceil_div(RT, 256)), unsigned(d.num_experts)), dim3(256), 0, st,
-                   a) != cudaSuccess)
-        return EP_ERR_CUDA;
-    return launch_result();
-}
 
 extern "C" int ep_dispatch(ep_dims_t d, const uint16_t* x, const int32_t* topk_idx, const int32_t* pair_row,
                            uint16_t* recv_x, int32_t* src_info, int32_t* status, ep_cfg_t cfg, void* stream) {

@@ -7,12 +7,13 @@
 // (source rank, token): the row of token (r, t) on rank d is the number of
 // tokens before it, in that order, that rank d receives.
 //
-// One CTA per source rank r.  Its first row on rank d is the sum over r' < r
-// of num_tokens_per_rank[r'][d]; within the rank, each thread owns a run of
-// consecutive tokens, and a block-wide exclusive scan of the runs' counts
-// (warp shuffles, then the warp totals) gives each run its first row, for one
-// destination rank after another.  CTA 0 also writes recv_tokens and the
-// per-expert receive counts rounded up to expert_alignment.
+// One CTA per (source rank r, destination rank d).  Its first row on rank d is
+// the sum over r' < r of num_tokens_per_rank[r'][d]; it then walks rank r's
+// tokens in tiles of 1024, one token per thread: a ballot gives each token's
+// place among the warp's sent tokens, and every warp scans the 32 warp counts
+// of the tile (shared memory) to find its base.  CTAs (0, d) also write
+// recv_tokens[d], and CTA (0, 0) the per-expert receive counts rounded up to
+// expert_alignment.
 #include <algorithm>
 #include <cstdint>
 
@@ -37,74 +38,62 @@ struct NormalLayoutArgs {
     int64_t capacity;
 };
 
-// Exclusive prefix of v over the CTA's threads (in thread order); all threads must call.
-__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_sums) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int32_t inc = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int32_t t = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += t;
-    }
-    if (lane == 31) warp_sums[warp] = inc;
-    __syncthreads();
-    if (warp == 0) {
-        const int nw = blockDim.x >> 5;
-        int32_t w = lane < nw ? warp_sums[lane] : 0;
-        int32_t wi = w;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int32_t t = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += t;
-        }
-        if (lane < nw) warp_sums[lane] = wi - w;
-    }
-    __syncthreads();
-    const int32_t base = warp_sums[warp] + inc - v;
-    __syncthreads();
-    return base;
-}
-
 __global__ void __launch_bounds__(kNormalThreads) normal_layout_kernel(NormalLayoutArgs a) {
     pdl_wait();  // nothing upstream is read before this
     pdl_launch_dependents();
-    __shared__ int32_t first_row[EP_MAX_RANKS];
-    __shared__ int32_t warp_sums[32];
-    const int r = blockIdx.x;
-    for (int d = threadIdx.x; d < a.R; d += blockDim.x) {
-        int32_t s = 0;
-        for (int q = 0; q < r; ++q) s += a.num_tokens_per_rank[q * a.R + d];
-        first_row[d] = s;
-        if (r == 0) {
-            int32_t tot = 0;
-            for (int q = 0; q < a.R; ++q) tot += a.num_tokens_per_rank[q * a.R + d];
-            a.recv_tokens[d] = tot;
+    __shared__ int32_t warp_cnt[kNormalThreads / 32];
+    __shared__ int32_t first_row;
+    const int r = blockIdx.x, d = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int kWarps = kNormalThreads / 32;
+    if (warp == 0) {
+        // lane q holds num_tokens_per_rank[q][d]: ranks before r give the first row
+        const int32_t n = lane < a.R ? a.num_tokens_per_rank[lane * a.R + d] : 0;
+        int32_t before = lane < r ? n : 0, all = n;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            before += __shfl_xor_sync(0xffffffffu, before, o);
+            all += __shfl_xor_sync(0xffffffffu, all, o);
+        }
+        if (lane == 0) {
+            first_row = before;
+            if (r == 0) a.recv_tokens[d] = all;
         }
     }
-    if (r == 0) {
+    if (r == 0 && d == 0) {
         for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
             const int32_t n = a.recv_count[e];
             a.num_recv_tokens_per_expert[e] = ((n + a.alignment - 1) / a.alignment) * a.alignment;
         }
     }
     __syncthreads();
-    const int per = (a.T + blockDim.x - 1) / blockDim.x;
-    const int t0 = min(a.T, int(threadIdx.x) * per), t1 = min(a.T, t0 + per);
-    const uint8_t* itr = a.is_token_in_rank + int64_t(r) * a.T * a.R;
-    int32_t* rows = a.token_recv_row + int64_t(r) * a.T * a.R;
+    int32_t running = first_row;
+    const uint8_t* itr = a.is_token_in_rank + int64_t(r) * a.T * a.R + d;
+    int32_t* rows = a.token_recv_row + int64_t(r) * a.T * a.R + d;
     bool overflow = false;
-    for (int d = 0; d < a.R; ++d) {
-        int32_t c = 0;
-        for (int t = t0; t < t1; ++t) c += itr[int64_t(t) * a.R + d] != 0;
-        int32_t row = first_row[d] + block_exclusive_scan(c, warp_sums);
-        for (int t = t0; t < t1; ++t) {
-            const bool sent = itr[int64_t(t) * a.R + d] != 0;
-            rows[int64_t(t) * a.R + d] = sent ? row : -1;
-            if (sent) {
-                overflow |= row >= a.capacity;
-                ++row;
-            }
+    int64_t t = threadIdx.x;
+    bool sent = t < a.T && itr[t * a.R] != 0;
+    for (int64_t t0 = 0; t0 < a.T; t0 += kNormalThreads, t += kNormalThreads) {
+        const int64_t tn = t + kNormalThreads;
+        const bool sent_next = tn < a.T && itr[tn * a.R] != 0;  // one tile ahead
+        const uint32_t bal = __ballot_sync(0xffffffffu, sent);
+        if (lane == 0) warp_cnt[warp] = __popc(bal);
+        __syncthreads();
+        const int32_t c = lane < kWarps ? warp_cnt[lane] : 0;
+        int32_t inc = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
         }
+        const int32_t warp_base = __shfl_sync(0xffffffffu, inc - c, warp);
+        const int32_t tile_total = __shfl_sync(0xffffffffu, inc, 31);
+        const int32_t row = running + warp_base + __popc(bal & lanemask_lt());
+        if (t < a.T) rows[t * a.R] = sent ? row : -1;
+        overflow |= sent && row >= a.capacity;
+        running += tile_total;
+        sent = sent_next;
+        __syncthreads();  // warp_cnt is rewritten by the next tile
     }
     if (__syncthreads_or(overflow) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_OVERFLOW);
 }
@@ -139,7 +128,8 @@ extern "C" int ep_normal_layout(ep_dims_t d, int32_t recv_capacity, int32_t expe
     a.E = d.num_experts;
     a.alignment = expert_alignment;
     a.capacity = recv_capacity;
-    if (launch_pdl(normal_layout_kernel, dim3(d.num_ranks), dim3(kNormalThreads), 0, static_cast<cudaStream_t>(stream),
+    if (launch_pdl(normal_layout_kernel, dim3(d.num_ranks, d.num_ranks), dim3(kNormalThreads), 0,
+                   static_cast<cudaStream_t>(stream),
                    a) != cudaSuccess)
         return EP_ERR_CUDA;
     return launch_result();

@@ -249,7 +249,8 @@ enum {
  *   workspace    >= ep_dispatch_fp8_workspace_bytes(d, scale_format) bytes, 16-byte
  *                aligned; scratch (contents ignored on entry, undefined on return)
  * out:
- *   recv_x       uint8 [E,CAP,H]   e4m3 codes of every written row (8-byte aligned)
+ *   recv_x       uint8 [E,CAP,H]   e4m3 codes of every written row (8-byte aligned;
+ *                16-byte aligned for the bulk path)
  *   recv_scales  EP_FP8_SCALE_F32 / _POW2: float [E, H/128, CAP];
  *                EP_FP8_SCALE_UE8M0: int32 [E, H/512, CAP], byte j of word w is the
  *                UE8M0 scale of channel group 4w+j.  This is the [E, CAP, groups]
@@ -258,6 +259,11 @@ enum {
  * Rows not written keep their contents.  Two launches: the cast (codes to every
  * live row, each token's scales once to the workspace), then a scale writer that
  * fills the column-major scale tensor with coalesced stores.
+ * cfg.variant: EP_VARIANT_BULK stages each bf16 row in shared memory with a bulk
+ * copy and bulk-stores the code rows (needs 2*H <= 16384 and a 16-byte aligned
+ * recv_x, else EP_ERR_UNSUPPORTED); EP_VARIANT_VECTOR moves rows through
+ * registers; EP_VARIANT_AUTO takes the bulk path when it applies.  Both give the
+ * same bits.
  */
 EP_API int ep_dispatch_fp8(ep_dims_t d, const uint16_t *x, const int32_t *topk_idx,
                            const int32_t *pair_row, const int32_t *recv_count,

@@ -23,21 +23,24 @@ def _free_memory():
     torch.cuda.empty_cache()
 
 
-def run_fp8(inp, E, fmt):
+VARIANTS = [ep.EP_VARIANT_BULK, ep.EP_VARIANT_VECTOR]
+
+
+def run_fp8(inp, E, fmt, cfg=None):
     idx = i32_dev(inp.topk_idx)
     act = u8_dev(inp.active)
     lay = ep.ep_layout(idx, act, E, hidden=inp.x.shape[2])
     codes, scales, src, st = ep.ep_dispatch_fp8(bf16_dev(inp.x), idx, lay.pair_row, lay.recv_count, E, fmt,
-                                                status=lay.status)
+                                                status=lay.status, cfg=cfg)
     torch.cuda.synchronize()
     return lay, codes, scales, src, int(st.item())
 
 
-def check_fp8(inp, E, fmt, tag):
+def check_fp8(inp, E, fmt, tag, cfg=None):
     ref = oracle.layout(inp.topk_idx, inp.active, E)
     pow2 = fmt != ep.EP_FP8_SCALE_F32
     w_codes, w_scales, w_ue, _ = oracle.dispatch_fp8(inp.x, inp.topk_idx, ref, pow2)
-    lay, codes, scales, src, st = run_fp8(inp, E, fmt)
+    lay, codes, scales, src, st = run_fp8(inp, E, fmt, cfg)
     check_layout(lay, ref, tag)
     assert st == ref.status
     cap = codes.shape[1]
@@ -63,20 +66,47 @@ def check_fp8(inp, E, fmt, tag):
             assert np.array_equal(s.view(np.uint32), w_scales[a:a + n].view(np.uint32)), f"{tag} scales {e}"
 
 
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("fmt", FORMATS)
 @pytest.mark.parametrize("name", ["decode", "sweep_T64_mask5", "replica_T256"])
-def test_fp8_dispatch_matches_oracle(name, fmt):
+def test_fp8_dispatch_matches_oracle(name, fmt, variant):
     w = inputs.replica(256) if name == "replica_T256" else inputs.named(name)
     inp = inputs.make_inputs(w)
     if w.num_extra:
         phys = oracle.reroute(inp.topk_idx, w.num_experts, w.num_extra)["topk_idx_phys"]
         inp = inputs.Inputs(phys, inp.topk_weights, inp.x, inp.active)
-    check_fp8(inp, w.num_physical, fmt, f"{name} fmt {fmt}")
+    check_fp8(inp, w.num_physical, fmt, f"{name} fmt {fmt} variant {variant}", dict(variant=variant))
 
 
 @pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("launch", [dict(max_ctas=1), dict(max_ctas=3, stages=2), dict(max_ctas=5, stages=3),
+                                    dict(max_ctas=2, stages=8)])
+def test_fp8_bulk_ring_wraps(fmt, launch):
+    # few CTAs and a shallow ring: each CTA walks many rows, every stage and code buffer is
+    # reused many times, and seven consumer warps share each row (stages=2: fewer stages than
+    # consumer warps).
+    w = inputs.sweep(32, masked=True)
+    inp = inputs.make_inputs(w)
+    check_fp8(inp, w.num_experts, fmt, f"ring {launch} fmt {fmt}", dict(variant=ep.EP_VARIANT_BULK, **launch))
+
+
+def test_fp8_wide_row_falls_back_to_vector():
+    # a bf16 row of 2 * 8704 bytes does not fit one bulk stage: AUTO takes the vector path,
+    # an explicit bulk request is refused
+    w = inputs.Workload("h8704", 2, 24, 3, 8, 8704)
+    inp = inputs.make_inputs(w)
+    check_fp8(inp, w.num_experts, ep.EP_FP8_SCALE_UE8M0, "H=8704 auto")
+    idx = i32_dev(inp.topk_idx)
+    lay = ep.ep_layout(idx, u8_dev(inp.active), w.num_experts, hidden=w.hidden)
+    with pytest.raises(ep.EPError):
+        ep.ep_dispatch_fp8(bf16_dev(inp.x), idx, lay.pair_row, lay.recv_count, w.num_experts,
+                           ep.EP_FP8_SCALE_UE8M0, cfg=dict(variant=ep.EP_VARIANT_BULK))
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("fmt", FORMATS)
 @pytest.mark.parametrize("magnitude", [0.0, 1e-30, 1e-3, 1e3, 1e30])
-def test_fp8_dispatch_extreme_values(fmt, magnitude):
+def test_fp8_dispatch_extreme_values(fmt, magnitude, variant):
     R, T, k, E, H = 2, 24, 3, 8, 1024
     rng = np.random.default_rng(int(magnitude * 7) % 97 + fmt)
     idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k).astype(np.int32)
@@ -86,14 +116,15 @@ def test_fp8_dispatch_extreme_values(fmt, magnitude):
     bits = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     w = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
     inp = inputs.Inputs(idx, w, bits, np.ones(R, np.uint8))
-    check_fp8(inp, E, fmt, f"magnitude {magnitude} fmt {fmt}")
+    check_fp8(inp, E, fmt, f"magnitude {magnitude} fmt {fmt} variant {variant}", dict(variant=variant))
 
 
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("fmt", [ep.EP_FP8_SCALE_F32, ep.EP_FP8_SCALE_POW2])
-def test_fp8_dispatch_small_hidden(fmt):
+def test_fp8_dispatch_small_hidden(fmt, variant):
     w = inputs.Workload("h128", 4, 40, 2, 8, 128)
     inp = inputs.make_inputs(w)
-    check_fp8(inp, w.num_experts, fmt, f"H=128 fmt {fmt}")
+    check_fp8(inp, w.num_experts, fmt, f"H=128 fmt {fmt} variant {variant}", dict(variant=variant))
 
 
 def test_fp8_dispatch_rejects_bad_hidden():

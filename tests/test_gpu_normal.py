@@ -95,3 +95,18 @@ def test_normal_mode_sixteen_ranks_bulk_combine():
     act = np.ones(R, np.uint8)
     act[7] = 0
     check_normal(inputs.Inputs(idx, wts, x, act), E, "R=16")
+
+
+@pytest.mark.parametrize("R,T", [(8, 1024), (8, 1025), (32, 2500)])
+def test_normal_layout_token_tiles(R, T):
+    """The receive rows are scanned 1024 tokens at a time: one tile exactly, one more token, a ragged
+    third tile at the largest rank count."""
+    k, E, H = 4, 2 * R, 128
+    rng = np.random.default_rng(R * 10007 + T)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k).astype(np.int32)
+    idx[0, ::7, 1] = -1                       # some unselected slots
+    x = inputs.bf16_tokens(rng, R * T, H).reshape(R, T, H)
+    wts = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+    act = np.ones(R, np.uint8)
+    act[R - 2] = 0
+    check_normal(inputs.Inputs(idx, wts, x, act), E, f"R={R} T={T}")
