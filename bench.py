@@ -96,18 +96,68 @@ def profiled_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """SM clock and clock-event reasons sampled while the timed region runs.
+
+    NVML (the library nvidia-smi reads) is polled every 5 ms from a thread, so even a timed
+    region of a few tens of milliseconds yields several samples; without NVML it falls back to
+    ``nvidia-smi -lms 200``.  The GPU is found by its PCI address, so the sample is of the device
+    the timed kernels ran on.  Nothing is ever set: clocks are only read.
+    """
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits worth reporting (idle, application clocks and sync boost are not)
+    REASON_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                   0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+    PERIOD_S = 0.005
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, device=None):
         self.gpu_index = gpu_index
+        self.device = device
         self.proc = None
+        self.thread = None
+        self.samples = []
+        self.max_mhz = None
         self.path = os.path.join("/tmp", f"ep_bench_clocks_{os.getpid()}.csv")
 
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        if self.device is not None:
+            import torch
+
+            pr = torch.cuda.get_device_properties(self.device)
+            try:
+                return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(
+                    f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0")
+            except Exception:
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu_index)
+
+    def _poll(self, nv, h):
+        reasons_of = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), int(reasons_of(h))))
+            except Exception:
+                pass
+            self.stop.wait(self.PERIOD_S)
+
     def __enter__(self):
+        import threading
+
+        try:
+            nv, h = self._nvml_handle()
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -118,6 +168,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -127,6 +180,15 @@ class ClockSampler:
             self.fh.close()
 
     def summary(self):
+        if self.thread is not None:
+            if not self.samples:
+                return None
+            seen = 0
+            for _, bits in self.samples:
+                seen |= bits
+            return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                    "reasons": sorted(name for bit, name in self.REASON_BITS.items() if seen & bit),
+                    "samples": len(self.samples), "source": "nvml, every 5 ms"}
         if self.proc is None:
             return None
         rows = []
@@ -144,7 +206,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(float(r[2]) for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": "nvidia-smi, every 200 ms"}
 
 
 # ----------------------------------------------------------------------------- rank plumbing
@@ -293,7 +355,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
     rank_barrier(world, local_rank)
     torch.cuda.synchronize(dev)
-    sampler = ClockSampler(gpu_index_of(local_rank))
+    sampler = ClockSampler(gpu_index_of(local_rank), dev)
     with sampler, torch.cuda.stream(stream):
         t_start.record(stream)
         for i in range(args.steps):
