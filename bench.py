@@ -295,7 +295,8 @@ def run_ours(args, rank, world, local_rank):
                             torch.empty((R, T, k), dtype=torch.int32, device=dev), status)
     stream = torch.cuda.Stream(dev)
     n_ev = 4
-    launches_per_step = 5 + (2 if reroute else 0)  # layout 3, dispatch 1, combine 1 (+ reroute 2)
+    layout_launches = 3 if ep.ep_layout_path(R, T, k, E, H) == ep.EP_LAYOUT_CHUNKED else 1
+    launches_per_step = layout_launches + 2 + (2 if reroute else 0)  # layout, dispatch, combine (+ reroute 2)
 
     idx_phys = rr_out["topk_idx_phys"] if reroute else idx_log
 

@@ -12,6 +12,7 @@ from .ep import (  # noqa: F401
     ep_dispatch_fp8,
     ep_layout,
     ep_layout_workspace_bytes,
+    ep_layout_path,
     ep_normal_combine,
     ep_normal_dispatch,
     ep_normal_layout,

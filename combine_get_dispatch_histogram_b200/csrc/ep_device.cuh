@@ -164,6 +164,40 @@ __device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
     return any != 0;
 }
 
+// ---------------------------------------------------------------- thread-block clusters
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// Barrier over every thread of the cluster; writes before it (shared, distributed
+// shared and global memory) are visible to every thread of the cluster after it.
+// Every thread of every CTA of the cluster must call it.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `cta` of this cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t cta) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(cta));
+    return r;
+}
+
+__device__ __forceinline__ int32_t ld_dsmem_s32(uint32_t addr) {
+    int32_t v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ uint32_t lanemask_lt() {

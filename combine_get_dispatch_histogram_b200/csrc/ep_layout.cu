@@ -59,6 +59,11 @@ constexpr int kSmallThreads = 1024;
 constexpr int kSmallMaxPairs = 32768;
 constexpr int kSmallMaxExperts = 1024;
 constexpr int kSmallMaxRanks = 32;
+constexpr int kSmallAutoPairs = 2048;  // AUTO takes the single-CTA path up to here
+constexpr int kClusterMaxCtas = 16;     // a non-portable cluster size (8 is the portable limit)
+constexpr int kClusterPairsPerCta = 1024;
+constexpr int64_t kClusterMaxPairs = 65536;
+constexpr int64_t kClusterAutoPairs = 32768;  // AUTO takes the cluster path up to here
 constexpr int kMaxWarps = 16;
 constexpr int kBatch = 8;           // 32-pair steps whose loads are issued together
 constexpr int kActiveSlots = 64;    // shared copy of the active mask (EP_MAX_RANKS)
@@ -236,7 +241,19 @@ __global__ void __launch_bounds__(32 * kScanWarps) layout_scan_kernel(LayoutArgs
     }
 }
 
-// Single CTA: the whole layout in one launch (small problems).
+// Single CTA: the whole layout in one launch (small problems).  The NW / R warps
+// of rank r split its tokens into consecutive parts, in (rank, part) order.
+//  1. the warp's first pairs are loaded while the tables (active mask,
+//     rank_of) and the zeroed warp histograms are set up;
+//  2. each warp walks its part in 32-pair steps: a pair's row within the part is
+//     its expert's running count in the warp histogram plus the matching lanes
+//     below it (ballot match), kept in registers (parked in pair_row when the
+//     part is longer than one round of loads); with k a power of two a token's
+//     k slots sit in k aligned lanes, and an OR over them gives its destination
+//     ranks (is_token_in_rank, num_tokens_per_rank) in the same step;
+//  3. per expert, the warp histograms are scanned in (rank, part) order into
+//     each warp's first row;
+//  4. each live pair adds its warp's first row for its expert.
 __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(LayoutArgs a) {
     pdl_wait();  // nothing upstream is read before this
     pdl_launch_dependents();
@@ -247,10 +264,6 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
     int32_t* tpr = smem + kActiveSlots;                        // [R][R]
     int32_t* rank_of = tpr + kSmallMaxRanks * kSmallMaxRanks;   // [E]
     int32_t* whist = rank_of + a.E;                            // [NW][E]
-    load_tables(a, act, rank_of);
-    for (int i = threadIdx.x; i < NW * a.E; i += blockDim.x) whist[i] = 0;
-    for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) tpr[i] = 0;
-    __syncthreads();
 
     // warps per rank and this warp's token range (in (rank, token) order)
     const int wpr = NW / a.R;  // R <= 32
@@ -258,47 +271,85 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
     const bool has_rank = r < a.R;
     const int tw = (a.T + wpr - 1) / wpr;
     const int wt0 = has_rank ? min(a.T, part * tw) : 0, wt1 = has_rank ? min(a.T, wt0 + tw) : 0;
-    const bool src_ok = has_rank && act[r] != 0;
     const int64_t pbase = has_rank ? (int64_t(r) * a.T + wt0) * a.k : 0;
     const int32_t* base = a.topk_idx + pbase;
     int32_t* rows = a.pair_row + pbase;
     const int np = (wt1 - wt0) * a.k;
-    int32_t* mine = whist + warp * a.E;
+    const bool one_round = np <= 32 * kBatch;
 
-    bool bad = false;
-    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
-        int ev[kBatch];
+    int ev[kBatch];  // the first round's experts need no table: load them before the barrier
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int p = p0 + u * 32 + lane;
-            ev[u] = p < np ? __ldg(base + p) : -1;
+    for (int u = 0; u < kBatch; ++u) {
+        const int p = u * 32 + lane;
+        ev[u] = p < np ? __ldg(base + p) : -1;
+    }
+    load_tables(a, act, rank_of);
+    for (int i = threadIdx.x; i < NW * a.E; i += blockDim.x) whist[i] = 0;
+    for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) tpr[i] = 0;
+    __syncthreads();
+
+    const bool src_ok = has_rank && act[r] != 0;
+    int32_t* mine = whist + warp * a.E;
+    const uint32_t below = lanemask_lt();
+    const bool lanes_per_token = (a.k & (a.k - 1)) == 0;  // k divides 32: a token is k aligned lanes
+    bool bad = false;
+    int rk[kBatch];  // rows within the part of the last round's pairs (-1: not live)
+    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+        if (p0 > 0) {
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int p = p0 + u * 32 + lane;
+                ev[u] = p < np ? __ldg(base + p) : -1;
+            }
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
+            rk[u] = -1;
+            if (p0 + u * 32 >= np) break;  // the same for the whole warp
+            const int p = p0 + u * 32 + lane;
             const int e = ev[u];
             bad |= (e < -1 || e >= a.E);
             const bool live = pair_live(e, a.E, src_ok, rank_of);
             const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
-            if (live && lane == __ffs(m) - 1) mine[e] += __popc(m);
+            const int32_t b = live ? mine[e] : 0;
             __syncwarp();
+            if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
+            __syncwarp();
+            rk[u] = live ? b + __popc(m & below) : -1;
+            if (!one_round && p < np) rows[p] = rk[u];
+            if (lanes_per_token) {
+                uint32_t dst = live ? (1u << rank_of[e]) : 0u;
+                for (int o = 1; o < a.k; o <<= 1) dst |= __shfl_xor_sync(0xffffffffu, dst, o);
+                const bool head = p < np && (lane & (a.k - 1)) == 0;
+                if (head) {
+                    uint8_t* itr = a.is_token_in_rank + ((pbase + p) / a.k) * a.R;
+                    for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((dst >> d) & 1u);
+                }
+                for (int d = 0; d < a.R; ++d) {
+                    const int n = __popc(__ballot_sync(0xffffffffu, head && ((dst >> d) & 1u)));
+                    if (lane == 0 && n) atomicAdd(tpr + r * a.R + d, n);
+                }
+            }
         }
     }
-    // destination-rank set of each token of this warp's part
-    for (int t0 = wt0; t0 < wt1; t0 += 32) {
-        const int t = t0 + lane;
-        uint64_t ranks = 0;
-        if (t < wt1) {
-            const int32_t* tb = a.topk_idx + (int64_t(r) * a.T + t) * a.k;
-            for (int j = 0; j < a.k; ++j) {
-                const int e = __ldg(tb + j);
-                if (pair_live(e, a.E, src_ok, rank_of)) ranks |= 1ull << rank_of[e];
+    if (!lanes_per_token) {
+        // destination-rank set of each token of this warp's part, one token per lane
+        for (int t0 = wt0; t0 < wt1; t0 += 32) {
+            const int t = t0 + lane;
+            uint64_t ranks = 0;
+            if (t < wt1) {
+                const int32_t* tb = a.topk_idx + (int64_t(r) * a.T + t) * a.k;
+                for (int j = 0; j < a.k; ++j) {
+                    const int e = __ldg(tb + j);
+                    if (pair_live(e, a.E, src_ok, rank_of)) ranks |= 1ull << rank_of[e];
+                }
+                uint8_t* itr = a.is_token_in_rank + (int64_t(r) * a.T + t) * a.R;
+                for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
             }
-            uint8_t* itr = a.is_token_in_rank + (int64_t(r) * a.T + t) * a.R;
-            for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
-        }
-        for (int d = 0; d < a.R; ++d) {
-            const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
-            if (lane == 0 && n) atomicAdd(tpr + r * a.R + d, n);
+            for (int d = 0; d < a.R; ++d) {
+                const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
+                if (lane == 0 && n) atomicAdd(tpr + r * a.R + d, n);
+            }
         }
     }
     if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
@@ -322,26 +373,200 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
     for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) a.num_tokens_per_rank[i] = tpr[i];
     __syncthreads();
 
-    const uint32_t below = lanemask_lt();
-    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
-        int ev[kBatch];
+    // rows = the warp's first row for the expert + the row within the part
+    if (one_round) {
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
-            const int p = p0 + u * 32 + lane;
-            ev[u] = p < np ? __ldg(base + p) : -1;
+            const int p = u * 32 + lane;
+            if (u * 32 >= np) break;
+            if (p < np) rows[p] = rk[u] >= 0 ? mine[ev[u]] + rk[u] : -1;
+        }
+    } else {
+        for (int p = lane; p < np; p += 32) {
+            const int32_t q = rows[p];  // written by this thread in step 2
+            if (q >= 0) rows[p] = mine[__ldg(base + p)] + q;
+        }
+    }
+}
+
+// Cluster path (EP_LAYOUT_CLUSTER): the single-CTA algorithm over a thread-block
+// cluster of CL CTAs, one per SM, whose shared memories are reachable from one
+// another.  The cluster's CL * 32 warps split each rank's tokens as the single
+// CTA's warps do (global warp g = CTA * 32 + warp, in (rank, part) order):
+//  1. each warp walks its part as in the single-CTA path (row within the part,
+//     destination ranks), into its CTA's shared memory;
+//  2. each CTA scans its own warps' histograms per expert and keeps its totals;
+//     after a cluster barrier, its first row per expert is the sum of the totals
+//     of the CTAs before it, read from their shared memory; the CTA holding a
+//     rank's first warp writes that rank's expert_rank_offset, the last CTA
+//     recv_count, CTA 0 the sum of every CTA's num_tokens_per_rank;
+//  3. each live pair's row is its CTA's first row + its warp's first row within
+//     the CTA + its row within the part;
+//  4. after a second cluster barrier (no shared memory is read across CTAs
+//     past it), the rank owners take num_tokens_per_expert from neighbouring
+//     offsets.
+__global__ void __launch_bounds__(kSmallThreads) layout_cluster_kernel(LayoutArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
+    extern __shared__ int32_t smem[];
+    constexpr int NW = kSmallThreads / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cta = int(cluster_ctarank()), CL = int(cluster_nctarank());
+    int32_t* act = smem;
+    int32_t* tpr = smem + kActiveSlots;                        // [R][R], this CTA's tokens
+    int32_t* rank_of = tpr + kSmallMaxRanks * kSmallMaxRanks;   // [E]
+    int32_t* ctot = rank_of + a.E;                             // [E] this CTA's live pairs per expert
+    int32_t* cbase = ctot + a.E;                               // [E] this CTA's first row per expert
+    int32_t* whist = cbase + a.E;                              // [NW][E]
+
+    // warps per rank and this warp's token range (in (rank, token) order)
+    const int wpr = CL * NW / a.R;  // R <= 32 <= CL * NW
+    const int gw = cta * NW + warp;
+    const int r = gw / wpr, part = gw - r * wpr;
+    const bool has_rank = r < a.R;
+    const int tw = (a.T + wpr - 1) / wpr;
+    const int wt0 = has_rank ? min(a.T, part * tw) : 0, wt1 = has_rank ? min(a.T, wt0 + tw) : 0;
+    const int64_t pbase = has_rank ? (int64_t(r) * a.T + wt0) * a.k : 0;
+    const int32_t* base = a.topk_idx + pbase;
+    int32_t* rows = a.pair_row + pbase;
+    const int np = (wt1 - wt0) * a.k;
+    const bool one_round = np <= 32 * kBatch;
+
+    int ev[kBatch];  // the first round's experts need no table: load them before the barrier
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+        const int p = u * 32 + lane;
+        ev[u] = p < np ? __ldg(base + p) : -1;
+    }
+    load_tables(a, act, rank_of);
+    for (int i = threadIdx.x; i < NW * a.E; i += blockDim.x) whist[i] = 0;
+    for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) tpr[i] = 0;
+    __syncthreads();
+
+    const bool src_ok = has_rank && act[r] != 0;
+    int32_t* mine = whist + warp * a.E;
+    const uint32_t below = lanemask_lt();
+    const bool lanes_per_token = (a.k & (a.k - 1)) == 0;  // k divides 32: a token is k aligned lanes
+    bool bad = false;
+    int rk[kBatch];  // rows within the part of the last round's pairs (-1: not live)
+    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+        if (p0 > 0) {
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int p = p0 + u * 32 + lane;
+                ev[u] = p < np ? __ldg(base + p) : -1;
+            }
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
+            rk[u] = -1;
+            if (p0 + u * 32 >= np) break;  // the same for the whole warp
             const int p = p0 + u * 32 + lane;
-            if (p0 + u * 32 >= np) break;
             const int e = ev[u];
+            bad |= (e < -1 || e >= a.E);
             const bool live = pair_live(e, a.E, src_ok, rank_of);
             const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
             const int32_t b = live ? mine[e] : 0;
             __syncwarp();
             if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
             __syncwarp();
-            if (p < np) rows[p] = live ? b + __popc(m & below) : -1;
+            rk[u] = live ? b + __popc(m & below) : -1;
+            if (!one_round && p < np) rows[p] = rk[u];
+            if (lanes_per_token) {
+                uint32_t dst = live ? (1u << rank_of[e]) : 0u;
+                for (int o = 1; o < a.k; o <<= 1) dst |= __shfl_xor_sync(0xffffffffu, dst, o);
+                const bool head = p < np && (lane & (a.k - 1)) == 0;
+                if (head) {
+                    uint8_t* itr = a.is_token_in_rank + ((pbase + p) / a.k) * a.R;
+                    for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((dst >> d) & 1u);
+                }
+                for (int d = 0; d < a.R; ++d) {
+                    const int n = __popc(__ballot_sync(0xffffffffu, head && ((dst >> d) & 1u)));
+                    if (lane == 0 && n) atomicAdd(tpr + r * a.R + d, n);
+                }
+            }
+        }
+    }
+    if (!lanes_per_token) {
+        for (int t0 = wt0; t0 < wt1; t0 += 32) {
+            const int t = t0 + lane;
+            uint64_t ranks = 0;
+            if (t < wt1) {
+                const int32_t* tb = a.topk_idx + (int64_t(r) * a.T + t) * a.k;
+                for (int j = 0; j < a.k; ++j) {
+                    const int e = __ldg(tb + j);
+                    if (pair_live(e, a.E, src_ok, rank_of)) ranks |= 1ull << rank_of[e];
+                }
+                uint8_t* itr = a.is_token_in_rank + (int64_t(r) * a.T + t) * a.R;
+                for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
+            }
+            for (int d = 0; d < a.R; ++d) {
+                const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
+                if (lane == 0 && n) atomicAdd(tpr + r * a.R + d, n);
+            }
+        }
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
+
+    // this CTA's warps, scanned per expert in warp order; ctot = the CTA's total
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        int32_t run = 0;
+        for (int w = 0; w < NW; ++w) {
+            const int32_t c = whist[w * a.E + e];
+            whist[w * a.E + e] = run;
+            run += c;
+        }
+        ctot[e] = run;
+    }
+    cluster_sync();  // every CTA's ctot and tpr are final
+
+    // ranks whose first warp (rank * wpr) is in this CTA
+    const int r_lo = (cta * NW + wpr - 1) / wpr;
+    const int r_hi = min(a.R, ((cta + 1) * NW + wpr - 1) / wpr);
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        int32_t b = 0;
+        for (int c = 0; c < cta; ++c) b += ld_dsmem_s32(dsmem_addr(ctot + e, uint32_t(c)));
+        cbase[e] = b;
+        for (int rr = r_lo; rr < r_hi; ++rr)
+            a.expert_rank_offset[int64_t(e) * a.R + rr] = b + whist[(rr * wpr - cta * NW) * a.E + e];
+        if (cta == CL - 1) {
+            const int32_t n = b + ctot[e];
+            a.recv_count[e] = n;
+            if (n > a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
+        }
+    }
+    if (cta == 0) {
+        for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) {
+            int32_t n = 0;
+            for (int c = 0; c < CL; ++c) n += ld_dsmem_s32(dsmem_addr(tpr + i, uint32_t(c)));
+            a.num_tokens_per_rank[i] = n;
+        }
+    }
+    __syncthreads();  // cbase
+
+    if (one_round) {
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = u * 32 + lane;
+            if (u * 32 >= np) break;
+            if (p < np) rows[p] = rk[u] >= 0 ? cbase[ev[u]] + mine[ev[u]] + rk[u] : -1;
+        }
+    } else {
+        for (int p = lane; p < np; p += 32) {
+            const int32_t q = rows[p];  // written by this thread in step 1
+            if (q >= 0) {
+                const int e = __ldg(base + p);
+                rows[p] = cbase[e] + mine[e] + q;
+            }
+        }
+    }
+    cluster_sync();  // expert_rank_offset and recv_count are written; no remote shared reads after this
+
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        for (int rr = r_lo; rr < r_hi; ++rr) {
+            const int32_t off = cbase[e] + whist[(rr * wpr - cta * NW) * a.E + e];
+            const int32_t next = rr + 1 < a.R ? a.expert_rank_offset[int64_t(e) * a.R + rr + 1] : a.recv_count[e];
+            a.num_tokens_per_expert[int64_t(rr) * a.E + e] = next - off;
         }
     }
 }
@@ -716,6 +941,87 @@ int fused_capacity(int threads, size_t smem) {
 
 using namespace ep;
 
+namespace ep {
+namespace {
+
+size_t cluster_smem_bytes(const ep_dims_t& d) {
+    return size_t(kActiveSlots + kSmallMaxRanks * kSmallMaxRanks + 3 * d.num_experts +
+                  (kSmallThreads / 32) * d.num_experts) * 4;
+}
+
+// CTAs of the layout cluster for `pairs` pairs: one per kClusterPairsPerCta, at
+// least 2, at most kClusterMaxCtas, and no more than the device can hold at once
+// (asked of the occupancy calculator once per size and cached).
+int cluster_ctas(int64_t pairs, size_t smem) {
+    static int max_ok[kClusterMaxCtas + 1] = {};  // 0 unknown, 1 fits, -1 does not
+    int cl = int(std::min<int64_t>(kClusterMaxCtas, std::max<int64_t>(2, ceil_div(pairs, kClusterPairsPerCta))));
+    for (; cl >= 2; cl = cl > 8 ? 8 : cl / 2) {
+        if (max_ok[cl] == 0) {
+            cudaLaunchConfig_t lc = {};
+            lc.gridDim = dim3(cl);
+            lc.blockDim = dim3(kSmallThreads);
+            lc.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = cl;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            lc.attrs = attr;
+            lc.numAttrs = 1;
+            int n = 0;
+            const bool ok = cudaOccupancyMaxActiveClusters(&n, layout_cluster_kernel, &lc) == cudaSuccess && n >= 1;
+            if (!ok) cudaGetLastError();
+            max_ok[cl] = ok ? 1 : -1;
+        }
+        if (max_ok[cl] > 0) return cl;
+    }
+    return 1;
+}
+
+size_t fused_smem_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
+    return size_t(2 * kActiveSlots + 2 * d.num_experts + lg.warps * d.num_experts) * 4;
+}
+
+// The path ep_layout takes for these dims and cfg, or a negative EP_ERR_* code.
+// AUTO, from graph replays on B200: one CTA up to kSmallAutoPairs pairs (8.6 us at 1024
+// pairs, 10.6 us at 2048); a cluster up to kClusterAutoPairs (10.6 us from 4096 to 16384
+// pairs, 12.7 us at 32768, where one CTA takes 14.7 to 74 us); the chunked path beyond
+// (about 17 to 19 us), which also beats the fused one (cooperative launch plus two grid
+// barriers, about 19 us).
+int resolve_layout_path(const ep_dims_t& d, const ep_cfg_t& cfg, const LayoutGeom& lg) {
+    const int64_t pairs = int64_t(d.num_ranks) * d.num_tokens * d.num_topk;
+    const bool tables_fit = d.num_ranks <= kSmallMaxRanks && d.num_experts <= kSmallMaxExperts;
+    const bool small_ok = tables_fit && pairs <= kSmallMaxPairs;
+    const bool cluster_ok = tables_fit && pairs <= kClusterMaxPairs;
+    switch (cfg.variant) {
+        case EP_VARIANT_AUTO:
+            if (small_ok && pairs <= kSmallAutoPairs) return EP_LAYOUT_SINGLE_CTA;
+            if (cluster_ok && pairs <= kClusterAutoPairs) return EP_LAYOUT_CLUSTER;
+            return EP_LAYOUT_CHUNKED;
+        case EP_LAYOUT_CHUNKED:
+            return EP_LAYOUT_CHUNKED;
+        case EP_LAYOUT_SINGLE_CTA:
+            return small_ok ? int(EP_LAYOUT_SINGLE_CTA) : int(EP_ERR_UNSUPPORTED);
+        case EP_LAYOUT_FUSED:
+            return lg.G <= kMaxFlags && lg.G <= fused_capacity(32 * lg.warps, fused_smem_bytes(d, lg))
+                       ? int(EP_LAYOUT_FUSED)
+                       : int(EP_ERR_UNSUPPORTED);
+        case EP_LAYOUT_CLUSTER:
+            return cluster_ok ? int(EP_LAYOUT_CLUSTER) : int(EP_ERR_UNSUPPORTED);
+        default:
+            return EP_ERR_INVALID;
+    }
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" int ep_layout_path(ep_dims_t d, ep_cfg_t cfg) {
+    const int rc = check_dims(d);
+    if (rc != EP_OK) return rc;
+    return resolve_layout_path(d, cfg, layout_geom(d));
+}
+
 extern "C" size_t ep_layout_workspace_bytes(ep_dims_t d) {
     if (check_dims(d) != EP_OK) return 0;
     const LayoutGeom lg = layout_geom(d);
@@ -764,18 +1070,11 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     a.cap = RT;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int64_t pairs = int64_t(d.num_ranks) * d.num_tokens * d.num_topk;
-    const bool small_ok = d.num_ranks <= kSmallMaxRanks && d.num_experts <= kSmallMaxExperts &&
-                          pairs <= kSmallMaxPairs;
+    const int path = resolve_layout_path(d, cfg, lg);
+    if (path < 0) return path;
     const int W = lg.warps;
-    const size_t fused_smem = size_t(2 * kActiveSlots + 2 * d.num_experts + W * d.num_experts) * 4;
-    const bool fused_ok = lg.G <= kMaxFlags && lg.G <= fused_capacity(32 * W, fused_smem);
-    // AUTO: the chunked path.  On B200 its three launches (about 17 us per call in a graph)
-    // beat the fused one (about 19 us: cooperative launch plus two grid barriers).
-    int path = cfg.variant;
-    if (path == EP_VARIANT_AUTO) path = EP_LAYOUT_CHUNKED;
     if (path == EP_LAYOUT_FUSED) {
-        if (!fused_ok) return EP_ERR_UNSUPPORTED;
+        const size_t fused_smem = fused_smem_bytes(d, lg);
         void* args[] = {&a};
         cudaLaunchConfig_t lc = {};
         lc.gridDim = dim3(lg.G);
@@ -793,8 +1092,32 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
         }
         return launch_result();
     }
+    if (path == EP_LAYOUT_CLUSTER) {
+        const size_t smem = cluster_smem_bytes(d);
+        if (cudaFuncSetAttribute(layout_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(layout_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess)
+            return EP_ERR_CUDA;
+        const int cl = cluster_ctas(int64_t(d.num_ranks) * d.num_tokens * d.num_topk, smem);
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(cl);
+        lc.blockDim = dim3(kSmallThreads);
+        lc.dynamicSmemBytes = smem;
+        lc.stream = s;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cl;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 2;
+        if (cudaLaunchKernelEx(&lc, layout_cluster_kernel, a) != cudaSuccess) return EP_ERR_CUDA;
+        return launch_result();
+    }
     if (path == EP_LAYOUT_SINGLE_CTA) {
-        if (!small_ok) return EP_ERR_UNSUPPORTED;
         const size_t smem = size_t(kActiveSlots + kSmallMaxRanks * kSmallMaxRanks + d.num_experts +
                                    (kSmallThreads / 32) * d.num_experts) * 4;
         if (smem > 48 * 1024 &&
@@ -805,7 +1128,6 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
             return EP_ERR_CUDA;
         return launch_result();
     }
-    if (path != EP_LAYOUT_CHUNKED) return EP_ERR_INVALID;
     const size_t count_smem = size_t(2 * kActiveSlots + 2 * d.num_experts) * 4;
     const size_t rank_smem = size_t(kActiveSlots + 2 * d.num_experts + W * d.num_experts) * 4;
     if (count_smem > 48 * 1024 &&

@@ -35,6 +35,10 @@ EP_FP8_SCALE_POW2 = 1
 EP_FP8_SCALE_UE8M0 = 2
 EP_VARIANT_BULK = 1
 EP_VARIANT_VECTOR = 2
+EP_LAYOUT_CHUNKED = 1
+EP_LAYOUT_SINGLE_CTA = 2
+EP_LAYOUT_FUSED = 3
+EP_LAYOUT_CLUSTER = 4
 
 _lib = None
 
@@ -71,6 +75,8 @@ def load_library(path: str = LIB_PATH):
     lib.ep_version.restype = ctypes.c_char_p
     lib.ep_layout_workspace_bytes.argtypes = [Dims]
     lib.ep_layout_workspace_bytes.restype = SZ
+    lib.ep_layout_path.argtypes = [Dims, Cfg]
+    lib.ep_layout_path.restype = ctypes.c_int
     lib.ep_layout.argtypes = [Dims, P, P, P, SZ, P, P, P, P, P, P, P, Cfg, P]
     lib.ep_layout.restype = ctypes.c_int
     lib.ep_dispatch.argtypes = [Dims, P, P, P, P, P, P, Cfg, P]
@@ -163,6 +169,15 @@ class DispatchLayout:
     expert_rank_offset: torch.Tensor     # int32 [E, R]
     pair_row: torch.Tensor               # int32 [R, T, k]
     status: torch.Tensor                 # int32 [1]
+
+
+def ep_layout_path(num_ranks: int, num_tokens: int, num_topk: int, num_experts: int, hidden: int = 8,
+                   cfg=None) -> int:
+    """The ``EP_LAYOUT_*`` path ``ep_layout`` takes for this shape and ``cfg`` (``ep_layout_path``)."""
+    rc = int(load_library().ep_layout_path(Dims(num_ranks, num_tokens, num_topk, num_experts, hidden), _cfg(cfg)))
+    if rc < 0:
+        _check("ep_layout_path", rc)
+    return rc
 
 
 def ep_layout_workspace_bytes(num_ranks: int, num_tokens: int, num_topk: int, num_experts: int,

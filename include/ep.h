@@ -115,12 +115,18 @@ typedef struct ep_cfg {
 } ep_cfg_t;
 
 /* Paths of ep_layout (ep_cfg_t.variant); they compute the same result.  AUTO
- * takes CHUNKED, the fastest on B200 at every measured shape. */
+ * takes, where it applies, SINGLE_CTA up to R*T*k = 2048 pairs, CLUSTER up to
+ * 32768, else CHUNKED: the fastest on B200 in each range (graph replays: 8.6 us
+ * at 1024 pairs; 10.6 us from 4096 to 16384 and 12.7 us at 32768 on the
+ * cluster, against 16.8 us chunked). */
 enum {
     EP_LAYOUT_CHUNKED = 1,    /* three launches over chunks of each rank's tokens; any shape */
     EP_LAYOUT_SINGLE_CTA = 2, /* one launch, one CTA; R <= 32, E <= 1024, R*T*k <= 32768 */
-    EP_LAYOUT_FUSED = 3       /* one cooperative launch with two grid barriers; needs the
+    EP_LAYOUT_FUSED = 3,      /* one cooperative launch with two grid barriers; needs the
                                  chunk grid to fit the device (else EP_ERR_UNSUPPORTED) */
+    EP_LAYOUT_CLUSTER = 4     /* one launch of a thread-block cluster of up to 16 CTAs that
+                                 share their histograms through distributed shared memory;
+                                 R <= 32, E <= 1024, R*T*k <= 65536 */
 };
 
 /* Data paths of ep_dispatch / ep_combine (ep_cfg_t.variant). */
@@ -138,6 +144,17 @@ EP_API const char *ep_version(void);
 
 /* Bytes of device workspace ep_layout needs for `d` (0 for an invalid shape). */
 EP_API size_t ep_layout_workspace_bytes(ep_dims_t d);
+
+/*
+ * ep_layout_path -- the path (EP_LAYOUT_*) ep_layout takes for these dims and
+ * cfg.variant, so a caller can tell how many kernels a call launches (CHUNKED:
+ * three; SINGLE_CTA, FUSED, CLUSTER: one).  The pages have no counterpart: it only
+ * reports this library's own choice.  Returns EP_ERR_INVALID for bad dims or
+ * an unknown variant and EP_ERR_UNSUPPORTED when the requested path cannot take
+ * the shape, exactly as ep_layout would; launches nothing.
+ */
+EP_API int ep_layout_path(ep_dims_t d, ep_cfg_t cfg);
+
 
 /*
  * ep_layout -- per-expert / per-rank histogram, prefix sums and stable rows.

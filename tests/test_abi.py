@@ -90,3 +90,35 @@ def test_host_validation_rejects_without_launching(lib):
     assert lib.ep_dispatch(good, odd, fake, fake, fake, fake, fake, cfg, None) == ep.EP_ERR_INVALID
     assert lib.ep_reroute(1, 4, 2, 0, 1, None, None, 0, None, None, None, None, None, cfg, None) \
         == ep.EP_ERR_INVALID
+
+
+def test_layout_path_choice(lib):
+    """AUTO takes one CTA up to 2048 pairs and a cluster up to 32768 (R <= 32, E <= 1024), the
+    chunked path beyond; explicit paths are honoured or refused exactly as ep_layout would."""
+    from combine_get_dispatch_histogram_b200 import ep
+
+    assert ep.ep_layout_path(2, 64, 2, 8) == ep.EP_LAYOUT_SINGLE_CTA          # 256 pairs
+    assert ep.ep_layout_path(8, 32, 8, 256) == ep.EP_LAYOUT_SINGLE_CTA        # 2048 pairs
+    assert ep.ep_layout_path(8, 64, 8, 256) == ep.EP_LAYOUT_CLUSTER           # 4096 pairs
+    assert ep.ep_layout_path(8, 512, 8, 256) == ep.EP_LAYOUT_CLUSTER          # 32768 pairs
+    assert ep.ep_layout_path(8, 1024, 8, 256) == ep.EP_LAYOUT_CHUNKED         # 65536 pairs
+    assert ep.ep_layout_path(8, 16, 8, 2048) == ep.EP_LAYOUT_CHUNKED          # E > 1024
+    assert ep.ep_layout_path(40, 8, 8, 80) == ep.EP_LAYOUT_CHUNKED            # R > 32
+    cluster = dict(variant=ep.EP_LAYOUT_CLUSTER)
+    assert ep.ep_layout_path(8, 1024, 8, 256, cfg=cluster) == ep.EP_LAYOUT_CLUSTER
+    with pytest.raises(ep.EPError) as ei:
+        ep.ep_layout_path(8, 2048, 8, 256, cfg=cluster)
+    assert ei.value.code == ep.EP_ERR_UNSUPPORTED
+    chunked = dict(variant=ep.EP_LAYOUT_CHUNKED)
+    assert ep.ep_layout_path(8, 16, 8, 256, cfg=chunked) == ep.EP_LAYOUT_CHUNKED
+    single = dict(variant=ep.EP_LAYOUT_SINGLE_CTA)
+    assert ep.ep_layout_path(8, 512, 8, 256, cfg=single) == ep.EP_LAYOUT_SINGLE_CTA   # 32768 pairs
+    with pytest.raises(ep.EPError) as ei:
+        ep.ep_layout_path(8, 1024, 8, 256, cfg=single)
+    assert ei.value.code == ep.EP_ERR_UNSUPPORTED
+    with pytest.raises(ep.EPError) as ei:
+        ep.ep_layout_path(8, 16, 8, 255)                                       # E % R != 0
+    assert ei.value.code == ep.EP_ERR_INVALID
+    with pytest.raises(ep.EPError) as ei:
+        ep.ep_layout_path(8, 16, 8, 256, cfg=dict(variant=9))
+    assert ei.value.code == ep.EP_ERR_INVALID

@@ -332,10 +332,10 @@ def test_vector_variant_rejects_wide_topk():
     assert ei.value.code == ep.EP_ERR_UNSUPPORTED
 
 
-LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED = 1, 2, 3
+LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER = 1, 2, 3, 4
 
 
-@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED])
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER])
 @pytest.mark.parametrize("name", ["tiny", "decode", "sweep_T16_mask5", "sweep_T512", "sweep_T256_mask5"])
 def test_layout_paths_match_oracle(name, path):
     w = inputs.named(name)
@@ -345,12 +345,14 @@ def test_layout_paths_match_oracle(name, path):
                f"{name} layout path {path}")
 
 
-@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED])
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER])
 @pytest.mark.parametrize("name", ["k1", "T1", "R1", "E_equals_R", "k32", "many_experts"])
 def test_layout_paths_edge_shapes(name, path):
     c = EDGE[name]
     if path == LAYOUT_SINGLE_CTA and (c["E"] > 1024 or c["R"] > 32 or c["R"] * c["T"] * c["k"] > 32768):
         pytest.skip("shape outside the single-CTA path's limits")
+    if path == LAYOUT_CLUSTER and (c["E"] > 1024 or c["R"] > 32 or c["R"] * c["T"] * c["k"] > 65536):
+        pytest.skip("shape outside the cluster path's limits")
     rng = np.random.default_rng(zlib.crc32(name.encode()) + 7)
     idx = _uniform_idx(rng, c["R"], c["T"], c["k"], c["E"])
     idx = np.where(rng.random(idx.shape) < 0.1, -1, idx)
@@ -363,7 +365,25 @@ def test_layout_paths_edge_shapes(name, path):
                f"{name} layout path {path}")
 
 
-@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED])
+@pytest.mark.parametrize("path", [LAYOUT_SINGLE_CTA, LAYOUT_CLUSTER])
+@pytest.mark.parametrize("R,T,k,E", [(2, 2000, 6, 64), (4, 2048, 4, 128), (32, 8, 8, 1024), (3, 700, 5, 96)])
+def test_single_cta_layout_long_parts(R, T, k, E, path):
+    """Single-CTA and cluster layouts where a warp's part is longer than one round of loads (rows
+    parked in pair_row between the passes), with k a power of two (destination ranks from an OR
+    over a token's lanes) and not (one token per lane), and a rank count that leaves warps idle;
+    the cluster cases also split ranks across CTAs and put several ranks in one CTA."""
+    rng = np.random.default_rng(R * 1000 + T + k)
+    idx = _uniform_idx(rng, R, T, k, E)
+    idx = np.where(rng.random(idx.shape) < 0.05, -1, idx)
+    act = np.ones(R, np.uint8)
+    act[R - 1] = 0
+    inp = _custom(R, T, k, E, 64, idx, active=act)
+    ref, packed, want = _oracle_all(inp, E)
+    _check_all(run_path(inp, E, 64, layout_cfg=dict(variant=path)), ref, packed, want,
+               f"path {path} R={R} T={T} k={k}")
+
+
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER])
 def test_layout_paths_overflow_and_bad_ids(path):
     R, T, k, E, H = 2, 16, 3, 4, 64
     idx = np.zeros((R, T, k), np.int32)
@@ -407,3 +427,17 @@ def test_fused_layout_in_cuda_graph_replays():
         g.replay()
         torch.cuda.synchronize()
         check_layout(lay, ref, "graph replay")
+
+
+@pytest.mark.parametrize("T", [64, 128, 200, 512, 1024])
+def test_cluster_layout_sizes(T):
+    """Cluster layout across its cluster sizes (one CTA per 1024 pairs, 2 to 16) and a ragged T."""
+    w = (inputs.sweep(T) if T in (64, 128, 512) else
+         inputs.Workload(f"T{T}", 8, T, 8, 256, 64, inactive=(3,) if T == 200 else ()))
+    inp = inputs.make_inputs(w, tokens=False)
+    ref = oracle.layout(inp.topk_idx, inp.active, w.num_experts)
+    lay = ep.ep_layout(i32_dev(inp.topk_idx), u8_dev(inp.active), w.num_experts, hidden=w.hidden,
+                       cfg=dict(variant=LAYOUT_CLUSTER))
+    torch.cuda.synchronize()
+    check_layout(lay, ref, f"cluster T={T}")
+    assert int(lay.status.item()) == ref.status
