@@ -63,7 +63,7 @@ constexpr int kSmallAutoPairs = 2048;  // AUTO takes the single-CTA path up to h
 constexpr int kClusterMaxCtas = 16;     // a non-portable cluster size (8 is the portable limit)
 constexpr int kClusterPairsPerCta = 1024;
 constexpr int64_t kClusterMaxPairs = 65536;
-constexpr int64_t kClusterAutoPairs = 32768;  // AUTO takes the cluster path up to here
+constexpr int64_t kClusterAutoPairs = 65536;  // AUTO takes the cluster path up to here
 constexpr int kMaxWarps = 16;
 constexpr int kBatch = 8;           // 32-pair steps whose loads are issued together
 constexpr int kActiveSlots = 64;    // shared copy of the active mask (EP_MAX_RANKS)
@@ -985,9 +985,9 @@ size_t fused_smem_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
 // The path ep_layout takes for these dims and cfg, or a negative EP_ERR_* code.
 // AUTO, from graph replays on B200: one CTA up to kSmallAutoPairs pairs (8.6 us at 1024
 // pairs, 10.6 us at 2048); a cluster up to kClusterAutoPairs (10.6 us from 4096 to 16384
-// pairs, 12.7 us at 32768, where one CTA takes 14.7 to 74 us); the chunked path beyond
-// (about 17 to 19 us), which also beats the fused one (cooperative launch plus two grid
-// barriers, about 19 us).
+// pairs, 12.7 us at 32768, 14.7 at 49152, 16.8 at 65536, where one CTA takes 14.7 to 74 us);
+// the chunked path beyond (about 17 to 19 us), which also beats the fused one (cooperative
+// launch plus two grid barriers, about 19 us).
 int resolve_layout_path(const ep_dims_t& d, const ep_cfg_t& cfg, const LayoutGeom& lg) {
     const int64_t pairs = int64_t(d.num_ranks) * d.num_tokens * d.num_topk;
     const bool tables_fit = d.num_ranks <= kSmallMaxRanks && d.num_experts <= kSmallMaxExperts;

@@ -116,7 +116,7 @@ typedef struct ep_cfg {
 
 /* Paths of ep_layout (ep_cfg_t.variant); they compute the same result.  AUTO
  * takes, where it applies, SINGLE_CTA up to R*T*k = 2048 pairs, CLUSTER up to
- * 32768, else CHUNKED: the fastest on B200 in each range (graph replays: 8.6 us
+ * 65536, else CHUNKED: the fastest on B200 in each range (graph replays: 8.6 us
  * at 1024 pairs; 10.6 us from 4096 to 16384 and 12.7 us at 32768 on the
  * cluster, against 16.8 us chunked). */
 enum {

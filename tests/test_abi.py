@@ -93,7 +93,7 @@ def test_host_validation_rejects_without_launching(lib):
 
 
 def test_layout_path_choice(lib):
-    """AUTO takes one CTA up to 2048 pairs and a cluster up to 32768 (R <= 32, E <= 1024), the
+    """AUTO takes one CTA up to 2048 pairs and a cluster up to 65536 (R <= 32, E <= 1024), the
     chunked path beyond; explicit paths are honoured or refused exactly as ep_layout would."""
     from combine_get_dispatch_histogram_b200 import ep
 
@@ -101,7 +101,8 @@ def test_layout_path_choice(lib):
     assert ep.ep_layout_path(8, 32, 8, 256) == ep.EP_LAYOUT_SINGLE_CTA        # 2048 pairs
     assert ep.ep_layout_path(8, 64, 8, 256) == ep.EP_LAYOUT_CLUSTER           # 4096 pairs
     assert ep.ep_layout_path(8, 512, 8, 256) == ep.EP_LAYOUT_CLUSTER          # 32768 pairs
-    assert ep.ep_layout_path(8, 1024, 8, 256) == ep.EP_LAYOUT_CHUNKED         # 65536 pairs
+    assert ep.ep_layout_path(8, 1024, 8, 256) == ep.EP_LAYOUT_CLUSTER         # 65536 pairs
+    assert ep.ep_layout_path(8, 1025, 8, 256) == ep.EP_LAYOUT_CHUNKED         # 65600 pairs
     assert ep.ep_layout_path(8, 16, 8, 2048) == ep.EP_LAYOUT_CHUNKED          # E > 1024
     assert ep.ep_layout_path(40, 8, 8, 80) == ep.EP_LAYOUT_CHUNKED            # R > 32
     cluster = dict(variant=ep.EP_LAYOUT_CLUSTER)
