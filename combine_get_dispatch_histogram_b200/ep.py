@@ -39,6 +39,8 @@ EP_LAYOUT_CHUNKED = 1
 EP_LAYOUT_SINGLE_CTA = 2
 EP_LAYOUT_FUSED = 3
 EP_LAYOUT_CLUSTER = 4
+EP_REROUTE_TWO_LAUNCH = 1
+EP_REROUTE_CLUSTER = 2
 
 _lib = None
 

@@ -60,7 +60,7 @@ def main():
                             device=dev)
         out = ep.ep_reroute(idx, w.num_experts, w.num_extra, status=status)
         calls.append(lambda: ep.ep_reroute(idx, w.num_experts, w.num_extra, workspace=rr_ws, out=out,
-                                           status=status, stream=stream))
+                                           status=status, stream=stream, cfg=cfg))
     if args.op in ("layout", "step"):
         calls.append(lambda: ep.ep_layout(idx_phys, act, E, hidden=H, workspace=ws, out=lay, status=status,
                                           stream=stream, cfg=dict(variant=args.layout_variant)))

@@ -365,7 +365,16 @@ EP_API int ep_normal_combine(ep_dims_t d, int32_t recv_capacity, const uint16_t 
                              const int32_t *token_recv_row, const uint8_t *active, uint16_t *out,
                              int32_t *status, ep_cfg_t cfg, void *stream);
 
-/* Bytes of device workspace ep_reroute needs. */
+/* Paths of ep_reroute (ep_cfg_t.variant); they compute the same result.  AUTO
+ * takes CLUSTER. */
+enum {
+    EP_REROUTE_TWO_LAUNCH = 1, /* count per CTA into the workspace, then sum, plan and expand */
+    EP_REROUTE_CLUSTER = 2     /* one launch of a thread-block cluster of up to 16 CTAs that
+                                  read each other's counts through distributed shared memory */
+};
+
+/* Bytes of device workspace ep_reroute needs (the two-launch path uses it; the
+ * cluster path does not, but every call is checked against this size). */
 EP_API size_t ep_reroute_workspace_bytes(int32_t num_ranks, int32_t num_tokens, int32_t num_topk,
                                   int32_t num_logical);
 

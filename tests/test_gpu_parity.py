@@ -283,7 +283,8 @@ def test_fuzz_small(seed):
     _check_all(res, ref, packed, want, f"fuzz{seed}")
 
 
-def test_reroute_small_cases():
+@pytest.mark.parametrize("variant", [ep.EP_REROUTE_CLUSTER, ep.EP_REROUTE_TWO_LAUNCH])
+def test_reroute_small_cases(variant):
     rng = np.random.default_rng(77)
     for it in range(20):
         E = int(rng.integers(1, 70))
@@ -292,11 +293,32 @@ def test_reroute_small_cases():
         k = int(rng.integers(1, min(E, 8) + 1))
         idx = inputs.zipf_topk(rng, R * T, E, k, 1.3).reshape(R, T, k)
         idx = np.where(rng.random(idx.shape) < 0.05, -1, idx).astype(np.int32)
-        rr = ep.ep_reroute(i32_dev(idx), E, extra)
+        rr = ep.ep_reroute(i32_dev(idx), E, extra, cfg=dict(variant=variant))
         torch.cuda.synchronize()
         rref = oracle.reroute(idx, E, extra)
         for key in ("load", "num_replicas", "phys_base", "topk_idx_phys"):
             assert np.array_equal(rr[key].cpu().numpy(), rref[key]), (it, key)
+
+
+@pytest.mark.parametrize("variant", [ep.EP_REROUTE_CLUSTER, ep.EP_REROUTE_TWO_LAUNCH])
+@pytest.mark.parametrize("R,T,k,E,extra", [(8, 2048, 6, 64, 16), (8, 4096, 8, 256, 64), (2, 3000, 4, 8192, 100),
+                                           (1, 1, 1, 1, 0), (4, 0, 2, 8, 3)])
+def test_reroute_paths_sizes(R, T, k, E, extra, variant):
+    """Both reroute paths from one slice to the largest cluster (16 CTAs), the most logical
+    experts (8192), one pair, no pairs, and a bad id (flagged, mapped to -1)."""
+    rng = np.random.default_rng(R * 7 + T + E)
+    if E <= 256:
+        idx = inputs.zipf_topk(rng, R * T, E, k, 1.2).reshape(R, T, k).astype(np.int32)
+    else:  # uniform ids (repeats allowed: the reroute counts pairs) without an [n, E] draw table
+        idx = rng.integers(0, E, size=(R, T, k)).astype(np.int32)
+    if idx.size > 3:
+        idx.reshape(-1)[3] = E + 5
+    rr = ep.ep_reroute(i32_dev(idx), E, extra, cfg=dict(variant=variant))
+    torch.cuda.synchronize()
+    rref = oracle.reroute(idx, E, extra)
+    for key in ("load", "num_replicas", "phys_base", "topk_idx_phys"):
+        assert np.array_equal(rr[key].cpu().numpy(), rref[key]), key
+    assert bool(int(rr["status"].item()) & ep.EP_STATUS_BAD_EXPERT) == (idx.size > 3)
 
 
 @pytest.mark.parametrize("variant", [1, 2])
