@@ -296,23 +296,30 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.Stream(dev)
     n_ev = 4
     layout_launches = 3 if ep.ep_layout_path(R, T, k, E, H) == ep.EP_LAYOUT_CHUNKED else 1
-    launches_per_step = layout_launches + 2 + (2 if reroute else 0)  # layout, dispatch, combine (+ reroute 2)
+    launches_per_step = layout_launches + 2 + (1 if reroute else 0)  # layout, dispatch, combine (+ reroute)
 
-    idx_phys = rr_out["topk_idx_phys"] if reroute else idx_log
+    # the step reads its inputs from and writes its result to the current buffer set (the end-to-end
+    # leg alternates two sets so that one step's copies overlap the next step's)
+    cur = {"b": dict(idx=idx_log, w=wts, act=act, x=x, out=out)}
+
+    def idx_phys():
+        return rr_out["topk_idx_phys"] if reroute else cur["b"]["idx"]
 
     def do_layout():
+        b = cur["b"]
         if reroute:
-            ep.ep_reroute(idx_log, w.num_experts, w.num_extra, workspace=rr_ws, out=rr_out, status=status,
+            ep.ep_reroute(b["idx"], w.num_experts, w.num_extra, workspace=rr_ws, out=rr_out, status=status,
                           stream=stream)
-        ep.ep_layout(idx_phys, act, E, hidden=H, workspace=lay_ws, out=lay, status=status, stream=stream)
+        ep.ep_layout(idx_phys(), b["act"], E, hidden=H, workspace=lay_ws, out=lay, status=status, stream=stream)
 
     def do_dispatch():
-        ep.ep_dispatch(x, idx_phys, lay.pair_row, E, recv_x=recv_x, src_info=src_info, status=status,
-                       stream=stream, cfg=args.dispatch_cfg)
+        ep.ep_dispatch(cur["b"]["x"], idx_phys(), lay.pair_row, E, recv_x=recv_x, src_info=src_info,
+                       status=status, stream=stream, cfg=args.dispatch_cfg)
 
     def do_combine():
-        ep.ep_combine(recv_x, idx_phys, wts, lay.pair_row, act, out=out, status=status, stream=stream,
-                      cfg=args.combine_cfg)
+        b = cur["b"]
+        ep.ep_combine(recv_x, idx_phys(), b["w"], lay.pair_row, b["act"], out=b["out"], status=status,
+                      stream=stream, cfg=args.combine_cfg)
 
     parts = (do_layout, do_dispatch, do_combine)
 
@@ -389,34 +396,64 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit(f"device status {int(status.item())} after the timed steps")
 
     # ---------------------------------------------------------------- e2e: host buffers
+    # Every step copies its inputs from pinned host memory and its result back.  Two device buffer
+    # sets alternate: step i's inputs go up on one copy stream while step i-1 computes and step i-2's
+    # result comes down on another (PCIe carries both directions at once).  A set is refilled only
+    # after the step that read it has finished, and its result buffer only after it has been read out.
     e2e = None
     if args.e2e_steps > 0:
         h_idx = torch.from_numpy(inp.topk_idx).pin_memory()
         h_w = torch.from_numpy(inp.topk_weights).pin_memory()
         h_act = torch.from_numpy(inp.active).pin_memory()
         h_x = torch.from_numpy(inp.x.view(np.int16)).pin_memory()
-        h_out = torch.empty((R, T, H), dtype=torch.int16).pin_memory()
+        h_out = [torch.empty((R, T, H), dtype=torch.int16).pin_memory() for _ in range(2)]
         h2d = h_idx.numel() * 4 + h_w.numel() * 4 + h_act.numel() + h_x.numel() * 2
-        d2h = h_out.numel() * 2
+        d2h = h_out[0].numel() * 2
+        sets = [cur["b"], dict(idx=torch.empty_like(idx_log), w=torch.empty_like(wts), act=torch.empty_like(act),
+                               x=torch.empty_like(x), out=torch.empty_like(out))]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        n = args.e2e_steps
         rank_barrier(world, local_rank)
         torch.cuda.synchronize(dev)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(args.e2e_steps):
-                idx_log.copy_(h_idx, non_blocking=True)
-                wts.copy_(h_w, non_blocking=True)
-                act.copy_(h_act, non_blocking=True)
-                x.view(torch.int16).copy_(h_x, non_blocking=True)
+        e0.record(stream)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for i in range(n):
+            b = i % 2
+            B = sets[b]
+            if i >= 2:
+                s_in.wait_event(ev_done[b])      # step i-2 has finished reading this set
+            with torch.cuda.stream(s_in):
+                B["idx"].copy_(h_idx, non_blocking=True)
+                B["w"].copy_(h_w, non_blocking=True)
+                B["act"].copy_(h_act, non_blocking=True)
+                B["x"].view(torch.int16).copy_(h_x, non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])     # step i-2's result has been read out of this set
+            cur["b"] = B
+            with torch.cuda.stream(stream):
                 step()
-                h_out.copy_(out.view(torch.int16), non_blocking=True)
-            e1.record(stream)
-            stream.synchronize()
+                ev_done[b].record(stream)
+            s_out.wait_event(ev_done[b])
+            with torch.cuda.stream(s_out):
+                h_out[b].copy_(B["out"].view(torch.int16), non_blocking=True)
+                ev_out[b].record(s_out)
+        for b in range(min(2, n)):
+            stream.wait_event(ev_out[b])
+        e1.record(stream)
+        stream.synchronize()
+        cur["b"] = sets[0]
         rank_barrier(world, local_rank)
-        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        e2e_ms = e0.elapsed_time(e1) / n
         e2e = dict(ms=e2e_ms, h2d=h2d, d2h=d2h)
-        assert np.array_equal(h_out.numpy(), out.view(torch.int16).cpu().numpy())
+        assert np.array_equal(h_out[(n - 1) % 2].numpy(), out.view(torch.int16).cpu().numpy())
 
     # ---------------------------------------------------------------- reduce over ranks
     total_ms, lay_ms, dis_ms, com_ms, e2e_ms = reduce_over_ranks(
