@@ -279,8 +279,9 @@ enum {
  * cfg.variant: EP_VARIANT_BULK stages each bf16 row in shared memory with a bulk
  * copy and bulk-stores the code rows (needs 2*H <= 16384 and a 16-byte aligned
  * recv_x, else EP_ERR_UNSUPPORTED); EP_VARIANT_VECTOR moves rows through
- * registers; EP_VARIANT_AUTO takes the bulk path when it applies.  Both give the
- * same bits.
+ * registers; EP_VARIANT_AUTO takes the bulk path when it applies, except with
+ * fp32 scales on at most 1024 tokens (R*T), where the vector path is faster.
+ * Both give the same bits.
  */
 EP_API int ep_dispatch_fp8(ep_dims_t d, const uint16_t *x, const int32_t *topk_idx,
                            const int32_t *pair_row, const int32_t *recv_count,
