@@ -241,71 +241,74 @@ __global__ void __launch_bounds__(32 * kScanWarps) layout_scan_kernel(LayoutArgs
     }
 }
 
-// Single CTA: the whole layout in one launch (small problems).  The NW / R warps
-// of rank r split its tokens into consecutive parts, in (rank, part) order.
-//  1. the warp's first pairs are loaded while the tables (active mask,
-//     rank_of) and the zeroed warp histograms are set up;
-//  2. each warp walks its part in 32-pair steps: a pair's row within the part is
-//     its expert's running count in the warp histogram plus the matching lanes
-//     below it (ballot match), kept in registers (parked in pair_row when the
-//     part is longer than one round of loads); with k a power of two a token's
-//     k slots sit in k aligned lanes, and an OR over them gives its destination
-//     ranks (is_token_in_rank, num_tokens_per_rank) in the same step;
-//  3. per expert, the warp histograms are scanned in (rank, part) order into
-//     each warp's first row;
-//  4. each live pair adds its warp's first row for its expert.
-__global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(LayoutArgs a) {
-    pdl_wait();  // nothing upstream is read before this
-    pdl_launch_dependents();
-    extern __shared__ int32_t smem[];
-    constexpr int NW = kSmallThreads / 32;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int32_t* act = smem;
-    int32_t* tpr = smem + kActiveSlots;                        // [R][R]
-    int32_t* rank_of = tpr + kSmallMaxRanks * kSmallMaxRanks;   // [E]
-    int32_t* whist = rank_of + a.E;                            // [NW][E]
+// ---------------------------------------------------------------------------
+// One-launch paths (single CTA, cluster).  Their warps -- 32 per CTA, a cluster's
+// numbered CTA * 32 + warp -- split each rank's tokens into consecutive parts in
+// (rank, part) order, and each warp walks its part once.
 
-    // warps per rank and this warp's token range (in (rank, token) order)
-    const int wpr = NW / a.R;  // R <= 32
-    const int r = warp / wpr, part = warp - r * wpr;
-    const bool has_rank = r < a.R;
+// A warp's part of the tokens: rank r, tokens [t0, t1), pairs from pbase on.
+struct WarpPart {
+    int r, t0, t1;
+    int64_t pbase;
+    int np;          // pairs of the part
+    bool has_rank;   // warps past the last rank have no part
+    bool one_round;  // np <= 32 * kBatch: the rows within the part stay in registers
+};
+
+__device__ __forceinline__ WarpPart warp_part(const LayoutArgs& a, int gw, int wpr) {
+    WarpPart w;
+    w.r = gw / wpr;
+    const int part = gw - w.r * wpr;
+    w.has_rank = w.r < a.R;
     const int tw = (a.T + wpr - 1) / wpr;
-    const int wt0 = has_rank ? min(a.T, part * tw) : 0, wt1 = has_rank ? min(a.T, wt0 + tw) : 0;
-    const int64_t pbase = has_rank ? (int64_t(r) * a.T + wt0) * a.k : 0;
-    const int32_t* base = a.topk_idx + pbase;
-    int32_t* rows = a.pair_row + pbase;
-    const int np = (wt1 - wt0) * a.k;
-    const bool one_round = np <= 32 * kBatch;
+    w.t0 = w.has_rank ? min(a.T, part * tw) : 0;
+    w.t1 = w.has_rank ? min(a.T, w.t0 + tw) : 0;
+    w.pbase = w.has_rank ? (int64_t(w.r) * a.T + w.t0) * a.k : 0;
+    w.np = (w.t1 - w.t0) * a.k;
+    w.one_round = w.np <= 32 * kBatch;
+    return w;
+}
 
-    int ev[kBatch];  // the first round's experts need no table: load them before the barrier
+// The part's first round of experts; it needs no table, so it is loaded before
+// the barrier that publishes them.
+__device__ __forceinline__ void load_first_round(const LayoutArgs& a, const WarpPart& w, int (&ev)[kBatch]) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
         const int p = u * 32 + lane;
-        ev[u] = p < np ? __ldg(base + p) : -1;
+        ev[u] = p < w.np ? __ldg(a.topk_idx + w.pbase + p) : -1;
     }
-    load_tables(a, act, rank_of);
-    for (int i = threadIdx.x; i < NW * a.E; i += blockDim.x) whist[i] = 0;
-    for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) tpr[i] = 0;
-    __syncthreads();
+}
 
-    const bool src_ok = has_rank && act[r] != 0;
-    int32_t* mine = whist + warp * a.E;
+// One pass over the part.  A pair's row within the part is its expert's running
+// count in the warp's histogram `mine` plus the matching lanes below it (ballot
+// match); it stays in rk (the last round's pairs) or, for a part longer than one
+// round, is parked in pair_row.  Each token's destination ranks go to
+// is_token_in_rank and its counts to tpr[r][*]: with k a power of two a token's
+// k slots sit in k aligned lanes and an OR over them gives the set, otherwise one
+// token per lane re-reads its slots.  True if this lane saw an id outside [-1, E).
+__device__ __forceinline__ bool walk_part(const LayoutArgs& a, const WarpPart& w, const int32_t* act,
+                                          const int32_t* rank_of, int32_t* mine, int32_t* tpr,
+                                          int (&ev)[kBatch], int (&rk)[kBatch]) {
+    const int lane = threadIdx.x & 31;
+    const bool src_ok = w.has_rank && act[w.r] != 0;
+    const int32_t* base = a.topk_idx + w.pbase;
+    int32_t* rows = a.pair_row + w.pbase;
     const uint32_t below = lanemask_lt();
     const bool lanes_per_token = (a.k & (a.k - 1)) == 0;  // k divides 32: a token is k aligned lanes
     bool bad = false;
-    int rk[kBatch];  // rows within the part of the last round's pairs (-1: not live)
-    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+    for (int p0 = 0; p0 < w.np; p0 += 32 * kBatch) {
         if (p0 > 0) {
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
                 const int p = p0 + u * 32 + lane;
-                ev[u] = p < np ? __ldg(base + p) : -1;
+                ev[u] = p < w.np ? __ldg(base + p) : -1;
             }
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             rk[u] = -1;
-            if (p0 + u * 32 >= np) break;  // the same for the whole warp
+            if (p0 + u * 32 >= w.np) break;  // the same for the whole warp
             const int p = p0 + u * 32 + lane;
             const int e = ev[u];
             bad |= (e < -1 || e >= a.E);
@@ -316,42 +319,91 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
             if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
             __syncwarp();
             rk[u] = live ? b + __popc(m & below) : -1;
-            if (!one_round && p < np) rows[p] = rk[u];
+            if (!w.one_round && p < w.np) rows[p] = rk[u];
             if (lanes_per_token) {
                 uint32_t dst = live ? (1u << rank_of[e]) : 0u;
                 for (int o = 1; o < a.k; o <<= 1) dst |= __shfl_xor_sync(0xffffffffu, dst, o);
-                const bool head = p < np && (lane & (a.k - 1)) == 0;
+                const bool head = p < w.np && (lane & (a.k - 1)) == 0;
                 if (head) {
-                    uint8_t* itr = a.is_token_in_rank + ((pbase + p) / a.k) * a.R;
+                    uint8_t* itr = a.is_token_in_rank + ((w.pbase + p) / a.k) * a.R;
                     for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((dst >> d) & 1u);
                 }
                 for (int d = 0; d < a.R; ++d) {
                     const int n = __popc(__ballot_sync(0xffffffffu, head && ((dst >> d) & 1u)));
-                    if (lane == 0 && n) atomicAdd(tpr + r * a.R + d, n);
+                    if (lane == 0 && n) atomicAdd(tpr + w.r * a.R + d, n);
                 }
             }
         }
     }
     if (!lanes_per_token) {
-        // destination-rank set of each token of this warp's part, one token per lane
-        for (int t0 = wt0; t0 < wt1; t0 += 32) {
+        for (int t0 = w.t0; t0 < w.t1; t0 += 32) {
             const int t = t0 + lane;
             uint64_t ranks = 0;
-            if (t < wt1) {
-                const int32_t* tb = a.topk_idx + (int64_t(r) * a.T + t) * a.k;
+            if (t < w.t1) {
+                const int32_t* tb = a.topk_idx + (int64_t(w.r) * a.T + t) * a.k;
                 for (int j = 0; j < a.k; ++j) {
                     const int e = __ldg(tb + j);
                     if (pair_live(e, a.E, src_ok, rank_of)) ranks |= 1ull << rank_of[e];
                 }
-                uint8_t* itr = a.is_token_in_rank + (int64_t(r) * a.T + t) * a.R;
+                uint8_t* itr = a.is_token_in_rank + (int64_t(w.r) * a.T + t) * a.R;
                 for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
             }
             for (int d = 0; d < a.R; ++d) {
                 const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
-                if (lane == 0 && n) atomicAdd(tpr + r * a.R + d, n);
+                if (lane == 0 && n) atomicAdd(tpr + w.r * a.R + d, n);
             }
         }
     }
+    return bad;
+}
+
+// Each live pair's row: first_row(e), the part's first row for its expert, plus
+// its row within the part.
+template <typename FirstRow>
+__device__ __forceinline__ void finish_rows(const LayoutArgs& a, const WarpPart& w, const int (&ev)[kBatch],
+                                            const int (&rk)[kBatch], FirstRow first_row) {
+    const int lane = threadIdx.x & 31;
+    int32_t* rows = a.pair_row + w.pbase;
+    if (w.one_round) {
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = u * 32 + lane;
+            if (u * 32 >= w.np) break;
+            if (p < w.np) rows[p] = rk[u] >= 0 ? first_row(ev[u]) + rk[u] : -1;
+        }
+    } else {
+        for (int p = lane; p < w.np; p += 32) {
+            const int32_t q = rows[p];  // written by this thread in walk_part
+            if (q >= 0) rows[p] = first_row(__ldg(a.topk_idx + w.pbase + p)) + q;
+        }
+    }
+}
+
+// Single CTA: the whole layout in one launch (small problems).  After the walk,
+// the warp histograms are scanned per expert in warp (= (rank, part)) order into
+// each warp's first row, which the pairs add.
+__global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(LayoutArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
+    extern __shared__ int32_t smem[];
+    constexpr int NW = kSmallThreads / 32;
+    const int warp = threadIdx.x >> 5;
+    int32_t* act = smem;
+    int32_t* tpr = smem + kActiveSlots;                        // [R][R]
+    int32_t* rank_of = tpr + kSmallMaxRanks * kSmallMaxRanks;   // [E]
+    int32_t* whist = rank_of + a.E;                            // [NW][E]
+
+    const int wpr = NW / a.R;  // warps per rank, R <= 32
+    const WarpPart w = warp_part(a, warp, wpr);
+    int ev[kBatch], rk[kBatch];
+    load_first_round(a, w, ev);
+    load_tables(a, act, rank_of);
+    for (int i = threadIdx.x; i < NW * a.E; i += blockDim.x) whist[i] = 0;
+    for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) tpr[i] = 0;
+    __syncthreads();
+
+    int32_t* mine = whist + warp * a.E;
+    const bool bad = walk_part(a, w, act, rank_of, mine, tpr, ev, rk);
     if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
 
     // scan the warp histograms per expert in warp order = (rank, part) order
@@ -360,9 +412,9 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
         for (int rr = 0; rr < a.R; ++rr) {
             const int32_t rank_first = run;
             a.expert_rank_offset[int64_t(e) * a.R + rr] = rank_first;
-            for (int w = rr * wpr; w < (rr + 1) * wpr; ++w) {
-                const int32_t c = whist[w * a.E + e];
-                whist[w * a.E + e] = run;
+            for (int wi = rr * wpr; wi < (rr + 1) * wpr; ++wi) {
+                const int32_t c = whist[wi * a.E + e];
+                whist[wi * a.E + e] = run;
                 run += c;
             }
             a.num_tokens_per_expert[int64_t(rr) * a.E + e] = run - rank_first;
@@ -372,29 +424,13 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
     }
     for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) a.num_tokens_per_rank[i] = tpr[i];
     __syncthreads();
-
-    // rows = the warp's first row for the expert + the row within the part
-    if (one_round) {
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int p = u * 32 + lane;
-            if (u * 32 >= np) break;
-            if (p < np) rows[p] = rk[u] >= 0 ? mine[ev[u]] + rk[u] : -1;
-        }
-    } else {
-        for (int p = lane; p < np; p += 32) {
-            const int32_t q = rows[p];  // written by this thread in step 2
-            if (q >= 0) rows[p] = mine[__ldg(base + p)] + q;
-        }
-    }
+    finish_rows(a, w, ev, rk, [&](int e) { return mine[e]; });
 }
 
 // Cluster path (EP_LAYOUT_CLUSTER): the single-CTA algorithm over a thread-block
 // cluster of CL CTAs, one per SM, whose shared memories are reachable from one
-// another.  The cluster's CL * 32 warps split each rank's tokens as the single
-// CTA's warps do (global warp g = CTA * 32 + warp, in (rank, part) order):
-//  1. each warp walks its part as in the single-CTA path (row within the part,
-//     destination ranks), into its CTA's shared memory;
+// another:
+//  1. each warp walks its part into its CTA's shared memory;
 //  2. each CTA scans its own warps' histograms per expert and keeps its totals;
 //     after a cluster barrier, its first row per expert is the sum of the totals
 //     of the CTAs before it, read from their shared memory; the CTA holding a
@@ -410,7 +446,7 @@ __global__ void __launch_bounds__(kSmallThreads) layout_cluster_kernel(LayoutArg
     pdl_launch_dependents();
     extern __shared__ int32_t smem[];
     constexpr int NW = kSmallThreads / 32;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const int cta = int(cluster_ctarank()), CL = int(cluster_nctarank());
     int32_t* act = smem;
     int32_t* tpr = smem + kActiveSlots;                        // [R][R], this CTA's tokens
@@ -419,101 +455,25 @@ __global__ void __launch_bounds__(kSmallThreads) layout_cluster_kernel(LayoutArg
     int32_t* cbase = ctot + a.E;                               // [E] this CTA's first row per expert
     int32_t* whist = cbase + a.E;                              // [NW][E]
 
-    // warps per rank and this warp's token range (in (rank, token) order)
-    const int wpr = CL * NW / a.R;  // R <= 32 <= CL * NW
-    const int gw = cta * NW + warp;
-    const int r = gw / wpr, part = gw - r * wpr;
-    const bool has_rank = r < a.R;
-    const int tw = (a.T + wpr - 1) / wpr;
-    const int wt0 = has_rank ? min(a.T, part * tw) : 0, wt1 = has_rank ? min(a.T, wt0 + tw) : 0;
-    const int64_t pbase = has_rank ? (int64_t(r) * a.T + wt0) * a.k : 0;
-    const int32_t* base = a.topk_idx + pbase;
-    int32_t* rows = a.pair_row + pbase;
-    const int np = (wt1 - wt0) * a.k;
-    const bool one_round = np <= 32 * kBatch;
-
-    int ev[kBatch];  // the first round's experts need no table: load them before the barrier
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-        const int p = u * 32 + lane;
-        ev[u] = p < np ? __ldg(base + p) : -1;
-    }
+    const int wpr = CL * NW / a.R;  // warps per rank, R <= 32 <= CL * NW
+    const WarpPart w = warp_part(a, cta * NW + warp, wpr);
+    int ev[kBatch], rk[kBatch];
+    load_first_round(a, w, ev);
     load_tables(a, act, rank_of);
     for (int i = threadIdx.x; i < NW * a.E; i += blockDim.x) whist[i] = 0;
     for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) tpr[i] = 0;
     __syncthreads();
 
-    const bool src_ok = has_rank && act[r] != 0;
     int32_t* mine = whist + warp * a.E;
-    const uint32_t below = lanemask_lt();
-    const bool lanes_per_token = (a.k & (a.k - 1)) == 0;  // k divides 32: a token is k aligned lanes
-    bool bad = false;
-    int rk[kBatch];  // rows within the part of the last round's pairs (-1: not live)
-    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
-        if (p0 > 0) {
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                const int p = p0 + u * 32 + lane;
-                ev[u] = p < np ? __ldg(base + p) : -1;
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            rk[u] = -1;
-            if (p0 + u * 32 >= np) break;  // the same for the whole warp
-            const int p = p0 + u * 32 + lane;
-            const int e = ev[u];
-            bad |= (e < -1 || e >= a.E);
-            const bool live = pair_live(e, a.E, src_ok, rank_of);
-            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
-            const int32_t b = live ? mine[e] : 0;
-            __syncwarp();
-            if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
-            __syncwarp();
-            rk[u] = live ? b + __popc(m & below) : -1;
-            if (!one_round && p < np) rows[p] = rk[u];
-            if (lanes_per_token) {
-                uint32_t dst = live ? (1u << rank_of[e]) : 0u;
-                for (int o = 1; o < a.k; o <<= 1) dst |= __shfl_xor_sync(0xffffffffu, dst, o);
-                const bool head = p < np && (lane & (a.k - 1)) == 0;
-                if (head) {
-                    uint8_t* itr = a.is_token_in_rank + ((pbase + p) / a.k) * a.R;
-                    for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((dst >> d) & 1u);
-                }
-                for (int d = 0; d < a.R; ++d) {
-                    const int n = __popc(__ballot_sync(0xffffffffu, head && ((dst >> d) & 1u)));
-                    if (lane == 0 && n) atomicAdd(tpr + r * a.R + d, n);
-                }
-            }
-        }
-    }
-    if (!lanes_per_token) {
-        for (int t0 = wt0; t0 < wt1; t0 += 32) {
-            const int t = t0 + lane;
-            uint64_t ranks = 0;
-            if (t < wt1) {
-                const int32_t* tb = a.topk_idx + (int64_t(r) * a.T + t) * a.k;
-                for (int j = 0; j < a.k; ++j) {
-                    const int e = __ldg(tb + j);
-                    if (pair_live(e, a.E, src_ok, rank_of)) ranks |= 1ull << rank_of[e];
-                }
-                uint8_t* itr = a.is_token_in_rank + (int64_t(r) * a.T + t) * a.R;
-                for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
-            }
-            for (int d = 0; d < a.R; ++d) {
-                const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
-                if (lane == 0 && n) atomicAdd(tpr + r * a.R + d, n);
-            }
-        }
-    }
+    const bool bad = walk_part(a, w, act, rank_of, mine, tpr, ev, rk);
     if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
 
     // this CTA's warps, scanned per expert in warp order; ctot = the CTA's total
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         int32_t run = 0;
-        for (int w = 0; w < NW; ++w) {
-            const int32_t c = whist[w * a.E + e];
-            whist[w * a.E + e] = run;
+        for (int wi = 0; wi < NW; ++wi) {
+            const int32_t c = whist[wi * a.E + e];
+            whist[wi * a.E + e] = run;
             run += c;
         }
         ctot[e] = run;
@@ -543,23 +503,7 @@ __global__ void __launch_bounds__(kSmallThreads) layout_cluster_kernel(LayoutArg
         }
     }
     __syncthreads();  // cbase
-
-    if (one_round) {
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int p = u * 32 + lane;
-            if (u * 32 >= np) break;
-            if (p < np) rows[p] = rk[u] >= 0 ? cbase[ev[u]] + mine[ev[u]] + rk[u] : -1;
-        }
-    } else {
-        for (int p = lane; p < np; p += 32) {
-            const int32_t q = rows[p];  // written by this thread in step 1
-            if (q >= 0) {
-                const int e = __ldg(base + p);
-                rows[p] = cbase[e] + mine[e] + q;
-            }
-        }
-    }
+    finish_rows(a, w, ev, rk, [&](int e) { return cbase[e] + mine[e]; });
     cluster_sync();  // expert_rank_offset and recv_count are written; no remote shared reads after this
 
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
