@@ -8,21 +8,31 @@
 // among its expert's live pairs in (source rank, token, slot) order: a stable
 // counting sort keyed by expert.
 //
-// Three paths compute the same result (ep_cfg_t.variant selects one; AUTO
-// takes the chunked path, measured fastest on B200).  Both sort with the same two ideas: lanes holding the same expert
-// are merged (a match mask built from one warp ballot per expert-id bit) so
-// one leader updates the group's count (a warp-aggregated update), and a
-// pair's row inside a run of 32 consecutive
+// Four paths compute the same result (ep_cfg_t.variant selects one; AUTO takes
+// the single CTA up to 2048 pairs, the cluster up to 65536, the chunked path
+// beyond: the fastest on B200 in each range).  All sort with the same two ideas:
+// lanes holding the same expert are merged (a match mask built from one warp
+// ballot per expert-id bit) so one leader updates the group's count (a
+// warp-aggregated update), and a pair's row inside a run of 32 consecutive
 // pairs is its running count plus its rank among equal experts to its left
 // (popc of the match mask below it).  Destination ranks come from a shared
 // table rank_of[e] (-1 when that rank is masked), so no pair test divides.
 //
-// Single-CTA path (EP_LAYOUT_SINGLE_CTA; R <= 32, E <= 1024, <= 32768 pairs;
-// AUTO up to 4096 pairs): one 1024-thread CTA, one launch, no workspace.  Each rank's tokens are split
-// among 32/R warps in (rank, token) order; every warp builds a private
-// histogram of its part, the CTA scans them over warps per expert (which also
-// yields expert_rank_offset, num_tokens_per_expert, recv_count), and every
-// warp then walks its part again assigning rows.
+// Single-CTA path (EP_LAYOUT_SINGLE_CTA; R <= 32, E <= 1024, <= 32768 pairs):
+// one 1024-thread CTA, one launch, no workspace.  Each rank's tokens are split
+// among 32/R warps in (rank, token) order; every warp walks its part once,
+// finding each pair's row within the part and each token's destination ranks;
+// the CTA scans the warp histograms per expert (which also yields
+// expert_rank_offset, num_tokens_per_expert, recv_count) and the pairs add
+// their warp's first row.
+//
+// Cluster path (EP_LAYOUT_CLUSTER; R <= 32, E <= 1024, <= 65536 pairs): the
+// same over a thread-block cluster of 2 to 16 CTAs whose shared memories see
+// one another; a CTA's first rows come from the other CTAs' totals, read
+// through distributed shared memory after a cluster barrier.
+//
+// Fused path (EP_LAYOUT_FUSED): the chunked path below in one cooperative
+// launch with two bounded grid barriers.
 //
 // Chunked path (EP_LAYOUT_CHUNKED; any shape): each rank's tokens are cut into
 // C contiguous chunks (chunk g = r*C + c, ordered like the sort key; about a

@@ -29,6 +29,17 @@
  *                  (GPU operations), with the placement rule "add one replica
  *                  at a time to the expert with the largest load/replicas,
  *                  ties to the lowest id".
+ *   ep_dispatch_fp8 -- Buffer.low_latency_dispatch with use_fp8=True (and its
+ *                  round_scale / use_ue8m0 options) on the NeMo page.
+ *   ep_normal_layout, ep_normal_dispatch, ep_normal_combine -- the normal
+ *                  (high-throughput) Buffer.dispatch / Buffer.combine of the
+ *                  NeMo page: one copy per destination rank, unweighted combine.
+ *   ep_replica_weight_sync, ep_replica_grad_reduce -- "Replica weight sync" and
+ *                  "Replica gradient reduction" of the UltraEP page.
+ *   ep_layout_noalloc, ep_layout_path and the *_workspace_bytes queries have
+ *                  no counterpart on the pages; they serve callers of this
+ *                  library (scratch without allocation, which path a call takes,
+ *                  scratch sizes).
  *
  * Conventions shared by every entry point
  *   - Every pointer argument is a DEVICE pointer owned by the caller, except
