@@ -19,7 +19,11 @@ Reported:
   roofline     the dominant kernel's achieved GB/s against the measured copy
                bandwidth of this GPU type (MEASURED_PEAKS.json);
   e2e          the same metric with host buffers: every step copies its inputs
-               from pinned host memory and reads the output back;
+               from pinned host memory and reads the output back; two device
+               buffer sets let one step's upload overlap the previous step's
+               download and compute;
+  clocks       SM clock (median) and clock-event reasons sampled through NVML
+               every 5 ms while the timed region runs;
   cpu_baseline the plain single-threaded CPU oracle on a bounded sample of the
                same workload (rank 0, one GPU only).
 
