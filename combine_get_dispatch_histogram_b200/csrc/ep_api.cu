@@ -1,5 +1,6 @@
 // ep_api.cu -- library-wide entry points (error names, version) and the host
 // helpers the launchers share (device queries, launch-error mapping).
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -10,8 +11,9 @@ namespace ep {
 
 namespace {
 constexpr int kMaxDevices = 64;
-int g_sms[kMaxDevices] = {0};
-int g_smem[kMaxDevices] = {0};
+// per-device caches; 0 = not asked yet (a race only repeats the same query)
+std::atomic<int> g_sms[kMaxDevices] = {};
+std::atomic<int> g_smem[kMaxDevices] = {};
 
 int current_device() {
     int dev = -1;
@@ -23,24 +25,24 @@ int current_device() {
 int sm_count() {
     const int dev = current_device();
     if (dev < 0) return -1;
-    if (g_sms[dev] == 0) {
-        int v = 0;
+    int v = g_sms[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
         if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-        g_sms[dev] = v;
+        g_sms[dev].store(v, std::memory_order_relaxed);
     }
-    return g_sms[dev];
+    return v;
 }
 
 int max_smem_optin() {
     const int dev = current_device();
     if (dev < 0) return 48 * 1024;
-    if (g_smem[dev] == 0) {
-        int v = 0;
+    int v = g_smem[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
         if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
             return 48 * 1024;
-        g_smem[dev] = v;
+        g_smem[dev].store(v, std::memory_order_relaxed);
     }
-    return g_smem[dev];
+    return v;
 }
 
 int launch_result() { return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA; }

@@ -33,6 +33,7 @@
 // current one, so it runs up to S stages ahead: S * k * piece bytes of loads
 // in flight per SM.
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 
 #include <cuda_bf16.h>
@@ -317,13 +318,15 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(CombineArgs a) {
 
 template <int U, bool NORMAL>
 int launch_combine_vec(const CombineArgs& a, const ep_cfg_t& cfg, int sms, cudaStream_t stream) {
-    static int per_sm[64] = {0};
+    static std::atomic<int> per_sm[64];  // resident CTAs per SM, per device; 0 = not asked yet
     int dev = 0;
     cudaGetDevice(&dev);
-    int& occ = per_sm[dev & 63];
-    if (occ == 0 &&
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, combine_vec_kernel<U, NORMAL>, 256, 0) != cudaSuccess)
-        return EP_ERR_CUDA;
+    int occ = per_sm[dev & 63].load(std::memory_order_relaxed);
+    if (occ == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, combine_vec_kernel<U, NORMAL>, 256, 0) != cudaSuccess)
+            return EP_ERR_CUDA;
+        per_sm[dev & 63].store(occ, std::memory_order_relaxed);
+    }
     int64_t grid = int64_t(sms) * std::max(1, occ);
     if (cfg.max_ctas > 0) grid = std::min<int64_t>(grid, cfg.max_ctas);
     const int64_t warps_needed = ceil_div(int64_t(a.R) * a.T * ceil_div(a.row_bytes >> 4, 32 * U), 1);

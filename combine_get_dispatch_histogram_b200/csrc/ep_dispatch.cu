@@ -29,6 +29,7 @@
 // the unit being refilled is prefetched one iteration ahead into registers
 // and parked in shared memory for the consumer.
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 
 #include "ep.h"
@@ -282,13 +283,15 @@ __global__ void __launch_bounds__(256) dispatch_vec_kernel(DispatchArgs a) {
 
 template <int U>
 int launch_dispatch_vec(const DispatchArgs& a, const ep_cfg_t& cfg, int sms, cudaStream_t stream) {
-    static int per_sm[64] = {0};
+    static std::atomic<int> per_sm[64];  // resident CTAs per SM, per device; 0 = not asked yet
     int dev = 0;
     cudaGetDevice(&dev);
-    int& occ = per_sm[dev & 63];
-    if (occ == 0 &&
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, dispatch_vec_kernel<U>, 256, 0) != cudaSuccess)
-        return EP_ERR_CUDA;
+    int occ = per_sm[dev & 63].load(std::memory_order_relaxed);
+    if (occ == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, dispatch_vec_kernel<U>, 256, 0) != cudaSuccess)
+            return EP_ERR_CUDA;
+        per_sm[dev & 63].store(occ, std::memory_order_relaxed);
+    }
     int64_t grid = int64_t(sms) * std::max(1, occ);
     if (cfg.max_ctas > 0) grid = std::min<int64_t>(grid, cfg.max_ctas);
     const int64_t units = (a.n_units / a.n_pieces) * ceil_div(a.row_bytes >> 4, 32 * U);

@@ -2,6 +2,8 @@
 // queries, launch-error mapping.  Internal to the library.
 #pragma once
 
+#include <algorithm>
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -52,6 +54,48 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 // Streaming-multiprocessor count of the current device (cached per device).
+// Which thread-block cluster sizes of one kernel the device can hold at once:
+// [device][CTAs], 0 = not asked yet, 1 = fits, -1 = does not (static storage,
+// so it starts zeroed; a race only repeats the same query).
+struct ClusterFitCache {
+    std::atomic<int> v[64][17];
+};
+
+// The largest cluster of at most `want` CTAs (trying want, then 8, 4, 2) of
+// `kernel` with `threads` threads and `smem` bytes of dynamic shared memory that
+// the current device can hold at once, as the occupancy calculator answers;
+// 1 if none.  Ask with the kernel's largest `smem` so that one answer holds for
+// every shape; the kernel's dynamic shared-memory limit must already allow it.
+template <typename... KArgs>
+int fitting_cluster(void (*kernel)(KArgs...), int want, int threads, size_t smem, ClusterFitCache& cache) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+    int cl = std::min(16, std::max(1, want));
+    for (; cl > 1; cl = cl > 8 ? 8 : cl / 2) {
+        int known = cache.v[dev][cl].load(std::memory_order_relaxed);
+        if (known == 0) {
+            cudaLaunchConfig_t lc = {};
+            lc.gridDim = dim3(cl);
+            lc.blockDim = dim3(threads);
+            lc.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = cl;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            lc.attrs = attr;
+            lc.numAttrs = 1;
+            int n = 0;
+            const bool ok = cudaOccupancyMaxActiveClusters(&n, kernel, &lc) == cudaSuccess && n >= 1;
+            if (!ok) cudaGetLastError();
+            known = ok ? 1 : -1;
+            cache.v[dev][cl].store(known, std::memory_order_relaxed);
+        }
+        if (known > 0) return cl;
+    }
+    return 1;
+}
+
 int sm_count();
 
 // Largest dynamic shared memory a CTA may opt into on the current device.

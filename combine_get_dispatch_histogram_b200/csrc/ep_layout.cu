@@ -870,24 +870,19 @@ size_t layout_ws_tpr_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
 
 // Largest grid of the fused kernel that can be co-resident on the current device (0 if none).
 int fused_capacity(int threads, size_t smem) {
-    static int cached[64][kMaxWarps + 1] = {};
+    // asked on every call: the answer depends on smem, and only the fused path asks
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
     int coop = 0;
     if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop) return 0;
-    int& c = cached[dev & 63][threads / 32];
-    if (c == 0) {
-        int per_sm = 0;
-        if (smem > 48 * 1024 &&
-            cudaFuncSetAttribute(layout_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-                cudaSuccess)
-            return 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel, threads, smem) !=
+    int per_sm = 0;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(layout_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
             cudaSuccess)
-            return 0;
-        c = per_sm * sm_count();
-    }
-    return c;
+        return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel, threads, smem) != cudaSuccess)
+        return 0;
+    return per_sm * sm_count();
 }
 
 }  // namespace
@@ -903,34 +898,7 @@ size_t cluster_smem_bytes(const ep_dims_t& d) {
                   (kSmallThreads / 32) * d.num_experts) * 4;
 }
 
-// CTAs of the layout cluster for `pairs` pairs: one per kClusterPairsPerCta, at
-// least 2, at most kClusterMaxCtas, and no more than the device can hold at once
-// (asked of the occupancy calculator once per size and cached).
-int cluster_ctas(int64_t pairs, size_t smem) {
-    static int max_ok[kClusterMaxCtas + 1] = {};  // 0 unknown, 1 fits, -1 does not
-    int cl = int(std::min<int64_t>(kClusterMaxCtas, std::max<int64_t>(2, ceil_div(pairs, kClusterPairsPerCta))));
-    for (; cl >= 2; cl = cl > 8 ? 8 : cl / 2) {
-        if (max_ok[cl] == 0) {
-            cudaLaunchConfig_t lc = {};
-            lc.gridDim = dim3(cl);
-            lc.blockDim = dim3(kSmallThreads);
-            lc.dynamicSmemBytes = smem;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = cl;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            lc.attrs = attr;
-            lc.numAttrs = 1;
-            int n = 0;
-            const bool ok = cudaOccupancyMaxActiveClusters(&n, layout_cluster_kernel, &lc) == cudaSuccess && n >= 1;
-            if (!ok) cudaGetLastError();
-            max_ok[cl] = ok ? 1 : -1;
-        }
-        if (max_ok[cl] > 0) return cl;
-    }
-    return 1;
-}
+ClusterFitCache g_layout_cluster_fit;
 
 size_t fused_smem_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
     return size_t(2 * kActiveSlots + 2 * d.num_experts + lg.warps * d.num_experts) * 4;
@@ -1048,12 +1016,19 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     }
     if (path == EP_LAYOUT_CLUSTER) {
         const size_t smem = cluster_smem_bytes(d);
-        if (cudaFuncSetAttribute(layout_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-                cudaSuccess ||
+        ep_dims_t widest = d;  // the largest shared-memory need of the path (E = kSmallMaxExperts)
+        widest.num_experts = kSmallMaxExperts;
+        const size_t smem_max = cluster_smem_bytes(widest);
+        if (cudaFuncSetAttribute(layout_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem_max)) != cudaSuccess ||
             cudaFuncSetAttribute(layout_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                 cudaSuccess)
             return EP_ERR_CUDA;
-        const int cl = cluster_ctas(int64_t(d.num_ranks) * d.num_tokens * d.num_topk, smem);
+        // one CTA per kClusterPairsPerCta pairs, 2 to kClusterMaxCtas, as many as fit at once
+        const int64_t pairs = int64_t(d.num_ranks) * d.num_tokens * d.num_topk;
+        const int want = int(std::min<int64_t>(kClusterMaxCtas,
+                                               std::max<int64_t>(2, ceil_div(pairs, kClusterPairsPerCta))));
+        const int cl = fitting_cluster(layout_cluster_kernel, want, kSmallThreads, smem_max, g_layout_cluster_fit);
         cudaLaunchConfig_t lc = {};
         lc.gridDim = dim3(cl);
         lc.blockDim = dim3(kSmallThreads);

@@ -265,35 +265,7 @@ __global__ void __launch_bounds__(kRerouteClusterThreads) reroute_cluster_kernel
 
 constexpr int kRerouteMaxBlocks = 256;
 
-// CTAs of the reroute cluster: one per kRerouteClusterPairsPerCta pairs, at most
-// kRerouteClusterMaxCtas, fewer if the device cannot hold that cluster at once
-// (asked of the occupancy calculator once per size and cached).
-int reroute_cluster_ctas(int64_t n_pairs, size_t smem) {
-    static int fits[kRerouteClusterMaxCtas + 1] = {};  // 0 unknown, 1 fits, -1 does not
-    int cl = int(std::min<int64_t>(kRerouteClusterMaxCtas,
-                                   std::max<int64_t>(1, ceil_div(n_pairs, kRerouteClusterPairsPerCta))));
-    for (; cl > 1; cl = cl > 8 ? 8 : cl / 2) {
-        if (fits[cl] == 0) {
-            cudaLaunchConfig_t lc = {};
-            lc.gridDim = dim3(cl);
-            lc.blockDim = dim3(kRerouteClusterThreads);
-            lc.dynamicSmemBytes = smem;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = cl;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            lc.attrs = attr;
-            lc.numAttrs = 1;
-            int n = 0;
-            const bool ok = cudaOccupancyMaxActiveClusters(&n, reroute_cluster_kernel, &lc) == cudaSuccess && n >= 1;
-            if (!ok) cudaGetLastError();
-            fits[cl] = ok ? 1 : -1;
-        }
-        if (fits[cl] > 0) return cl;
-    }
-    return 1;
-}
+ClusterFitCache g_reroute_cluster_fit;
 
 int reroute_blocks(int64_t n_pairs) {
     const int64_t by_size = ceil_div(n_pairs, int64_t(kRerouteThreads) * 4);
@@ -350,12 +322,17 @@ extern "C" int ep_reroute(int32_t num_ranks, int32_t num_tokens, int32_t num_top
     if (variant != EP_REROUTE_CLUSTER && variant != EP_REROUTE_TWO_LAUNCH) return EP_ERR_INVALID;
     if (variant == EP_REROUTE_CLUSTER) {
         const size_t smem = size_t(4 * num_logical + 1) * 4;
-        if (cudaFuncSetAttribute(reroute_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-                cudaSuccess ||
+        const size_t smem_max = size_t(4 * kRerouteMaxLogical + 1) * 4;  // the path's largest need
+        if (cudaFuncSetAttribute(reroute_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem_max)) != cudaSuccess ||
             cudaFuncSetAttribute(reroute_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                 cudaSuccess)
             return EP_ERR_CUDA;
-        const int cl = reroute_cluster_ctas(n_pairs, smem);
+        // one CTA per kRerouteClusterPairsPerCta pairs, up to kRerouteClusterMaxCtas, as many as fit
+        const int want = int(std::min<int64_t>(kRerouteClusterMaxCtas,
+                                               std::max<int64_t>(1, ceil_div(n_pairs, kRerouteClusterPairsPerCta))));
+        const int cl = fitting_cluster(reroute_cluster_kernel, want, kRerouteClusterThreads, smem_max,
+                                       g_reroute_cluster_fit);
         a.per_block = std::max<int64_t>(1, ceil_div(n_pairs, cl));
         cudaLaunchConfig_t lc = {};
         lc.gridDim = dim3(cl);
