@@ -540,20 +540,27 @@ def oracle_sample(w: inputs.Workload, sample_tokens: int, inp=None):
     x = np.ascontiguousarray(inp.x[:, :Ts])
     wts = np.ascontiguousarray(inp.topk_weights[:, :Ts])
     E, H, R = w.num_physical, w.hidden, w.num_ranks
+    stages = {}
     t0 = time.perf_counter()
     if w.num_extra:
         idx = oracle.reroute(idx, w.num_experts, w.num_extra)["topk_idx_phys"]
+        stages["reroute"] = time.perf_counter() - t0
+    t1 = time.perf_counter()
     ref = oracle.layout(idx, inp.active, E)
+    t2 = time.perf_counter()
     packed, _ = oracle.dispatch(x, idx, ref)
+    t3 = time.perf_counter()
     oracle.combine(packed, ref.list_base[:-1], idx, wts, ref.pair_row, inp.active, E)
-    secs = time.perf_counter() - t0
+    t4 = time.perf_counter()
+    stages.update(layout=t2 - t1, dispatch=t3 - t2, combine=t4 - t3)
+    secs = t4 - t0
     live = int(ref.recv_count.sum())
     sent = int(ref.is_token_in_rank.reshape(R * Ts, R).max(axis=1).sum())
     d_b, c_b = algorithmic_bytes(H, sent, live, R * Ts)
     return dict(value=round((d_b + c_b) / secs / 1e9, 3), unit="GB/s", cores=1, kind="oracle",
                 sample=f"first {Ts} of {w.num_tokens} tokens of each of the {R} ranks "
                        f"(reroute + layout + dispatch + combine, single-threaded C, float64 combine)",
-                seconds=round(secs, 3))
+                seconds=round(secs, 3), stage_seconds={k_: round(v, 4) for k_, v in stages.items()})
 
 
 def cpu_model():
@@ -579,6 +586,9 @@ def run_reference(args, world):
     value = statistics.median(s["value"] for s in samples)
     base = dict(samples[0])
     base["value"] = value
+    base["seconds"] = round(secs, 3)
+    base["stage_seconds"] = {k_: round(statistics.median(s_["stage_seconds"][k_] for s_ in samples), 4)
+                             for k_ in samples[0]["stage_seconds"]}
     base["host_cores"] = os.cpu_count()
     base["cpu_model"] = cpu_model()
     return {
