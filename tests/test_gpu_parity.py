@@ -463,3 +463,25 @@ def test_cluster_layout_sizes(T):
     torch.cuda.synchronize()
     check_layout(lay, ref, f"cluster T={T}")
     assert int(lay.status.item()) == ref.status
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_one_launch_layout_fuzz(seed):
+    """Random shapes within the one-launch paths' limits (R <= 32, E <= 1024), each through the
+    single-CTA, cluster and chunked paths: every layout output bit-exact against the oracle."""
+    rng = np.random.default_rng(9000 + seed)
+    R = int(rng.integers(1, 33))
+    E = R * int(rng.integers(1, max(2, 1024 // R + 1)))
+    k = int(rng.integers(1, min(E, 32) + 1))
+    T = int(rng.choice([0, 1, int(rng.integers(2, 40)), int(rng.integers(40, 300))]))
+    T = min(T, 32768 // (R * k))                    # within the single-CTA limit
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k) if T else \
+        np.zeros((R, 0, k), np.int64)
+    idx = np.where(rng.random(idx.shape) < 0.1, -1, idx).astype(np.int32)
+    act = (rng.random(R) > 0.2).astype(np.uint8)
+    ref = oracle.layout(idx, act, E)
+    for path in (LAYOUT_SINGLE_CTA, LAYOUT_CLUSTER, LAYOUT_CHUNKED):
+        lay = ep.ep_layout(i32_dev(idx), u8_dev(act), E, hidden=8, cfg=dict(variant=path))
+        torch.cuda.synchronize()
+        check_layout(lay, ref, f"seed {seed} R={R} T={T} k={k} E={E} path {path}")
+        assert int(lay.status.item()) == ref.status, (seed, path)
