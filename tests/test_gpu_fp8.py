@@ -138,3 +138,29 @@ def test_fp8_dispatch_rejects_bad_hidden():
     x = torch.zeros((R, T, 200), dtype=torch.bfloat16, device=dev())
     with pytest.raises(ep.EPError):
         ep.ep_dispatch_fp8(x, idx, pr, rc, E)                          # not a multiple of 128
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_fp8_dispatch_fuzz(seed):
+    """Random shapes (H any multiple of 128 up to 8192, so 1 to 8 consumer warps and different ring
+    depths on the bulk path), masks, unselected slots, all scale formats, both data paths."""
+    rng = np.random.default_rng(7000 + seed)
+    fmt = FORMATS[seed % 3]
+    R = int(rng.integers(1, 9))
+    E = R * int(rng.integers(1, 17))
+    k = int(rng.integers(1, min(E, 8) + 1))
+    T = int(rng.choice([0, 1, int(rng.integers(2, 65))]))
+    unit = 512 if fmt == ep.EP_FP8_SCALE_UE8M0 else 128
+    H = unit * int(rng.integers(1, 8192 // unit + 1))
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k) if T else \
+        np.zeros((R, 0, k), np.int64)
+    idx = np.where(rng.random(idx.shape) < 0.1, -1, idx).astype(np.int32)
+    scale = 10.0 ** rng.uniform(-4, 4, size=(R, T, 1))
+    x = (rng.standard_normal((R, T, H)) * scale).astype(np.float32)
+    bits = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    w = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+    act = (rng.random(R) > 0.2).astype(np.uint8)
+    inp = inputs.Inputs(idx, w, bits, act)
+    for variant in VARIANTS:
+        check_fp8(inp, E, fmt, f"seed {seed} R={R} T={T} k={k} E={E} H={H} fmt {fmt} variant {variant}",
+                  dict(variant=variant))
