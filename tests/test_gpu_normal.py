@@ -110,3 +110,29 @@ def test_normal_layout_token_tiles(R, T):
     act = np.ones(R, np.uint8)
     act[R - 2] = 0
     check_normal(inputs.Inputs(idx, wts, x, act), E, f"R={R} T={T}")
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_normal_mode_fuzz(seed):
+    """Random shapes up to 32 ranks, alignments, receive capacities (some too small), unselected
+    slots, a mask flipped before combine; both data paths where they apply."""
+    rng = np.random.default_rng(5000 + seed)
+    R = int(rng.integers(1, 33))
+    E = R * int(rng.integers(1, 9))
+    k = int(rng.integers(1, min(E, 8) + 1))
+    T = int(rng.choice([0, 1, int(rng.integers(2, 100))]))
+    H = 8 * int(rng.integers(1, 65))
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k) if T else \
+        np.zeros((R, 0, k), np.int64)
+    idx = np.where(rng.random(idx.shape) < 0.1, -1, idx).astype(np.int32)
+    x = inputs.bf16_tokens(rng, R * T, H).reshape(R, T, H)
+    wts = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+    act = (rng.random(R) > 0.2).astype(np.uint8)
+    now = act.copy()
+    now[int(rng.integers(0, R))] ^= 1
+    alignment = int(rng.choice([1, 4, 32]))
+    capacity = None if seed % 4 else int(rng.integers(0, R * T + 1))
+    cfgs = [dict(variant=1), dict(variant=2)] if R <= 8 else [None]
+    for cfg in cfgs:
+        check_normal(inputs.Inputs(idx, wts, x, act), E, f"seed {seed} R={R} T={T} k={k} H={H} cfg {cfg}",
+                     alignment=alignment, capacity=capacity, active_combine=now, cfg=cfg)
