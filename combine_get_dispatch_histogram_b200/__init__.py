@@ -13,6 +13,7 @@ from .ep import (  # noqa: F401
     ep_layout,
     ep_layout_workspace_bytes,
     ep_layout_path,
+    ep_diag_wait_timeout,
     ep_normal_combine,
     ep_normal_dispatch,
     ep_normal_layout,

@@ -664,6 +664,14 @@ __device__ bool grid_barrier(uint64_t* flags, int G, uint64_t value, int32_t* st
     return passed != 0;
 }
 
+// Diagnostic (ep_diag_wait_timeout): one CTA enters the fused path's grid barrier
+// as if the grid had two CTAs, so it waits for a flag that nothing sets; the
+// bounded wait gives up after kWaitTimeoutNs, flags EP_STATUS_TIMEOUT and the
+// kernel returns, leaving the context usable.
+__global__ void __launch_bounds__(32) diag_wait_timeout_kernel(uint64_t* flags, int32_t* status) {
+    grid_barrier(flags, 2, 1, status);
+}
+
 __global__ void __launch_bounds__(32 * kMaxWarps) layout_fused_kernel(LayoutArgs a) {
     pdl_wait();  // nothing upstream is read before this
     pdl_launch_dependents();
@@ -1072,5 +1080,11 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
             cudaSuccess ||
         launch_pdl(layout_rank_kernel, dim3(lg.G), dim3(32 * W), rank_smem, s, a) != cudaSuccess)
         return EP_ERR_CUDA;
+    return launch_result();
+}
+
+extern "C" int ep_diag_wait_timeout(void* flags, int32_t* status, void* stream) {
+    if (!flags || !status || (reinterpret_cast<uintptr_t>(flags) & 7u)) return EP_ERR_INVALID;
+    diag_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t*>(flags), status);
     return launch_result();
 }

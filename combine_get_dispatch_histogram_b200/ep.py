@@ -79,6 +79,8 @@ def load_library(path: str = LIB_PATH):
     lib.ep_layout_workspace_bytes.restype = SZ
     lib.ep_layout_path.argtypes = [Dims, Cfg]
     lib.ep_layout_path.restype = ctypes.c_int
+    lib.ep_diag_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    lib.ep_diag_wait_timeout.restype = ctypes.c_int
     lib.ep_layout.argtypes = [Dims, P, P, P, SZ, P, P, P, P, P, P, P, Cfg, P]
     lib.ep_layout.restype = ctypes.c_int
     lib.ep_dispatch.argtypes = [Dims, P, P, P, P, P, P, Cfg, P]
@@ -180,6 +182,22 @@ def ep_layout_path(num_ranks: int, num_tokens: int, num_topk: int, num_experts: 
     if rc < 0:
         _check("ep_layout_path", rc)
     return rc
+
+
+def ep_diag_wait_timeout(flags: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """Run the bounded-wait diagnostic (``ep_diag_wait_timeout``); returns the status word.
+
+    With ``flags`` None, a zeroed 16-byte buffer is used, so the wait runs out (about 2 s).
+    """
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if flags is None:
+        flags = torch.zeros(2, dtype=torch.int64, device=dev)
+    _need(flags, "flags", torch.int64, (2,), dev)
+    status = _status(dev, status)
+    _check("ep_diag_wait_timeout", lib.ep_diag_wait_timeout(_ptr(flags), _ptr(status), _stream(dev, stream)))
+    return status
 
 
 def ep_layout_workspace_bytes(num_ranks: int, num_tokens: int, num_topk: int, num_experts: int,

@@ -166,6 +166,19 @@ EP_API size_t ep_layout_workspace_bytes(ep_dims_t d);
  */
 EP_API int ep_layout_path(ep_dims_t d, ep_cfg_t cfg);
 
+/*
+ * ep_diag_wait_timeout -- diagnostic of the bounded waits (the pages have no
+ * counterpart).  One CTA enters the grid barrier of the fused layout path as if
+ * the grid had two CTAs, so it waits for a flag that nothing sets; after the
+ * library's wait limit (2 s) it gives up, ORs EP_STATUS_TIMEOUT into *status and
+ * returns.  Nothing faults or hangs and the context stays usable: this shows
+ * how every bounded wait of the library ends.
+ * in:  flags   >= 16 bytes of device memory, 8-byte aligned, zero-filled (a
+ *              nonzero second word, 1 or 2, lets the wait pass at once)
+ * out: status  int32 device word
+ */
+EP_API int ep_diag_wait_timeout(void *flags, int32_t *status, void *stream);
+
 
 /*
  * ep_layout -- per-expert / per-rank histogram, prefix sums and stable rows.
