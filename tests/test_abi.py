@@ -123,3 +123,21 @@ def test_layout_path_choice(lib):
     with pytest.raises(ep.EPError) as ei:
         ep.ep_layout_path(8, 16, 8, 256, cfg=dict(variant=9))
     assert ei.value.code == ep.EP_ERR_INVALID
+
+
+def test_fp8_workspace_and_diag_validation(lib):
+    """FP8 scratch = one scale word per 128 channels (per 512 for UE8M0) per token, 16-byte
+    rounded; 0 for a hidden size the cast cannot take.  The wait diagnostic rejects null or
+    misaligned pointers on the host, before any launch."""
+    import ctypes
+
+    from combine_get_dispatch_histogram_b200 import ep
+
+    assert ep.ep_dispatch_fp8_workspace_bytes(8, 4096, 8, 256, 7168, ep.EP_FP8_SCALE_F32) == 8 * 4096 * 56 * 4
+    assert ep.ep_dispatch_fp8_workspace_bytes(8, 4096, 8, 256, 7168, ep.EP_FP8_SCALE_UE8M0) == 8 * 4096 * 14 * 4
+    assert ep.ep_dispatch_fp8_workspace_bytes(1, 3, 1, 8, 128, ep.EP_FP8_SCALE_POW2) == 16   # 12 B -> 16
+    assert ep.ep_dispatch_fp8_workspace_bytes(2, 4, 2, 8, 200, ep.EP_FP8_SCALE_F32) == 0     # H % 128 != 0
+    word = ctypes.c_int32(0)
+    assert lib.ep_diag_wait_timeout(None, ctypes.byref(word), None) == ep.EP_ERR_INVALID
+    assert lib.ep_diag_wait_timeout(ctypes.c_void_p(4), ctypes.byref(word), None) == ep.EP_ERR_INVALID
+    assert lib.ep_diag_wait_timeout(ctypes.c_void_p(8), None, None) == ep.EP_ERR_INVALID
