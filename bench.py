@@ -24,8 +24,9 @@ Reported:
                download and compute;
   clocks       SM clock (median) and clock-event reasons sampled through NVML
                every 5 ms while the timed region runs;
-  cpu_baseline the plain single-threaded CPU oracle on a bounded sample of the
-               same workload (rank 0, one GPU only).
+  cpu_baseline the plain single-threaded CPU oracle, pinned to one host core,
+               over the same workload once (rank 0, one GPU only), timed per
+               stage.
 
 ``--impl reference`` times that CPU oracle alone as the reference arm.
 Multi-GPU (torchrun): every rank runs an independent replica (the emulated
@@ -244,6 +245,22 @@ def whole_job_gbs(total_bytes: float, ms: float) -> float:
     return total_bytes / (ms * 1e-3) / 1e9
 
 
+def stats_ms(samples):
+    """Median, min and max of per-call times (ms)."""
+    return {"median": statistics.median(samples), "min": min(samples), "max": max(samples)}
+
+
+def config_of(w: inputs.Workload, world: int) -> dict:
+    """The workload description both arms report (identical dicts for the same run)."""
+    R, T, H = w.num_ranks, w.num_tokens, w.hidden
+    slab_bytes = w.num_physical * R * T * H * 2
+    return {"workload": f"{w.name} " + " ".join(f"{k_}={v}" for k_, v in w.describe().items()),
+            **w.describe(), "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
+            "emulated_ep_ranks": R,
+            "l2": "no flush: inputs larger than L2 (x %.0f MB, receive slab %.1f GB)"
+                  % (R * T * H * 2 / 1e6, slab_bytes / 1e9)}
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def algorithmic_bytes(H: int, tokens_sent: int, live_pairs: int, tokens_out: int):
@@ -251,17 +268,14 @@ def algorithmic_bytes(H: int, tokens_sent: int, live_pairs: int, tokens_out: int
     return row * (tokens_sent + live_pairs), row * (live_pairs + tokens_out)
 
 
-def run_ours(args, rank, world, local_rank):
+def run_ours(args, rank, world, local_rank, w, inp):
     import torch
-    import torch.distributed as dist
 
     from combine_get_dispatch_histogram_b200 import ep
 
     ep.load_library()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = inputs.named(args.workload)
-    inp = inputs.make_inputs(w)
     R, T, k, H = w.num_ranks, w.num_tokens, w.num_topk, w.hidden
     E = w.num_physical
     cap = R * T
@@ -381,21 +395,22 @@ def run_ours(args, rank, world, local_rank):
     rank_barrier(world, local_rank)
     total_ms = t_start.elapsed_time(t_end)
     if graphs is None:
-        lay_ms = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
-        dis_ms = sum(e[1].elapsed_time(e[2]) for e in events) / args.steps
-        com_ms = sum(e[2].elapsed_time(e[3]) for e in events) / args.steps
+        per_part = [[e[i].elapsed_time(e[i + 1]) for e in events] for i in range(len(parts))]
     else:
-        part_ms = []
+        # each part replayed alone as its own graph, one event pair per replay
+        per_part = []
         for g in graphs[1:]:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
             with torch.cuda.stream(stream):
-                e0.record(stream)
-                for _ in range(args.steps):
+                for e0, e1 in evs:
+                    e0.record(stream)
                     g.replay()
-                e1.record(stream)
+                    e1.record(stream)
             stream.synchronize()
-            part_ms.append(e0.elapsed_time(e1) / args.steps)
-        lay_ms, dis_ms, com_ms = part_ms
+            per_part.append([e0.elapsed_time(e1) for e0, e1 in evs])
+    part_stats = [stats_ms(v) for v in per_part]
+    lay_ms, dis_ms, com_ms = (st["median"] for st in part_stats)
     if int(status.item()) != 0:
         raise SystemExit(f"device status {int(status.item())} after the timed steps")
 
@@ -460,8 +475,10 @@ def run_ours(args, rank, world, local_rank):
         assert np.array_equal(h_out[(n - 1) % 2].numpy(), out.view(torch.int16).cpu().numpy())
 
     # ---------------------------------------------------------------- reduce over ranks
-    total_ms, lay_ms, dis_ms, com_ms, e2e_ms = reduce_over_ranks(
-        [total_ms, lay_ms, dis_ms, com_ms, e2e["ms"] if e2e else 0.0], world, dev, "max")
+    flat = [v for st in part_stats for v in (st["median"], st["min"], st["max"])]
+    total_ms, e2e_ms, *flat = reduce_over_ranks([total_ms, e2e["ms"] if e2e else 0.0] + flat, world, dev, "max")
+    part_stats = [dict(median=flat[3 * i], min=flat[3 * i + 1], max=flat[3 * i + 2]) for i in range(len(parts))]
+    lay_ms, dis_ms, com_ms = (st["median"] for st in part_stats)
     ms_per_step = total_ms / args.steps
     step_bytes = d_bytes + c_bytes
     (job_bytes,) = reduce_over_ranks([step_bytes], world, dev, "sum")
@@ -485,14 +502,13 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"{w.name} " + " ".join(f"{k_}={v}" for k_, v in w.describe().items()),
-                   **w.describe(), "parallelism": f"replicas{world}" if world > 1 else "single-gpu",
-                   "emulated_ep_ranks": R,
-                   "l2": "no flush: inputs larger than L2 (x %.0f MB, receive slab %.1f GB)"
-                         % (R * T * H * 2 / 1e6, slab_bytes / 1e9)},
+        "config": config_of(w, world),
         "dispatch_us": round(dis_ms * 1e3, 2),
         "combine_us": round(com_ms * 1e3, 2),
         "layout_us": round(lay_ms * 1e3, 2),
+        "kernel_us": {name: {k_: round(v * 1e3, 2) for k_, v in st.items()}
+                      for name, st in zip(("layout", "dispatch", "combine"), part_stats)},
+        "kernel_us_stat": "median over the timed steps (min, max beside it); max over ranks",
         "dispatch_gbs": round(dis_gbs, 1),
         "combine_gbs": round(com_gbs, 1),
         "dispatch_frac_of_8tbs": round(dis_gbs / NOMINAL_HBM_GBS, 4),
@@ -530,37 +546,65 @@ def gpu_index_of(local_rank: int) -> int:
 
 # ----------------------------------------------------------------------------- CPU oracle arm
 
-def oracle_sample(w: inputs.Workload, sample_tokens: int, inp=None):
-    """Time the CPU oracle on the first `sample_tokens` tokens of every rank of the workload."""
+class one_core:
+    """Pin the calling thread to one host core for the duration (restores the old set after)."""
+
+    def __enter__(self):
+        self.old = None
+        self.core = None
+        try:
+            self.old = os.sched_getaffinity(0)
+            self.core = min(self.old)
+            os.sched_setaffinity(0, {self.core})
+        except (AttributeError, OSError):
+            self.old = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.old is not None:
+            os.sched_setaffinity(0, self.old)
+
+
+def oracle_sample(w: inputs.Workload, sample_tokens=None, inp=None):
+    """Time the CPU oracle, pinned to one core, stage by stage.
+
+    ``sample_tokens`` None (the default) runs the whole workload once; a number
+    runs the first that many tokens of every rank.
+    """
     import oracle
 
     inp = inp if inp is not None else inputs.make_inputs(w)
-    Ts = min(sample_tokens, w.num_tokens)
+    Ts = w.num_tokens if sample_tokens is None else min(int(sample_tokens), w.num_tokens)
     idx = np.ascontiguousarray(inp.topk_idx[:, :Ts])
     x = np.ascontiguousarray(inp.x[:, :Ts])
     wts = np.ascontiguousarray(inp.topk_weights[:, :Ts])
     E, H, R = w.num_physical, w.hidden, w.num_ranks
+    oracle.load()
     stages = {}
-    t0 = time.perf_counter()
-    if w.num_extra:
-        idx = oracle.reroute(idx, w.num_experts, w.num_extra)["topk_idx_phys"]
-        stages["reroute"] = time.perf_counter() - t0
-    t1 = time.perf_counter()
-    ref = oracle.layout(idx, inp.active, E)
-    t2 = time.perf_counter()
-    packed, _ = oracle.dispatch(x, idx, ref)
-    t3 = time.perf_counter()
-    oracle.combine(packed, ref.list_base[:-1], idx, wts, ref.pair_row, inp.active, E)
-    t4 = time.perf_counter()
+    with one_core() as pin:
+        t0 = time.perf_counter()
+        if w.num_extra:
+            idx = oracle.reroute(idx, w.num_experts, w.num_extra)["topk_idx_phys"]
+            stages["reroute"] = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        ref = oracle.layout(idx, inp.active, E)
+        t2 = time.perf_counter()
+        packed, _ = oracle.dispatch(x, idx, ref)
+        t3 = time.perf_counter()
+        oracle.combine(packed, ref.list_base[:-1], idx, wts, ref.pair_row, inp.active, E)
+        t4 = time.perf_counter()
+    del packed
     stages.update(layout=t2 - t1, dispatch=t3 - t2, combine=t4 - t3)
     secs = t4 - t0
     live = int(ref.recv_count.sum())
     sent = int(ref.is_token_in_rank.reshape(R * Ts, R).max(axis=1).sum())
     d_b, c_b = algorithmic_bytes(H, sent, live, R * Ts)
+    what = ("the whole workload" if Ts == w.num_tokens else f"first {Ts} of {w.num_tokens} tokens of each rank")
     return dict(value=round((d_b + c_b) / secs / 1e9, 3), unit="GB/s", cores=1, kind="oracle",
-                sample=f"first {Ts} of {w.num_tokens} tokens of each of the {R} ranks "
-                       f"(reroute + layout + dispatch + combine, single-threaded C, float64 combine)",
-                seconds=round(secs, 3), stage_seconds={k_: round(v, 4) for k_, v in stages.items()})
+                sample=f"{what}: {R} ranks x {Ts} tokens (reroute + layout + dispatch + combine, "
+                       f"single-threaded C, float64 combine, one pass)",
+                pinned_core=pin.core, seconds=round(secs, 3),
+                stage_seconds={k_: round(v, 4) for k_, v in stages.items()})
 
 
 def cpu_model():
@@ -605,8 +649,7 @@ def run_reference(args, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{w.name} " + " ".join(f"{k_}={v}" for k_, v in w.describe().items()),
-                   **w.describe(), "parallelism": "cpu-oracle"},
+        "config": config_of(w, world),
         "cpu_baseline": base,
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -635,8 +678,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--graph", action="store_true",
                     help="replay the step as a CUDA graph (per-kernel split from per-kernel graphs)")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=1024,
-                    help="tokens per rank in the CPU oracle's timed sample")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=None,
+                    help="tokens per rank in the CPU oracle's timed pass (default: the whole workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dispatch-cfg", type=parse_cfg, default=None,
                     help="launch config of ep_dispatch, e.g. max_ctas=296,stages=7")
@@ -665,9 +708,11 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local_rank))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        w = inputs.named(args.workload)
+        inp = inputs.make_inputs(w)
+        line = run_ours(args, rank, world, local_rank, w, inp)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            cb = oracle_sample(inputs.named(args.workload), args.cpu_sample_tokens)
+            cb = oracle_sample(w, args.cpu_sample_tokens, inp)
             cb["host_cores"] = os.cpu_count()
             cb["cpu_model"] = cpu_model()
             line["cpu_baseline"] = cb

@@ -108,3 +108,24 @@ def run_path(inp, E, H, *, active_combine=None, cfg=None, y=None, layout_cfg=Non
     out, _ = ep.ep_combine(recv_x if y is None else y, idx, w, lay.pair_row, act_c, status=status, cfg=cfg)
     torch.cuda.synchronize()
     return dict(lay=lay, recv_x=recv_x, src_info=src_info, out=out, status=int(status.item()))
+
+
+def check_combine_full(out: torch.Tensor, packed: np.ndarray, ref: oracle.Layout, topk_idx: np.ndarray,
+                       topk_weights: np.ndarray, active: np.ndarray, E: int, tag: str = "",
+                       chunk_tokens: int = 4096):
+    """Every output row of a combine against the float64 oracle, in chunks of tokens.
+
+    The oracle runs on ``chunk_tokens`` (rank, token) pairs at a time, so host
+    memory stays bounded at any size while no row goes unchecked.
+    """
+    R, T = topk_idx.shape[:2]
+    got_all = out.view(R * T, -1)
+    n = R * T
+    for lo in range(0, n, chunk_tokens):
+        hi = min(n, lo + chunk_tokens)
+        g = np.arange(lo, hi, dtype=np.int64)
+        tokens = np.stack([g // T, g % T], axis=1).astype(np.int32)
+        want, _ = oracle.combine(packed, ref.list_base[:-1], topk_idx, topk_weights, ref.pair_row, active, E,
+                                 tokens=tokens)
+        check_close(bf16_host(got_all[lo:hi]), want, f"{tag} tokens [{lo}, {hi})")
+    return n

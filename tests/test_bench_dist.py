@@ -66,3 +66,31 @@ def test_reference_arm_under_torchrun_prints_once():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_reports_our_config_and_a_pinned_full_pass():
+    """The reference arm names the same config dict as our arm and times the whole workload on one core."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "1",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "1", "--steps", "2", "--warmup", "3", "--workload", "tiny"]
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = json.loads([l for l in res.stdout.splitlines() if l.startswith("{")][0])
+    sys.path.insert(0, ROOT)
+    import bench
+    from combine_get_dispatch_histogram_b200 import inputs
+
+    assert line["config"] == bench.config_of(inputs.tiny(), 1)
+    cb = line["cpu_baseline"]
+    assert cb["cores"] == 1 and cb["pinned_core"] is not None
+    assert cb["sample"].startswith("the whole workload")
+    assert set(cb["stage_seconds"]) == {"layout", "dispatch", "combine"}
+
+
+def test_kernel_time_statistics():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    st = bench.stats_ms([3.0, 1.0, 2.0, 10.0, 2.5])
+    assert st == {"median": 2.5, "min": 1.0, "max": 10.0}

@@ -4,8 +4,9 @@ Runs in the launch configuration the benchmark times (default ep_cfg).  The
 receive slab alone is [256, 32768, 7168] bf16 = 120.26 GB; the test skips
 when the device cannot hold it.  Layout, handle and src_info are compared in
 full; payload rows are compared in full when the host has the memory for the
-oracle's packed rows (3.76 GB), else on a seeded sample of experts; combine
-is compared on a seeded sample of 4096 tokens.
+oracle's packed rows (3.76 GB), else on a seeded sample of experts; every one
+of the 32768 combine output rows is compared with the float64 oracle, which
+runs in chunks of 4096 tokens.
 """
 import numpy as np
 import pytest
@@ -13,7 +14,7 @@ import torch
 
 import oracle
 from combine_get_dispatch_histogram_b200 import inputs
-from gpu_util import bf16_host, check_close, check_dispatch, check_layout, run_path, valid_rows
+from gpu_util import bf16_host, check_combine_full, check_dispatch, check_layout, run_path
 
 pytestmark = pytest.mark.gpu
 
@@ -56,13 +57,10 @@ def test_prefill_full_size():
             assert np.array_equal(got, inp.x[src[:, 0], src[:, 1]])
         packed = None
 
-    rng = np.random.default_rng(1)
-    tokens = np.stack([rng.integers(0, R, 4096), rng.integers(0, T, 4096)], axis=1)
     if packed is None:
         packed, _ = oracle.dispatch(inp.x, inp.topk_idx, ref)
-    want, _ = oracle.combine(packed, ref.list_base[:-1], inp.topk_idx, inp.topk_weights, ref.pair_row,
-                             inp.active, E, tokens=tokens)
-    got = bf16_host(res["out"])[tokens[:, 0], tokens[:, 1]]
-    check_close(got, want, "prefill combine")
+    checked = check_combine_full(res["out"], packed, ref, inp.topk_idx, inp.topk_weights, inp.active, E,
+                                 "prefill combine")
+    assert checked == R * T
     del res
     torch.cuda.empty_cache()
