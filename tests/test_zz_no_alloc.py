@@ -41,11 +41,17 @@ def _empty_layout(R, T, k, E, dev):
         torch.zeros(1, dtype=torch.int32, device=dev))
 
 
-def test_noalloc_layout_equals_workspace_layout_on_two_calls_in_a_row():
+@pytest.mark.parametrize("variant", [0, ep.EP_LAYOUT_FUSED])
+def test_noalloc_layout_equals_workspace_layout_on_two_calls_in_a_row(variant):
+    """AUTO takes the chunked / cluster paths; FUSED reads the barrier epoch the array keeps between calls.
+
+    The two shapes have different chunk grids (128 and 32 chunks), so the second call
+    starts from the first call's epoch and flags in the shared array.
+    """
     fn = _bind()
     dev = torch.device("cuda:0")
     stream = torch.cuda.current_stream(dev)
-    for w in (inputs.prefill(), inputs.sweep(64, masked=True)):
+    for w in (inputs.prefill(), inputs.sweep(64, masked=True), inputs.prefill()):
         inp = inputs.make_inputs(w, tokens=False)
         R, T, k, E = w.num_ranks, w.num_tokens, w.num_topk, w.num_physical
         idx = torch.from_numpy(inp.topk_idx).to(dev)
@@ -57,7 +63,8 @@ def test_noalloc_layout_equals_workspace_layout_on_two_calls_in_a_row():
                 ctypes.c_void_p(got.num_tokens_per_rank.data_ptr()),
                 ctypes.c_void_p(got.is_token_in_rank.data_ptr()), ctypes.c_void_p(got.recv_count.data_ptr()),
                 ctypes.c_void_p(got.expert_rank_offset.data_ptr()), ctypes.c_void_p(got.pair_row.data_ptr()),
-                ctypes.c_void_p(got.status.data_ptr()), ep.Cfg(0, 0, 0, 0), ctypes.c_void_p(stream.cuda_stream))
+                ctypes.c_void_p(got.status.data_ptr()), ep.Cfg(0, 0, 0, variant),
+                ctypes.c_void_p(stream.cuda_stream))
         assert rc == ep.EP_OK, ep.ep_strerror(rc)
         torch.cuda.synchronize()
         for key in KEYS:
