@@ -22,6 +22,7 @@ from .ep import (  # noqa: F401
     ep_reroute,
     ep_reroute_workspace_bytes,
     ep_strerror,
+    ep_topk_idx_to_int32,
     ep_version,
     load_library,
 )

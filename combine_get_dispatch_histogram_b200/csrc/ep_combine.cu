@@ -389,6 +389,7 @@ using namespace ep;
 extern "C" int ep_combine(ep_dims_t d, const uint16_t* y, const int32_t* topk_idx, const float* topk_weights,
                           const int32_t* pair_row, const uint8_t* active, uint16_t* out, int32_t* status,
                           ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_combine");
     int rc = check_dims(d);
     if (rc != EP_OK) return rc;
     const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
@@ -423,6 +424,7 @@ extern "C" int ep_combine(ep_dims_t d, const uint16_t* y, const int32_t* topk_id
 extern "C" int ep_normal_combine(ep_dims_t d, int32_t recv_capacity, const uint16_t* y,
                                  const int32_t* token_recv_row, const uint8_t* active, uint16_t* out,
                                  int32_t* status, ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_normal_combine");
     int rc = check_dims(d);
     if (rc != EP_OK) return rc;
     if (recv_capacity < 0) return EP_ERR_INVALID;

@@ -325,6 +325,7 @@ using namespace ep;
 
 extern "C" int ep_dispatch(ep_dims_t d, const uint16_t* x, const int32_t* topk_idx, const int32_t* pair_row,
                            uint16_t* recv_x, int32_t* src_info, int32_t* status, ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_dispatch");
     int rc = check_dims(d);
     if (rc != EP_OK) return rc;
     const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
@@ -384,6 +385,7 @@ extern "C" int ep_normal_dispatch(ep_dims_t d, int32_t recv_capacity, const uint
                                   const float* topk_weights, const uint8_t* active, const int32_t* token_recv_row,
                                   uint16_t* recv_x, int32_t* recv_topk_idx, float* recv_topk_weights,
                                   int32_t* src_info, int32_t* status, ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_normal_dispatch");
     int rc = check_dims(d);
     if (rc != EP_OK) return rc;
     if (recv_capacity < 0) return EP_ERR_INVALID;

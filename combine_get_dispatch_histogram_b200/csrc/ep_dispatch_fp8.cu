@@ -407,6 +407,7 @@ extern "C" int ep_dispatch_fp8(ep_dims_t d, const uint16_t* x, const int32_t* to
                                const int32_t* recv_count, int32_t scale_format, void* workspace,
                                size_t workspace_bytes, uint8_t* recv_x, void* recv_scales, int32_t* src_info,
                                int32_t* status, ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_dispatch_fp8");
     int rc = check_dims(d);
     if (rc != EP_OK) return rc;
     if (scale_format != EP_FP8_SCALE_F32 && scale_format != EP_FP8_SCALE_POW2 && scale_format != EP_FP8_SCALE_UE8M0)

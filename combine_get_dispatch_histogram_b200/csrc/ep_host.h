@@ -7,10 +7,23 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "ep.h"
 
 namespace ep {
+
+// NVTX range named after the entry point, open for the duration of the host
+// call (validation and launches), so a timeline tool shows which C-ABI call
+// enqueued which kernels.  Without a tool attached a push/pop costs a few
+// nanoseconds.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define EP_NVTX_RANGE(name) ::ep::NvtxRange ep_nvtx_range_(name)
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

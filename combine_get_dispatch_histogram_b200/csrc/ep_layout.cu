@@ -93,7 +93,9 @@ struct LayoutArgs {
     int32_t* expert_rank_offset;
     int32_t* pair_row;
     int32_t* status;
-    int R, T, k, E, E_local;
+    int R, T, k, E, E_local;  // R: ranks of the EP world (mask, destinations, is_token_in_rank width)
+    int Rs, r0;        // source ranks laid out (rows of topk_idx), the first one's rank: R and 0 for
+                       // the whole world, 1 and the caller's rank for a rank-local layout
     int key_bits;      // bits that tell experts apart: ceil(log2(E))
     int C, G;          // chunks per rank, chunks
     int chunk_tokens;  // tokens per chunk (the last chunk of a rank may be shorter)
@@ -113,6 +115,7 @@ __device__ __forceinline__ ChunkGeom chunk_of(const LayoutArgs& a, int g) {
 }
 
 // act[] <- active mask, rank_of[e] <- destination rank of e, or -1 if it is masked.
+// act[] is indexed by world rank; source row r is rank r0 + r.
 __device__ __forceinline__ void load_tables(const LayoutArgs& a, int32_t* act, int32_t* rank_of) {
     for (int i = threadIdx.x; i < a.R; i += blockDim.x) act[i] = a.active[i];
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_count_kernel(LayoutArgs
     __syncthreads();
 
     const ChunkGeom cg = chunk_of(a, blockIdx.x);
-    const bool src_ok = act[cg.r] != 0;
+    const bool src_ok = act[a.r0 + cg.r] != 0;
     const int64_t pbase = (int64_t(cg.r) * a.T + cg.t0) * a.k;
     const int32_t* base = a.topk_idx + pbase;
     const int np = (cg.t1 - cg.t0) * a.k;
@@ -232,14 +235,14 @@ __global__ void __launch_bounds__(32 * kScanWarps) layout_scan_kernel(LayoutArgs
     }
     __syncthreads();
     if (ok) {
-        for (int r = warp; r < a.R; r += kScanWarps) {
+        for (int r = warp; r < a.Rs; r += kScanWarps) {
             const int32_t off = a.chunk_hist[int64_t(r) * a.C * a.E + e];
-            const int32_t next = r + 1 < a.R ? a.chunk_hist[int64_t(r + 1) * a.C * a.E + e] : total[lane];
-            a.expert_rank_offset[int64_t(e) * a.R + r] = off;
+            const int32_t next = r + 1 < a.Rs ? a.chunk_hist[int64_t(r + 1) * a.C * a.E + e] : total[lane];
+            a.expert_rank_offset[int64_t(e) * a.Rs + r] = off;
             a.num_tokens_per_expert[int64_t(r) * a.E + e] = next - off;
         }
     }
-    const int RR = a.R * a.R;
+    const int RR = a.Rs * a.R;
     for (int pr = blockIdx.x * kScanWarps + warp; pr < RR; pr += gridDim.x * kScanWarps) {
         const int r = pr / a.R, d = pr - r * a.R;
         const int32_t* col = a.chunk_tpr + int64_t(r) * a.C * a.R + d;
@@ -269,7 +272,7 @@ __device__ __forceinline__ WarpPart warp_part(const LayoutArgs& a, int gw, int w
     WarpPart w;
     w.r = gw / wpr;
     const int part = gw - w.r * wpr;
-    w.has_rank = w.r < a.R;
+    w.has_rank = w.r < a.Rs;
     const int tw = (a.T + wpr - 1) / wpr;
     w.t0 = w.has_rank ? min(a.T, part * tw) : 0;
     w.t1 = w.has_rank ? min(a.T, w.t0 + tw) : 0;
@@ -301,7 +304,7 @@ __device__ __forceinline__ bool walk_part(const LayoutArgs& a, const WarpPart& w
                                           const int32_t* rank_of, int32_t* mine, int32_t* tpr,
                                           int (&ev)[kBatch], int (&rk)[kBatch]) {
     const int lane = threadIdx.x & 31;
-    const bool src_ok = w.has_rank && act[w.r] != 0;
+    const bool src_ok = w.has_rank && act[a.r0 + w.r] != 0;
     const int32_t* base = a.topk_idx + w.pbase;
     int32_t* rows = a.pair_row + w.pbase;
     const uint32_t below = lanemask_lt();
@@ -403,13 +406,13 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
     int32_t* rank_of = tpr + kSmallMaxRanks * kSmallMaxRanks;   // [E]
     int32_t* whist = rank_of + a.E;                            // [NW][E]
 
-    const int wpr = NW / a.R;  // warps per rank, R <= 32
+    const int wpr = NW / a.Rs;  // warps per source rank, Rs <= 32
     const WarpPart w = warp_part(a, warp, wpr);
     int ev[kBatch], rk[kBatch];
     load_first_round(a, w, ev);
     load_tables(a, act, rank_of);
     for (int i = threadIdx.x; i < NW * a.E; i += blockDim.x) whist[i] = 0;
-    for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) tpr[i] = 0;
+    for (int i = threadIdx.x; i < a.Rs * a.R; i += blockDim.x) tpr[i] = 0;
     __syncthreads();
 
     int32_t* mine = whist + warp * a.E;
@@ -419,9 +422,9 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
     // scan the warp histograms per expert in warp order = (rank, part) order
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         int32_t run = 0;
-        for (int rr = 0; rr < a.R; ++rr) {
+        for (int rr = 0; rr < a.Rs; ++rr) {
             const int32_t rank_first = run;
-            a.expert_rank_offset[int64_t(e) * a.R + rr] = rank_first;
+            a.expert_rank_offset[int64_t(e) * a.Rs + rr] = rank_first;
             for (int wi = rr * wpr; wi < (rr + 1) * wpr; ++wi) {
                 const int32_t c = whist[wi * a.E + e];
                 whist[wi * a.E + e] = run;
@@ -432,7 +435,7 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
         a.recv_count[e] = run;
         if (run > a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
     }
-    for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) a.num_tokens_per_rank[i] = tpr[i];
+    for (int i = threadIdx.x; i < a.Rs * a.R; i += blockDim.x) a.num_tokens_per_rank[i] = tpr[i];
     __syncthreads();
     finish_rows(a, w, ev, rk, [&](int e) { return mine[e]; });
 }
@@ -465,13 +468,13 @@ __global__ void __launch_bounds__(kSmallThreads) layout_cluster_kernel(LayoutArg
     int32_t* cbase = ctot + a.E;                               // [E] this CTA's first row per expert
     int32_t* whist = cbase + a.E;                              // [NW][E]
 
-    const int wpr = CL * NW / a.R;  // warps per rank, R <= 32 <= CL * NW
+    const int wpr = CL * NW / a.Rs;  // warps per source rank, Rs <= 32 <= CL * NW
     const WarpPart w = warp_part(a, cta * NW + warp, wpr);
     int ev[kBatch], rk[kBatch];
     load_first_round(a, w, ev);
     load_tables(a, act, rank_of);
     for (int i = threadIdx.x; i < NW * a.E; i += blockDim.x) whist[i] = 0;
-    for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) tpr[i] = 0;
+    for (int i = threadIdx.x; i < a.Rs * a.R; i += blockDim.x) tpr[i] = 0;
     __syncthreads();
 
     int32_t* mine = whist + warp * a.E;
@@ -492,13 +495,13 @@ __global__ void __launch_bounds__(kSmallThreads) layout_cluster_kernel(LayoutArg
 
     // ranks whose first warp (rank * wpr) is in this CTA
     const int r_lo = (cta * NW + wpr - 1) / wpr;
-    const int r_hi = min(a.R, ((cta + 1) * NW + wpr - 1) / wpr);
+    const int r_hi = min(a.Rs, ((cta + 1) * NW + wpr - 1) / wpr);
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         int32_t b = 0;
         for (int c = 0; c < cta; ++c) b += ld_dsmem_s32(dsmem_addr(ctot + e, uint32_t(c)));
         cbase[e] = b;
         for (int rr = r_lo; rr < r_hi; ++rr)
-            a.expert_rank_offset[int64_t(e) * a.R + rr] = b + whist[(rr * wpr - cta * NW) * a.E + e];
+            a.expert_rank_offset[int64_t(e) * a.Rs + rr] = b + whist[(rr * wpr - cta * NW) * a.E + e];
         if (cta == CL - 1) {
             const int32_t n = b + ctot[e];
             a.recv_count[e] = n;
@@ -506,7 +509,7 @@ __global__ void __launch_bounds__(kSmallThreads) layout_cluster_kernel(LayoutArg
         }
     }
     if (cta == 0) {
-        for (int i = threadIdx.x; i < a.R * a.R; i += blockDim.x) {
+        for (int i = threadIdx.x; i < a.Rs * a.R; i += blockDim.x) {
             int32_t n = 0;
             for (int c = 0; c < CL; ++c) n += ld_dsmem_s32(dsmem_addr(tpr + i, uint32_t(c)));
             a.num_tokens_per_rank[i] = n;
@@ -519,7 +522,7 @@ __global__ void __launch_bounds__(kSmallThreads) layout_cluster_kernel(LayoutArg
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         for (int rr = r_lo; rr < r_hi; ++rr) {
             const int32_t off = cbase[e] + whist[(rr * wpr - cta * NW) * a.E + e];
-            const int32_t next = rr + 1 < a.R ? a.expert_rank_offset[int64_t(e) * a.R + rr + 1] : a.recv_count[e];
+            const int32_t next = rr + 1 < a.Rs ? a.expert_rank_offset[int64_t(e) * a.Rs + rr + 1] : a.recv_count[e];
             a.num_tokens_per_expert[int64_t(rr) * a.E + e] = next - off;
         }
     }
@@ -540,7 +543,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_rank_kernel(LayoutArgs 
 
     const int g = blockIdx.x;
     const ChunkGeom cg = chunk_of(a, g);
-    const bool src_ok = act[cg.r] != 0;
+    const bool src_ok = act[a.r0 + cg.r] != 0;
 
     // 1. first rows of this chunk (written by the scan)
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) first[e] = a.chunk_hist[int64_t(g) * a.E + e];
@@ -694,7 +697,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_fused_kernel(LayoutArgs
 
     const int g = blockIdx.x;
     const ChunkGeom cg = chunk_of(a, g);
-    const bool src_ok = act[cg.r] != 0;
+    const bool src_ok = act[a.r0 + cg.r] != 0;
     const int tw = (cg.t1 - cg.t0 + W - 1) / W;
     const int wt0 = min(cg.t1, cg.t0 + warp * tw), wt1 = min(cg.t1, wt0 + tw);
     const int64_t pbase = (int64_t(cg.r) * a.T + wt0) * a.k;
@@ -788,16 +791,16 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_fused_kernel(LayoutArgs
         }
         __syncthreads();
         if (ok) {
-            for (int r = warp; r < a.R; r += W) {
+            for (int r = warp; r < a.Rs; r += W) {
                 const int32_t off = a.chunk_hist[int64_t(r) * a.C * a.E + e];
-                const int32_t next = r + 1 < a.R ? a.chunk_hist[int64_t(r + 1) * a.C * a.E + e] : col_total[lane];
-                a.expert_rank_offset[int64_t(e) * a.R + r] = off;
+                const int32_t next = r + 1 < a.Rs ? a.chunk_hist[int64_t(r + 1) * a.C * a.E + e] : col_total[lane];
+                a.expert_rank_offset[int64_t(e) * a.Rs + r] = off;
                 a.num_tokens_per_expert[int64_t(r) * a.E + e] = next - off;
             }
         }
         __syncthreads();
     }
-    const int RR = a.R * a.R;
+    const int RR = a.Rs * a.R;
     for (int pr = g * W + warp; pr < RR; pr += a.G * W) {
         const int r = pr / a.R, d = pr - r * a.R;
         const int32_t* colp = a.chunk_tpr + int64_t(r) * a.C * a.R + d;
@@ -848,20 +851,246 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_fused_kernel(LayoutArgs
     if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned long long*>(a.sync), epoch + 1);
 }
 
+// ---------------------------------------------------------------------------
+// Look-back path (EP_LAYOUT_LOOKBACK): the chunked algorithm in ONE ordinary
+// launch, one CTA per chunk, with no grid-wide barrier.  A chunk's first rows
+// need only the histograms of the chunks before it, so each CTA
+//   A. counts its chunk (warp histograms kept in shared memory, destination
+//      ranks, per-destination token counts), writes the chunk histogram and
+//      publishes it with a release flag;
+//   B. waits (bounded) for the flags of the chunks before it only -- CTAs are
+//      dispatched in index order, so those have started -- and sums their
+//      histograms, all its threads loading in parallel;
+//   C. assigns rows as the rank kernel does.
+// The owners of the per-rank outputs are the chunks that can see them: the
+// first chunk of rank r writes expert_rank_offset[:, r], the last chunk of rank
+// r num_tokens_per_expert[r] and num_tokens_per_rank[r], the last chunk of all
+// recv_count.  Flags use the fused path's epoch scheme (shared workspace
+// prefix): the last CTA advances the epoch once every CTA has published, hence
+// has read it.
+__global__ void __launch_bounds__(32 * kMaxWarps) layout_lookback_kernel(LayoutArgs a) {
+    pdl_wait();  // nothing upstream is read before this
+    pdl_launch_dependents();
+    extern __shared__ int32_t smem[];
+    __shared__ int passed;
+    const int NT = blockDim.x;
+    const int W = NT >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int32_t* act = smem;
+    int32_t* tpr = smem + kActiveSlots;
+    int32_t* rank_of = smem + 2 * kActiveSlots;
+    int32_t* first = rank_of + a.E;       // [E] rows of the chunks before this one
+    int32_t* rank_first = first + a.E;    // [E] rows of the chunks of the ranks before this chunk's rank
+    int32_t* part = rank_first + a.E;     // [2][NT] partial sums of phase B
+    int32_t* whist = part + 2 * NT;       // [W][E]
+    const uint64_t epoch = *reinterpret_cast<volatile uint64_t*>(a.sync);
+    uint64_t* flags = a.sync + 1;
+    const uint64_t value = 2 * (epoch + 1);
+    load_tables(a, act, rank_of);
+    for (int i = threadIdx.x; i < W * a.E; i += NT) whist[i] = 0;
+    for (int d = threadIdx.x; d < a.R; d += NT) tpr[d] = 0;
+    __syncthreads();
+
+    const int g = blockIdx.x;
+    const ChunkGeom cg = chunk_of(a, g);
+    const bool src_ok = act[a.r0 + cg.r] != 0;
+    const int tw = (cg.t1 - cg.t0 + W - 1) / W;
+    const int wt0 = min(cg.t1, cg.t0 + warp * tw), wt1 = min(cg.t1, wt0 + tw);
+    const int64_t pbase = (int64_t(cg.r) * a.T + wt0) * a.k;
+    const int32_t* base = a.topk_idx + pbase;
+    int32_t* rows = a.pair_row + pbase;
+    const int np = (wt1 - wt0) * a.k;
+    int32_t* mine = whist + warp * a.E;
+
+    // ---- A: warp histograms, destination ranks, chunk histogram, publish
+    bool bad = false;
+    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+        int ev[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            ev[u] = p < np ? __ldg(base + p) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int e = ev[u];
+            bad |= (e < -1 || e >= a.E);
+            const bool live = pair_live(e, a.E, src_ok, rank_of);
+            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
+            if (live && lane == __ffs(m) - 1) mine[e] += __popc(m);
+            __syncwarp();
+        }
+    }
+    for (int t0 = wt0; t0 < wt1; t0 += 32) {
+        const int t = t0 + lane;
+        uint64_t ranks = 0;
+        if (t < wt1) {
+            const int32_t* tb = a.topk_idx + (int64_t(cg.r) * a.T + t) * a.k;
+            for (int j = 0; j < a.k; ++j) {
+                const int e = __ldg(tb + j);
+                if (pair_live(e, a.E, src_ok, rank_of)) ranks |= 1ull << rank_of[e];
+            }
+            uint8_t* itr = a.is_token_in_rank + (int64_t(cg.r) * a.T + t) * a.R;
+            for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
+        }
+        for (int d = 0; d < a.R; ++d) {
+            const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
+            if (lane == 0 && n) atomicAdd(tpr + d, n);
+        }
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
+    int32_t* own = a.chunk_hist + int64_t(g) * a.E;
+    for (int e = threadIdx.x; e < a.E; e += NT) {
+        int32_t s = 0;
+        for (int w = 0; w < W; ++w) s += whist[w * a.E + e];
+        own[e] = s;
+    }
+    for (int d = threadIdx.x; d < a.R; d += NT) a.chunk_tpr[int64_t(g) * a.R + d] = tpr[d];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        st_release_u64(flags + g, value);
+    }
+
+    // ---- B: wait for the chunks before this one (bounded), then sum their histograms
+    if (warp == 0) {
+        bool ok = true;
+        const uint64_t t0 = global_timer_ns();
+        for (int b = 0; b < g && ok; b += 32) {
+            const int gg = b + lane;
+            for (uint32_t it = 0;; ++it) {
+                const bool here = gg >= g || ld_acquire_u64(flags + gg) >= value;
+                if (__all_sync(0xffffffffu, here)) break;
+                if ((it & 63u) == 63u && __any_sync(0xffffffffu, global_timer_ns() - t0 > kWaitTimeoutNs)) {
+                    ok = false;
+                    break;
+                }
+            }
+            ok = __all_sync(0xffffffffu, ok);
+        }
+        if (lane == 0) passed = ok;
+    }
+    __syncthreads();
+    if (g == a.G - 1 && threadIdx.x == 0)  // every CTA has read the epoch (or the wait gave up)
+        atomicMax(reinterpret_cast<unsigned long long*>(a.sync), epoch + 1);
+    if (!passed) {
+        if (threadIdx.x == 0) flag_status(a.status, EP_STATUS_TIMEOUT);
+        return;
+    }
+    const int rC = cg.r * a.C;  // first chunk of this chunk's rank
+    {
+        // thread (e, q): expert e, chunks gg = q, q + P, ... (P = NT / E parts when E <= NT)
+        const int P = a.E <= NT ? NT / a.E : 1;
+        for (int e0 = 0; e0 < a.E; e0 += NT / P) {
+            const int e = e0 + threadIdx.x % (NT / P);
+            const int q = threadIdx.x / (NT / P);
+            int32_t s_before = 0, s_rank = 0;
+            if (e < a.E && q < P) {
+                int gg = q;
+#pragma unroll 1
+                for (; gg + 7 * P < g; gg += 8 * P) {
+                    int32_t v[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) v[u] = a.chunk_hist[int64_t(gg + u * P) * a.E + e];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        if (gg + u * P < rC) s_before += v[u];
+                        else s_rank += v[u];
+                    }
+                }
+                for (; gg < g; gg += P) {
+                    const int32_t v = a.chunk_hist[int64_t(gg) * a.E + e];
+                    if (gg < rC) s_before += v;
+                    else s_rank += v;
+                }
+            }
+            if (q < P) {
+                part[threadIdx.x] = s_before;
+                part[NT + threadIdx.x] = s_rank;
+            }
+            __syncthreads();
+            if (q == 0 && e < a.E) {
+                int32_t b = 0, r = 0;
+                for (int qq = 0; qq < P; ++qq) {
+                    b += part[qq * (NT / P) + (e - e0)];
+                    r += part[NT + qq * (NT / P) + (e - e0)];
+                }
+                rank_first[e] = b;
+                first[e] = b + r;
+            }
+            __syncthreads();
+        }
+    }
+    if (g == rC) {
+        for (int e = threadIdx.x; e < a.E; e += NT) a.expert_rank_offset[int64_t(e) * a.Rs + cg.r] = first[e];
+    }
+    if (g == rC + a.C - 1) {
+        for (int e = threadIdx.x; e < a.E; e += NT)
+            a.num_tokens_per_expert[int64_t(cg.r) * a.E + e] = first[e] - rank_first[e] + own[e];
+        for (int d = warp; d < a.R; d += W) {
+            int32_t t = 0;
+            for (int c = lane; c < a.C; c += 32) t += a.chunk_tpr[int64_t(rC + c) * a.R + d];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+            if (lane == 0) a.num_tokens_per_rank[int64_t(cg.r) * a.R + d] = t;
+        }
+    }
+    if (g == a.G - 1) {
+        for (int e = threadIdx.x; e < a.E; e += NT) {
+            const int32_t n = first[e] + own[e];
+            a.recv_count[e] = n;
+            if (n > a.cap) flag_status(a.status, EP_STATUS_OVERFLOW);
+        }
+    }
+
+    // ---- C: per-warp first rows, then rows
+    for (int e = threadIdx.x; e < a.E; e += NT) {
+        int32_t run = first[e];
+        for (int w = 0; w < W; ++w) {
+            const int32_t v = whist[w * a.E + e];
+            whist[w * a.E + e] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    const uint32_t below = lanemask_lt();
+    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
+        int ev[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            ev[u] = p < np ? __ldg(base + p) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int p = p0 + u * 32 + lane;
+            if (p0 + u * 32 >= np) break;
+            const int e = ev[u];
+            const bool live = pair_live(e, a.E, src_ok, rank_of);
+            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
+            const int32_t b = live ? mine[e] : 0;
+            __syncwarp();
+            if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
+            __syncwarp();
+            if (p < np) rows[p] = live ? b + __popc(m & below) : -1;
+        }
+    }
+}
+
 struct LayoutGeom {
     int C, G, chunk_tokens, warps;
 };
 
-// Chunks per rank, tokens per chunk and warps per CTA for a shape.
-LayoutGeom layout_geom(const ep_dims_t& d) {
+// Chunks per source rank, tokens per chunk and warps per CTA for a shape whose
+// routing has Rs source ranks (Rs = R for the whole world, 1 for one rank).
+LayoutGeom layout_geom(const ep_dims_t& d, int Rs) {
     LayoutGeom lg;
-    const int64_t pairs = int64_t(d.num_ranks) * d.num_tokens * d.num_topk;
+    const int64_t pairs = int64_t(Rs) * d.num_tokens * d.num_topk;
     const int64_t target = std::min<int64_t>(kMaxChunks, std::max<int64_t>(kTargetChunks, ceil_div(pairs, kPairsPerChunk)));
-    int64_t C = std::max<int64_t>(1, ceil_div(target, d.num_ranks));
+    int64_t C = std::max<int64_t>(1, ceil_div(target, Rs));
     C = std::max<int64_t>(1, std::min<int64_t>(C, d.num_tokens));
     lg.chunk_tokens = int(std::max<int64_t>(1, ceil_div(d.num_tokens, C)));
     lg.C = int(std::max<int64_t>(1, ceil_div(std::max(d.num_tokens, 1), lg.chunk_tokens)));
-    lg.G = d.num_ranks * lg.C;
+    lg.G = Rs * lg.C;
     // warp-private histograms of the rank kernel: W * E ints within ~96 KB
     const int64_t per_warp = int64_t(d.num_experts) * 4;
     lg.warps = int(std::max<int64_t>(1, std::min<int64_t>(kMaxWarps, (96 * 1024) / per_warp)));
@@ -912,14 +1141,18 @@ size_t fused_smem_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
     return size_t(2 * kActiveSlots + 2 * d.num_experts + lg.warps * d.num_experts) * 4;
 }
 
+size_t lookback_smem_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
+    return size_t(2 * kActiveSlots + 3 * d.num_experts + 2 * 32 * lg.warps + lg.warps * d.num_experts) * 4;
+}
+
 // The path ep_layout takes for these dims and cfg, or a negative EP_ERR_* code.
 // AUTO, from graph replays on B200: one CTA up to kSmallAutoPairs pairs (8.6 us at 1024
 // pairs, 10.6 us at 2048); a cluster up to kClusterAutoPairs (10.6 us from 4096 to 16384
 // pairs, 12.7 us at 32768, 14.7 at 49152, 16.8 at 65536, where one CTA takes 14.7 to 74 us);
 // the chunked path beyond (about 17 to 19 us), which also beats the fused one (cooperative
 // launch plus two grid barriers, about 19 us).
-int resolve_layout_path(const ep_dims_t& d, const ep_cfg_t& cfg, const LayoutGeom& lg) {
-    const int64_t pairs = int64_t(d.num_ranks) * d.num_tokens * d.num_topk;
+int resolve_layout_path(const ep_dims_t& d, int Rs, const ep_cfg_t& cfg, const LayoutGeom& lg) {
+    const int64_t pairs = int64_t(Rs) * d.num_tokens * d.num_topk;
     const bool tables_fit = d.num_ranks <= kSmallMaxRanks && d.num_experts <= kSmallMaxExperts;
     const bool small_ok = tables_fit && pairs <= kSmallMaxPairs;
     const bool cluster_ok = tables_fit && pairs <= kClusterMaxPairs;
@@ -938,10 +1171,23 @@ int resolve_layout_path(const ep_dims_t& d, const ep_cfg_t& cfg, const LayoutGeo
                        : int(EP_ERR_UNSUPPORTED);
         case EP_LAYOUT_CLUSTER:
             return cluster_ok ? int(EP_LAYOUT_CLUSTER) : int(EP_ERR_UNSUPPORTED);
+        case EP_LAYOUT_LOOKBACK:
+            return lg.G <= kMaxFlags && lookback_smem_bytes(d, lg) <= size_t(max_smem_optin())
+                       ? int(EP_LAYOUT_LOOKBACK)
+                       : int(EP_ERR_UNSUPPORTED);
         default:
             return EP_ERR_INVALID;
     }
 }
+
+size_t layout_ws_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
+    return kSyncBytes + layout_ws_hist_bytes(d, lg) + layout_ws_tpr_bytes(d, lg);
+}
+
+int layout_run(const ep_dims_t& d, int Rs, int r0, const int32_t* topk_idx, const uint8_t* active, void* workspace,
+               int32_t* num_tokens_per_expert, int32_t* num_tokens_per_rank, uint8_t* is_token_in_rank,
+               int32_t* recv_count, int32_t* expert_rank_offset, int32_t* pair_row, int32_t* status,
+               const ep_cfg_t& cfg, cudaStream_t s);
 
 }  // namespace
 }  // namespace ep
@@ -949,20 +1195,19 @@ int resolve_layout_path(const ep_dims_t& d, const ep_cfg_t& cfg, const LayoutGeo
 extern "C" int ep_layout_path(ep_dims_t d, ep_cfg_t cfg) {
     const int rc = check_dims(d);
     if (rc != EP_OK) return rc;
-    return resolve_layout_path(d, cfg, layout_geom(d));
+    return resolve_layout_path(d, d.num_ranks, cfg, layout_geom(d, d.num_ranks));
 }
 
 extern "C" size_t ep_layout_workspace_bytes(ep_dims_t d) {
     if (check_dims(d) != EP_OK) return 0;
-    const LayoutGeom lg = layout_geom(d);
-    return kSyncBytes + layout_ws_hist_bytes(d, lg) + layout_ws_tpr_bytes(d, lg);
+    return layout_ws_bytes(d, layout_geom(d, d.num_ranks));
 }
 
 extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* active, void* workspace,
                          size_t workspace_bytes, int32_t* num_tokens_per_expert, int32_t* num_tokens_per_rank,
                          uint8_t* is_token_in_rank, int32_t* recv_count, int32_t* expert_rank_offset,
                          int32_t* pair_row, int32_t* status, ep_cfg_t cfg, void* stream) {
-    (void)cfg;
+    EP_NVTX_RANGE("ep_layout");
     int rc = check_dims(d);
     if (rc != EP_OK) return rc;
     const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
@@ -971,8 +1216,50 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     if (RT > 0 && (!topk_idx || !is_token_in_rank || !pair_row)) return EP_ERR_INVALID;
     const size_t need = ep_layout_workspace_bytes(d);
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return EP_ERR_INVALID;
+    return layout_run(d, d.num_ranks, 0, topk_idx, active, workspace, num_tokens_per_expert, num_tokens_per_rank,
+                      is_token_in_rank, recv_count, expert_rank_offset, pair_row, status, cfg,
+                      static_cast<cudaStream_t>(stream));
+}
 
-    const LayoutGeom lg = layout_geom(d);
+// Rank-local layout: the same kernels over one source rank's routing (Rs = 1),
+// with the mask and destinations of the whole world.  Its per-source outputs are
+// one row; the offset within each expert (always 0 for a lone source) and the
+// receive counts (equal to the local counts) go to the workspace tail.
+extern "C" size_t ep_layout_local_workspace_bytes(ep_dims_t d) {
+    if (check_dims(d) != EP_OK) return 0;
+    return layout_ws_bytes(d, layout_geom(d, 1)) + 2 * round_up16(size_t(d.num_experts) * 4);
+}
+
+extern "C" int ep_layout_local(ep_dims_t d, int32_t rank, const int32_t* topk_idx, const uint8_t* active,
+                               void* workspace, size_t workspace_bytes, int32_t* num_tokens_per_expert,
+                               int32_t* num_tokens_per_rank, uint8_t* is_token_in_rank, int32_t* local_row,
+                               int32_t* status, ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_layout_local");
+    int rc = check_dims(d);
+    if (rc != EP_OK) return rc;
+    if (rank < 0 || rank >= d.num_ranks) return EP_ERR_INVALID;
+    if (!active || !num_tokens_per_expert || !num_tokens_per_rank) return EP_ERR_INVALID;
+    if (d.num_tokens > 0 && (!topk_idx || !is_token_in_rank || !local_row)) return EP_ERR_INVALID;
+    const LayoutGeom lg = layout_geom(d, 1);
+    const size_t base = layout_ws_bytes(d, lg);
+    if (!workspace || workspace_bytes < ep_layout_local_workspace_bytes(d) || !aligned16(workspace))
+        return EP_ERR_INVALID;
+    char* ws = static_cast<char*>(workspace);
+    int32_t* offset_scratch = reinterpret_cast<int32_t*>(ws + base);
+    int32_t* count_scratch = reinterpret_cast<int32_t*>(ws + base + round_up16(size_t(d.num_experts) * 4));
+    return layout_run(d, 1, rank, topk_idx, active, workspace, num_tokens_per_expert, num_tokens_per_rank,
+                      is_token_in_rank, count_scratch, offset_scratch, local_row, status, cfg,
+                      static_cast<cudaStream_t>(stream));
+}
+
+namespace ep {
+namespace {
+
+int layout_run(const ep_dims_t& d, int Rs, int r0, const int32_t* topk_idx, const uint8_t* active, void* workspace,
+               int32_t* num_tokens_per_expert, int32_t* num_tokens_per_rank, uint8_t* is_token_in_rank,
+               int32_t* recv_count, int32_t* expert_rank_offset, int32_t* pair_row, int32_t* status,
+               const ep_cfg_t& cfg, cudaStream_t s) {
+    const LayoutGeom lg = layout_geom(d, Rs);
     LayoutArgs a;
     a.topk_idx = topk_idx;
     a.active = active;
@@ -988,6 +1275,8 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     a.pair_row = pair_row;
     a.status = status;
     a.R = d.num_ranks;
+    a.Rs = Rs;
+    a.r0 = r0;
     a.T = d.num_tokens;
     a.k = d.num_topk;
     a.E = d.num_experts;
@@ -997,10 +1286,9 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     a.C = lg.C;
     a.G = lg.G;
     a.chunk_tokens = lg.chunk_tokens;
-    a.cap = RT;
+    a.cap = int64_t(d.num_ranks) * d.num_tokens;
 
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const int path = resolve_layout_path(d, cfg, lg);
+    const int path = resolve_layout_path(d, Rs, cfg, lg);
     if (path < 0) return path;
     const int W = lg.warps;
     if (path == EP_LAYOUT_FUSED) {
@@ -1022,6 +1310,16 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
         }
         return launch_result();
     }
+    if (path == EP_LAYOUT_LOOKBACK) {
+        const size_t smem = lookback_smem_bytes(d, lg);
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(layout_lookback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+                cudaSuccess)
+            return EP_ERR_CUDA;
+        if (launch_pdl(layout_lookback_kernel, dim3(lg.G), dim3(32 * W), smem, s, a) != cudaSuccess)
+            return EP_ERR_CUDA;
+        return launch_result();
+    }
     if (path == EP_LAYOUT_CLUSTER) {
         const size_t smem = cluster_smem_bytes(d);
         ep_dims_t widest = d;  // the largest shared-memory need of the path (E = kSmallMaxExperts)
@@ -1033,7 +1331,7 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
                 cudaSuccess)
             return EP_ERR_CUDA;
         // one CTA per kClusterPairsPerCta pairs, 2 to kClusterMaxCtas, as many as fit at once
-        const int64_t pairs = int64_t(d.num_ranks) * d.num_tokens * d.num_topk;
+        const int64_t pairs = int64_t(Rs) * d.num_tokens * d.num_topk;
         const int want = int(std::min<int64_t>(kClusterMaxCtas,
                                                std::max<int64_t>(2, ceil_div(pairs, kClusterPairsPerCta))));
         const int cl = fitting_cluster(layout_cluster_kernel, want, kSmallThreads, smem_max, g_layout_cluster_fit);
@@ -1083,7 +1381,11 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     return launch_result();
 }
 
+}  // namespace
+}  // namespace ep
+
 extern "C" int ep_diag_wait_timeout(void* flags, int32_t* status, void* stream) {
+    EP_NVTX_RANGE("ep_diag_wait_timeout");
     if (!flags || !status || (reinterpret_cast<uintptr_t>(flags) & 7u)) return EP_ERR_INVALID;
     diag_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t*>(flags), status);
     return launch_result();

@@ -107,6 +107,7 @@ extern "C" int ep_normal_layout(ep_dims_t d, int32_t recv_capacity, int32_t expe
                                 const uint8_t* is_token_in_rank, const int32_t* num_tokens_per_rank,
                                 const int32_t* recv_count, int32_t* token_recv_row, int32_t* recv_tokens,
                                 int32_t* num_recv_tokens_per_expert, int32_t* status, ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_normal_layout");
     (void)cfg;
     int rc = check_dims(d);
     if (rc != EP_OK) return rc;

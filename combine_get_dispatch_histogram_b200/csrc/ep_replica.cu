@@ -109,6 +109,7 @@ using namespace ep;
 extern "C" int ep_replica_weight_sync(int32_t num_logical, int32_t num_physical, const int32_t* phys_base,
                                       int64_t param_bytes, const void* master, void* replicas, int32_t* status,
                                       ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_replica_weight_sync");
     (void)cfg;
     const int rc = check_replica_args(num_logical, num_physical, phys_base, param_bytes, master, replicas);
     if (rc != EP_OK || param_bytes == 0) return rc;
@@ -125,6 +126,7 @@ extern "C" int ep_replica_weight_sync(int32_t num_logical, int32_t num_physical,
 extern "C" int ep_replica_grad_reduce(int32_t num_logical, int32_t num_physical, const int32_t* phys_base,
                                       int64_t num_params, const float* replica_grads, float* master_grads,
                                       int32_t* status, ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_replica_grad_reduce");
     (void)cfg;
     if (num_params < 0) return EP_ERR_INVALID;
     const int rc = check_replica_args(num_logical, num_physical, phys_base, num_params * 4, replica_grads, master_grads);

@@ -288,6 +288,7 @@ extern "C" int ep_reroute(int32_t num_ranks, int32_t num_tokens, int32_t num_top
                           int32_t num_extra, const int32_t* topk_idx_logical, void* workspace,
                           size_t workspace_bytes, int32_t* load, int32_t* num_replicas, int32_t* phys_base,
                           int32_t* topk_idx_phys, int32_t* status, ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_reroute");
     if (num_ranks <= 0 || num_tokens < 0 || num_topk <= 0 || num_logical <= 0 || num_extra < 0)
         return EP_ERR_INVALID;
     if (num_logical > kRerouteMaxLogical || num_topk > EP_MAX_TOPK) return EP_ERR_UNSUPPORTED;

@@ -8,7 +8,10 @@ non-zero return code.  There is no fallback: if ``libep.so`` is missing or no
 GPU is present, the call fails loudly.
 
 Tensor conventions (R ranks, T tokens per rank, k slots, E experts, H hidden,
-CAP = R*T slab rows per expert) follow ``include/ep.h``.
+CAP = R*T slab rows per expert) follow ``include/ep.h``.  Routing ids
+(``topk_idx``) may be int32 or int64; int64 ids are converted on the device by
+``ep_topk_idx_to_int32`` (saturating, so ids outside the int32 range are
+flagged as bad experts rather than wrapped) before the call.
 """
 from __future__ import annotations
 
@@ -39,6 +42,7 @@ EP_LAYOUT_CHUNKED = 1
 EP_LAYOUT_SINGLE_CTA = 2
 EP_LAYOUT_FUSED = 3
 EP_LAYOUT_CLUSTER = 4
+EP_LAYOUT_LOOKBACK = 5
 EP_REROUTE_TWO_LAUNCH = 1
 EP_REROUTE_CLUSTER = 2
 
@@ -54,6 +58,12 @@ class EPError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("num_ranks", ctypes.c_int32), ("num_tokens", ctypes.c_int32), ("num_topk", ctypes.c_int32),
                 ("num_experts", ctypes.c_int32), ("hidden", ctypes.c_int32)]
+
+
+class PeerTable(ctypes.Structure):
+    """``ep_peer_table_t``: device arrays of R uint64 addresses (slabs, src_info, flag words)."""
+
+    _fields_ = [("slab", ctypes.c_void_p), ("src_info", ctypes.c_void_p), ("flags", ctypes.c_void_p)]
 
 
 class Cfg(ctypes.Structure):
@@ -105,6 +115,33 @@ def load_library(path: str = LIB_PATH):
     lib.ep_reroute_workspace_bytes.restype = SZ
     lib.ep_reroute.argtypes = [I32, I32, I32, I32, I32, P, P, SZ, P, P, P, P, P, Cfg, P]
     lib.ep_reroute.restype = ctypes.c_int
+    lib.ep_topk_idx_to_int32.argtypes = [P, P, ctypes.c_int64, P]
+    lib.ep_topk_idx_to_int32.restype = ctypes.c_int
+    U64 = ctypes.c_uint64
+    lib.ep_layout_local_workspace_bytes.argtypes = [Dims]
+    lib.ep_layout_local_workspace_bytes.restype = SZ
+    lib.ep_layout_local.argtypes = [Dims, I32, P, P, P, SZ, P, P, P, P, P, Cfg, P]
+    lib.ep_layout_local.restype = ctypes.c_int
+    lib.ep_peer_offsets.argtypes = [I32, I32, I32, P, P, P]
+    lib.ep_peer_offsets.restype = ctypes.c_int
+    lib.ep_dispatch_peer_workspace_bytes.argtypes = []
+    lib.ep_dispatch_peer_workspace_bytes.restype = SZ
+    lib.ep_dispatch_peer.argtypes = [Dims, I32, PeerTable, P, P, P, P, P, U64, P, SZ, P, Cfg, P]
+    lib.ep_dispatch_peer.restype = ctypes.c_int
+    lib.ep_wait_peers.argtypes = [I32, P, U64, P, P, P]
+    lib.ep_wait_peers.restype = ctypes.c_int
+    lib.ep_signal_peers.argtypes = [I32, I32, P, P, U64, P]
+    lib.ep_signal_peers.restype = ctypes.c_int
+    lib.ep_peer_recv_count.argtypes = [I32, I32, I32, P, P, P]
+    lib.ep_peer_recv_count.restype = ctypes.c_int
+    lib.ep_combine_peer.argtypes = [Dims, I32, P, P, P, P, P, P, P, P, Cfg, P]
+    lib.ep_combine_peer.restype = ctypes.c_int
+    lib.ep_ipc_export.argtypes = [P, P, ctypes.POINTER(U64)]
+    lib.ep_ipc_export.restype = ctypes.c_int
+    lib.ep_ipc_import.argtypes = [P, U64, ctypes.POINTER(P), ctypes.POINTER(P)]
+    lib.ep_ipc_import.restype = ctypes.c_int
+    lib.ep_ipc_close.argtypes = [P]
+    lib.ep_ipc_close.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -162,6 +199,34 @@ def _status(device, status):
     return _need(status, "status", torch.int32, device=device)
 
 
+def ep_topk_idx_to_int32(topk_idx: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """int64 routing ids to the library's int32 form (``ep_topk_idx_to_int32``).
+
+    Ids outside the int32 range saturate to -2^31 or 2^31 - 1, which every
+    kernel flags as a bad expert; -1 and ids in range are kept.
+    """
+    lib = load_library()
+    _need(topk_idx, "topk_idx", torch.int64)
+    dev = topk_idx.device
+    if out is None:
+        out = torch.empty(topk_idx.shape, dtype=torch.int32, device=dev)
+    _need(out, "out", torch.int32, tuple(topk_idx.shape), dev)
+    with torch.cuda.device(dev):
+        rc = lib.ep_topk_idx_to_int32(_ptr(topk_idx), _ptr(out), topk_idx.numel(), _stream(dev, stream))
+    _check("ep_topk_idx_to_int32", rc)
+    if stream is not None:
+        out.record_stream(stream)  # the kernels that read it run on `stream`
+    return out
+
+
+def _idx32(topk_idx: torch.Tensor, name: str, stream=None) -> torch.Tensor:
+    """Routing ids as int32: int32 passes through, int64 is converted on the device."""
+    if isinstance(topk_idx, torch.Tensor) and topk_idx.dtype == torch.int64:
+        return ep_topk_idx_to_int32(topk_idx, stream=stream)
+    return _need(topk_idx, name, torch.int32)
+
+
 @dataclasses.dataclass
 class DispatchLayout:
     """Outputs of :func:`ep_layout`: the layout plus the dispatch / combine handle."""
@@ -215,7 +280,7 @@ def ep_layout(topk_idx: torch.Tensor, active: torch.Tensor, num_experts: int, *,
     zero-filled before its first use and reserved for ep_layout calls afterwards.
     """
     lib = load_library()
-    _need(topk_idx, "topk_idx", torch.int32)
+    topk_idx = _idx32(topk_idx, "topk_idx", stream)
     if topk_idx.dim() != 3:
         raise ValueError("topk_idx must be [R, T, k]")
     R, T, k = topk_idx.shape
@@ -264,7 +329,7 @@ def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, pair_row: torch.Tensor,
         raise ValueError("x must be [R, T, H]")
     R, T, H = x.shape
     dev = x.device
-    _need(topk_idx, "topk_idx", torch.int32, device=dev)
+    topk_idx = _need(_idx32(topk_idx, "topk_idx", stream), "topk_idx", torch.int32, device=dev)
     if topk_idx.dim() != 3 or tuple(topk_idx.shape[:2]) != (R, T):
         raise ValueError("topk_idx must be [R, T, k]")
     k = topk_idx.shape[2]
@@ -303,7 +368,7 @@ def ep_dispatch_fp8(x: torch.Tensor, topk_idx: torch.Tensor, pair_row: torch.Ten
         raise ValueError("x must be [R, T, H]")
     R, T, H = x.shape
     dev = x.device
-    _need(topk_idx, "topk_idx", torch.int32, device=dev)
+    topk_idx = _need(_idx32(topk_idx, "topk_idx", stream), "topk_idx", torch.int32, device=dev)
     if topk_idx.dim() != 3 or tuple(topk_idx.shape[:2]) != (R, T):
         raise ValueError("topk_idx must be [R, T, k]")
     k = topk_idx.shape[2]
@@ -354,7 +419,7 @@ def ep_combine(y: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tens
         raise ValueError("y must be [E, R*T, H]")
     E, cap, H = y.shape
     dev = y.device
-    _need(topk_idx, "topk_idx", torch.int32, device=dev)
+    topk_idx = _need(_idx32(topk_idx, "topk_idx", stream), "topk_idx", torch.int32, device=dev)
     if topk_idx.dim() != 3:
         raise ValueError("topk_idx must be [R, T, k]")
     R, T, k = topk_idx.shape
@@ -386,7 +451,7 @@ def ep_reroute(topk_idx_logical: torch.Tensor, num_logical: int, num_extra: int,
     Returns a dict with ``load``, ``num_replicas``, ``phys_base``, ``topk_idx_phys``, ``status``.
     """
     lib = load_library()
-    _need(topk_idx_logical, "topk_idx_logical", torch.int32)
+    topk_idx_logical = _idx32(topk_idx_logical, "topk_idx_logical", stream)
     if topk_idx_logical.dim() != 3:
         raise ValueError("topk_idx_logical must be [R, T, k]")
     R, T, k = topk_idx_logical.shape
@@ -499,7 +564,7 @@ def ep_normal_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_weights: to
     _need(x, "x", torch.bfloat16)
     R, T, H = x.shape
     dev = x.device
-    _need(topk_idx, "topk_idx", torch.int32, device=dev)
+    topk_idx = _need(_idx32(topk_idx, "topk_idx", stream), "topk_idx", torch.int32, device=dev)
     k = topk_idx.shape[2]
     _need(topk_weights, "topk_weights", torch.float32, (R, T, k), dev)
     _need(active, "active", torch.uint8, (R,), dev)
@@ -592,3 +657,227 @@ def ep_replica_grad_reduce(replica_grads: torch.Tensor, phys_base: torch.Tensor,
                                         _stream(dev, stream))
     _check("ep_replica_grad_reduce", rc)
     return master_grads
+
+
+# ----------------------------------------------------------------------------- EP across GPUs (one process per GPU)
+
+EP_IPC_HANDLE_BYTES = 64
+
+
+@dataclasses.dataclass
+class LocalLayout:
+    """Outputs of :func:`ep_layout_local` for one source rank."""
+
+    num_tokens_per_expert: torch.Tensor  # int32 [E] (the row every rank all-gathers)
+    num_tokens_per_rank: torch.Tensor    # int32 [R]
+    is_token_in_rank: torch.Tensor       # uint8 [T, R]
+    local_row: torch.Tensor              # int32 [T, k]
+    status: torch.Tensor                 # int32 [1]
+
+
+def ep_layout_local_workspace_bytes(num_ranks: int, num_tokens: int, num_topk: int, num_experts: int,
+                                    hidden: int = 8) -> int:
+    return int(load_library().ep_layout_local_workspace_bytes(Dims(num_ranks, num_tokens, num_topk, num_experts,
+                                                                   hidden)))
+
+
+def ep_layout_local(topk_idx: torch.Tensor, active: torch.Tensor, rank: int, num_experts: int, *, hidden: int = 8,
+                    workspace: Optional[torch.Tensor] = None, out: Optional[LocalLayout] = None,
+                    status: Optional[torch.Tensor] = None, cfg=None, stream=None) -> LocalLayout:
+    """Layout of one rank's own routing (``ep_layout_local``); ``topk_idx`` is that rank's [T, k]."""
+    lib = load_library()
+    topk_idx = _idx32(topk_idx, "topk_idx", stream)
+    if topk_idx.dim() != 2:
+        raise ValueError("topk_idx must be [T, k] (this rank's routing)")
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    R = active.shape[0]
+    E = int(num_experts)
+    _need(active, "active", torch.uint8, (R,), dev)
+    dims = Dims(R, T, k, E, hidden)
+    ws_bytes = int(lib.ep_layout_local_workspace_bytes(dims))
+    if workspace is None:
+        workspace = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, device=dev)
+    if out is None:
+        out = LocalLayout(torch.empty(E, dtype=torch.int32, device=dev), torch.empty(R, dtype=torch.int32, device=dev),
+                          torch.empty((T, R), dtype=torch.uint8, device=dev),
+                          torch.empty((T, k), dtype=torch.int32, device=dev), _status(dev, status))
+    else:
+        _need(out.num_tokens_per_expert, "num_tokens_per_expert", torch.int32, (E,), dev)
+        _need(out.num_tokens_per_rank, "num_tokens_per_rank", torch.int32, (R,), dev)
+        _need(out.is_token_in_rank, "is_token_in_rank", torch.uint8, (T, R), dev)
+        _need(out.local_row, "local_row", torch.int32, (T, k), dev)
+        if status is not None:
+            out.status = _need(status, "status", torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.ep_layout_local(dims, int(rank), _ptr(topk_idx), _ptr(active), _ptr(workspace), workspace.numel(),
+                                 _ptr(out.num_tokens_per_expert), _ptr(out.num_tokens_per_rank),
+                                 _ptr(out.is_token_in_rank), _ptr(out.local_row), _ptr(out.status), _cfg(cfg),
+                                 _stream(dev, stream))
+    _check("ep_layout_local", rc)
+    return out
+
+
+def ep_peer_offsets(counts, rank: int):
+    """Host derivation (``ep_peer_offsets``; no GPU): ``(expert_rank_offset [E], recv_count [E/R])`` of ``rank``.
+
+    ``counts`` is the all-gathered ``[R, E]`` int32 count matrix on the host (numpy or a CPU tensor).
+    """
+    import numpy as np
+
+    c = np.ascontiguousarray(counts.numpy() if isinstance(counts, torch.Tensor) else counts, dtype=np.int32)
+    if c.ndim != 2:
+        raise ValueError("counts must be [R, E]")
+    R, E = c.shape
+    offs = np.zeros(E, np.int32)
+    recv = np.zeros(E // R if R else 0, np.int32)
+    rc = load_library().ep_peer_offsets(R, E, int(rank), c.ctypes.data, offs.ctypes.data, recv.ctypes.data)
+    _check("ep_peer_offsets", rc)
+    return offs, recv
+
+
+def ep_dispatch_peer_workspace_bytes() -> int:
+    return int(load_library().ep_dispatch_peer_workspace_bytes())
+
+
+def _addr_table(t: torch.Tensor, name: str, R: int, dev):
+    return _need(t, name, torch.int64, (R,), dev)
+
+
+def ep_dispatch_peer(x: torch.Tensor, topk_idx: torch.Tensor, local_row: torch.Tensor, counts: torch.Tensor,
+                     active: torch.Tensor, rank: int, slab_table: torch.Tensor, src_info_table: torch.Tensor,
+                     flag_table: torch.Tensor, signal: int, workspace: torch.Tensor, *,
+                     status: Optional[torch.Tensor] = None, cfg=None, stream=None) -> torch.Tensor:
+    """Send this rank's rows to every destination's slab and signal (``ep_dispatch_peer``). Returns ``status``.
+
+    The three tables are int64 device tensors of R addresses (see ``ep_peer_table_t``).
+    """
+    lib = load_library()
+    _need(x, "x", torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError("x must be [T, H] (this rank's tokens)")
+    T, H = x.shape
+    dev = x.device
+    topk_idx = _need(_idx32(topk_idx, "topk_idx", stream), "topk_idx", torch.int32, device=dev)
+    k = topk_idx.shape[1]
+    _need(local_row, "local_row", torch.int32, (T, k), dev)
+    R, E = counts.shape
+    _need(counts, "counts", torch.int32, (R, E), dev)
+    _need(active, "active", torch.uint8, (R,), dev)
+    table = PeerTable(_ptr(_addr_table(slab_table, "slab_table", R, dev)),
+                      _ptr(_addr_table(src_info_table, "src_info_table", R, dev)),
+                      _ptr(_addr_table(flag_table, "flag_table", R, dev)))
+    _need(workspace, "workspace", torch.uint8, device=dev)
+    status = _status(dev, status)
+    with torch.cuda.device(dev):
+        rc = lib.ep_dispatch_peer(Dims(R, T, k, E, H), int(rank), table, _ptr(x), _ptr(topk_idx), _ptr(local_row),
+                                  _ptr(counts), _ptr(active), int(signal), _ptr(workspace), workspace.numel(),
+                                  _ptr(status), _cfg(cfg), _stream(dev, stream))
+    _check("ep_dispatch_peer", rc)
+    return status
+
+
+def ep_wait_peers(flags: torch.Tensor, signal: int, active: torch.Tensor, *, status: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """Bounded wait until ``flags[s] >= signal`` for every active rank s (``ep_wait_peers``). Returns ``status``."""
+    lib = load_library()
+    dev = flags.device
+    R = flags.shape[0]
+    _need(flags, "flags", torch.int64, (R,), dev)
+    _need(active, "active", torch.uint8, (R,), dev)
+    status = _status(dev, status)
+    with torch.cuda.device(dev):
+        rc = lib.ep_wait_peers(R, _ptr(flags), int(signal), _ptr(active), _ptr(status), _stream(dev, stream))
+    _check("ep_wait_peers", rc)
+    return status
+
+
+def ep_signal_peers(flag_table: torch.Tensor, rank: int, active: torch.Tensor, signal: int, *, stream=None):
+    """Release ``signal`` into word ``rank`` of every active rank's flags (``ep_signal_peers``)."""
+    lib = load_library()
+    dev = flag_table.device
+    R = flag_table.shape[0]
+    _addr_table(flag_table, "flag_table", R, dev)
+    _need(active, "active", torch.uint8, (R,), dev)
+    with torch.cuda.device(dev):
+        rc = lib.ep_signal_peers(R, int(rank), _ptr(flag_table), _ptr(active), int(signal), _stream(dev, stream))
+    _check("ep_signal_peers", rc)
+
+
+def ep_peer_recv_count(counts: torch.Tensor, rank: int, *, out: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """Rows each local expert of ``rank`` receives, from the device count matrix (``ep_peer_recv_count``)."""
+    lib = load_library()
+    dev = counts.device
+    R, E = counts.shape
+    _need(counts, "counts", torch.int32, (R, E), dev)
+    if out is None:
+        out = torch.empty(E // R, dtype=torch.int32, device=dev)
+    _need(out, "out", torch.int32, (E // R,), dev)
+    with torch.cuda.device(dev):
+        rc = lib.ep_peer_recv_count(R, E, int(rank), _ptr(counts), _ptr(out), _stream(dev, stream))
+    _check("ep_peer_recv_count", rc)
+    return out
+
+
+def ep_combine_peer(slab_table: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                    local_row: torch.Tensor, counts: torch.Tensor, active: torch.Tensor, rank: int, hidden: int, *,
+                    out: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None, cfg=None,
+                    stream=None):
+    """Weighted gather of this rank's tokens from every rank's expert outputs (``ep_combine_peer``).
+
+    Returns ``(out [T, H] bf16, status)``.
+    """
+    lib = load_library()
+    dev = topk_weights.device
+    topk_idx = _need(_idx32(topk_idx, "topk_idx", stream), "topk_idx", torch.int32, device=dev)
+    T, k = topk_idx.shape
+    R, E = counts.shape
+    _addr_table(slab_table, "slab_table", R, dev)
+    _need(topk_weights, "topk_weights", torch.float32, (T, k), dev)
+    _need(local_row, "local_row", torch.int32, (T, k), dev)
+    _need(counts, "counts", torch.int32, (R, E), dev)
+    _need(active, "active", torch.uint8, (R,), dev)
+    H = int(hidden)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (T, H), dev)
+    status = _status(dev, status)
+    with torch.cuda.device(dev):
+        rc = lib.ep_combine_peer(Dims(R, T, k, E, H), int(rank), _ptr(slab_table), _ptr(topk_idx),
+                                 _ptr(topk_weights), _ptr(local_row), _ptr(counts), _ptr(active), _ptr(out),
+                                 _ptr(status), _cfg(cfg), _stream(dev, stream))
+    _check("ep_combine_peer", rc)
+    return out, status
+
+
+def ep_ipc_export(t: torch.Tensor):
+    """``(handle bytes, offset)`` of the allocation holding ``t`` (``ep_ipc_export``), to send to other ranks."""
+    lib = load_library()
+    if not t.is_cuda:
+        raise ValueError("t must be a CUDA tensor")
+    buf = ctypes.create_string_buffer(EP_IPC_HANDLE_BYTES)
+    off = ctypes.c_uint64(0)
+    with torch.cuda.device(t.device):
+        rc = lib.ep_ipc_export(_ptr(t), buf, ctypes.byref(off))
+    _check("ep_ipc_export", rc)
+    return buf.raw, int(off.value)
+
+
+def ep_ipc_import(handle: bytes, offset: int, device=None):
+    """Map another process's exported buffer (``ep_ipc_import``): ``(address, base)``; close with ``ep_ipc_close``."""
+    lib = load_library()
+    if len(handle) != EP_IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle is {EP_IPC_HANDLE_BYTES} bytes")
+    ptr, base = ctypes.c_void_p(), ctypes.c_void_p()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        rc = lib.ep_ipc_import(ctypes.create_string_buffer(handle, EP_IPC_HANDLE_BYTES), int(offset),
+                               ctypes.byref(ptr), ctypes.byref(base))
+    _check("ep_ipc_import", rc)
+    return int(ptr.value), int(base.value)
+
+
+def ep_ipc_close(base: int):
+    """Unmap a buffer mapped by :func:`ep_ipc_import` (``ep_ipc_close``)."""
+    _check("ep_ipc_close", load_library().ep_ipc_close(ctypes.c_void_p(base)))

@@ -36,6 +36,12 @@
  *                  NeMo page: one copy per destination rank, unweighted combine.
  *   ep_replica_weight_sync, ep_replica_grad_reduce -- "Replica weight sync" and
  *                  "Replica gradient reduction" of the UltraEP page.
+ *   ep_layout_local, ep_dispatch_peer, ep_wait_peers, ep_signal_peers,
+ *   ep_combine_peer (+ ep_peer_offsets, ep_peer_recv_count, ep_ipc_*) -- the
+ *                  same low-latency dispatch / combine between processes that
+ *                  each own one GPU, over NVLink peer memory (section at the end).
+ *   ep_topk_idx_to_int32 -- the int64 topk_idx of the NeMo page's Buffer calls
+ *                  in the int32 form of the nixl PR, saturating out-of-range ids.
  *   ep_layout_noalloc, ep_layout_path and the *_workspace_bytes queries have
  *                  no counterpart on the pages; they serve callers of this
  *                  library (scratch without allocation, which path a call takes,
@@ -52,7 +58,8 @@
  *     k = num_topk, E = num_experts, H = hidden, CAP = R*T (slab rows per
  *     expert).
  *   - topk_idx is int32 (the index width the nixl PR made the default);
- *     -1 means "no selection".  A pair (r,t,j) is LIVE when
+ *     -1 means "no selection".  Routing held as int64 (the NeMo page's dtype)
+ *     is converted once by ep_topk_idx_to_int32.  A pair (r,t,j) is LIVE when
  *     0 <= e = topk_idx[r,t,j] < E, active[r] != 0 and active[e/E_local] != 0:
  *     a masked rank neither sends nor receives.
  *   - Data errors never trap.  Kernels OR bits into *status (int32, device,
@@ -135,9 +142,13 @@ enum {
     EP_LAYOUT_SINGLE_CTA = 2, /* one launch, one CTA; R <= 32, E <= 1024, R*T*k <= 32768 */
     EP_LAYOUT_FUSED = 3,      /* one cooperative launch with two grid barriers; needs the
                                  chunk grid to fit the device (else EP_ERR_UNSUPPORTED) */
-    EP_LAYOUT_CLUSTER = 4     /* one launch of a thread-block cluster of up to 16 CTAs that
+    EP_LAYOUT_CLUSTER = 4,    /* one launch of a thread-block cluster of up to 16 CTAs that
                                  share their histograms through distributed shared memory;
                                  R <= 32, E <= 1024, R*T*k <= 65536 */
+    EP_LAYOUT_LOOKBACK = 5    /* one ordinary launch, one CTA per chunk: each CTA publishes its
+                                 chunk's histogram with a release flag and waits (bounded) only
+                                 for the chunks before it; any shape whose chunk grid has at most
+                                 255 chunks (every supported shape) */
 };
 
 /* Data paths of ep_dispatch / ep_combine (ep_cfg_t.variant). */
@@ -179,6 +190,25 @@ EP_API int ep_layout_path(ep_dims_t d, ep_cfg_t cfg);
  */
 EP_API int ep_diag_wait_timeout(void *flags, int32_t *status, void *stream);
 
+
+/*
+ * ep_topk_idx_to_int32 -- routing ids in the page's int64 form to the int32
+ * form every other entry point reads.
+ *
+ * Buffer.get_dispatch_layout and Buffer.dispatch on the NeMo AutoModel page
+ * "nemo_automodel.components.moe.uccl_ep.buffer" take topk_idx as
+ * torch.int64; the ai-dynamo/nixl PR "nixl_ep: Optimize low-latency NVLink
+ * path" made 32-bit indices the default, which this library uses.
+ * in:  topk_idx64 int64 [n]   8-byte aligned
+ * out: topk_idx32 int32 [n]   4-byte aligned; every element written
+ * Each id is converted with saturation: -1 and every id in [-2^31, 2^31) keep
+ * their value, larger ids become 2^31 - 1 and smaller ones -2^31.  Both
+ * saturated values lie outside [-1, E) for every supported E, so the layout,
+ * dispatch, combine and reroute kernels drop those pairs and raise
+ * EP_STATUS_BAD_EXPERT instead of sending a wrapped id to a real expert.
+ * One launch on `stream`; n == 0 enqueues nothing.
+ */
+EP_API int ep_topk_idx_to_int32(const int64_t *topk_idx64, int32_t *topk_idx32, int64_t n, void *stream);
 
 /*
  * ep_layout -- per-expert / per-rank histogram, prefix sums and stable rows.
@@ -234,7 +264,9 @@ enum { EP_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024 };
  *   - The first call on a device looks up that device's scratch address
  *     (cudaGetSymbolAddress with the device current) and caches it; make
  *     that first call before any stream capture.  EP_ERR_CUDA if the lookup
- *     fails.
+ *     fails.  The cache is per context: after a cudaDeviceReset the next
+ *     call looks the address up again (the new context's copy of the array
+ *     starts zeroed, as the barrier state requires).
  *   - All calls on a device share the one array and it keeps the last call's
  *     contents.  It is zero when the library is loaded, as the layout's
  *     barrier state requires, and every call leaves that state ready for the
@@ -447,6 +479,156 @@ EP_API int ep_replica_weight_sync(int32_t num_logical, int32_t num_physical, con
 EP_API int ep_replica_grad_reduce(int32_t num_logical, int32_t num_physical, const int32_t *phys_base,
                                   int64_t num_params, const float *replica_grads, float *master_grads,
                                   int32_t *status, ep_cfg_t cfg, void *stream);
+
+/*
+ * ---------------------------------------------------------------------------
+ * Expert parallelism across GPUs: one process per GPU, rank r of R.
+ *
+ * The low-latency dispatch / combine of the NeMo AutoModel page
+ * "nemo_automodel.components.moe.uccl_ep.buffer" (Buffer.low_latency_dispatch,
+ * Buffer.low_latency_combine; intranode NVLink) store token rows straight into
+ * the destination rank's receive buffer and signal arrival with flags; the
+ * ai-dynamo/nixl PR "nixl_ep: Optimize low-latency NVLink path" keeps a table of
+ * peer pointers and an active-rank mask that lets the ranks that are still up
+ * carry on.  The entry points below are that transport over NVLink / NVSwitch
+ * peer memory.  One step, in stream order on every rank:
+ *   1. ep_layout_local on the rank's own routing; the caller all-gathers the
+ *      [E] num_tokens_per_expert of every rank into counts [R, E] (a collective
+ *      of R * E int32, e.g. NCCL all_gather);
+ *   2. ep_dispatch_peer: rows into every destination's slab, then a release flag;
+ *   3. ep_wait_peers on the rank's arrival flags (bounded), ep_peer_recv_count;
+ *   4. the experts run on the local slab and write their outputs;
+ *   5. ep_signal_peers into every rank's "ready" flags, ep_wait_peers on the
+ *      rank's own ready flags;
+ *   6. ep_combine_peer gathers the weighted outputs back into the rank's tokens.
+ * Receive layout: expert e (on rank d = e / E_local, local expert le) keeps its
+ * rows in (source rank, token, slot) order in d's slab [E_local, CAP, H],
+ * CAP = R * T: the row of source r's pair is expert_rank_offset[e][r] (from the
+ * count matrix) + local_row, exactly the single-GPU layout of ep_layout.
+ * Peer memory is touched only by plain 16-byte loads / stores and 8-byte
+ * release / acquire flag accesses (no bulk copy, no multicast).  A masked rank
+ * (active[d] == 0) is neither written, read, signalled nor waited for.  Signals
+ * are 64-bit values that grow from step to step (a wait passes when the flag is
+ * >= the value), so flag words never need clearing; zero them once.
+ * ---------------------------------------------------------------------------
+ */
+
+/* Addresses, valid in the calling process, of every rank's buffers: device
+ * arrays of num_ranks uint64 each (entry d = rank d's buffer; the caller's own
+ * rank included).  Map peers' buffers with ep_ipc_export / ep_ipc_import. */
+typedef struct ep_peer_table {
+    const uint64_t *slab;      /* rank d's receive slab, bf16 [E_local, CAP, H], 16-byte aligned */
+    const uint64_t *src_info;  /* rank d's src_info, int32 [E_local, CAP, 2] */
+    const uint64_t *flags;     /* rank d's arrival flag words, uint64 [R]; word s is written by source s */
+} ep_peer_table_t;
+
+/* Bytes of the workspace ep_layout_local needs for `d` (0 for an invalid shape). */
+EP_API size_t ep_layout_local_workspace_bytes(ep_dims_t d);
+
+/*
+ * ep_layout_local -- ep_layout over ONE source rank's routing (Buffer.get_dispatch_layout
+ * as each rank of a real EP world runs it on its own tokens).
+ * in:  rank                 this process's rank r
+ *      topk_idx   int32 [T,k] rank r's routing
+ *      active     uint8 [R]   the world's active-rank mask (pairs of a masked source or
+ *                             destination are not live)
+ *      workspace  >= ep_layout_local_workspace_bytes(d), 16-byte aligned, zeroed once
+ *                 before first use, reserved for ep_layout_local calls (as for ep_layout)
+ * out: num_tokens_per_expert int32 [E]   r's live pairs per expert (the row to all-gather)
+ *      num_tokens_per_rank   int32 [R]   r's tokens with >= 1 live pair on rank d
+ *      is_token_in_rank      uint8 [T,R]
+ *      local_row             int32 [T,k] row of each live pair among r's live pairs of its
+ *                                        expert, in (token, slot) order; -1 if not live
+ */
+EP_API int ep_layout_local(ep_dims_t d, int32_t rank, const int32_t *topk_idx, const uint8_t *active,
+                           void *workspace, size_t workspace_bytes, int32_t *num_tokens_per_expert,
+                           int32_t *num_tokens_per_rank, uint8_t *is_token_in_rank, int32_t *local_row,
+                           int32_t *status, ep_cfg_t cfg, void *stream);
+
+/*
+ * ep_peer_offsets -- HOST function (no GPU): from the all-gathered count matrix,
+ * counts int32 [R,E] (host), the first row of source `rank` inside every expert,
+ * expert_rank_offset int32 [E] (host) = sum over r' < rank of counts[r'][e], and
+ * the rows each of `rank`'s experts receives, recv_count int32 [E/R] (host) =
+ * sum over r' of counts[r'][rank * E/R + le].  For callers that bring the counts
+ * to the host; the device path derives the same values inside its kernels.
+ * EP_ERR_INVALID for bad arguments or a sum beyond int32.
+ */
+EP_API int ep_peer_offsets(int32_t num_ranks, int32_t num_experts, int32_t rank, const int32_t *counts,
+                           int32_t *expert_rank_offset, int32_t *recv_count);
+
+/* Bytes of workspace ep_dispatch_peer needs (a CTA-completion counter). */
+EP_API size_t ep_dispatch_peer_workspace_bytes(void);
+
+/*
+ * ep_dispatch_peer -- send rank r's token rows to the experts' slabs on every rank.
+ * in:  peers      the table above
+ *      x          bf16 [T,H]   rank r's tokens, 16-byte aligned
+ *      topk_idx   int32 [T,k], local_row int32 [T,k] (ep_layout_local on the same routing)
+ *      counts     int32 [R,E]  device, every rank's num_tokens_per_expert (all-gathered)
+ *      active     uint8 [R]    mask at dispatch time (masked destinations are skipped)
+ *      signal     value released into word r of every active destination's flags after
+ *                 the last row (use a value larger than every earlier step's)
+ *      workspace  >= ep_dispatch_peer_workspace_bytes(), 8-byte aligned, zeroed once,
+ *                 reserved for this rank's ep_dispatch_peer calls (ordered on the GPU)
+ * out (in the destination ranks' memory): slab rows and src_info (src_rank, src_token)
+ *      of every live pair; rows >= CAP are flagged EP_STATUS_OVERFLOW and not written.
+ * A masked source (active[r] == 0) sends and signals nothing.  The call launches even
+ * with T = 0, so the flags still go out.
+ */
+EP_API int ep_dispatch_peer(ep_dims_t d, int32_t rank, ep_peer_table_t peers, const uint16_t *x,
+                            const int32_t *topk_idx, const int32_t *local_row, const int32_t *counts,
+                            const uint8_t *active, uint64_t signal, void *workspace, size_t workspace_bytes,
+                            int32_t *status, ep_cfg_t cfg, void *stream);
+
+/*
+ * ep_wait_peers -- bounded wait until flags[s] >= signal for every active rank s.
+ * flags uint64 [R] in this rank's memory (8-byte aligned).  Each wait gives up
+ * after the library's wait limit (2 s): EP_STATUS_TIMEOUT is OR-ed into *status
+ * and the kernel returns, so the context stays usable; kernels after it in the
+ * stream then see the peers' writes only if no timeout was reported.
+ */
+EP_API int ep_wait_peers(int32_t num_ranks, const uint64_t *flags, uint64_t signal, const uint8_t *active,
+                         int32_t *status, void *stream);
+
+/*
+ * ep_signal_peers -- after the kernels before it in the stream, release `signal`
+ * into word `rank` of every active rank d's flags; peer_flags is a device array of
+ * R addresses (rank d's flag words).  Nothing is sent when rank itself is masked.
+ */
+EP_API int ep_signal_peers(int32_t num_ranks, int32_t rank, const uint64_t *peer_flags, const uint8_t *active,
+                           uint64_t signal, void *stream);
+
+/* recv_count int32 [E/R] (device) = rows each local expert of `rank` receives,
+ * summed over the count matrix counts int32 [R,E] (device). */
+EP_API int ep_peer_recv_count(int32_t num_ranks, int32_t num_experts, int32_t rank, const int32_t *counts,
+                              int32_t *recv_count, void *stream);
+
+/*
+ * ep_combine_peer -- rank r's weighted gather of its tokens' expert outputs.
+ * in:  y_slabs   device [R] addresses of every rank's expert outputs, bf16 [E_local, CAP, H]
+ *                (rows as ep_dispatch_peer placed them)
+ *      topk_idx, topk_weights float [T,k], local_row, counts, active (mask at combine time)
+ * out: out bf16 [T,H] = bf16_rne(sum over j = 0..k-1 of w[t,j] * y[row of (t,j)]) in
+ *      float32 from +0, over live slots whose destination is active; zeros if active[r] == 0.
+ */
+EP_API int ep_combine_peer(ep_dims_t d, int32_t rank, const uint64_t *y_slabs, const int32_t *topk_idx,
+                           const float *topk_weights, const int32_t *local_row, const int32_t *counts,
+                           const uint8_t *active, uint16_t *out, int32_t *status, ep_cfg_t cfg, void *stream);
+
+/* CUDA IPC handles for the peer table: a handle is EP_IPC_HANDLE_BYTES of host memory. */
+enum { EP_IPC_HANDLE_BYTES = 64 };
+
+/* The IPC handle of the allocation that holds device pointer `ptr` and ptr's byte
+ * offset inside it (host outputs), to send to the other ranks. */
+EP_API int ep_ipc_export(const void *ptr, void *handle, uint64_t *offset);
+
+/* Map another process's exported buffer: *ptr = its address here, *base = the mapping
+ * to pass to ep_ipc_close.  A process cannot import its own handles (CUDA refuses). */
+EP_API int ep_ipc_import(const void *handle, uint64_t offset, void **ptr, void **base);
+
+/* Unmap a buffer mapped by ep_ipc_import. */
+EP_API int ep_ipc_close(void *base);
 
 #ifdef __cplusplus
 }

@@ -12,8 +12,8 @@ import torch
 
 import oracle
 from combine_get_dispatch_histogram_b200 import ep, inputs
-from gpu_util import (bf16_dev, bf16_host, check_close, check_dispatch, check_layout, dev, f32_dev, i32_dev,
-                      run_path, u8_dev)
+from gpu_util import (bf16_dev, bf16_host, check_close, check_combine_full, check_dispatch, check_layout, dev,
+                      f32_dev, i32_dev, run_path, u8_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -103,10 +103,6 @@ def test_replica_workload_full_size():
     phys = inputs.Inputs(rref["topk_idx_phys"], inp.topk_weights, inp.x, inp.active)
     ref = oracle.layout(phys.topk_idx, phys.active, E)
     packed, _ = oracle.dispatch(phys.x, phys.topk_idx, ref)
-    rng = np.random.default_rng(3)
-    tokens = np.stack([rng.integers(0, w.num_ranks, 3000), rng.integers(0, w.num_tokens, 3000)], axis=1)
-    want, _ = oracle.combine(packed, ref.list_base[:-1], phys.topk_idx, phys.topk_weights, ref.pair_row,
-                             phys.active, E, tokens=tokens)
     # the GPU runs on its own rerouted ids
     idx = rr["topk_idx_phys"]
     status = torch.zeros(1, dtype=torch.int32, device=dev())
@@ -116,8 +112,8 @@ def test_replica_workload_full_size():
     torch.cuda.synchronize()
     check_layout(lay, ref, "replica")
     check_dispatch(recv_x, src_info, ref, packed, "replica")
-    got = bf16_host(out)[tokens[:, 0], tokens[:, 1]]
-    check_close(got, want, "replica")
+    checked = check_combine_full(out, packed, ref, phys.topk_idx, phys.topk_weights, phys.active, E, "replica")
+    assert checked == w.num_ranks * w.num_tokens
     assert int(status.item()) == 0
 
 
@@ -354,10 +350,10 @@ def test_vector_variant_rejects_wide_topk():
     assert ei.value.code == ep.EP_ERR_UNSUPPORTED
 
 
-LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER = 1, 2, 3, 4
+LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER, LAYOUT_LOOKBACK = 1, 2, 3, 4, 5
 
 
-@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER])
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER, LAYOUT_LOOKBACK])
 @pytest.mark.parametrize("name", ["tiny", "decode", "sweep_T16_mask5", "sweep_T512", "sweep_T256_mask5"])
 def test_layout_paths_match_oracle(name, path):
     w = inputs.named(name)
@@ -367,7 +363,7 @@ def test_layout_paths_match_oracle(name, path):
                f"{name} layout path {path}")
 
 
-@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER])
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER, LAYOUT_LOOKBACK])
 @pytest.mark.parametrize("name", ["k1", "T1", "R1", "E_equals_R", "k32", "many_experts"])
 def test_layout_paths_edge_shapes(name, path):
     c = EDGE[name]
@@ -405,7 +401,7 @@ def test_single_cta_layout_long_parts(R, T, k, E, path):
                f"path {path} R={R} T={T} k={k}")
 
 
-@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER])
+@pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER, LAYOUT_LOOKBACK])
 def test_layout_paths_overflow_and_bad_ids(path):
     R, T, k, E, H = 2, 16, 3, 4, 64
     idx = np.zeros((R, T, k), np.int32)
@@ -468,7 +464,7 @@ def test_cluster_layout_sizes(T):
 @pytest.mark.parametrize("seed", range(40))
 def test_one_launch_layout_fuzz(seed):
     """Random shapes within the one-launch paths' limits (R <= 32, E <= 1024), each through the
-    single-CTA, cluster and chunked paths: every layout output bit-exact against the oracle."""
+    single-CTA, cluster, chunked and look-back paths: every layout output bit-exact against the oracle."""
     rng = np.random.default_rng(9000 + seed)
     R = int(rng.integers(1, 33))
     E = R * int(rng.integers(1, max(2, 1024 // R + 1)))
@@ -480,8 +476,38 @@ def test_one_launch_layout_fuzz(seed):
     idx = np.where(rng.random(idx.shape) < 0.1, -1, idx).astype(np.int32)
     act = (rng.random(R) > 0.2).astype(np.uint8)
     ref = oracle.layout(idx, act, E)
-    for path in (LAYOUT_SINGLE_CTA, LAYOUT_CLUSTER, LAYOUT_CHUNKED):
+    for path in (LAYOUT_SINGLE_CTA, LAYOUT_CLUSTER, LAYOUT_CHUNKED, LAYOUT_LOOKBACK):
         lay = ep.ep_layout(i32_dev(idx), u8_dev(act), E, hidden=8, cfg=dict(variant=path))
         torch.cuda.synchronize()
         check_layout(lay, ref, f"seed {seed} R={R} T={T} k={k} E={E} path {path}")
         assert int(lay.status.item()) == ref.status, (seed, path)
+
+
+def test_lookback_and_fused_layouts_share_a_workspace_across_shapes():
+    """The look-back and fused paths keep their flags in the same workspace prefix; alternating
+    them over shapes with different chunk grids never lets a stale flag pass for a current one."""
+    ws = torch.zeros(ep.ep_layout_workspace_bytes(8, 4096, 8, 256, 7168) + 4096, dtype=torch.uint8, device=dev())
+    cases = [inputs.prefill(), inputs.decode(), inputs.sweep(16, masked=True), inputs.replica(), inputs.sweep(512)]
+    for it, w in enumerate(cases * 2):
+        inp = inputs.make_inputs(w, tokens=False)
+        E = w.num_experts
+        ref = oracle.layout(inp.topk_idx, inp.active, E)
+        for path in (LAYOUT_LOOKBACK, LAYOUT_FUSED, LAYOUT_LOOKBACK):
+            lay = ep.ep_layout(i32_dev(inp.topk_idx), u8_dev(inp.active), E, hidden=w.hidden, workspace=ws,
+                               cfg=dict(variant=path))
+            torch.cuda.synchronize()
+            check_layout(lay, ref, f"call {it} {w.name} path {path}")
+            assert int(lay.status.item()) == ref.status
+
+
+@pytest.mark.parametrize("T", [1, 33, 4096, 8192])
+def test_lookback_layout_many_chunks(T):
+    """Prefill-style Zipf routing through the look-back path, from one token per rank to 148 chunks."""
+    w = inputs.Workload(f"zipf_T{T}", 8, T, 8, 256, 64, routing="zipf", zipf_s=1.2, inactive=(6,) if T == 33 else ())
+    inp = inputs.make_inputs(w, tokens=False)
+    ref = oracle.layout(inp.topk_idx, inp.active, w.num_experts)
+    lay = ep.ep_layout(i32_dev(inp.topk_idx), u8_dev(inp.active), w.num_experts, hidden=w.hidden,
+                       cfg=dict(variant=LAYOUT_LOOKBACK))
+    torch.cuda.synchronize()
+    check_layout(lay, ref, f"lookback T={T}")
+    assert int(lay.status.item()) == ref.status
