@@ -474,9 +474,33 @@ def run_ours(args, rank, world, local_rank, w, inp):
         e2e = dict(ms=e2e_ms, h2d=h2d, d2h=d2h)
         assert np.array_equal(h_out[(n - 1) % 2].numpy(), out.view(torch.int16).cpu().numpy())
 
+    # ---------------------------------------------------------------- dispatch ceilings (after the timed region)
+    # The paced dispatch kernel with its row loads left out: mode 0 times the scatter's stores alone,
+    # mode 1 the stores plus the paced prefetch of the rows -- the dispatch's own HBM traffic with no
+    # store waiting for a read.  Each is timed like the steps: warm-up, then one event pair per call.
+    ceil_ms = []
+    for mode in (0, 1):
+        def ceiling_call():
+            ep.ep_diag_dispatch_ceiling(cur["b"]["x"], idx_phys(), lay.pair_row, E, mode, recv_x=recv_x,
+                                        src_info=src_info, status=status, stream=stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                ceiling_call()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for e0, e1 in evs:
+                e0.record(stream)
+                ceiling_call()
+                e1.record(stream)
+        stream.synchronize()
+        ceil_ms.append(statistics.median(e0.elapsed_time(e1) for e0, e1 in evs))
+    if int(status.item()) != 0:
+        raise SystemExit(f"device status {int(status.item())} after the ceiling calls")
+
     # ---------------------------------------------------------------- reduce over ranks
     flat = [v for st in part_stats for v in (st["median"], st["min"], st["max"])]
-    total_ms, e2e_ms, *flat = reduce_over_ranks([total_ms, e2e["ms"] if e2e else 0.0] + flat, world, dev, "max")
+    total_ms, e2e_ms, c0_ms, c1_ms, *flat = reduce_over_ranks(
+        [total_ms, e2e["ms"] if e2e else 0.0] + ceil_ms + flat, world, dev, "max")
     part_stats = [dict(median=flat[3 * i], min=flat[3 * i + 1], max=flat[3 * i + 2]) for i in range(len(parts))]
     lay_ms, dis_ms, com_ms = (st["median"] for st in part_stats)
     ms_per_step = total_ms / args.steps
@@ -519,6 +543,14 @@ def run_ours(args, rank, world, local_rank, w, inp):
                      "traffic": profiled_traffic(dom[0], w.name),
                      "algorithmic_bytes": dom[1]},
         "gpu_launches": launches_per_step * args.steps,
+        "dispatch_ceiling": {
+            "what": "the paced dispatch kernel without its row loads (ep_diag_dispatch_ceiling), timed after the "
+                    "steps: stores alone, and stores plus the paced L2 prefetch of the rows (the dispatch's HBM "
+                    "traffic with no store waiting on a read)",
+            "stores_only_us": round(c0_ms * 1e3, 2),
+            "stores_and_row_reads_us": round(c1_ms * 1e3, 2),
+            "dispatch_over_stores_and_reads": round(dis_ms / c1_ms, 4),
+        },
     }
     if args.graph:
         line["graph"] = True

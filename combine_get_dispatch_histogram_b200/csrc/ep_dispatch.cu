@@ -41,6 +41,13 @@ namespace {
 
 constexpr uint32_t kDispatchPieceMax = 16384;  // largest row piece staged at once
 constexpr int kDispatchMaxStages = 16;
+// Paced reads (EP_VARIANT_PACED), measured on B200 at the prefill shape: one CTA per SM with a
+// 14-stage ring, L2 prefetches issued in the first 6 us of every 40 us, ~300 KB of rows ahead per
+// CTA (about 45 MB of L2 in all).
+constexpr uint64_t kPacePeriodNs = 40000;
+constexpr uint64_t kPaceWindowNs = 6000;
+constexpr int64_t kPaceAheadBytes = 300 * 1024;
+constexpr int kPaceMinUnitsPerCta = 64;  // AUTO paces only runs long enough to span several periods
 
 struct DispatchArgs {
     const uint8_t* x;
@@ -64,6 +71,12 @@ struct DispatchArgs {
     uint32_t stage_bytes;
     int stages;
     int64_t n_units;
+    // Paced reads (read_period_ns 0: off).  The rows a CTA will stage next are brought into L2
+    // by prefetches issued only while globaltimer % read_period_ns < read_window_ns, up to
+    // read_ahead units past the one being stored, so every SM reads in the same short windows
+    // and HBM serves the stores alone in between; the staging loads then hit L2.
+    uint64_t read_period_ns, read_window_ns;
+    int read_ahead;
 };
 
 struct UnitMeta {
@@ -97,7 +110,10 @@ __device__ __forceinline__ uint32_t piece_size(const DispatchArgs& a, int q) {
     return q + 1 < a.n_pieces ? a.piece_bytes : uint32_t(a.row_bytes - int64_t(q) * a.piece_bytes);
 }
 
-template <bool NORMAL>
+// NOLOAD (the ceiling diagnostic only): the row loads are left out and the zeroed ring is
+// stored as it is, so the kernel issues the dispatch's row stores (and, paced, its L2 prefetches)
+// without waiting for any read.
+template <bool NORMAL, bool NOLOAD>
 __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x;
@@ -106,6 +122,10 @@ __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
     int2* meta = reinterpret_cast<int2*>(full + S);  // [S][32] (e, row) of the staged unit
     int2* slot = meta + S * 32;                       // [S][32] normal mode: (slot expert, weight bits)
 
+    if (NOLOAD)
+        for (size_t i = lane; i < size_t(S) * a.stage_bytes / 16; i += 32)
+            reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (NOLOAD) fence_proxy_async_shared();  // the zeroed ring is read by the bulk stores
     if (lane == 0) {
         for (int s = 0; s < S; ++s) mbar_init(smem_u32(full + s), 1);
         mbar_init_fence();
@@ -118,6 +138,34 @@ __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
     const int64_t my_n = first < a.n_units ? (a.n_units - 1 - first) / step + 1 : 0;
     const uint64_t pol_load = policy_evict_first();
     const uint64_t pol_store = policy_evict_first();
+    const uint64_t pol_prefetch = policy_evict_last();
+
+    // Paced reads: after each unit, inside the read window (or when fewer than a ring's worth of
+    // units are prefetched), prefetch the rows of units [pf, i + read_ahead) that have a live slot.
+    // Lane j checks unit pf + j, so 32 units go per round.
+    int64_t pf = my_n < S ? my_n : S;  // the first S units are loaded straight from HBM
+    auto pace_reads = [&](int64_t i) {
+        int go = 0;
+        if (lane == 0)
+            go = pf <= i + S || global_timer_ns() % a.read_period_ns < a.read_window_ns;
+        if (!__shfl_sync(0xffffffffu, go, 0)) return;
+        const int64_t want = (i + a.read_ahead) < my_n ? (i + a.read_ahead) : my_n;
+        for (; pf < want; pf += 32) {
+            const int64_t v = pf + lane;
+            if (v >= want) continue;
+            const int64_t u = first + v * step;
+            const int64_t tok = u / a.n_pieces;
+            bool live = false;
+            for (int j = 0; j < a.k; ++j) {
+                const int row = __ldg(a.pair_row + tok * a.k + j);
+                live |= row >= 0 && row < a.cap;
+            }
+            const int q = int(u - tok * a.n_pieces);
+            if (live) bulk_prefetch_l2(a.x + tok * a.row_bytes + int64_t(q) * a.piece_bytes, piece_size(a, q),
+                                       pol_prefetch);
+        }
+        if (pf > want) pf = want;
+    };
 
     // Stage unit i: park its routing in shared memory and start the row load.
     auto issue = [&](int64_t i, UnitMeta m) {
@@ -136,7 +184,7 @@ __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
         __syncwarp();
         if (lane == 0) {
             const uint32_t bar = smem_u32(full + s);
-            if (any) {
+            if (any && !NOLOAD) {
                 const uint32_t bytes = piece_size(a, q);
                 mbar_arrive_expect_tx(bar, bytes);
                 const uint8_t* src = a.x + (u / a.n_pieces) * a.row_bytes + int64_t(q) * a.piece_bytes;
@@ -190,6 +238,7 @@ __global__ void __launch_bounds__(32) dispatch_kernel(DispatchArgs a) {
             }
         }
         bulk_commit();
+        if (a.read_period_ns != 0) pace_reads(i);
         // refill the stage of unit i-1 with unit i-1+S once its stores have read it
         const int64_t refill = i - 1 + S;
         if (i >= 1 && refill < my_n) {
@@ -302,7 +351,7 @@ int launch_dispatch_vec(const DispatchArgs& a, const ep_cfg_t& cfg, int sms, cud
 }
 
 // Stage count from the shared-memory budget, then the bulk-path launch.
-template <bool NORMAL>
+template <bool NORMAL, bool NOLOAD = false>
 int launch_bulk_dispatch(DispatchArgs& a, const ep_cfg_t& cfg, int64_t grid, int budget, cudaStream_t stream) {
     const size_t per_stage = size_t(a.stage_bytes) + 8 + 2 * 256;
     int stages = cfg.stages > 0 ? cfg.stages : int(budget / per_stage);
@@ -310,34 +359,18 @@ int launch_bulk_dispatch(DispatchArgs& a, const ep_cfg_t& cfg, int64_t grid, int
     a.stages = stages;
     const size_t smem = size_t(stages) * per_stage;
     if (smem > size_t(max_smem_optin())) return EP_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(dispatch_kernel<NORMAL>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(dispatch_kernel<NORMAL, NOLOAD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem)) != cudaSuccess)
         return EP_ERR_CUDA;
-    if (launch_pdl(dispatch_kernel<NORMAL>, dim3(unsigned(grid)), dim3(32), smem, stream, a) != cudaSuccess)
+    if (launch_pdl(dispatch_kernel<NORMAL, NOLOAD>, dim3(unsigned(grid)), dim3(32), smem, stream, a) != cudaSuccess)
         return EP_ERR_CUDA;
     return launch_result();
 }
 
-}  // namespace
-}  // namespace ep
-
-using namespace ep;
-
-extern "C" int ep_dispatch(ep_dims_t d, const uint16_t* x, const int32_t* topk_idx, const int32_t* pair_row,
-                           uint16_t* recv_x, int32_t* src_info, int32_t* status, ep_cfg_t cfg, void* stream) {
-    EP_NVTX_RANGE("ep_dispatch");
-    int rc = check_dims(d);
-    if (rc != EP_OK) return rc;
+// The low-latency arguments of a (validated) ep_dispatch call.
+int fill_dispatch_args(DispatchArgs& a, const ep_dims_t& d, const uint16_t* x, const int32_t* topk_idx,
+                       const int32_t* pair_row, uint16_t* recv_x, int32_t* src_info, int32_t* status) {
     const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
-    if (RT == 0 || d.hidden == 0) return EP_OK;
-    if (!x || !topk_idx || !pair_row || !recv_x || !src_info) return EP_ERR_INVALID;
-    if (!aligned16(x) || !aligned16(recv_x) || (reinterpret_cast<uintptr_t>(src_info) & 7u)) return EP_ERR_INVALID;
-
-    const int variant = cfg.variant != EP_VARIANT_AUTO ? cfg.variant : EP_VARIANT_BULK;
-    if (variant != EP_VARIANT_BULK && variant != EP_VARIANT_VECTOR) return EP_ERR_INVALID;
-    if (variant == EP_VARIANT_VECTOR && d.num_topk > kVecKMax) return EP_ERR_UNSUPPORTED;
-
-    DispatchArgs a;
     a.x = reinterpret_cast<const uint8_t*>(x);
     a.topk_idx = topk_idx;
     a.pair_row = pair_row;
@@ -362,9 +395,70 @@ extern "C" int ep_dispatch(ep_dims_t d, const uint16_t* x, const int32_t* topk_i
     if (int64_t(a.n_pieces - 1) * a.piece_bytes >= a.row_bytes) return EP_ERR_UNSUPPORTED;
     a.stage_bytes = uint32_t((a.piece_bytes + 127) & ~127u);
     a.n_units = RT * a.n_pieces;
+    a.read_period_ns = 0;
+    a.read_window_ns = 0;
+    a.read_ahead = 0;
+    return EP_OK;
+}
+
+// AUTO paces the reads when every CTA of a one-per-SM grid has enough units to span several
+// read periods (prefill-sized dispatches); short dispatches keep the two-CTA bulk path.
+bool paced_by_default(const DispatchArgs& a, int sms) {
+    return a.n_units >= int64_t(kPaceMinUnitsPerCta) * sms;
+}
+
+// Grid, stages and (for the paced path) the read schedule, then the bulk-path launch.  `prefetch`
+// (default: as paced) turns the paced read schedule on; the ceiling diagnostic may turn it off.
+template <bool NORMAL, bool NOLOAD = false>
+int run_bulk_dispatch(DispatchArgs& a, const ep_cfg_t& cfg, bool paced, int sms, cudaStream_t stream,
+                      int prefetch = -1) {
+    // default grid: 2 CTAs per SM, or 1 with paced reads (one deep ring per SM); cfg.max_ctas
+    // sets the grid (and so the CTAs sharing an SM)
+    int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas) : int64_t(sms) * (paced ? 1 : 2);
+    grid = std::max<int64_t>(1, std::min<int64_t>(grid, a.n_units));
+    const int ctas_per_sm = int(std::max<int64_t>(1, ceil_div(grid, sms)));
+    int budget = std::max(1, max_smem_optin() / ctas_per_sm - 1024);
+    if (paced && prefetch != 0) {
+        a.read_period_ns = kPacePeriodNs;
+        a.read_window_ns = kPaceWindowNs;
+        a.read_ahead = int(std::max<int64_t>(1, kPaceAheadBytes / std::max<int64_t>(1, a.stage_bytes)));
+    }
+    if (paced) {
+        // the ring of the measured schedule: 14 stages (fewer if the budget is smaller)
+        if (cfg.stages <= 0) budget = std::min(budget, 14 * int(a.stage_bytes + 8 + 2 * 256));
+    }
+    return launch_bulk_dispatch<NORMAL, NOLOAD>(a, cfg, grid, budget, stream);
+}
+
+}  // namespace
+}  // namespace ep
+
+using namespace ep;
+
+extern "C" int ep_dispatch(ep_dims_t d, const uint16_t* x, const int32_t* topk_idx, const int32_t* pair_row,
+                           uint16_t* recv_x, int32_t* src_info, int32_t* status, ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_dispatch");
+    int rc = check_dims(d);
+    if (rc != EP_OK) return rc;
+    const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
+    if (RT == 0 || d.hidden == 0) return EP_OK;
+    if (!x || !topk_idx || !pair_row || !recv_x || !src_info) return EP_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(recv_x) || (reinterpret_cast<uintptr_t>(src_info) & 7u)) return EP_ERR_INVALID;
+
+    const int requested = cfg.variant;
+    if (requested != EP_VARIANT_AUTO && requested != EP_VARIANT_BULK && requested != EP_VARIANT_VECTOR &&
+        requested != EP_VARIANT_PACED)
+        return EP_ERR_INVALID;
+    if (requested == EP_VARIANT_VECTOR && d.num_topk > kVecKMax) return EP_ERR_UNSUPPORTED;
+
+    DispatchArgs a;
+    rc = fill_dispatch_args(a, d, x, topk_idx, pair_row, recv_x, src_info, status);
+    if (rc != EP_OK) return rc;
 
     const int sms = sm_count();
     if (sms <= 0) return EP_ERR_CUDA;
+    const int variant = requested != EP_VARIANT_AUTO ? requested
+                        : (paced_by_default(a, sms) ? EP_VARIANT_PACED : EP_VARIANT_BULK);
     if (variant == EP_VARIANT_VECTOR) {
         cudaStream_t st = static_cast<cudaStream_t>(stream);
         switch (cfg.threads) {
@@ -373,12 +467,7 @@ extern "C" int ep_dispatch(ep_dims_t d, const uint16_t* x, const int32_t* topk_i
             default: return launch_dispatch_vec<4>(a, cfg, sms, st);
         }
     }
-    // default 2 CTAs per SM; cfg.max_ctas sets the grid (and so the CTAs sharing an SM)
-    int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas) : int64_t(sms) * 2;
-    grid = std::max<int64_t>(1, std::min<int64_t>(grid, a.n_units));
-    const int ctas_per_sm = int(std::max<int64_t>(1, ceil_div(grid, sms)));
-    const int budget = std::max(1, max_smem_optin() / ctas_per_sm - 1024);
-    return launch_bulk_dispatch<false>(a, cfg, grid, budget, static_cast<cudaStream_t>(stream));
+    return run_bulk_dispatch<false>(a, cfg, variant == EP_VARIANT_PACED, sms, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int ep_normal_dispatch(ep_dims_t d, int32_t recv_capacity, const uint16_t* x, const int32_t* topk_idx,
@@ -422,11 +511,33 @@ extern "C" int ep_normal_dispatch(ep_dims_t d, int32_t recv_capacity, const uint
     if (int64_t(a.n_pieces - 1) * a.piece_bytes >= a.row_bytes) return EP_ERR_UNSUPPORTED;
     a.stage_bytes = uint32_t((a.piece_bytes + 127) & ~127u);
     a.n_units = RT * a.n_pieces;
+    a.read_period_ns = 0;
+    a.read_window_ns = 0;
+    a.read_ahead = 0;
     const int sms = sm_count();
     if (sms <= 0) return EP_ERR_CUDA;
-    int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas) : int64_t(sms) * 2;
-    grid = std::max<int64_t>(1, std::min<int64_t>(grid, a.n_units));
-    const int ctas_per_sm = int(std::max<int64_t>(1, ceil_div(grid, sms)));
-    const int budget = std::max(1, max_smem_optin() / ctas_per_sm - 1024);
-    return launch_bulk_dispatch<true>(a, cfg, grid, budget, static_cast<cudaStream_t>(stream));
+    // normal mode has only the bulk data path: PACED (or AUTO on a long dispatch) paces its reads,
+    // any other variant runs it unpaced
+    const bool paced = cfg.variant == EP_VARIANT_PACED || (cfg.variant == EP_VARIANT_AUTO && paced_by_default(a, sms));
+    return run_bulk_dispatch<true>(a, cfg, paced, sms, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int ep_diag_dispatch_ceiling(ep_dims_t d, const uint16_t* x, const int32_t* topk_idx,
+                                        const int32_t* pair_row, uint16_t* recv_x, int32_t* src_info, int32_t mode,
+                                        int32_t* status, ep_cfg_t cfg, void* stream) {
+    EP_NVTX_RANGE("ep_diag_dispatch_ceiling");
+    int rc = check_dims(d);
+    if (rc != EP_OK) return rc;
+    if (mode != 0 && mode != 1) return EP_ERR_INVALID;
+    const int64_t RT = int64_t(d.num_ranks) * d.num_tokens;
+    if (RT == 0 || d.hidden == 0) return EP_OK;
+    if (!x || !topk_idx || !pair_row || !recv_x || !src_info) return EP_ERR_INVALID;
+    if (!aligned16(x) || !aligned16(recv_x) || (reinterpret_cast<uintptr_t>(src_info) & 7u)) return EP_ERR_INVALID;
+    DispatchArgs a;
+    rc = fill_dispatch_args(a, d, x, topk_idx, pair_row, recv_x, src_info, status);
+    if (rc != EP_OK) return rc;
+    const int sms = sm_count();
+    if (sms <= 0) return EP_ERR_CUDA;
+    // the paced path's grid and ring, its L2 prefetch schedule in mode 1
+    return run_bulk_dispatch<false, true>(a, cfg, true, sms, static_cast<cudaStream_t>(stream), mode);
 }

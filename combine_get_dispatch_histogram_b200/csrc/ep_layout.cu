@@ -297,11 +297,12 @@ __device__ __forceinline__ void load_first_round(const LayoutArgs& a, const Warp
 // count in the warp's histogram `mine` plus the matching lanes below it (ballot
 // match); it stays in rk (the last round's pairs) or, for a part longer than one
 // round, is parked in pair_row.  Each token's destination ranks go to
-// is_token_in_rank and its counts to tpr[r][*]: with k a power of two a token's
+// is_token_in_rank and its counts to tpr_row[*] (the part's source rank's row of
+// per-destination token counts): with k a power of two a token's
 // k slots sit in k aligned lanes and an OR over them gives the set, otherwise one
 // token per lane re-reads its slots.  True if this lane saw an id outside [-1, E).
 __device__ __forceinline__ bool walk_part(const LayoutArgs& a, const WarpPart& w, const int32_t* act,
-                                          const int32_t* rank_of, int32_t* mine, int32_t* tpr,
+                                          const int32_t* rank_of, int32_t* mine, int32_t* tpr_row,
                                           int (&ev)[kBatch], int (&rk)[kBatch]) {
     const int lane = threadIdx.x & 31;
     const bool src_ok = w.has_rank && act[a.r0 + w.r] != 0;
@@ -343,7 +344,7 @@ __device__ __forceinline__ bool walk_part(const LayoutArgs& a, const WarpPart& w
                 }
                 for (int d = 0; d < a.R; ++d) {
                     const int n = __popc(__ballot_sync(0xffffffffu, head && ((dst >> d) & 1u)));
-                    if (lane == 0 && n) atomicAdd(tpr + w.r * a.R + d, n);
+                    if (lane == 0 && n) atomicAdd(tpr_row + d, n);
                 }
             }
         }
@@ -363,7 +364,7 @@ __device__ __forceinline__ bool walk_part(const LayoutArgs& a, const WarpPart& w
             }
             for (int d = 0; d < a.R; ++d) {
                 const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
-                if (lane == 0 && n) atomicAdd(tpr + w.r * a.R + d, n);
+                if (lane == 0 && n) atomicAdd(tpr_row + d, n);
             }
         }
     }
@@ -416,7 +417,7 @@ __global__ void __launch_bounds__(kSmallThreads) layout_single_cta_kernel(Layout
     __syncthreads();
 
     int32_t* mine = whist + warp * a.E;
-    const bool bad = walk_part(a, w, act, rank_of, mine, tpr, ev, rk);
+    const bool bad = walk_part(a, w, act, rank_of, mine, tpr + (w.has_rank ? w.r * a.R : 0), ev, rk);
     if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
 
     // scan the warp histograms per expert in warp order = (rank, part) order
@@ -478,7 +479,7 @@ __global__ void __launch_bounds__(kSmallThreads) layout_cluster_kernel(LayoutArg
     __syncthreads();
 
     int32_t* mine = whist + warp * a.E;
-    const bool bad = walk_part(a, w, act, rank_of, mine, tpr, ev, rk);
+    const bool bad = walk_part(a, w, act, rank_of, mine, tpr + (w.has_rank ? w.r * a.R : 0), ev, rk);
     if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
 
     // this CTA's warps, scanned per expert in warp order; ctot = the CTA's total
@@ -892,56 +893,27 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_lookback_kernel(LayoutA
 
     const int g = blockIdx.x;
     const ChunkGeom cg = chunk_of(a, g);
-    const bool src_ok = act[a.r0 + cg.r] != 0;
+    // this warp's part of the chunk: the walk of the one-launch paths, rows within the part kept
+    WarpPart w;
+    w.r = cg.r;
+    w.has_rank = true;
     const int tw = (cg.t1 - cg.t0 + W - 1) / W;
-    const int wt0 = min(cg.t1, cg.t0 + warp * tw), wt1 = min(cg.t1, wt0 + tw);
-    const int64_t pbase = (int64_t(cg.r) * a.T + wt0) * a.k;
-    const int32_t* base = a.topk_idx + pbase;
-    int32_t* rows = a.pair_row + pbase;
-    const int np = (wt1 - wt0) * a.k;
+    w.t0 = min(cg.t1, cg.t0 + warp * tw);
+    w.t1 = min(cg.t1, w.t0 + tw);
+    w.pbase = (int64_t(cg.r) * a.T + w.t0) * a.k;
+    w.np = (w.t1 - w.t0) * a.k;
+    w.one_round = w.np <= 32 * kBatch;
     int32_t* mine = whist + warp * a.E;
+    int ev[kBatch], rk[kBatch];
+    load_first_round(a, w, ev);
 
-    // ---- A: warp histograms, destination ranks, chunk histogram, publish
-    bool bad = false;
-    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
-        int ev[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int p = p0 + u * 32 + lane;
-            ev[u] = p < np ? __ldg(base + p) : -1;
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int e = ev[u];
-            bad |= (e < -1 || e >= a.E);
-            const bool live = pair_live(e, a.E, src_ok, rank_of);
-            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
-            if (live && lane == __ffs(m) - 1) mine[e] += __popc(m);
-            __syncwarp();
-        }
-    }
-    for (int t0 = wt0; t0 < wt1; t0 += 32) {
-        const int t = t0 + lane;
-        uint64_t ranks = 0;
-        if (t < wt1) {
-            const int32_t* tb = a.topk_idx + (int64_t(cg.r) * a.T + t) * a.k;
-            for (int j = 0; j < a.k; ++j) {
-                const int e = __ldg(tb + j);
-                if (pair_live(e, a.E, src_ok, rank_of)) ranks |= 1ull << rank_of[e];
-            }
-            uint8_t* itr = a.is_token_in_rank + (int64_t(cg.r) * a.T + t) * a.R;
-            for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((ranks >> d) & 1u);
-        }
-        for (int d = 0; d < a.R; ++d) {
-            const int n = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
-            if (lane == 0 && n) atomicAdd(tpr + d, n);
-        }
-    }
+    // ---- A: warp histograms and rows within the parts, destination ranks, chunk histogram, publish
+    const bool bad = walk_part(a, w, act, rank_of, mine, tpr, ev, rk);
     if (__syncthreads_or(bad) && threadIdx.x == 0) flag_status(a.status, EP_STATUS_BAD_EXPERT);
     int32_t* own = a.chunk_hist + int64_t(g) * a.E;
     for (int e = threadIdx.x; e < a.E; e += NT) {
         int32_t s = 0;
-        for (int w = 0; w < W; ++w) s += whist[w * a.E + e];
+        for (int ww = 0; ww < W; ++ww) s += whist[ww * a.E + e];
         own[e] = s;
     }
     for (int d = threadIdx.x; d < a.R; d += NT) a.chunk_tpr[int64_t(g) * a.R + d] = tpr[d];
@@ -1042,38 +1014,17 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_lookback_kernel(LayoutA
         }
     }
 
-    // ---- C: per-warp first rows, then rows
+    // ---- C: per-warp first rows, then each live pair's row = its warp's first row + its row in the part
     for (int e = threadIdx.x; e < a.E; e += NT) {
         int32_t run = first[e];
-        for (int w = 0; w < W; ++w) {
-            const int32_t v = whist[w * a.E + e];
-            whist[w * a.E + e] = run;
+        for (int ww = 0; ww < W; ++ww) {
+            const int32_t v = whist[ww * a.E + e];
+            whist[ww * a.E + e] = run;
             run += v;
         }
     }
     __syncthreads();
-    const uint32_t below = lanemask_lt();
-    for (int p0 = 0; p0 < np; p0 += 32 * kBatch) {
-        int ev[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int p = p0 + u * 32 + lane;
-            ev[u] = p < np ? __ldg(base + p) : -1;
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int p = p0 + u * 32 + lane;
-            if (p0 + u * 32 >= np) break;
-            const int e = ev[u];
-            const bool live = pair_live(e, a.E, src_ok, rank_of);
-            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
-            const int32_t b = live ? mine[e] : 0;
-            __syncwarp();
-            if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
-            __syncwarp();
-            if (p < np) rows[p] = live ? b + __popc(m & below) : -1;
-        }
-    }
+    finish_rows(a, w, ev, rk, [&](int e) { return mine[e]; });
 }
 
 struct LayoutGeom {
@@ -1149,8 +1100,9 @@ size_t lookback_smem_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
 // AUTO, from graph replays on B200: one CTA up to kSmallAutoPairs pairs (8.6 us at 1024
 // pairs, 10.6 us at 2048); a cluster up to kClusterAutoPairs (10.6 us from 4096 to 16384
 // pairs, 12.7 us at 32768, 14.7 at 49152, 16.8 at 65536, where one CTA takes 14.7 to 74 us);
-// the chunked path beyond (about 17 to 19 us), which also beats the fused one (cooperative
-// launch plus two grid barriers, about 19 us).
+// the look-back path beyond, one launch (prefill, 262144 pairs: 21.5 us per stream launch
+// against 25.9 for the three chunked launches and 20.3 for the fused cooperative launch,
+// which is slower in a graph); the chunked path only if the chunk grid outgrows the flags.
 int resolve_layout_path(const ep_dims_t& d, int Rs, const ep_cfg_t& cfg, const LayoutGeom& lg) {
     const int64_t pairs = int64_t(Rs) * d.num_tokens * d.num_topk;
     const bool tables_fit = d.num_ranks <= kSmallMaxRanks && d.num_experts <= kSmallMaxExperts;
@@ -1160,6 +1112,7 @@ int resolve_layout_path(const ep_dims_t& d, int Rs, const ep_cfg_t& cfg, const L
         case EP_VARIANT_AUTO:
             if (small_ok && pairs <= kSmallAutoPairs) return EP_LAYOUT_SINGLE_CTA;
             if (cluster_ok && pairs <= kClusterAutoPairs) return EP_LAYOUT_CLUSTER;
+            if (lg.G <= kMaxFlags && lookback_smem_bytes(d, lg) <= size_t(max_smem_optin())) return EP_LAYOUT_LOOKBACK;
             return EP_LAYOUT_CHUNKED;
         case EP_LAYOUT_CHUNKED:
             return EP_LAYOUT_CHUNKED;

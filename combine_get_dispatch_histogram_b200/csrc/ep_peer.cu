@@ -209,21 +209,29 @@ __global__ void __launch_bounds__(kPeerThreads) dispatch_peer_kernel(PeerArgs a)
 // ---------------------------------------------------------------------------- waits and signals
 
 // Thread s waits until this rank's flag word s holds at least `signal`, for every
-// active source s, giving up after kWaitTimeoutNs (EP_STATUS_TIMEOUT).
+// active source s, giving up after kWaitTimeoutNs (EP_STATUS_TIMEOUT).  With
+// wait_ns, the nanoseconds it waited for source s (until the flag or the give-up)
+// are added to wait_ns[s].
 __global__ void __launch_bounds__(EP_MAX_RANKS) wait_peers_kernel(const uint64_t* flags, int R, uint64_t signal,
-                                                                  const uint8_t* active, int32_t* status) {
+                                                                  const uint8_t* active, int32_t* status,
+                                                                  int64_t* wait_ns) {
     pdl_wait();
     const int s = threadIdx.x;
     if (s >= R || active[s] == 0) return;
     const uint64_t t0 = global_timer_ns();
+    uint64_t t = t0;
     for (uint32_t it = 0;; ++it) {
-        if (ld_acquire_sys_u64(flags + s) >= signal) return;
-        if ((it & 63u) == 63u && global_timer_ns() - t0 > kWaitTimeoutNs) {
-            flag_status(status, EP_STATUS_TIMEOUT);
-            return;
+        if (ld_acquire_sys_u64(flags + s) >= signal) break;
+        if ((it & 63u) == 63u) {
+            t = global_timer_ns();
+            if (t - t0 > kWaitTimeoutNs) {
+                flag_status(status, EP_STATUS_TIMEOUT);
+                break;
+            }
         }
         __nanosleep(64);
     }
+    if (wait_ns) wait_ns[s] += int64_t(global_timer_ns() - t0);
 }
 
 // Thread d releases `signal` into word `rank` of every active rank d's flags.
@@ -453,12 +461,13 @@ extern "C" int ep_dispatch_peer(ep_dims_t d, int32_t rank, ep_peer_table_t peers
 }
 
 extern "C" int ep_wait_peers(int32_t num_ranks, const uint64_t* flags, uint64_t signal, const uint8_t* active,
-                             int32_t* status, void* stream) {
+                             int64_t* wait_ns, int32_t* status, void* stream) {
     EP_NVTX_RANGE("ep_wait_peers");
-    if (num_ranks <= 0 || num_ranks > EP_MAX_RANKS || !flags || !active || !status || !aligned8(flags))
+    if (num_ranks <= 0 || num_ranks > EP_MAX_RANKS || !flags || !active || !status || !aligned8(flags) ||
+        (wait_ns && !aligned8(wait_ns)))
         return EP_ERR_INVALID;
     if (launch_pdl(wait_peers_kernel, dim3(1), dim3(EP_MAX_RANKS), 0, static_cast<cudaStream_t>(stream), flags,
-                   int(num_ranks), signal, active, status) != cudaSuccess)
+                   int(num_ranks), signal, active, status, wait_ns) != cudaSuccess)
         return EP_ERR_CUDA;
     return launch_result();
 }

@@ -38,6 +38,7 @@ EP_FP8_SCALE_POW2 = 1
 EP_FP8_SCALE_UE8M0 = 2
 EP_VARIANT_BULK = 1
 EP_VARIANT_VECTOR = 2
+EP_VARIANT_PACED = 3
 EP_LAYOUT_CHUNKED = 1
 EP_LAYOUT_SINGLE_CTA = 2
 EP_LAYOUT_FUSED = 3
@@ -95,6 +96,8 @@ def load_library(path: str = LIB_PATH):
     lib.ep_layout.restype = ctypes.c_int
     lib.ep_dispatch.argtypes = [Dims, P, P, P, P, P, P, Cfg, P]
     lib.ep_dispatch.restype = ctypes.c_int
+    lib.ep_diag_dispatch_ceiling.argtypes = [Dims, P, P, P, P, P, I32, P, Cfg, P]
+    lib.ep_diag_dispatch_ceiling.restype = ctypes.c_int
     lib.ep_combine.argtypes = [Dims, P, P, P, P, P, P, P, Cfg, P]
     lib.ep_combine.restype = ctypes.c_int
     lib.ep_dispatch_fp8.argtypes = [Dims, P, P, P, P, I32, P, SZ, P, P, P, P, Cfg, P]
@@ -128,7 +131,7 @@ def load_library(path: str = LIB_PATH):
     lib.ep_dispatch_peer_workspace_bytes.restype = SZ
     lib.ep_dispatch_peer.argtypes = [Dims, I32, PeerTable, P, P, P, P, P, U64, P, SZ, P, Cfg, P]
     lib.ep_dispatch_peer.restype = ctypes.c_int
-    lib.ep_wait_peers.argtypes = [I32, P, U64, P, P, P]
+    lib.ep_wait_peers.argtypes = [I32, P, U64, P, P, P, P]
     lib.ep_wait_peers.restype = ctypes.c_int
     lib.ep_signal_peers.argtypes = [I32, I32, P, P, U64, P]
     lib.ep_signal_peers.restype = ctypes.c_int
@@ -140,6 +143,8 @@ def load_library(path: str = LIB_PATH):
     lib.ep_ipc_export.restype = ctypes.c_int
     lib.ep_ipc_import.argtypes = [P, U64, ctypes.POINTER(P), ctypes.POINTER(P)]
     lib.ep_ipc_import.restype = ctypes.c_int
+    lib.ep_recv_stats_accumulate.argtypes = [I32, P, P, P]
+    lib.ep_recv_stats_accumulate.restype = ctypes.c_int
     lib.ep_ipc_close.argtypes = [P]
     lib.ep_ipc_close.restype = ctypes.c_int
     _lib = lib
@@ -347,6 +352,38 @@ def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, pair_row: torch.Tensor,
         rc = lib.ep_dispatch(Dims(R, T, k, E, H), _ptr(x), _ptr(topk_idx), _ptr(pair_row), _ptr(recv_x),
                              _ptr(src_info), _ptr(status), _cfg(cfg), _stream(dev, stream))
     _check("ep_dispatch", rc)
+    return recv_x, src_info, status
+
+
+def ep_diag_dispatch_ceiling(x: torch.Tensor, topk_idx: torch.Tensor, pair_row: torch.Tensor, num_experts: int,
+                             mode: int, *, recv_x: Optional[torch.Tensor] = None,
+                             src_info: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                             cfg=None, stream=None):
+    """The paced dispatch without its row loads (``ep_diag_dispatch_ceiling``): a ceiling instrument.
+
+    ``mode`` 0: the row stores alone; 1: the stores plus the paced L2 prefetches of the rows.
+    The slab rows written hold zeros.  Returns ``(recv_x, src_info, status)``.
+    """
+    lib = load_library()
+    _need(x, "x", torch.bfloat16)
+    R, T, H = x.shape
+    dev = x.device
+    topk_idx = _need(_idx32(topk_idx, "topk_idx", stream), "topk_idx", torch.int32, device=dev)
+    k = topk_idx.shape[2]
+    _need(pair_row, "pair_row", torch.int32, (R, T, k), dev)
+    E = int(num_experts)
+    cap = R * T
+    if recv_x is None:
+        recv_x = torch.empty((E, cap, H), dtype=torch.bfloat16, device=dev)
+    if src_info is None:
+        src_info = torch.empty((E, cap, 2), dtype=torch.int32, device=dev)
+    _need(recv_x, "recv_x", torch.bfloat16, (E, cap, H), dev)
+    _need(src_info, "src_info", torch.int32, (E, cap, 2), dev)
+    status = _status(dev, status)
+    with torch.cuda.device(dev):
+        rc = lib.ep_diag_dispatch_ceiling(Dims(R, T, k, E, H), _ptr(x), _ptr(topk_idx), _ptr(pair_row), _ptr(recv_x),
+                                          _ptr(src_info), int(mode), _ptr(status), _cfg(cfg), _stream(dev, stream))
+    _check("ep_diag_dispatch_ceiling", rc)
     return recv_x, src_info, status
 
 
@@ -778,17 +815,23 @@ def ep_dispatch_peer(x: torch.Tensor, topk_idx: torch.Tensor, local_row: torch.T
     return status
 
 
-def ep_wait_peers(flags: torch.Tensor, signal: int, active: torch.Tensor, *, status: Optional[torch.Tensor] = None,
-                  stream=None) -> torch.Tensor:
-    """Bounded wait until ``flags[s] >= signal`` for every active rank s (``ep_wait_peers``). Returns ``status``."""
+def ep_wait_peers(flags: torch.Tensor, signal: int, active: torch.Tensor, *, wait_ns: Optional[torch.Tensor] = None,
+                  status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Bounded wait until ``flags[s] >= signal`` for every active rank s (``ep_wait_peers``). Returns ``status``.
+
+    ``wait_ns`` (int64 [R]) accumulates the nanoseconds waited for each source.
+    """
     lib = load_library()
     dev = flags.device
     R = flags.shape[0]
     _need(flags, "flags", torch.int64, (R,), dev)
     _need(active, "active", torch.uint8, (R,), dev)
+    if wait_ns is not None:
+        _need(wait_ns, "wait_ns", torch.int64, (R,), dev)
     status = _status(dev, status)
     with torch.cuda.device(dev):
-        rc = lib.ep_wait_peers(R, _ptr(flags), int(signal), _ptr(active), _ptr(status), _stream(dev, stream))
+        rc = lib.ep_wait_peers(R, _ptr(flags), int(signal), _ptr(active), _ptr(wait_ns), _ptr(status),
+                               _stream(dev, stream))
     _check("ep_wait_peers", rc)
     return status
 
@@ -850,6 +893,19 @@ def ep_combine_peer(slab_table: torch.Tensor, topk_idx: torch.Tensor, topk_weigh
                                  _ptr(status), _cfg(cfg), _stream(dev, stream))
     _check("ep_combine_peer", rc)
     return out, status
+
+
+def ep_recv_stats_accumulate(recv_count: torch.Tensor, stats: torch.Tensor, *, stream=None) -> torch.Tensor:
+    """``stats += recv_count`` on the device (``ep_recv_stats_accumulate``): cumulative receive counts."""
+    lib = load_library()
+    dev = recv_count.device
+    n = recv_count.numel()
+    _need(recv_count, "recv_count", torch.int32, (n,), dev)
+    _need(stats, "stats", torch.int32, (n,), dev)
+    with torch.cuda.device(dev):
+        rc = lib.ep_recv_stats_accumulate(n, _ptr(recv_count), _ptr(stats), _stream(dev, stream))
+    _check("ep_recv_stats_accumulate", rc)
+    return stats
 
 
 def ep_ipc_export(t: torch.Tensor):

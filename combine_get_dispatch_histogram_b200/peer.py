@@ -108,8 +108,10 @@ class PeerRank:
                                    self.src_info_table, self.arrival_table, signal, self.bufs.dispatch_ws,
                                    status=status, stream=stream)
 
-    def wait_arrivals(self, signal: int, active: torch.Tensor, *, status=None, stream=None) -> torch.Tensor:
-        return ep.ep_wait_peers(self.bufs.arrival, signal, active, status=status, stream=stream)
+    def wait_arrivals(self, signal: int, active: torch.Tensor, *, wait_ns=None, status=None,
+                      stream=None) -> torch.Tensor:
+        """Bounded wait for every active source's rows; ``wait_ns`` (int64 [R]) accumulates the time per source."""
+        return ep.ep_wait_peers(self.bufs.arrival, signal, active, wait_ns=wait_ns, status=status, stream=stream)
 
     def recv_count(self, counts: torch.Tensor, *, stream=None) -> torch.Tensor:
         return ep.ep_peer_recv_count(counts, self.rank, stream=stream)

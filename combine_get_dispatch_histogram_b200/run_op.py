@@ -20,7 +20,7 @@ from . import ep, inputs
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("--op", choices=["layout", "dispatch", "dispatch_fp8", "combine", "reroute", "step",
+    ap.add_argument("--op", choices=["layout", "dispatch", "dispatch_ceiling", "dispatch_fp8", "combine", "reroute", "step",
                                      "normal_layout", "normal_dispatch", "normal_combine", "weight_sync",
                                      "grad_reduce"], required=True)
     ap.add_argument("--params", type=int, default=1 << 22, help="weight_sync / grad_reduce: float32 params per expert")
@@ -31,12 +31,13 @@ def main():
     ap.add_argument("--graph", action="store_true", help="time CUDA-graph replays of the calls")
     ap.add_argument("--variant", type=int, default=0, help="ep_cfg_t.variant of dispatch / combine")
     ap.add_argument("--layout-variant", type=int, default=0, help="ep_cfg_t.variant of layout")
+    ap.add_argument("--mode", type=int, default=0, help="dispatch_ceiling: 0 stores only, 1 stores + row prefetch")
     args = ap.parse_args()
 
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
     w = inputs.named(args.workload)
-    need_x = args.op in ("dispatch", "dispatch_fp8", "step") or args.op.startswith("normal_")
+    need_x = args.op in ("dispatch", "dispatch_ceiling", "dispatch_fp8", "step") or args.op.startswith("normal_")
     inp = inputs.make_inputs(w, tokens=need_x or args.op == "combine")
     R, T, k, H, E = w.num_ranks, w.num_tokens, w.num_topk, w.hidden, w.num_physical
     cap = R * T
@@ -102,7 +103,7 @@ def main():
         calls.append(lambda: ep.ep_dispatch_fp8(x, idx_phys, lay.pair_row, lay.recv_count, E, args.scale_format,
                                                 workspace=fp8_ws, recv_x=codes, recv_scales=scales,
                                                 src_info=src_info, status=status, stream=stream, cfg=cfg))
-    if args.op in ("dispatch", "combine", "step"):
+    if args.op in ("dispatch", "dispatch_ceiling", "combine", "step"):
         recv_x = torch.empty((E, cap, H), dtype=torch.bfloat16, device=dev)
         src_info = torch.empty((E, cap, 2), dtype=torch.int32, device=dev)
         x = (torch.from_numpy(inp.x.view(np.int16)).to(dev).view(torch.bfloat16) if inp.x is not None else
@@ -113,6 +114,9 @@ def main():
         if args.op in ("dispatch", "step"):
             calls.append(lambda: ep.ep_dispatch(x, idx_phys, lay.pair_row, E, recv_x=recv_x, src_info=src_info,
                                                 status=status, stream=stream, cfg=cfg))
+        if args.op == "dispatch_ceiling":
+            calls.append(lambda: ep.ep_diag_dispatch_ceiling(x, idx_phys, lay.pair_row, E, args.mode, recv_x=recv_x,
+                                                             src_info=src_info, status=status, stream=stream, cfg=cfg))
         if args.op in ("combine", "step"):
             calls.append(lambda: ep.ep_combine(recv_x, idx_phys, wts, lay.pair_row, act, out=out, status=status,
                                                stream=stream, cfg=cfg))
@@ -156,6 +160,8 @@ def main():
         algo = 2 * H * (sent + sends) if args.op == "normal_dispatch" else 2 * H * (sends + R * T)
     elif args.op in ("dispatch", "dispatch_fp8"):
         algo = 2 * H * sent + per_pair[args.op] * live
+    elif args.op == "dispatch_ceiling":
+        algo = 2 * H * (live + (sent if args.mode == 1 else 0))
     elif args.op == "combine":
         algo = 2 * H * (live + R * T)
     print(json.dumps({"op": args.op, "workload": w.name, "us_per_call": round(us, 2), "graph": args.graph,

@@ -42,7 +42,8 @@
  *                  each own one GPU, over NVLink peer memory (section at the end).
  *   ep_topk_idx_to_int32 -- the int64 topk_idx of the NeMo page's Buffer calls
  *                  in the int32 form of the nixl PR, saturating out-of-range ids.
- *   ep_layout_noalloc, ep_layout_path and the *_workspace_bytes queries have
+ *   ep_layout_noalloc, ep_layout_path, the ep_diag_* instruments and the
+ *                  *_workspace_bytes queries have
  *                  no counterpart on the pages; they serve callers of this
  *                  library (scratch without allocation, which path a call takes,
  *                  scratch sizes).
@@ -155,7 +156,12 @@ enum {
 enum {
     EP_VARIANT_AUTO = 0,      /* the faster path for the shape, as measured on B200 */
     EP_VARIANT_BULK = 1,      /* rows staged in shared memory by bulk async copies */
-    EP_VARIANT_VECTOR = 2     /* rows moved through registers as 16-byte vectors */
+    EP_VARIANT_VECTOR = 2,    /* rows moved through registers as 16-byte vectors */
+    EP_VARIANT_PACED = 3      /* ep_dispatch / ep_normal_dispatch: the bulk path with paced reads --
+                                 one CTA per SM, and the rows about to be staged are prefetched into
+                                 L2 only inside a short window that recurs on the GPU-wide clock,
+                                 so HBM serves reads in bursts and the row stores alone in between
+                                 (the same bits; AUTO takes it for long dispatches) */
 };
 
 /* Human-readable name of an EP_OK / EP_ERR_* code (static storage). */
@@ -189,6 +195,22 @@ EP_API int ep_layout_path(ep_dims_t d, ep_cfg_t cfg);
  * out: status  int32 device word
  */
 EP_API int ep_diag_wait_timeout(void *flags, int32_t *status, void *stream);
+
+/*
+ * ep_diag_dispatch_ceiling -- a measurement instrument (the pages have no
+ * counterpart): the paced dispatch kernel (EP_VARIANT_PACED's grid and ring)
+ * with its row loads left out, to time what HBM gives the dispatch's traffic
+ * when no store waits for a read.
+ *   mode 0: only the row stores and src_info of every live pair, from a zeroed
+ *           ring -- the ceiling of the scatter's writes alone;
+ *   mode 1: those stores plus the paced L2 prefetches of the token rows -- the
+ *           dispatch's own HBM traffic with no store waiting on it.
+ * Arguments and checks as ep_dispatch; the slab rows it writes hold zeros, not
+ * tokens, and src_info holds the true (src_rank, src_token).
+ */
+EP_API int ep_diag_dispatch_ceiling(ep_dims_t d, const uint16_t *x, const int32_t *topk_idx,
+                                    const int32_t *pair_row, uint16_t *recv_x, int32_t *src_info, int32_t mode,
+                                    int32_t *status, ep_cfg_t cfg, void *stream);
 
 
 /*
@@ -394,7 +416,9 @@ EP_API int ep_normal_layout(ep_dims_t d, int32_t recv_capacity, int32_t expert_a
                             int32_t *status, ep_cfg_t cfg, void *stream);
 
 /*
- * ep_normal_dispatch -- send each token row once per destination rank.
+ * ep_normal_dispatch -- send each token row once per destination rank (the bulk data path;
+ * cfg.variant EP_VARIANT_PACED paces its reads, AUTO does so for long dispatches, any other
+ * value runs it unpaced).
  * in:  x bf16 [R,T,H], topk_idx int32 [R,T,k], topk_weights float [R,T,k], active uint8 [R]
  *      (the mask ep_layout used), token_recv_row from ep_normal_layout
  * out (rows [0, min(recv_tokens[d], recv_capacity)) of every rank d; others untouched):
@@ -587,9 +611,12 @@ EP_API int ep_dispatch_peer(ep_dims_t d, int32_t rank, ep_peer_table_t peers, co
  * after the library's wait limit (2 s): EP_STATUS_TIMEOUT is OR-ed into *status
  * and the kernel returns, so the context stays usable; kernels after it in the
  * stream then see the peers' writes only if no timeout was reported.
+ * wait_ns int64 [R] (device, may be NULL): the nanoseconds spent waiting for each
+ * source are ADDED to wait_ns[s] -- the page's dispatch_wait_recv_cost_stats (a
+ * cumulative per-source wait time that localises a slow rank); masked sources add 0.
  */
 EP_API int ep_wait_peers(int32_t num_ranks, const uint64_t *flags, uint64_t signal, const uint8_t *active,
-                         int32_t *status, void *stream);
+                         int64_t *wait_ns, int32_t *status, void *stream);
 
 /*
  * ep_signal_peers -- after the kernels before it in the stream, release `signal`
@@ -615,6 +642,14 @@ EP_API int ep_peer_recv_count(int32_t num_ranks, int32_t num_experts, int32_t ra
 EP_API int ep_combine_peer(ep_dims_t d, int32_t rank, const uint64_t *y_slabs, const int32_t *topk_idx,
                            const float *topk_weights, const int32_t *local_row, const int32_t *counts,
                            const uint8_t *active, uint16_t *out, int32_t *status, ep_cfg_t cfg, void *stream);
+
+/*
+ * ep_recv_stats_accumulate -- stats[i] += recv_count[i] for i < num (int32, device):
+ * the page's cumulative_local_expert_recv_stats of Buffer.low_latency_dispatch, a
+ * running per-expert receive count for EP load-balance monitoring.  Pass ep_layout's
+ * recv_count (num = E) or ep_peer_recv_count's (num = E / R).
+ */
+EP_API int ep_recv_stats_accumulate(int32_t num, const int32_t *recv_count, int32_t *stats, void *stream);
 
 /* CUDA IPC handles for the peer table: a handle is EP_IPC_HANDLE_BYTES of host memory. */
 enum { EP_IPC_HANDLE_BYTES = 64 };

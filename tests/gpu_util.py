@@ -95,15 +95,19 @@ def check_close(got_bf16: np.ndarray, want_f64: np.ndarray, tag: str = ""):
         raise AssertionError(f"{tag} combine out of tolerance at {i}: gpu {g[i]} oracle {want_f64[i]}")
 
 
-def run_path(inp, E, H, *, active_combine=None, cfg=None, y=None, layout_cfg=None):
-    """layout -> dispatch -> combine on the GPU. Returns host/device results."""
+def run_path(inp, E, H, *, active_combine=None, cfg=None, y=None, layout_cfg=None, dispatch_cfg=None):
+    """layout -> dispatch -> combine on the GPU. Returns host/device results.
+
+    ``cfg`` goes to dispatch and combine, ``dispatch_cfg`` (if given) to dispatch alone.
+    """
     idx = i32_dev(inp.topk_idx)
     act = u8_dev(inp.active)
     x = bf16_dev(inp.x)
     w = f32_dev(inp.topk_weights)
     status = torch.zeros(1, dtype=torch.int32, device=dev())
     lay = ep.ep_layout(idx, act, E, hidden=H, status=status, cfg=layout_cfg)
-    recv_x, src_info, _ = ep.ep_dispatch(x, idx, lay.pair_row, E, status=status, cfg=cfg)
+    recv_x, src_info, _ = ep.ep_dispatch(x, idx, lay.pair_row, E, status=status,
+                                         cfg=cfg if dispatch_cfg is None else dispatch_cfg)
     act_c = act if active_combine is None else u8_dev(active_combine)
     out, _ = ep.ep_combine(recv_x if y is None else y, idx, w, lay.pair_row, act_c, status=status, cfg=cfg)
     torch.cuda.synchronize()

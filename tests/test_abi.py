@@ -94,7 +94,8 @@ def test_host_validation_rejects_without_launching(lib):
 
 def test_layout_path_choice(lib):
     """AUTO takes one CTA up to 2048 pairs and a cluster up to 65536 (R <= 32, E <= 1024), the
-    chunked path beyond; explicit paths are honoured or refused exactly as ep_layout would."""
+    one-launch look-back path beyond; explicit paths are honoured or refused exactly as ep_layout
+    would."""
     from combine_get_dispatch_histogram_b200 import ep
 
     assert ep.ep_layout_path(2, 64, 2, 8) == ep.EP_LAYOUT_SINGLE_CTA          # 256 pairs
@@ -102,9 +103,16 @@ def test_layout_path_choice(lib):
     assert ep.ep_layout_path(8, 64, 8, 256) == ep.EP_LAYOUT_CLUSTER           # 4096 pairs
     assert ep.ep_layout_path(8, 512, 8, 256) == ep.EP_LAYOUT_CLUSTER          # 32768 pairs
     assert ep.ep_layout_path(8, 1024, 8, 256) == ep.EP_LAYOUT_CLUSTER         # 65536 pairs
-    assert ep.ep_layout_path(8, 1025, 8, 256) == ep.EP_LAYOUT_CHUNKED         # 65600 pairs
-    assert ep.ep_layout_path(8, 16, 8, 2048) == ep.EP_LAYOUT_CHUNKED          # E > 1024
-    assert ep.ep_layout_path(40, 8, 8, 80) == ep.EP_LAYOUT_CHUNKED            # R > 32
+    assert ep.ep_layout_path(8, 1025, 8, 256) == ep.EP_LAYOUT_LOOKBACK        # 65600 pairs
+    assert ep.ep_layout_path(8, 4096, 8, 256) == ep.EP_LAYOUT_LOOKBACK        # prefill, 262144 pairs
+    assert ep.ep_layout_path(40, 8, 8, 80) == ep.EP_LAYOUT_LOOKBACK           # R > 32
+    # E > 1024: the look-back CTA's shared memory grows with E; where the device cannot give it
+    # (here, with no device, the 48 KB every CUDA device offers) the chunked path takes the shape
+    wide = (ep.EP_LAYOUT_LOOKBACK, ep.EP_LAYOUT_CHUNKED)
+    assert ep.ep_layout_path(8, 16, 8, 2048) in wide
+    assert ep.ep_layout_path(64, 2048, 8, 8192) in wide
+    lookback = dict(variant=ep.EP_LAYOUT_LOOKBACK)
+    assert ep.ep_layout_path(8, 16, 8, 256, cfg=lookback) == ep.EP_LAYOUT_LOOKBACK
     cluster = dict(variant=ep.EP_LAYOUT_CLUSTER)
     assert ep.ep_layout_path(8, 1024, 8, 256, cfg=cluster) == ep.EP_LAYOUT_CLUSTER
     with pytest.raises(ep.EPError) as ei:

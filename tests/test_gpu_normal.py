@@ -26,8 +26,9 @@ def run_normal(inp, E, alignment=1, capacity=None, active_combine=None, cfg=None
     nd = ep.ep_normal_dispatch(bf16_dev(inp.x), idx, f32_dev(inp.topk_weights), act, nl, E, status=lay.status,
                                cfg=cfg)
     act_c = act if active_combine is None else u8_dev(active_combine)
+    ccfg = cfg if not cfg or cfg.get("variant") != ep.EP_VARIANT_PACED else {**cfg, "variant": 0}  # dispatch only
     out, _ = ep.ep_normal_combine(nd["recv_x"] if y is None else y, nl, act_c, E, idx.shape[2], status=lay.status,
-                                  cfg=cfg)
+                                  cfg=ccfg)
     torch.cuda.synchronize()
     return lay, nl, nd, out
 
@@ -77,7 +78,8 @@ def test_normal_mode_worst_tokens_capacity(capacity):
     check_normal(inputs.make_inputs(w), w.num_experts, f"cap {capacity}", capacity=capacity)
 
 
-@pytest.mark.parametrize("cfg", [dict(variant=1), dict(variant=2), dict(variant=1, max_ctas=3, stages=2)])
+@pytest.mark.parametrize("cfg", [dict(variant=1), dict(variant=2), dict(variant=1, max_ctas=3, stages=2),
+                                 dict(variant=3), dict(variant=3, max_ctas=2, stages=2)])
 def test_normal_mode_paths_and_mask_flip(cfg):
     w = inputs.sweep(32, masked=True)
     inp = inputs.make_inputs(w)

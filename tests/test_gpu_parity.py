@@ -340,6 +340,33 @@ def test_variants_edge_shapes(name, variant):
     _check_all(run_path(inp, c["E"], c["H"], cfg=dict(variant=variant)), ref, packed, want, f"{name} v{variant}")
 
 
+PACED = [dict(variant=3), dict(variant=3, max_ctas=1, stages=2), dict(variant=3, max_ctas=5, stages=3),
+         dict(variant=3, max_ctas=7, stages=16)]
+
+
+@pytest.mark.parametrize("cfg", PACED)
+@pytest.mark.parametrize("name", ["tiny", "decode", "sweep_T64_mask5", "sweep_T512"])
+def test_paced_dispatch_matches_oracle(name, cfg):
+    """The paced bulk path (prefetches gated by the GPU clock) moves the same bits; tiny grids make
+    one CTA walk many units, so the prefetch cursor runs through many windows and ring wraps."""
+    w = inputs.named(name)
+    inp = inputs.make_inputs(w)
+    ref, packed, want = _oracle_all(inp, w.num_experts)
+    _check_all(run_path(inp, w.num_experts, w.hidden, dispatch_cfg=cfg), ref, packed, want, f"{name} {cfg}")
+
+
+@pytest.mark.parametrize("name", ["k1", "T1", "R1", "E_equals_R", "k32", "wide_H"])
+def test_paced_dispatch_edge_shapes(name):
+    c = EDGE[name]
+    rng = np.random.default_rng(zlib.crc32(name.encode()) + 3)
+    idx = _uniform_idx(rng, c["R"], c["T"], c["k"], c["E"])
+    idx = np.where(rng.random(idx.shape) < 0.1, -1, idx)
+    inp = _custom(c["R"], c["T"], c["k"], c["E"], c["H"], idx)
+    ref, packed, want = _oracle_all(inp, c["E"])
+    for cfg in (dict(variant=3), dict(variant=3, max_ctas=2, stages=2)):
+        _check_all(run_path(inp, c["E"], c["H"], dispatch_cfg=cfg), ref, packed, want, f"{name} {cfg}")
+
+
 def test_vector_variant_rejects_wide_topk():
     R, T, k, E, H = 2, 4, 9, 16, 64
     idx = torch.zeros((R, T, k), dtype=torch.int32, device=dev())
@@ -511,3 +538,40 @@ def test_lookback_layout_many_chunks(T):
     torch.cuda.synchronize()
     check_layout(lay, ref, f"lookback T={T}")
     assert int(lay.status.item()) == ref.status
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("name", ["decode", "sweep_T64_mask5"])
+def test_dispatch_ceiling_instrument(name, mode):
+    """The ceiling instrument writes zeros to exactly the dispatch's rows and the true src_info."""
+    w = inputs.named(name)
+    inp = inputs.make_inputs(w)
+    R, T, E, H = w.num_ranks, w.num_tokens, w.num_experts, w.hidden
+    ref = oracle.layout(inp.topk_idx, inp.active, E)
+    idx = i32_dev(inp.topk_idx)
+    lay = ep.ep_layout(idx, u8_dev(inp.active), E, hidden=H)
+    recv_x = torch.full((E, R * T, H), 3.0, dtype=torch.bfloat16, device=dev())
+    src_info = torch.full((E, R * T, 2), -9, dtype=torch.int32, device=dev())
+    _, _, st = ep.ep_diag_dispatch_ceiling(bf16_dev(inp.x), idx, lay.pair_row, E, mode, recv_x=recv_x,
+                                           src_info=src_info)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for e in range(E):
+        a, b = int(ref.list_base[e]), int(ref.list_base[e + 1])
+        assert np.array_equal(src_info[e, :b - a].cpu().numpy(), ref.src_list[a:b]), e
+        assert bool((recv_x[e, :b - a] == 0).all()), e
+        assert bool((recv_x[e, b - a:] == 3.0).all()) and bool((src_info[e, b - a:] == -9).all()), e
+
+
+def test_cumulative_receive_stats_over_calls():
+    """ep_recv_stats_accumulate over three layouts equals the sum of the oracle's receive counts."""
+    stats = torch.zeros(256, dtype=torch.int32, device=dev())
+    want = np.zeros(256, np.int64)
+    for name in ("decode", "sweep_T16_mask5", "sweep_T64"):
+        w = inputs.named(name)
+        inp = inputs.make_inputs(w, tokens=False)
+        lay = ep.ep_layout(i32_dev(inp.topk_idx), u8_dev(inp.active), w.num_experts, hidden=w.hidden)
+        ep.ep_recv_stats_accumulate(lay.recv_count, stats)
+        want += oracle.layout(inp.topk_idx, inp.active, w.num_experts).recv_count
+    torch.cuda.synchronize()
+    assert np.array_equal(stats.cpu().numpy(), want)

@@ -202,3 +202,29 @@ def test_ipc_export_reports_the_offset_inside_the_allocation():
     h1, off1 = ep.ep_ipc_export(t[4096:])
     assert len(h0) == ep.EP_IPC_HANDLE_BYTES and h0 == h1
     assert off1 - off0 == 4096
+
+
+def test_wait_cost_and_receive_stats():
+    """Per-source wait time accumulates (a sender that never comes costs the full wait limit) and the
+    cumulative receive counts of a rank's experts add up over steps."""
+    w = inputs.tiny()
+    inp = inputs.make_inputs(w)
+    E = w.num_experts
+    inp4 = inputs.Inputs(np.concatenate([inp.topk_idx, inp.topk_idx]), np.concatenate([inp.topk_weights] * 2),
+                         np.concatenate([inp.x, inp.x]), np.ones(4, np.uint8))
+    ranks, *_ = _run_world(inp4, E, w.hidden, signal=1, skip_sender=2)
+    wait_ns = torch.zeros(4, dtype=torch.int64, device=dev())
+    st = ranks[1].wait_arrivals(1, u8_dev(inp4.active), wait_ns=wait_ns)
+    torch.cuda.synchronize()
+    assert int(st.item()) == ep.EP_STATUS_TIMEOUT
+    ns = wait_ns.cpu().numpy()
+    assert ns[2] >= 2_000_000_000                      # the missing sender: the whole wait limit
+    assert all(ns[s] < 1_000_000_000 for s in (0, 1, 3))
+    ref = oracle.layout(inp4.topk_idx, inp4.active, E)
+    El = E // 4
+    stats = torch.zeros(El, dtype=torch.int32, device=dev())
+    for step in (2, 3, 4):
+        ranks, lays, counts, recv, status, waits, idx, act_c = _run_world(inp4, E, w.hidden, signal=step, world=ranks)
+        ep.ep_recv_stats_accumulate(recv[1], stats)
+    torch.cuda.synchronize()
+    assert np.array_equal(stats.cpu().numpy(), 3 * ref.recv_count[El:2 * El])
