@@ -44,6 +44,11 @@ struct DispatchFp8Args {
     int64_t cap;
     int64_t n_tok;
     int stages;            // bulk path: bf16 row stages per CTA
+    // bulk path, paced reads (read_period_ns 0: off): the producer prefetches the rows it will
+    // stage next into L2 only while globaltimer % read_period_ns < read_window_ns, up to
+    // read_ahead rows past the one it is loading (as ep_dispatch's EP_VARIANT_PACED)
+    uint64_t read_period_ns, read_window_ns;
+    int read_ahead;
 };
 
 template <int FMT>
@@ -222,9 +227,14 @@ __global__ void __launch_bounds__(256) dispatch_fp8_kernel(DispatchFp8Args a) {
 // The first of the two barriers per row also ORs the consumers' wait timeouts,
 // so all of them leave the loop together and no barrier is left waiting.
 constexpr int kFp8MaxConsumers = 8;
-constexpr int kFp8MaxStages = 8;
+constexpr int kFp8MaxStages = 16;
 constexpr uint32_t kFp8RowMax = 16384;  // largest bf16 row the bulk path stages whole
 constexpr int kFp8Bar = 1;              // named barrier of the consumer warps
+// paced reads: the schedule of ep_dispatch's EP_VARIANT_PACED
+constexpr uint64_t kFp8PacePeriodNs = 40000;
+constexpr uint64_t kFp8PaceWindowNs = 6000;
+constexpr int64_t kFp8PaceAheadBytes = 300 * 1024;
+constexpr int kFp8PaceMinRowsPerCta = 64;
 
 template <int FMT>
 __global__ void __launch_bounds__(32 * (1 + kFp8MaxConsumers)) dispatch_fp8_bulk_kernel(DispatchFp8Args a) {
@@ -268,6 +278,28 @@ __global__ void __launch_bounds__(32 * (1 + kFp8MaxConsumers)) dispatch_fp8_bulk
                 row = __ldg(a.pair_row + p);
             }
         };
+        const uint64_t pol_prefetch = policy_evict_last();
+        int64_t pf = my_n < S ? my_n : S;  // rows [0, pf) are loaded straight or prefetched
+        // paced reads: in the read window (or when fewer than a ring's worth of rows are
+        // prefetched), prefetch rows [pf, i + read_ahead) that have a live slot, lane j row pf + j
+        auto pace_reads = [&](int64_t i) {
+            int go = 0;
+            if (lane == 0) go = pf <= i + S || global_timer_ns() % a.read_period_ns < a.read_window_ns;
+            if (!__shfl_sync(0xffffffffu, go, 0)) return;
+            const int64_t want = (i + a.read_ahead) < my_n ? (i + a.read_ahead) : my_n;
+            for (; pf < want; pf += 32) {
+                const int64_t v = pf + lane;
+                if (v >= want) continue;
+                const int64_t tok = first + v * step;
+                bool live = false;
+                for (int j = 0; j < a.k; ++j) {
+                    const int r = __ldg(a.pair_row + tok * a.k + j);
+                    live |= r >= 0 && r < a.cap;
+                }
+                if (live) bulk_prefetch_l2(a.x + tok * int64_t(row_bytes), row_bytes, pol_prefetch);
+            }
+            if (pf > want) pf = want;
+        };
         int e_next = -1, row_next = -1;
         if (my_n > 0) routing(0, e_next, row_next);
         for (int64_t i = 0; i < my_n; ++i) {
@@ -298,6 +330,7 @@ __global__ void __launch_bounds__(32 * (1 + kFp8MaxConsumers)) dispatch_fp8_bulk
             } else {
                 mbar_arrive(bar);
             }
+            if (a.read_period_ns != 0) pace_reads(i);
         }
         return;
     }
@@ -439,22 +472,30 @@ extern "C" int ep_dispatch_fp8(ep_dims_t d, const uint16_t* x, const int32_t* to
     a.recv_count = recv_count;
     a.cap = RT;
     a.n_tok = RT;
+    a.read_period_ns = 0;
+    a.read_window_ns = 0;
+    a.read_ahead = 0;
     const int sms = sm_count();
     if (sms <= 0) return EP_ERR_CUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (cfg.variant != EP_VARIANT_AUTO && cfg.variant != EP_VARIANT_BULK && cfg.variant != EP_VARIANT_VECTOR)
+    if (cfg.variant != EP_VARIANT_AUTO && cfg.variant != EP_VARIANT_BULK && cfg.variant != EP_VARIANT_VECTOR &&
+        cfg.variant != EP_VARIANT_PACED)
         return EP_ERR_INVALID;
     const bool bulk_fits = uint32_t(d.hidden) * 2 <= kFp8RowMax && aligned16(recv_x);
-    if (cfg.variant == EP_VARIANT_BULK && !bulk_fits) return EP_ERR_UNSUPPORTED;
+    if ((cfg.variant == EP_VARIANT_BULK || cfg.variant == EP_VARIANT_PACED) && !bulk_fits) return EP_ERR_UNSUPPORTED;
+    // paced reads: asked for, or AUTO on the bulk path with enough rows per SM to span several
+    // read periods (the rule of ep_dispatch)
+    const bool paced = cfg.variant == EP_VARIANT_PACED ||
+                       (cfg.variant == EP_VARIANT_AUTO && bulk_fits && RT >= int64_t(kFp8PaceMinRowsPerCta) * sms);
     cudaError_t lerr;
     // AUTO: the bulk path, except fp32 scales on at most 1024 tokens, where the vector path's
     // finer units won on B200 (22.2 against 24.1 us at 8 ranks x 128 tokens; the bulk path leads
     // from 4096 tokens on: 68.6 against 77.9 us)
     const bool auto_vector = cfg.variant == EP_VARIANT_AUTO && scale_format == EP_FP8_SCALE_F32 && RT <= 1024;
     if (cfg.variant != EP_VARIANT_VECTOR && bulk_fits && !auto_vector) {
-        // default 2 CTAs per SM; cfg.max_ctas sets the grid.  W consumer warps split a
-        // row's 512-channel pieces evenly (7 at H = 7168, 8 at H = 4096).
-        int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas) : int64_t(sms) * 2;
+        // default 2 CTAs per SM (1 with paced reads, with a deeper ring); cfg.max_ctas sets the
+        // grid.  W consumer warps split a row's 512-channel pieces evenly (7 at H = 7168, 8 at 4096).
+        int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas) : int64_t(sms) * (paced ? 1 : 2);
         grid = std::max<int64_t>(1, std::min<int64_t>(grid, RT));
         const int ctas_per_sm = int(std::max<int64_t>(1, ceil_div(grid, sms)));
         const int np = int(ceil_div(d.hidden, 512));
@@ -464,7 +505,14 @@ extern "C" int ep_dispatch_fp8(ep_dims_t d, const uint16_t* x, const int32_t* to
         const size_t per_stage = stage_bytes + 16 + 32 * 8;                    // row, two mbarriers, routing
         const long budget = long(max_smem_optin()) / ctas_per_sm - 1024 - long(fixed);
         int stages = cfg.stages > 0 ? cfg.stages : int(std::max(0L, budget) / long(per_stage));
+        if (!paced && cfg.stages <= 0) stages = std::min(stages, 8);  // the unpaced path's measured ring
+        if (paced && cfg.stages <= 0) stages = std::min(stages, 14);
         stages = std::max(2, std::min(kFp8MaxStages, stages));
+        if (paced) {
+            a.read_period_ns = kFp8PacePeriodNs;
+            a.read_window_ns = kFp8PaceWindowNs;
+            a.read_ahead = int(std::max<int64_t>(1, kFp8PaceAheadBytes / int64_t(stage_bytes)));
+        }
         a.stages = stages;
         const size_t smem = size_t(stages) * per_stage + fixed;
         if (smem > size_t(max_smem_optin())) return EP_ERR_UNSUPPORTED;

@@ -1033,10 +1033,12 @@ struct LayoutGeom {
 
 // Chunks per source rank, tokens per chunk and warps per CTA for a shape whose
 // routing has Rs source ranks (Rs = R for the whole world, 1 for one rank).
-LayoutGeom layout_geom(const ep_dims_t& d, int Rs) {
+// `chunks` > 0 asks for that many chunks in all instead of one per kPairsPerChunk pairs.
+LayoutGeom layout_geom(const ep_dims_t& d, int Rs, int chunks = 0) {
     LayoutGeom lg;
     const int64_t pairs = int64_t(Rs) * d.num_tokens * d.num_topk;
-    const int64_t target = std::min<int64_t>(kMaxChunks, std::max<int64_t>(kTargetChunks, ceil_div(pairs, kPairsPerChunk)));
+    const int64_t target = chunks > 0 ? std::min<int64_t>(kMaxChunks, chunks)
+                                      : std::min<int64_t>(kMaxChunks, std::max<int64_t>(kTargetChunks, ceil_div(pairs, kPairsPerChunk)));
     int64_t C = std::max<int64_t>(1, ceil_div(target, Rs));
     C = std::max<int64_t>(1, std::min<int64_t>(C, d.num_tokens));
     lg.chunk_tokens = int(std::max<int64_t>(1, ceil_div(d.num_tokens, C)));
@@ -1138,9 +1140,9 @@ size_t layout_ws_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
 }
 
 int layout_run(const ep_dims_t& d, int Rs, int r0, const int32_t* topk_idx, const uint8_t* active, void* workspace,
-               int32_t* num_tokens_per_expert, int32_t* num_tokens_per_rank, uint8_t* is_token_in_rank,
-               int32_t* recv_count, int32_t* expert_rank_offset, int32_t* pair_row, int32_t* status,
-               const ep_cfg_t& cfg, cudaStream_t s);
+               size_t workspace_bytes, int32_t* num_tokens_per_expert, int32_t* num_tokens_per_rank,
+               uint8_t* is_token_in_rank, int32_t* recv_count, int32_t* expert_rank_offset, int32_t* pair_row,
+               int32_t* status, const ep_cfg_t& cfg, cudaStream_t s);
 
 }  // namespace
 }  // namespace ep
@@ -1148,7 +1150,7 @@ int layout_run(const ep_dims_t& d, int Rs, int r0, const int32_t* topk_idx, cons
 extern "C" int ep_layout_path(ep_dims_t d, ep_cfg_t cfg) {
     const int rc = check_dims(d);
     if (rc != EP_OK) return rc;
-    return resolve_layout_path(d, d.num_ranks, cfg, layout_geom(d, d.num_ranks));
+    return resolve_layout_path(d, d.num_ranks, cfg, layout_geom(d, d.num_ranks, cfg.max_ctas));
 }
 
 extern "C" size_t ep_layout_workspace_bytes(ep_dims_t d) {
@@ -1169,8 +1171,8 @@ extern "C" int ep_layout(ep_dims_t d, const int32_t* topk_idx, const uint8_t* ac
     if (RT > 0 && (!topk_idx || !is_token_in_rank || !pair_row)) return EP_ERR_INVALID;
     const size_t need = ep_layout_workspace_bytes(d);
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return EP_ERR_INVALID;
-    return layout_run(d, d.num_ranks, 0, topk_idx, active, workspace, num_tokens_per_expert, num_tokens_per_rank,
-                      is_token_in_rank, recv_count, expert_rank_offset, pair_row, status, cfg,
+    return layout_run(d, d.num_ranks, 0, topk_idx, active, workspace, workspace_bytes, num_tokens_per_expert,
+                      num_tokens_per_rank, is_token_in_rank, recv_count, expert_rank_offset, pair_row, status, cfg,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -1193,14 +1195,15 @@ extern "C" int ep_layout_local(ep_dims_t d, int32_t rank, const int32_t* topk_id
     if (rank < 0 || rank >= d.num_ranks) return EP_ERR_INVALID;
     if (!active || !num_tokens_per_expert || !num_tokens_per_rank) return EP_ERR_INVALID;
     if (d.num_tokens > 0 && (!topk_idx || !is_token_in_rank || !local_row)) return EP_ERR_INVALID;
-    const LayoutGeom lg = layout_geom(d, 1);
+    const LayoutGeom lg = layout_geom(d, 1, cfg.max_ctas);
     const size_t base = layout_ws_bytes(d, lg);
-    if (!workspace || workspace_bytes < ep_layout_local_workspace_bytes(d) || !aligned16(workspace))
+    if (!workspace || workspace_bytes < ep_layout_local_workspace_bytes(d) || !aligned16(workspace) ||
+        workspace_bytes < base + 2 * round_up16(size_t(d.num_experts) * 4))
         return EP_ERR_INVALID;
     char* ws = static_cast<char*>(workspace);
     int32_t* offset_scratch = reinterpret_cast<int32_t*>(ws + base);
     int32_t* count_scratch = reinterpret_cast<int32_t*>(ws + base + round_up16(size_t(d.num_experts) * 4));
-    return layout_run(d, 1, rank, topk_idx, active, workspace, num_tokens_per_expert, num_tokens_per_rank,
+    return layout_run(d, 1, rank, topk_idx, active, workspace, base, num_tokens_per_expert, num_tokens_per_rank,
                       is_token_in_rank, count_scratch, offset_scratch, local_row, status, cfg,
                       static_cast<cudaStream_t>(stream));
 }
@@ -1209,10 +1212,12 @@ namespace ep {
 namespace {
 
 int layout_run(const ep_dims_t& d, int Rs, int r0, const int32_t* topk_idx, const uint8_t* active, void* workspace,
-               int32_t* num_tokens_per_expert, int32_t* num_tokens_per_rank, uint8_t* is_token_in_rank,
-               int32_t* recv_count, int32_t* expert_rank_offset, int32_t* pair_row, int32_t* status,
-               const ep_cfg_t& cfg, cudaStream_t s) {
-    const LayoutGeom lg = layout_geom(d, Rs);
+               size_t workspace_bytes, int32_t* num_tokens_per_expert, int32_t* num_tokens_per_rank,
+               uint8_t* is_token_in_rank, int32_t* recv_count, int32_t* expert_rank_offset, int32_t* pair_row,
+               int32_t* status, const ep_cfg_t& cfg, cudaStream_t s) {
+    // cfg.max_ctas: the chunk count of the chunked, fused and look-back paths (their grids)
+    const LayoutGeom lg = layout_geom(d, Rs, cfg.max_ctas);
+    if (workspace_bytes < layout_ws_bytes(d, lg)) return EP_ERR_INVALID;
     LayoutArgs a;
     a.topk_idx = topk_idx;
     a.active = active;

@@ -111,9 +111,15 @@ def small_slab() -> Workload:
     return Workload("small_slab", 8, 512, 8, 32, 7168)
 
 
+def paced_slab() -> Workload:
+    """A 2.8 GB slab with 83 rows per SM: long enough for the paced dispatch (about six read periods),
+    small enough for detailed hardware-counter captures."""
+    return Workload("paced_slab", 8, 1536, 8, 16, 7168)
+
+
 def named(name: str) -> Workload:
     table = {"tiny": tiny(), "decode": decode(), "prefill": prefill(), "replica": replica(),
-             "small_slab": small_slab()}
+             "small_slab": small_slab(), "paced_slab": paced_slab()}
     if name in table:
         return table[name]
     if name.startswith("sweep_T"):

@@ -31,6 +31,7 @@ def main():
     ap.add_argument("--graph", action="store_true", help="time CUDA-graph replays of the calls")
     ap.add_argument("--variant", type=int, default=0, help="ep_cfg_t.variant of dispatch / combine")
     ap.add_argument("--layout-variant", type=int, default=0, help="ep_cfg_t.variant of layout")
+    ap.add_argument("--layout-ctas", type=int, default=0, help="ep_cfg_t.max_ctas of layout: chunk count")
     ap.add_argument("--mode", type=int, default=0, help="dispatch_ceiling: 0 stores only, 1 stores + row prefetch")
     args = ap.parse_args()
 
@@ -64,7 +65,8 @@ def main():
                                            status=status, stream=stream, cfg=cfg))
     if args.op in ("layout", "step"):
         calls.append(lambda: ep.ep_layout(idx_phys, act, E, hidden=H, workspace=ws, out=lay, status=status,
-                                          stream=stream, cfg=dict(variant=args.layout_variant)))
+                                          stream=stream, cfg=dict(variant=args.layout_variant,
+                                                                  max_ctas=args.layout_ctas)))
     if args.op in ("weight_sync", "grad_reduce"):
         if not w.num_extra:
             raise SystemExit("weight_sync / grad_reduce need a workload with replicas (e.g. replica)")

@@ -126,8 +126,9 @@ typedef struct ep_dims {
 /* Launch tuning (cf. Buffer.get_dispatch_config / get_combine_config and
  * num_sms on the NeMo page).  A zero field means "choose automatically". */
 typedef struct ep_cfg {
-    int32_t max_ctas;     /* CTAs of the row-moving kernels (dispatch: the grid, default
-                             2 per SM; combine: a cap, default 1 per SM) */
+    int32_t max_ctas;     /* CTAs of the row-moving kernels: the grid of dispatch (default 2
+                             per SM, 1 on the paced path) and of the vector combine (default:
+                             as many as fit at once); a cap for the bulk combine (default 1 per SM) */
     int32_t threads;      /* threads per CTA where the kernel allows a choice */
     int32_t stages;       /* shared-memory pipeline depth of dispatch / combine */
     int32_t variant;      /* dispatch / combine data path: EP_VARIANT_* */

@@ -23,7 +23,7 @@ def _free_memory():
     torch.cuda.empty_cache()
 
 
-VARIANTS = [ep.EP_VARIANT_BULK, ep.EP_VARIANT_VECTOR]
+VARIANTS = [ep.EP_VARIANT_BULK, ep.EP_VARIANT_VECTOR, ep.EP_VARIANT_PACED]
 
 
 def run_fp8(inp, E, fmt, cfg=None):
@@ -164,3 +164,13 @@ def test_fp8_dispatch_fuzz(seed):
     for variant in VARIANTS:
         check_fp8(inp, E, fmt, f"seed {seed} R={R} T={T} k={k} E={E} H={H} fmt {fmt} variant {variant}",
                   dict(variant=variant))
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("launch", [dict(max_ctas=1), dict(max_ctas=3, stages=2), dict(max_ctas=4, stages=14)])
+def test_fp8_paced_ring_wraps(fmt, launch):
+    """The paced bulk path with few CTAs: each producer walks many rows, so its prefetch cursor runs
+    through many read windows and the ring wraps many times."""
+    w = inputs.sweep(64, masked=True)
+    inp = inputs.make_inputs(w)
+    check_fp8(inp, w.num_experts, fmt, f"paced {launch} fmt {fmt}", dict(variant=ep.EP_VARIANT_PACED, **launch))

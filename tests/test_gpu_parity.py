@@ -341,7 +341,7 @@ def test_variants_edge_shapes(name, variant):
 
 
 PACED = [dict(variant=3), dict(variant=3, max_ctas=1, stages=2), dict(variant=3, max_ctas=5, stages=3),
-         dict(variant=3, max_ctas=7, stages=16)]
+         dict(variant=3, max_ctas=7, stages=15)]   # 15 stages of a 14 KB row: the deepest ring that fits
 
 
 @pytest.mark.parametrize("cfg", PACED)
