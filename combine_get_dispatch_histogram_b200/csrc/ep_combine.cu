@@ -327,10 +327,15 @@ int launch_combine_vec(const CombineArgs& a, const ep_cfg_t& cfg, int sms, cudaS
             return EP_ERR_CUDA;
         per_sm[dev & 63].store(occ, std::memory_order_relaxed);
     }
-    // default: the CTAs that fit at once; cfg.max_ctas sets the grid (more than fit at once makes a
-    // second wave that fills the SMs whose warps finish first)
-    int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas) : int64_t(sms) * std::max(1, occ);
-    const int64_t warps_needed = ceil_div(int64_t(a.R) * a.T * ceil_div(a.row_bytes >> 4, 32 * U), 1);
+    // default: the CTAs that fit at once, or three times as many for a large problem (>= 128 units
+    // per resident warp), whose later waves fill the SMs that finish first (B200, 8 x 4096 tokens:
+    // 635-637 against 655 us; no change at 8 x 512 tokens or the replica shape, slower at decode);
+    // cfg.max_ctas sets the grid
+    const int64_t resident = int64_t(sms) * std::max(1, occ);
+    const int64_t units = int64_t(a.R) * a.T * ceil_div(a.row_bytes >> 4, 32 * U);
+    int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas)
+                   : (units >= 128 * resident * (256 / 32) ? 3 * resident : resident);
+    const int64_t warps_needed = units;
     grid = std::max<int64_t>(1, std::min<int64_t>(grid, ceil_div(warps_needed, 8)));
     if (launch_pdl(combine_vec_kernel<U, NORMAL>, dim3(unsigned(grid)), dim3(256), 0, stream, a) != cudaSuccess)
         return EP_ERR_CUDA;

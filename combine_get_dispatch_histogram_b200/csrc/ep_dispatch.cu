@@ -47,7 +47,13 @@ constexpr int kDispatchMaxStages = 16;
 constexpr uint64_t kPacePeriodNs = 40000;
 constexpr uint64_t kPaceWindowNs = 6000;
 constexpr int64_t kPaceAheadBytes = 300 * 1024;
-constexpr int kPaceMinUnitsPerCta = 64;  // AUTO paces only runs long enough to span several periods
+// AUTO paces a low-latency dispatch only where it measured faster on B200: rows whose k stores
+// add up to >= 96 KB (so a 14-row ring holds about one read period of stores) and >= 16 rows per
+// SM.  Prefill (k = 8, 14 KB rows): 670 against 770 us; 8 x 512 tokens: 89.6 against 96.2 us.
+// It lost where the stores per row are smaller: the replica workload (k = 6, 8 KB rows) 255
+// against 172 us, normal mode (one row per destination rank) 849 against 455 us.
+constexpr int kPaceMinUnitsPerCta = 16;
+constexpr int64_t kPaceMinStoreBytesPerRow = 96 * 1024;
 
 struct DispatchArgs {
     const uint8_t* x;
@@ -401,10 +407,10 @@ int fill_dispatch_args(DispatchArgs& a, const ep_dims_t& d, const uint16_t* x, c
     return EP_OK;
 }
 
-// AUTO paces the reads when every CTA of a one-per-SM grid has enough units to span several
-// read periods (prefill-sized dispatches); short dispatches keep the two-CTA bulk path.
+// AUTO's choice for a low-latency dispatch (see kPaceMinStoreBytesPerRow).
 bool paced_by_default(const DispatchArgs& a, int sms) {
-    return a.n_units >= int64_t(kPaceMinUnitsPerCta) * sms;
+    return a.n_pieces == 1 && a.n_units >= int64_t(kPaceMinUnitsPerCta) * sms &&
+           int64_t(a.k) * a.row_bytes >= kPaceMinStoreBytesPerRow;
 }
 
 // Grid, stages and (for the paced path) the read schedule, then the bulk-path launch.  `prefetch`
@@ -516,9 +522,9 @@ extern "C" int ep_normal_dispatch(ep_dims_t d, int32_t recv_capacity, const uint
     a.read_ahead = 0;
     const int sms = sm_count();
     if (sms <= 0) return EP_ERR_CUDA;
-    // normal mode has only the bulk data path: PACED (or AUTO on a long dispatch) paces its reads,
-    // any other variant runs it unpaced
-    const bool paced = cfg.variant == EP_VARIANT_PACED || (cfg.variant == EP_VARIANT_AUTO && paced_by_default(a, sms));
+    // normal mode has only the bulk data path: PACED paces its reads (it measured slower at prefill,
+    // so AUTO does not), any other variant runs it unpaced
+    const bool paced = cfg.variant == EP_VARIANT_PACED;
     return run_bulk_dispatch<true>(a, cfg, paced, sms, static_cast<cudaStream_t>(stream));
 }
 

@@ -234,7 +234,6 @@ constexpr int kFp8Bar = 1;              // named barrier of the consumer warps
 constexpr uint64_t kFp8PacePeriodNs = 40000;
 constexpr uint64_t kFp8PaceWindowNs = 6000;
 constexpr int64_t kFp8PaceAheadBytes = 300 * 1024;
-constexpr int kFp8PaceMinRowsPerCta = 64;
 
 template <int FMT>
 __global__ void __launch_bounds__(32 * (1 + kFp8MaxConsumers)) dispatch_fp8_bulk_kernel(DispatchFp8Args a) {
@@ -483,10 +482,9 @@ extern "C" int ep_dispatch_fp8(ep_dims_t d, const uint16_t* x, const int32_t* to
         return EP_ERR_INVALID;
     const bool bulk_fits = uint32_t(d.hidden) * 2 <= kFp8RowMax && aligned16(recv_x);
     if ((cfg.variant == EP_VARIANT_BULK || cfg.variant == EP_VARIANT_PACED) && !bulk_fits) return EP_ERR_UNSUPPORTED;
-    // paced reads: asked for, or AUTO on the bulk path with enough rows per SM to span several
-    // read periods (the rule of ep_dispatch)
-    const bool paced = cfg.variant == EP_VARIANT_PACED ||
-                       (cfg.variant == EP_VARIANT_AUTO && bulk_fits && RT >= int64_t(kFp8PaceMinRowsPerCta) * sms);
+    // paced reads only when asked for: at prefill on B200 they did not pay here (UE8M0 437 against
+    // 440 us; fp32 scales 605 against 491 us, the one-CTA-per-SM grid halving the casting warps)
+    const bool paced = cfg.variant == EP_VARIANT_PACED;
     cudaError_t lerr;
     // AUTO: the bulk path, except fp32 scales on at most 1024 tokens, where the vector path's
     // finer units won on B200 (22.2 against 24.1 us at 8 ranks x 128 tokens; the bulk path leads

@@ -861,7 +861,8 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_fused_kernel(LayoutArgs
 //      publishes it with a release flag;
 //   B. waits (bounded) for the flags of the chunks before it only -- CTAs are
 //      dispatched in index order, so those have started -- and sums their
-//      histograms, all its threads loading in parallel;
+//      histograms, each warp a stripe of them with 16-byte loads all in flight,
+//      the warps' sums added up in shared memory;
 //   C. assigns rows as the rank kernel does.
 // The owners of the per-rank outputs are the chunks that can see them: the
 // first chunk of rank r writes expert_rank_offset[:, r], the last chunk of rank
@@ -881,13 +882,13 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_lookback_kernel(LayoutA
     int32_t* rank_of = smem + 2 * kActiveSlots;
     int32_t* first = rank_of + a.E;       // [E] rows of the chunks before this one
     int32_t* rank_first = first + a.E;    // [E] rows of the chunks of the ranks before this chunk's rank
-    int32_t* part = rank_first + a.E;     // [2][NT] partial sums of phase B
-    int32_t* whist = part + 2 * NT;       // [W][E]
+    int32_t* whist = rank_first + a.E;    // [W][E]
     const uint64_t epoch = *reinterpret_cast<volatile uint64_t*>(a.sync);
     uint64_t* flags = a.sync + 1;
     const uint64_t value = 2 * (epoch + 1);
     load_tables(a, act, rank_of);
     for (int i = threadIdx.x; i < W * a.E; i += NT) whist[i] = 0;
+    for (int e = threadIdx.x; e < a.E; e += NT) first[e] = rank_first[e] = 0;
     for (int d = threadIdx.x; d < a.R; d += NT) tpr[d] = 0;
     __syncthreads();
 
@@ -949,49 +950,53 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_lookback_kernel(LayoutA
         return;
     }
     const int rC = cg.r * a.C;  // first chunk of this chunk's rank
-    {
-        // thread (e, q): expert e, chunks gg = q, q + P, ... (P = NT / E parts when E <= NT)
-        const int P = a.E <= NT ? NT / a.E : 1;
-        for (int e0 = 0; e0 < a.E; e0 += NT / P) {
-            const int e = e0 + threadIdx.x % (NT / P);
-            const int q = threadIdx.x / (NT / P);
-            int32_t s_before = 0, s_rank = 0;
-            if (e < a.E && q < P) {
-                int gg = q;
-#pragma unroll 1
-                for (; gg + 7 * P < g; gg += 8 * P) {
-                    int32_t v[8];
+    // warp w sums chunks w, w + W, ... below g (16-byte loads of four experts when E % 4 == 0, so a
+    // lane's loads of all its chunks are in flight together), split at rC into the ranks before this
+    // chunk's rank and this rank's earlier chunks; the warps' partial sums meet in shared memory
+    if ((a.E & 3) == 0) {
+        const int E4 = a.E >> 2;
+        for (int e4 = lane; e4 < E4; e4 += 32) {
+            int4 sb = make_int4(0, 0, 0, 0), sr = sb;
+            int gg = warp;
+            for (; gg + 7 * W < g; gg += 8 * W) {
+                int4 v[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) v[u] = a.chunk_hist[int64_t(gg + u * P) * a.E + e];
+                for (int u = 0; u < 8; ++u)
+                    v[u] = reinterpret_cast<const int4*>(a.chunk_hist + int64_t(gg + u * W) * a.E)[e4];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        if (gg + u * P < rC) s_before += v[u];
-                        else s_rank += v[u];
-                    }
-                }
-                for (; gg < g; gg += P) {
-                    const int32_t v = a.chunk_hist[int64_t(gg) * a.E + e];
-                    if (gg < rC) s_before += v;
-                    else s_rank += v;
+                for (int u = 0; u < 8; ++u) {
+                    int4& acc = gg + u * W < rC ? sb : sr;
+                    acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
                 }
             }
-            if (q < P) {
-                part[threadIdx.x] = s_before;
-                part[NT + threadIdx.x] = s_rank;
+            for (; gg < g; gg += W) {
+                const int4 v = reinterpret_cast<const int4*>(a.chunk_hist + int64_t(gg) * a.E)[e4];
+                int4& acc = gg < rC ? sb : sr;
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
             }
-            __syncthreads();
-            if (q == 0 && e < a.E) {
-                int32_t b = 0, r = 0;
-                for (int qq = 0; qq < P; ++qq) {
-                    b += part[qq * (NT / P) + (e - e0)];
-                    r += part[NT + qq * (NT / P) + (e - e0)];
-                }
-                rank_first[e] = b;
-                first[e] = b + r;
+            const int e = 4 * e4;
+            if (sb.x | sb.y | sb.z | sb.w) {
+                atomicAdd(rank_first + e, sb.x); atomicAdd(rank_first + e + 1, sb.y);
+                atomicAdd(rank_first + e + 2, sb.z); atomicAdd(rank_first + e + 3, sb.w);
             }
-            __syncthreads();
+            if (sb.x | sb.y | sb.z | sb.w | sr.x | sr.y | sr.z | sr.w) {
+                atomicAdd(first + e, sb.x + sr.x); atomicAdd(first + e + 1, sb.y + sr.y);
+                atomicAdd(first + e + 2, sb.z + sr.z); atomicAdd(first + e + 3, sb.w + sr.w);
+            }
+        }
+    } else {
+        for (int e = lane; e < a.E; e += 32) {
+            int32_t sb = 0, sr = 0;
+            for (int gg = warp; gg < g; gg += W) {
+                const int32_t v = a.chunk_hist[int64_t(gg) * a.E + e];
+                if (gg < rC) sb += v;
+                else sr += v;
+            }
+            if (sb) atomicAdd(rank_first + e, sb);
+            if (sb | sr) atomicAdd(first + e, sb + sr);
         }
     }
+    __syncthreads();
     if (g == rC) {
         for (int e = threadIdx.x; e < a.E; e += NT) a.expert_rank_offset[int64_t(e) * a.Rs + cg.r] = first[e];
     }
@@ -1095,7 +1100,7 @@ size_t fused_smem_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
 }
 
 size_t lookback_smem_bytes(const ep_dims_t& d, const LayoutGeom& lg) {
-    return size_t(2 * kActiveSlots + 3 * d.num_experts + 2 * 32 * lg.warps + lg.warps * d.num_experts) * 4;
+    return size_t(2 * kActiveSlots + 3 * d.num_experts + lg.warps * d.num_experts) * 4;
 }
 
 // The path ep_layout takes for these dims and cfg, or a negative EP_ERR_* code.

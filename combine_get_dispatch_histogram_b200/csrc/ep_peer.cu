@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(256) peer_recv_count_kernel(const int32_t* cou
 // Slots are taken in groups of kPeerSlotGroup: a lane issues the group's loads,
 // then accumulates them in slot order.
 template <int U>
-__global__ void __launch_bounds__(kPeerThreads) combine_peer_kernel(PeerArgs a) {
+__global__ void __launch_bounds__(kPeerThreads, 1) combine_peer_kernel(PeerArgs a) {
     extern __shared__ int32_t off[];  // [E]
     __shared__ int32_t act[EP_MAX_RANKS];
     pdl_wait();

@@ -30,6 +30,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--graph", action="store_true", help="time CUDA-graph replays of the calls")
     ap.add_argument("--variant", type=int, default=0, help="ep_cfg_t.variant of dispatch / combine")
+    ap.add_argument("--max-ctas", type=int, default=0, help="ep_cfg_t.max_ctas of dispatch / combine")
     ap.add_argument("--layout-variant", type=int, default=0, help="ep_cfg_t.variant of layout")
     ap.add_argument("--layout-ctas", type=int, default=0, help="ep_cfg_t.max_ctas of layout: chunk count")
     ap.add_argument("--mode", type=int, default=0, help="dispatch_ceiling: 0 stores only, 1 stores + row prefetch")
@@ -45,7 +46,7 @@ def main():
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     idx = torch.from_numpy(inp.topk_idx).to(dev)
     act = torch.from_numpy(inp.active).to(dev)
-    cfg = dict(variant=args.variant)
+    cfg = dict(variant=args.variant, max_ctas=args.max_ctas)
     stream = torch.cuda.Stream(dev)
 
     if w.num_extra:

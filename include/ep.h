@@ -158,11 +158,14 @@ enum {
     EP_VARIANT_AUTO = 0,      /* the faster path for the shape, as measured on B200 */
     EP_VARIANT_BULK = 1,      /* rows staged in shared memory by bulk async copies */
     EP_VARIANT_VECTOR = 2,    /* rows moved through registers as 16-byte vectors */
-    EP_VARIANT_PACED = 3      /* ep_dispatch / ep_normal_dispatch: the bulk path with paced reads --
-                                 one CTA per SM, and the rows about to be staged are prefetched into
-                                 L2 only inside a short window that recurs on the GPU-wide clock,
-                                 so HBM serves reads in bursts and the row stores alone in between
-                                 (the same bits; AUTO takes it for long dispatches) */
+    EP_VARIANT_PACED = 3      /* ep_dispatch, ep_normal_dispatch, ep_dispatch_fp8: the bulk path
+                                 with paced reads -- one CTA per SM, and the rows about to be staged
+                                 are prefetched into L2 only inside a short window that recurs on
+                                 the GPU-wide clock, so HBM serves reads in bursts and the row stores
+                                 alone in between (the same bits).  AUTO takes it for ep_dispatch
+                                 when a row's k stores add up to >= 96 KB and every SM has >= 16
+                                 rows (e.g. 8 x 4096 tokens, top-8, H = 7168), where it measured
+                                 faster */
 };
 
 /* Human-readable name of an EP_OK / EP_ERR_* code (static storage). */
@@ -656,7 +659,9 @@ EP_API int ep_recv_stats_accumulate(int32_t num, const int32_t *recv_count, int3
 enum { EP_IPC_HANDLE_BYTES = 64 };
 
 /* The IPC handle of the allocation that holds device pointer `ptr` and ptr's byte
- * offset inside it (host outputs), to send to the other ranks. */
+ * offset inside it (host outputs), to send to the other ranks.  The allocation must be
+ * an ordinary device allocation (cudaMalloc, or PyTorch's caching allocator without
+ * expandable segments); virtual-memory-managed ones have no IPC handle (EP_ERR_CUDA). */
 EP_API int ep_ipc_export(const void *ptr, void *handle, uint64_t *offset);
 
 /* Map another process's exported buffer: *ptr = its address here, *base = the mapping
