@@ -511,6 +511,7 @@ def run_ours(args, rank, world, local_rank, w, inp):
     com_gbs = c_bytes / (com_ms * 1e-3) / 1e9
     peak, peak_kind = measured_hbm_gbs()
     d_name, c_name = kernel_names(args, k)
+    dispatch_path = ep.ep_dispatch_path(R, T, k, E, H, cfg=args.dispatch_cfg)
     dom = (d_name, d_bytes, dis_ms) if dis_ms >= com_ms else (c_name, c_bytes, com_ms)
     achieved = dom[1] / (dom[2] * 1e-3) / 1e9
     line = {
@@ -543,13 +544,17 @@ def run_ours(args, rank, world, local_rank, w, inp):
                      "traffic": profiled_traffic(dom[0], w.name),
                      "algorithmic_bytes": dom[1]},
         "gpu_launches": launches_per_step * args.steps,
+        "dispatch_path": {ep.EP_VARIANT_BULK: "bulk", ep.EP_VARIANT_PACED: "paced",
+                          ep.EP_VARIANT_VECTOR: "vector"}.get(dispatch_path, str(dispatch_path)),
         "dispatch_ceiling": {
             "what": "the paced dispatch kernel without its row loads (ep_diag_dispatch_ceiling), timed after the "
                     "steps: stores alone, and stores plus the paced L2 prefetch of the rows (the dispatch's HBM "
-                    "traffic with no store waiting on a read)",
+                    "traffic with no store waiting on a read); compared with the dispatch only when the dispatch "
+                    "itself took the paced path",
             "stores_only_us": round(c0_ms * 1e3, 2),
             "stores_and_row_reads_us": round(c1_ms * 1e3, 2),
-            "dispatch_over_stores_and_reads": round(dis_ms / c1_ms, 4),
+            "dispatch_over_stores_and_reads": (round(dis_ms / c1_ms, 4) if dispatch_path == ep.EP_VARIANT_PACED
+                                               else None),
         },
     }
     if args.graph:

@@ -547,3 +547,19 @@ extern "C" int ep_diag_dispatch_ceiling(ep_dims_t d, const uint16_t* x, const in
     // the paced path's grid and ring, its L2 prefetch schedule in mode 1
     return run_bulk_dispatch<false, true>(a, cfg, true, sms, static_cast<cudaStream_t>(stream), mode);
 }
+
+extern "C" int ep_dispatch_path(ep_dims_t d, ep_cfg_t cfg) {
+    int rc = check_dims(d);
+    if (rc != EP_OK) return rc;
+    if (cfg.variant != EP_VARIANT_AUTO && cfg.variant != EP_VARIANT_BULK && cfg.variant != EP_VARIANT_VECTOR &&
+        cfg.variant != EP_VARIANT_PACED)
+        return EP_ERR_INVALID;
+    if (cfg.variant == EP_VARIANT_VECTOR && d.num_topk > kVecKMax) return EP_ERR_UNSUPPORTED;
+    if (cfg.variant != EP_VARIANT_AUTO) return cfg.variant;
+    DispatchArgs a;
+    rc = fill_dispatch_args(a, d, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+    if (rc != EP_OK) return rc;
+    const int sms = sm_count();
+    if (sms <= 0) return EP_ERR_CUDA;
+    return paced_by_default(a, sms) ? EP_VARIANT_PACED : EP_VARIANT_BULK;
+}

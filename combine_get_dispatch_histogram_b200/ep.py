@@ -96,6 +96,8 @@ def load_library(path: str = LIB_PATH):
     lib.ep_layout.restype = ctypes.c_int
     lib.ep_dispatch.argtypes = [Dims, P, P, P, P, P, P, Cfg, P]
     lib.ep_dispatch.restype = ctypes.c_int
+    lib.ep_dispatch_path.argtypes = [Dims, Cfg]
+    lib.ep_dispatch_path.restype = ctypes.c_int
     lib.ep_diag_dispatch_ceiling.argtypes = [Dims, P, P, P, P, P, I32, P, Cfg, P]
     lib.ep_diag_dispatch_ceiling.restype = ctypes.c_int
     lib.ep_combine.argtypes = [Dims, P, P, P, P, P, P, P, Cfg, P]
@@ -353,6 +355,16 @@ def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, pair_row: torch.Tensor,
                              _ptr(src_info), _ptr(status), _cfg(cfg), _stream(dev, stream))
     _check("ep_dispatch", rc)
     return recv_x, src_info, status
+
+
+def ep_dispatch_path(num_ranks: int, num_tokens: int, num_topk: int, num_experts: int, hidden: int,
+                     cfg=None) -> int:
+    """The ``EP_VARIANT_*`` data path ``ep_dispatch`` takes for this shape and ``cfg`` (``ep_dispatch_path``)."""
+    with torch.cuda.device(torch.cuda.current_device()):
+        rc = int(load_library().ep_dispatch_path(Dims(num_ranks, num_tokens, num_topk, num_experts, hidden), _cfg(cfg)))
+    if rc < 0:
+        _check("ep_dispatch_path", rc)
+    return rc
 
 
 def ep_diag_dispatch_ceiling(x: torch.Tensor, topk_idx: torch.Tensor, pair_row: torch.Tensor, num_experts: int,

@@ -326,6 +326,14 @@ EP_API int ep_dispatch(ep_dims_t d, const uint16_t *x, const int32_t *topk_idx,
                 const int32_t *pair_row, uint16_t *recv_x, int32_t *src_info,
                 int32_t *status, ep_cfg_t cfg, void *stream);
 
+/*
+ * ep_dispatch_path -- the data path (EP_VARIANT_BULK, _VECTOR or _PACED) that
+ * ep_dispatch takes for these dims and cfg.variant on the current device (AUTO
+ * resolved); EP_ERR_* as ep_dispatch would return for bad dims or variant.  The
+ * pages have no counterpart: it reports this library's choice.  Launches nothing.
+ */
+EP_API int ep_dispatch_path(ep_dims_t d, ep_cfg_t cfg);
+
 /* Scale formats of ep_dispatch_fp8 (NeMo page, Buffer.low_latency_dispatch:
  * use_fp8, round_scale, use_ue8m0). */
 enum {

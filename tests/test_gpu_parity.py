@@ -575,3 +575,19 @@ def test_cumulative_receive_stats_over_calls():
         want += oracle.layout(inp.topk_idx, inp.active, w.num_experts).recv_count
     torch.cuda.synchronize()
     assert np.array_equal(stats.cpu().numpy(), want)
+
+
+def test_dispatch_path_choice():
+    """AUTO paces the dispatch only where a row's k stores add up to >= 96 KB with >= 16 rows per SM."""
+    assert ep.ep_dispatch_path(8, 4096, 8, 256, 7168) == ep.EP_VARIANT_PACED     # prefill
+    assert ep.ep_dispatch_path(8, 512, 8, 256, 7168) == ep.EP_VARIANT_PACED      # 27 rows per SM
+    assert ep.ep_dispatch_path(8, 128, 8, 256, 7168) == ep.EP_VARIANT_BULK       # decode: 7 rows per SM
+    assert ep.ep_dispatch_path(8, 2048, 6, 80, 4096) == ep.EP_VARIANT_BULK       # replica: 48 KB per row
+    assert ep.ep_dispatch_path(8, 128, 8, 256, 7168, cfg=dict(variant=2)) == ep.EP_VARIANT_VECTOR
+    assert ep.ep_dispatch_path(8, 128, 8, 256, 7168, cfg=dict(variant=3)) == ep.EP_VARIANT_PACED
+    with pytest.raises(ep.EPError) as ei:
+        ep.ep_dispatch_path(2, 4, 9, 16, 64, cfg=dict(variant=2))
+    assert ei.value.code == ep.EP_ERR_UNSUPPORTED
+    with pytest.raises(ep.EPError) as ei:
+        ep.ep_dispatch_path(2, 4, 2, 16, 64, cfg=dict(variant=7))
+    assert ei.value.code == ep.EP_ERR_INVALID
