@@ -21,6 +21,7 @@ from . import ep, inputs
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--op", choices=["layout", "dispatch", "dispatch_ceiling", "dispatch_fp8", "combine", "reroute", "step",
+                                     "peer_dispatch", "peer_combine",
                                      "normal_layout", "normal_dispatch", "normal_combine", "weight_sync",
                                      "grad_reduce"], required=True)
     ap.add_argument("--params", type=int, default=1 << 22, help="weight_sync / grad_reduce: float32 params per expert")
@@ -39,7 +40,8 @@ def main():
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
     w = inputs.named(args.workload)
-    need_x = args.op in ("dispatch", "dispatch_ceiling", "dispatch_fp8", "step") or args.op.startswith("normal_")
+    need_x = args.op in ("dispatch", "dispatch_ceiling", "dispatch_fp8", "step") or args.op.startswith("normal_") \
+        or args.op.startswith("peer_")
     inp = inputs.make_inputs(w, tokens=need_x or args.op == "combine")
     R, T, k, H, E = w.num_ranks, w.num_tokens, w.num_topk, w.hidden, w.num_physical
     cap = R * T
@@ -123,6 +125,31 @@ def main():
         if args.op in ("combine", "step"):
             calls.append(lambda: ep.ep_combine(recv_x, idx_phys, wts, lay.pair_row, act, out=out, status=status,
                                                stream=stream, cfg=cfg))
+    if args.op.startswith("peer_"):
+        # every emulated rank's kernel in turn on one stream (its own buffers, reached through the
+        # address tables as peer memory would be); the signals grow from call to call
+        from . import peer
+
+        ranks = peer.emulated_world(R, E, T, k, H, dev)
+        x = torch.from_numpy(inp.x.view(np.int16)).to(dev).view(torch.bfloat16)
+        wts = torch.from_numpy(inp.topk_weights).to(dev)
+        idxs = [idx_phys[r].contiguous() for r in range(R)]
+        lays = [ranks[r].layout(idxs[r], act, status=status) for r in range(R)]
+        counts = torch.stack([lay_r.num_tokens_per_expert for lay_r in lays])
+        outs = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+        sig = [0]
+
+        def peer_dispatch():
+            sig[0] += 1
+            for r in range(R):
+                ranks[r].dispatch(x[r], idxs[r], lays[r], counts, act, sig[0], status=status, stream=stream)
+
+        def peer_combine():
+            for r in range(R):
+                ranks[r].combine(idxs[r], wts[r], lays[r], counts, act, out=outs[r], status=status, stream=stream)
+
+        peer_dispatch()
+        calls.append(peer_dispatch if args.op == "peer_dispatch" else peer_combine)
     torch.cuda.synchronize()
 
     def run_all():
@@ -161,6 +188,10 @@ def main():
     elif args.op in ("normal_dispatch", "normal_combine"):
         sends = int(nl["recv_tokens"].sum().item())     # (token, destination rank) rows
         algo = 2 * H * (sent + sends) if args.op == "normal_dispatch" else 2 * H * (sends + R * T)
+    elif args.op == "peer_dispatch":
+        algo = 2 * H * (sent + live)
+    elif args.op == "peer_combine":
+        algo = 2 * H * (live + R * T)
     elif args.op in ("dispatch", "dispatch_fp8"):
         algo = 2 * H * sent + per_pair[args.op] * live
     elif args.op == "dispatch_ceiling":
