@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(256) peer_recv_count_kernel(const int32_t* cou
 // Slots are taken in groups of kPeerSlotGroup: a lane issues the group's loads,
 // then accumulates them in slot order.
 template <int U>
-__global__ void __launch_bounds__(kPeerThreads, 1) combine_peer_kernel(PeerArgs a) {
+__global__ void __launch_bounds__(kPeerThreads, 2) combine_peer_kernel(PeerArgs a) {
     extern __shared__ int32_t off[];  // [E]
     __shared__ int32_t act[EP_MAX_RANKS];
     pdl_wait();
@@ -523,8 +523,8 @@ extern "C" int ep_combine_peer(ep_dims_t d, int32_t rank, const uint64_t* y_slab
     a.rank = rank;
     a.cap = int64_t(d.num_ranks) * d.num_tokens;
     a.row_bytes = int64_t(d.hidden) * 2;
-    const int64_t units = int64_t(d.num_tokens) * ceil_div(a.row_bytes >> 4, 32 * 2);
-    return launch_peer_stream(combine_peer_kernel<2>, a, int(std::min<int64_t>(units, INT32_MAX)), cfg,
+    const int64_t units = int64_t(d.num_tokens) * ceil_div(a.row_bytes >> 4, 32 * 1);
+    return launch_peer_stream(combine_peer_kernel<1>, a, int(std::min<int64_t>(units, INT32_MAX)), cfg,
                               static_cast<cudaStream_t>(stream));
 }
 
