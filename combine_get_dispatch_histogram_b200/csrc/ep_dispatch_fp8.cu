@@ -226,7 +226,8 @@ __global__ void __launch_bounds__(256) dispatch_fp8_kernel(DispatchFp8Args a) {
 // apart only modulo 2) cannot mistake the stage's previous fill for row i.
 // The first of the two barriers per row also ORs the consumers' wait timeouts,
 // so all of them leave the loop together and no barrier is left waiting.
-constexpr int kFp8MaxConsumers = 8;
+constexpr int kFp8MaxConsumers = 16;
+constexpr int kFp8DefaultConsumers = 8;  // per CTA unless cfg.threads asks for more (up to kFp8MaxConsumers)
 constexpr int kFp8MaxStages = 16;
 constexpr uint32_t kFp8RowMax = 16384;  // largest bf16 row the bulk path stages whole
 constexpr int kFp8Bar = 1;              // named barrier of the consumer warps
@@ -497,7 +498,10 @@ extern "C" int ep_dispatch_fp8(ep_dims_t d, const uint16_t* x, const int32_t* to
         grid = std::max<int64_t>(1, std::min<int64_t>(grid, RT));
         const int ctas_per_sm = int(std::max<int64_t>(1, ceil_div(grid, sms)));
         const int np = int(ceil_div(d.hidden, 512));
-        const int consumers = int(ceil_div(np, ceil_div(np, kFp8MaxConsumers)));
+        // W consumer warps split a row's pieces evenly: by default at most kFp8DefaultConsumers
+        // (7 at H = 7168: two pieces each); cfg.threads = 32 * (1 + W) asks for W of them
+        const int want = cfg.threads >= 64 ? std::min(kFp8MaxConsumers, cfg.threads / 32 - 1) : kFp8DefaultConsumers;
+        const int consumers = int(ceil_div(np, ceil_div(np, want)));
         const size_t stage_bytes = (size_t(d.hidden) * 2 + 127) & ~size_t(127);
         const size_t fixed = 2 * ((size_t(d.hidden) + 127) & ~size_t(127));  // two code rows
         const size_t per_stage = stage_bytes + 16 + 32 * 8;                    // row, two mbarriers, routing

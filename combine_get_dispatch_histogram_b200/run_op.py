@@ -32,6 +32,8 @@ def main():
     ap.add_argument("--graph", action="store_true", help="time CUDA-graph replays of the calls")
     ap.add_argument("--variant", type=int, default=0, help="ep_cfg_t.variant of dispatch / combine")
     ap.add_argument("--max-ctas", type=int, default=0, help="ep_cfg_t.max_ctas of dispatch / combine")
+    ap.add_argument("--threads", type=int, default=0, help="ep_cfg_t.threads of dispatch / combine")
+    ap.add_argument("--stages", type=int, default=0, help="ep_cfg_t.stages of dispatch / combine")
     ap.add_argument("--layout-variant", type=int, default=0, help="ep_cfg_t.variant of layout")
     ap.add_argument("--layout-ctas", type=int, default=0, help="ep_cfg_t.max_ctas of layout: chunk count")
     ap.add_argument("--mode", type=int, default=0, help="dispatch_ceiling: 0 stores only, 1 stores + row prefetch")
@@ -48,7 +50,7 @@ def main():
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     idx = torch.from_numpy(inp.topk_idx).to(dev)
     act = torch.from_numpy(inp.active).to(dev)
-    cfg = dict(variant=args.variant, max_ctas=args.max_ctas)
+    cfg = dict(variant=args.variant, max_ctas=args.max_ctas, threads=args.threads, stages=args.stages)
     stream = torch.cuda.Stream(dev)
 
     if w.num_extra:

@@ -366,6 +366,8 @@ enum {
  * Rows not written keep their contents.  Two launches: the cast (codes to every
  * live row, each token's scales once to the workspace), then a scale writer that
  * fills the column-major scale tensor with coalesced stores.
+ * cfg.threads (bulk path): 32 * (1 + W) asks for W casting warps per CTA (1 to 16; default:
+ * up to 8, split evenly over the row's 512-channel pieces).
  * cfg.variant: EP_VARIANT_BULK stages each bf16 row in shared memory with a bulk
  * copy and bulk-stores the code rows (needs 2*H <= 16384 and a 16-byte aligned
  * recv_x, else EP_ERR_UNSUPPORTED); EP_VARIANT_VECTOR moves rows through

@@ -167,10 +167,20 @@ def test_fp8_dispatch_fuzz(seed):
 
 
 @pytest.mark.parametrize("fmt", FORMATS)
-@pytest.mark.parametrize("launch", [dict(max_ctas=1), dict(max_ctas=3, stages=2), dict(max_ctas=4, stages=14)])
+@pytest.mark.parametrize("launch", [dict(max_ctas=1), dict(max_ctas=3, stages=2), dict(max_ctas=4, stages=14),
+                                    dict(max_ctas=2, threads=32 * 15), dict(threads=32 * 17)])
 def test_fp8_paced_ring_wraps(fmt, launch):
     """The paced bulk path with few CTAs: each producer walks many rows, so its prefetch cursor runs
     through many read windows and the ring wraps many times."""
     w = inputs.sweep(64, masked=True)
     inp = inputs.make_inputs(w)
     check_fp8(inp, w.num_experts, fmt, f"paced {launch} fmt {fmt}", dict(variant=ep.EP_VARIANT_PACED, **launch))
+
+
+@pytest.mark.parametrize("threads", [32 * 2, 32 * 8, 32 * 15, 32 * 17])
+def test_fp8_consumer_warp_counts(threads):
+    """One to sixteen casting warps per CTA (cfg.threads = 32 * (1 + W)) give the same bits."""
+    w = inputs.sweep(64, masked=True)
+    inp = inputs.make_inputs(w)
+    check_fp8(inp, w.num_experts, ep.EP_FP8_SCALE_UE8M0, f"threads {threads}",
+              dict(variant=ep.EP_VARIANT_BULK, threads=threads, max_ctas=7))
