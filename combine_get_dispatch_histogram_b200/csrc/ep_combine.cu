@@ -231,9 +231,10 @@ __global__ void combine_kernel(CombineArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Vector path (EP_VARIANT_VECTOR, k <= 8): every warp owns a contiguous,
-// balanced range of units (token, piece of 32*U 16-byte columns).  At a token
-// boundary lane j reads slot j's routing and the slot pointers and weights are
+// Vector path (EP_VARIANT_VECTOR, k <= 8): the warps take units (token, piece of
+// 32*U 16-byte columns) strided from the end of the token range (low-latency
+// mode) or in contiguous ranges (normal mode).  At a new token
+// lane j reads slot j's routing and the slot pointers and weights are
 // broadcast with shuffles; then each lane issues all k * U 16-byte loads of
 // its columns at once (L1 bypassed, 256-byte L2 fetch), accumulates in slot
 // order and stores its U result vectors.
@@ -253,15 +254,28 @@ __global__ void __launch_bounds__(256) combine_vec_kernel(CombineArgs a) {
     const int piece_vec = 32 * U;
     const int np = (nvec + piece_vec - 1) / piece_vec;
     const int64_t n_units = int64_t(a.R) * a.T * np;
-    const int64_t q = n_units / warps, rem = n_units % warps;
-    const int64_t u0 = gw * q + (gw < rem ? gw : rem);
-    const int64_t u1 = u0 + q + (gw < rem ? 1 : 0);
+    // Low-latency mode takes units strided from the end: warp gw takes units n-1-gw, n-1-gw-W, ...
+    // (W = warps), so at any moment the grid works on one window of consecutive tokens, whose rows of
+    // the busy experts are neighbours in the slabs, and it starts with the tokens dispatched last,
+    // whose rows may still sit in L2.  (Contiguous ranges per warp read ~W scattered regions at once:
+    // 649 against 606 us for the whole prefill combine on B200, 682 against 626 us right after a
+    // dispatch.)  Normal mode keeps contiguous, balanced ranges per warp: its rows are per destination
+    // rank in (source, token) order, and the strided order measured slower there (457 against 444 us).
+    int64_t my_n, u0 = 0;
+    if (NORMAL) {
+        const int64_t q = n_units / warps, rem = n_units % warps;
+        u0 = gw * q + (gw < rem ? gw : rem);
+        my_n = q + (gw < rem ? 1 : 0);
+    } else {
+        my_n = gw < n_units ? (n_units - 1 - gw) / warps + 1 : 0;
+    }
 
     int64_t cur_tok = -1;
     uint32_t mask = 0;
     const uint8_t* src[kVecKMax];
     float wt[kVecKMax];
-    for (int64_t u = u0; u < u1; ++u) {
+    for (int64_t i = 0; i < my_n; ++i) {
+        const int64_t u = NORMAL ? u0 + i : n_units - 1 - gw - i * warps;
         const int64_t tok = u / np;
         const int pc = int(u - tok * np);
         if (tok != cur_tok) {
@@ -327,14 +341,14 @@ int launch_combine_vec(const CombineArgs& a, const ep_cfg_t& cfg, int sms, cudaS
             return EP_ERR_CUDA;
         per_sm[dev & 63].store(occ, std::memory_order_relaxed);
     }
-    // default: the CTAs that fit at once, or three times as many for a large problem (>= 128 units
-    // per resident warp), whose later waves fill the SMs that finish first (B200, 8 x 4096 tokens:
-    // 635-637 against 655 us; no change at 8 x 512 tokens or the replica shape, slower at decode);
-    // cfg.max_ctas sets the grid
+    // default: the CTAs that fit at once (low-latency mode, strided units: a 3x grid measured
+    // slower, 619 against 606 us at 8 x 4096 tokens); in normal mode (contiguous unit ranges) three
+    // times that for a large problem (>= 128 units per resident warp), whose later waves fill the SMs
+    // that finish first; cfg.max_ctas sets the grid
     const int64_t resident = int64_t(sms) * std::max(1, occ);
     const int64_t units = int64_t(a.R) * a.T * ceil_div(a.row_bytes >> 4, 32 * U);
     int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas)
-                   : (units >= 128 * resident * (256 / 32) ? 3 * resident : resident);
+                   : (NORMAL && units >= 128 * resident * (256 / 32) ? 3 * resident : resident);
     const int64_t warps_needed = units;
     grid = std::max<int64_t>(1, std::min<int64_t>(grid, ceil_div(warps_needed, 8)));
     if (launch_pdl(combine_vec_kernel<U, NORMAL>, dim3(unsigned(grid)), dim3(256), 0, stream, a) != cudaSuccess)
