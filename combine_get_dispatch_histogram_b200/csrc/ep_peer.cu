@@ -133,8 +133,8 @@ __device__ __forceinline__ PeerSlot peer_slot(const PeerArgs& a, const int32_t* 
 
 // ---------------------------------------------------------------------------- dispatch
 
-// Warps own contiguous, balanced ranges of units (token, piece of 32*U 16-byte
-// columns).  A lane loads its columns of the token row once and stores them to
+// Warps take units (token, piece of 32*U 16-byte columns) strided over the grid.
+// A lane loads its columns of the token row once and stores them to
 // every destination row; the row's (src_rank, src_token) goes to the
 // destination's src_info.  After its last store every thread fences at system
 // scope; the CTA that finishes last releases signal into every active
@@ -156,14 +156,15 @@ __global__ void __launch_bounds__(kPeerThreads) dispatch_peer_kernel(PeerArgs a)
     const int piece_vec = 32 * U;
     const int np = (nvec + piece_vec - 1) / piece_vec;
     const int64_t n_units = int64_t(a.T) * np;
-    const int64_t q = n_units / warps, rem = n_units % warps;
-    const int64_t u0 = gw * q + (gw < rem ? gw : rem);
-    const int64_t u1 = u0 + q + (gw < rem ? 1 : 0);
+    // units strided over the warps, so the grid works on one window of consecutive tokens at a time
+    // (the rows it writes to a busy expert are neighbours in its slab)
+    const int64_t my_n = gw < n_units ? (n_units - 1 - gw) / warps + 1 : 0;
 
     int64_t cur_tok = -1;
     uint32_t mask = 0;
     uint64_t my_addr = 0;
-    for (int64_t u = u0; u < u1; ++u) {
+    for (int64_t i = 0; i < my_n; ++i) {
+        const int64_t u = gw + i * warps;
         const int64_t t = u / np;
         const int pc = int(u - t * np);
         if (t != cur_tok) {
@@ -278,6 +279,8 @@ __global__ void __launch_bounds__(kPeerThreads, 2) combine_peer_kernel(PeerArgs 
     const int piece_vec = 32 * U;
     const int np = (nvec + piece_vec - 1) / piece_vec;
     const int64_t n_units = int64_t(a.T) * np;
+    // contiguous, balanced ranges of units per warp: on the emulated world this ran 963 us at
+    // prefill against 1144 us with units strided over the grid from the last token
     const int64_t q = n_units / warps, rem = n_units % warps;
     const int64_t u0 = gw * q + (gw < rem ? gw : rem);
     const int64_t u1 = u0 + q + (gw < rem ? 1 : 0);
