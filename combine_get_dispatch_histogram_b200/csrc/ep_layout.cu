@@ -78,7 +78,16 @@ constexpr int kMaxWarps = 16;
 constexpr int kBatch = 8;           // 32-pair steps whose loads are issued together
 constexpr int kActiveSlots = 64;    // shared copy of the active mask (EP_MAX_RANKS)
 constexpr int kMaxFlags = 255;      // >= kMaxChunks + EP_MAX_RANKS - 1
-constexpr size_t kSyncBytes = size_t(1 + kMaxFlags) * 8;  // epoch + flags, at offset 0 of the workspace
+constexpr int kFlagsPerLane = (kMaxFlags + 31) / 32;  // flags one lane of the look-back wait polls
+constexpr int kSumChunks = 8;  // chunk histograms a look-back warp loads at once (x 2 columns per lane)
+// Look-back flags sit kLookbackFlagWords words apart, one per 256 bytes: every CTA polls the
+// flags of the chunks before it, and packed into a few lines those polls queue behind each other.
+// (Fused-path flags are the first kMaxFlags words after the epoch; every flag word only ever holds
+// values of past epochs, below the current one, so the two paths can share the region.)
+constexpr int kLookbackFlagWords = 32;
+// epoch + flags, at offset 0 of the workspace; what follows starts on a 256-byte boundary
+constexpr size_t kSyncBytes = (size_t(1 + kMaxFlags * kLookbackFlagWords) * 8 + 255) / 256 * 256;
+static_assert(kSyncBytes % 16 == 0, "the chunk histograms after the flags are read 16 bytes at a time");
 
 struct LayoutArgs {
     const int32_t* topk_idx;
@@ -293,6 +302,29 @@ __device__ __forceinline__ void load_first_round(const LayoutArgs& a, const Warp
     }
 }
 
+// A token's destination-rank set (bit d = rank d, d < 8) spread to one byte per
+// rank: bytes 0-3 in the low word, 4-7 in the high word, each 0 or 1.
+__device__ __forceinline__ uint32_t rank_bytes_lo(uint32_t dst) { return ((dst & 0xFu) * 0x00204081u) & 0x01010101u; }
+__device__ __forceinline__ uint32_t rank_bytes_hi(uint32_t dst) {
+    return (((dst >> 4) & 0xFu) * 0x00204081u) & 0x01010101u;
+}
+
+// Adds a warp's per-lane byte counters of destination ranks (one byte per rank,
+// ranks 0-3 in lo, 4-7 in hi) to tpr_row[0..R).  Widened to 16-bit fields before
+// the warp sum: a lane counts at most kBatch tokens between two calls.
+__device__ __forceinline__ void flush_rank_counts(uint32_t lo, uint32_t hi, int R, int32_t* tpr_row) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t w0 = __reduce_add_sync(0xffffffffu, __byte_perm(lo, 0, 0x4140));  // ranks 0, 1
+    const uint32_t w1 = __reduce_add_sync(0xffffffffu, __byte_perm(lo, 0, 0x4342));  // ranks 2, 3
+    const uint32_t w2 = __reduce_add_sync(0xffffffffu, __byte_perm(hi, 0, 0x4140));  // ranks 4, 5
+    const uint32_t w3 = __reduce_add_sync(0xffffffffu, __byte_perm(hi, 0, 0x4342));  // ranks 6, 7
+    if (lane < R) {
+        const uint32_t wv = lane < 2 ? w0 : lane < 4 ? w1 : lane < 6 ? w2 : w3;
+        const int n = int((lane & 1) ? (wv >> 16) : (wv & 0xFFFFu));
+        if (n) atomicAdd(tpr_row + lane, n);
+    }
+}
+
 // One pass over the part.  A pair's row within the part is its expert's running
 // count in the warp's histogram `mine` plus the matching lanes below it (ballot
 // match); it stays in rk (the last round's pairs) or, for a part longer than one
@@ -301,6 +333,13 @@ __device__ __forceinline__ void load_first_round(const LayoutArgs& a, const Warp
 // per-destination token counts): with k a power of two a token's
 // k slots sit in k aligned lanes and an OR over them gives the set, otherwise one
 // token per lane re-reads its slots.  True if this lane saw an id outside [-1, E).
+//
+// The kernels that call this run it once per launch, so the 32-pair steps are a
+// rolled loop over one copy of the body (an unrolled copy per step runs from a
+// cold instruction cache): step u takes ev[0] and rotates ev/rk by one, which
+// after kBatch steps leaves both in their original order.  With R <= 8 a token's
+// ranks are written as one word of bytes and counted in per-lane byte counters,
+// summed over the warp once per round.
 __device__ __forceinline__ bool walk_part(const LayoutArgs& a, const WarpPart& w, const int32_t* act,
                                           const int32_t* rank_of, int32_t* mine, int32_t* tpr_row,
                                           int (&ev)[kBatch], int (&rk)[kBatch]) {
@@ -310,6 +349,10 @@ __device__ __forceinline__ bool walk_part(const LayoutArgs& a, const WarpPart& w
     int32_t* rows = a.pair_row + w.pbase;
     const uint32_t below = lanemask_lt();
     const bool lanes_per_token = (a.k & (a.k - 1)) == 0;  // k divides 32: a token is k aligned lanes
+    const bool packed = lanes_per_token && a.R <= 8;
+    // a token's row of is_token_in_rank as one store when R is 8 (or 4) and the buffer allows it
+    const uintptr_t itr_base = reinterpret_cast<uintptr_t>(a.is_token_in_rank);
+    const int itr_word = (a.R == 8 && (itr_base & 7u) == 0) ? 8 : (a.R == 4 && (itr_base & 3u) == 0) ? 4 : 0;
     bool bad = false;
     for (int p0 = 0; p0 < w.np; p0 += 32 * kBatch) {
         if (p0 > 0) {
@@ -319,35 +362,59 @@ __device__ __forceinline__ bool walk_part(const LayoutArgs& a, const WarpPart& w
                 ev[u] = p < w.np ? __ldg(base + p) : -1;
             }
         }
-#pragma unroll
+        uint32_t cnt_lo = 0, cnt_hi = 0;
+#pragma unroll 1
         for (int u = 0; u < kBatch; ++u) {
-            rk[u] = -1;
-            if (p0 + u * 32 >= w.np) break;  // the same for the whole warp
-            const int p = p0 + u * 32 + lane;
-            const int e = ev[u];
-            bad |= (e < -1 || e >= a.E);
-            const bool live = pair_live(e, a.E, src_ok, rank_of);
-            const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
-            const int32_t b = live ? mine[e] : 0;
-            __syncwarp();
-            if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
-            __syncwarp();
-            rk[u] = live ? b + __popc(m & below) : -1;
-            if (!w.one_round && p < w.np) rows[p] = rk[u];
-            if (lanes_per_token) {
-                uint32_t dst = live ? (1u << rank_of[e]) : 0u;
-                for (int o = 1; o < a.k; o <<= 1) dst |= __shfl_xor_sync(0xffffffffu, dst, o);
-                const bool head = p < w.np && (lane & (a.k - 1)) == 0;
-                if (head) {
+            const int e = ev[0];
+            int r = -1;
+            if (p0 + u * 32 < w.np) {  // the same for the whole warp
+                const int p = p0 + u * 32 + lane;
+                bad |= (e < -1 || e >= a.E);
+                const bool live = pair_live(e, a.E, src_ok, rank_of);
+                const uint32_t m = match_key(uint32_t(e), a.key_bits, __ballot_sync(0xffffffffu, live));
+                const int32_t b = live ? mine[e] : 0;
+                __syncwarp();
+                if (live && lane == __ffs(m) - 1) mine[e] = b + __popc(m);
+                __syncwarp();
+                r = live ? b + __popc(m & below) : -1;
+                if (!w.one_round && p < w.np) rows[p] = r;
+                if (lanes_per_token) {
+                    uint32_t dst = live ? (1u << rank_of[e]) : 0u;
+                    for (int o = 1; o < a.k; o <<= 1) dst |= __shfl_xor_sync(0xffffffffu, dst, o);
+                    const bool head = p < w.np && (lane & (a.k - 1)) == 0;
                     uint8_t* itr = a.is_token_in_rank + ((w.pbase + p) / a.k) * a.R;
-                    for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((dst >> d) & 1u);
-                }
-                for (int d = 0; d < a.R; ++d) {
-                    const int n = __popc(__ballot_sync(0xffffffffu, head && ((dst >> d) & 1u)));
-                    if (lane == 0 && n) atomicAdd(tpr_row + d, n);
+                    if (packed) {
+                        const uint32_t lo = rank_bytes_lo(dst), hi = rank_bytes_hi(dst);
+                        if (head) {
+                            if (itr_word == 8) {
+                                *reinterpret_cast<uint2*>(itr) = make_uint2(lo, hi);
+                            } else if (itr_word == 4) {
+                                *reinterpret_cast<uint32_t*>(itr) = lo;
+                            } else {
+                                for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((dst >> d) & 1u);
+                            }
+                            cnt_lo += lo;
+                            cnt_hi += hi;
+                        }
+                    } else {
+                        if (head)
+                            for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((dst >> d) & 1u);
+                        for (int d = 0; d < a.R; ++d) {
+                            const int n = __popc(__ballot_sync(0xffffffffu, head && ((dst >> d) & 1u)));
+                            if (lane == 0 && n) atomicAdd(tpr_row + d, n);
+                        }
+                    }
                 }
             }
+#pragma unroll
+            for (int i = 0; i < kBatch - 1; ++i) {
+                ev[i] = ev[i + 1];
+                rk[i] = rk[i + 1];
+            }
+            ev[kBatch - 1] = e;
+            rk[kBatch - 1] = r;
         }
+        if (packed) flush_rank_counts(cnt_lo, cnt_hi, a.R, tpr_row);
     }
     if (!lanes_per_token) {
         for (int t0 = w.t0; t0 < w.t1; t0 += 32) {
@@ -860,9 +927,10 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_fused_kernel(LayoutArgs
 //      ranks, per-destination token counts), writes the chunk histogram and
 //      publishes it with a release flag;
 //   B. waits (bounded) for the flags of the chunks before it only -- CTAs are
-//      dispatched in index order, so those have started -- and sums their
-//      histograms, each warp a stripe of them with 16-byte loads all in flight,
-//      the warps' sums added up in shared memory;
+//      dispatched in index order, so those have started; one warp polls them
+//      all, each lane its up to eight flags per round trip -- then sums their
+//      histograms: warp w takes chunks w, w + W, ... with all its 16-byte
+//      loads in flight, and the warps' sums meet in shared memory;
 //   C. assigns rows as the rank kernel does.
 // The owners of the per-rank outputs are the chunks that can see them: the
 // first chunk of rank r writes expert_rank_offset[:, r], the last chunk of rank
@@ -874,7 +942,6 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_lookback_kernel(LayoutA
     pdl_wait();  // nothing upstream is read before this
     pdl_launch_dependents();
     extern __shared__ int32_t smem[];
-    __shared__ int passed;
     const int NT = blockDim.x;
     const int W = NT >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int32_t* act = smem;
@@ -883,14 +950,6 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_lookback_kernel(LayoutA
     int32_t* first = rank_of + a.E;       // [E] rows of the chunks before this one
     int32_t* rank_first = first + a.E;    // [E] rows of the chunks of the ranks before this chunk's rank
     int32_t* whist = rank_first + a.E;    // [W][E]
-    const uint64_t epoch = *reinterpret_cast<volatile uint64_t*>(a.sync);
-    uint64_t* flags = a.sync + 1;
-    const uint64_t value = 2 * (epoch + 1);
-    load_tables(a, act, rank_of);
-    for (int i = threadIdx.x; i < W * a.E; i += NT) whist[i] = 0;
-    for (int e = threadIdx.x; e < a.E; e += NT) first[e] = rank_first[e] = 0;
-    for (int d = threadIdx.x; d < a.R; d += NT) tpr[d] = 0;
-    __syncthreads();
 
     const int g = blockIdx.x;
     const ChunkGeom cg = chunk_of(a, g);
@@ -904,9 +963,18 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_lookback_kernel(LayoutA
     w.pbase = (int64_t(cg.r) * a.T + w.t0) * a.k;
     w.np = (w.t1 - w.t0) * a.k;
     w.one_round = w.np <= 32 * kBatch;
-    int32_t* mine = whist + warp * a.E;
     int ev[kBatch], rk[kBatch];
-    load_first_round(a, w, ev);
+    load_first_round(a, w, ev);  // in flight while the tables are set up
+
+    const uint64_t epoch = *reinterpret_cast<volatile uint64_t*>(a.sync);
+    uint64_t* flags = a.sync + 1;
+    const uint64_t value = 2 * (epoch + 1);
+    load_tables(a, act, rank_of);
+    for (int i = threadIdx.x; i < W * a.E; i += NT) whist[i] = 0;
+    for (int e = threadIdx.x; e < a.E; e += NT) first[e] = rank_first[e] = 0;
+    for (int d = threadIdx.x; d < a.R; d += NT) tpr[d] = 0;
+    __syncthreads();
+    int32_t* mine = whist + warp * a.E;
 
     // ---- A: warp histograms and rows within the parts, destination ranks, chunk histogram, publish
     const bool bad = walk_part(a, w, act, rank_of, mine, tpr, ev, rk);
@@ -918,27 +986,33 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_lookback_kernel(LayoutA
         own[e] = s;
     }
     for (int d = threadIdx.x; d < a.R; d += NT) a.chunk_tpr[int64_t(g) * a.R + d] = tpr[d];
+    // the barrier orders every thread's writes of the chunk before thread 0's release (the release
+    // is cumulative), so the flag needs no further fence
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        st_release_u64(flags + g, value);
-    }
+    if (threadIdx.x == 0) st_release_u64(flags + int64_t(g) * kLookbackFlagWords, value);
 
-    // ---- B: wait for the chunks before this one (bounded), then sum their histograms
+    // ---- B: wait (bounded) for the chunks before this one, then sum their histograms
+    __shared__ int passed;
     if (warp == 0) {
         bool ok = true;
         const uint64_t t0 = global_timer_ns();
-        for (int b = 0; b < g && ok; b += 32) {
-            const int gg = b + lane;
-            for (uint32_t it = 0;; ++it) {
-                const bool here = gg >= g || ld_acquire_u64(flags + gg) >= value;
-                if (__all_sync(0xffffffffu, here)) break;
-                if ((it & 63u) == 63u && __any_sync(0xffffffffu, global_timer_ns() - t0 > kWaitTimeoutNs)) {
-                    ok = false;
-                    break;
-                }
+        uint32_t need = 0;  // bit q: chunk lane + 32 q is before this one and not yet seen published
+#pragma unroll
+        for (int q = 0; q < kFlagsPerLane; ++q) need |= uint32_t(lane + 32 * q < g) << q;
+        for (uint32_t it = 0;; ++it) {
+            uint64_t seen[kFlagsPerLane];
+#pragma unroll
+            for (int q = 0; q < kFlagsPerLane; ++q)
+                seen[q] = (need >> q) & 1u ? ld_acquire_u64(flags + int64_t(lane + 32 * q) * kLookbackFlagWords)
+                                           : value;
+#pragma unroll
+            for (int q = 0; q < kFlagsPerLane; ++q)
+                if (seen[q] >= value) need &= ~(1u << q);
+            if (__all_sync(0xffffffffu, need == 0)) break;
+            if ((it & 63u) == 63u && __any_sync(0xffffffffu, global_timer_ns() - t0 > kWaitTimeoutNs)) {
+                ok = false;
+                break;
             }
-            ok = __all_sync(0xffffffffu, ok);
         }
         if (lane == 0) passed = ok;
     }
@@ -950,50 +1024,61 @@ __global__ void __launch_bounds__(32 * kMaxWarps) layout_lookback_kernel(LayoutA
         return;
     }
     const int rC = cg.r * a.C;  // first chunk of this chunk's rank
-    // warp w sums chunks w, w + W, ... below g (16-byte loads of four experts when E % 4 == 0, so a
-    // lane's loads of all its chunks are in flight together), split at rC into the ranks before this
-    // chunk's rank and this rank's earlier chunks; the warps' partial sums meet in shared memory
-    if ((a.E & 3) == 0) {
-        const int E4 = a.E >> 2;
-        for (int e4 = lane; e4 < E4; e4 += 32) {
-            int4 sb = make_int4(0, 0, 0, 0), sr = sb;
-            int gg = warp;
-            for (; gg + 7 * W < g; gg += 8 * W) {
-                int4 v[8];
+    {
+        // split at rC into the ranks before this chunk's rank and this rank's earlier chunks.  When
+        // E % 4 == 0: warp w takes chunks w, w + W, ...; lane l the 16-byte columns (four experts)
+        // l, l + 32, ... of each, kSumChunks chunks by two columns of loads in flight per lane; the
+        // warps' sums meet in shared memory.
+        if ((a.E & 3) == 0) {
+            const int E4 = a.E >> 2;
+            for (int c0 = lane; c0 < E4; c0 += 64) {
+                const int c1 = c0 + 32;
+                int4 sb0 = make_int4(0, 0, 0, 0), sr0 = sb0, sb1 = sb0, sr1 = sb0;
+                for (int gg = warp; gg < g; gg += kSumChunks * W) {
+                    int4 v0[kSumChunks], v1[kSumChunks];
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    v[u] = reinterpret_cast<const int4*>(a.chunk_hist + int64_t(gg + u * W) * a.E)[e4];
+                    for (int u = 0; u < kSumChunks; ++u) {
+                        const int gu = gg + u * W;
+                        const int4* row = reinterpret_cast<const int4*>(a.chunk_hist + int64_t(gu) * a.E);
+                        v0[u] = gu < g ? row[c0] : make_int4(0, 0, 0, 0);
+                        v1[u] = (gu < g && c1 < E4) ? row[c1] : make_int4(0, 0, 0, 0);
+                    }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    int4& acc = gg + u * W < rC ? sb : sr;
-                    acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+                    for (int u = 0; u < kSumChunks; ++u) {
+                        const bool before = gg + u * W < rC;
+                        int4& a0 = before ? sb0 : sr0;
+                        int4& a1 = before ? sb1 : sr1;
+                        a0.x += v0[u].x; a0.y += v0[u].y; a0.z += v0[u].z; a0.w += v0[u].w;
+                        a1.x += v1[u].x; a1.y += v1[u].y; a1.z += v1[u].z; a1.w += v1[u].w;
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int c = h ? c1 : c0;
+                    if (c >= E4) break;
+                    const int4 sb = h ? sb1 : sb0, sr = h ? sr1 : sr0;
+                    const int e = 4 * c;
+                    if (sb.x | sb.y | sb.z | sb.w) {
+                        atomicAdd(rank_first + e, sb.x); atomicAdd(rank_first + e + 1, sb.y);
+                        atomicAdd(rank_first + e + 2, sb.z); atomicAdd(rank_first + e + 3, sb.w);
+                    }
+                    if (sb.x | sb.y | sb.z | sb.w | sr.x | sr.y | sr.z | sr.w) {
+                        atomicAdd(first + e, sb.x + sr.x); atomicAdd(first + e + 1, sb.y + sr.y);
+                        atomicAdd(first + e + 2, sb.z + sr.z); atomicAdd(first + e + 3, sb.w + sr.w);
+                    }
                 }
             }
-            for (; gg < g; gg += W) {
-                const int4 v = reinterpret_cast<const int4*>(a.chunk_hist + int64_t(gg) * a.E)[e4];
-                int4& acc = gg < rC ? sb : sr;
-                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        } else {
+            for (int e = lane; e < a.E; e += 32) {
+                int32_t sb = 0, sr = 0;
+                for (int gg = warp; gg < g; gg += W) {
+                    const int32_t v = a.chunk_hist[int64_t(gg) * a.E + e];
+                    if (gg < rC) sb += v;
+                    else sr += v;
+                }
+                if (sb) atomicAdd(rank_first + e, sb);
+                if (sb | sr) atomicAdd(first + e, sb + sr);
             }
-            const int e = 4 * e4;
-            if (sb.x | sb.y | sb.z | sb.w) {
-                atomicAdd(rank_first + e, sb.x); atomicAdd(rank_first + e + 1, sb.y);
-                atomicAdd(rank_first + e + 2, sb.z); atomicAdd(rank_first + e + 3, sb.w);
-            }
-            if (sb.x | sb.y | sb.z | sb.w | sr.x | sr.y | sr.z | sr.w) {
-                atomicAdd(first + e, sb.x + sr.x); atomicAdd(first + e + 1, sb.y + sr.y);
-                atomicAdd(first + e + 2, sb.z + sr.z); atomicAdd(first + e + 3, sb.w + sr.w);
-            }
-        }
-    } else {
-        for (int e = lane; e < a.E; e += 32) {
-            int32_t sb = 0, sr = 0;
-            for (int gg = warp; gg < g; gg += W) {
-                const int32_t v = a.chunk_hist[int64_t(gg) * a.E + e];
-                if (gg < rC) sb += v;
-                else sr += v;
-            }
-            if (sb) atomicAdd(rank_first + e, sb);
-            if (sb | sr) atomicAdd(first + e, sb + sr);
         }
     }
     __syncthreads();

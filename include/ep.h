@@ -245,7 +245,7 @@ EP_API int ep_topk_idx_to_int32(const int64_t *topk_idx64, int32_t *topk_idx32, 
  *   workspace             >= ep_layout_workspace_bytes(d) bytes, 16-byte aligned,
  *                         owned by the caller.  Zero-fill it once before its first
  *                         use (e.g. cudaMemset) and keep it for ep_layout calls
- *                         only: its first 2 KiB carry barrier state from call to
+ *                         only: its first 64 KiB carry barrier state from call to
  *                         call (cf. Buffer.clean_low_latency_buffer on the NeMo
  *                         page); the rest is scratch.  Calls sharing a workspace
  *                         must be ordered on the GPU.

@@ -52,13 +52,14 @@ def test_error_names_and_version(lib):
 def test_workspace_sizes(lib):
     from combine_get_dispatch_histogram_b200 import ep
 
-    # 2 KiB of barrier state, then per chunk E + R ints; chunks: one per 2048 pairs, at least 32
-    # and at most 148 in all, a whole number per rank.  8 ranks x 4096 tokens x top-8: 128 chunks.
-    sync = 2048
+    # 64 KiB of barrier state (the epoch and up to 255 chunk flags, one per 256 bytes), then per
+    # chunk E + R ints; chunks: one per 2048 pairs, at least 32 and at most 148 in all, a whole
+    # number per rank.  8 ranks x 4096 tokens x top-8: 128 chunks.
+    sync = 65536
     assert ep.ep_layout_workspace_bytes(8, 4096, 8, 256, 7168) == sync + 128 * 256 * 4 + 128 * 8 * 4
     assert ep.ep_layout_workspace_bytes(8, 65536, 8, 256, 7168) == sync + 152 * 256 * 4 + 152 * 8 * 4
     assert ep.ep_layout_workspace_bytes(8, 128, 8, 256, 7168) == sync + 32 * 256 * 4 + 32 * 8 * 4
-    assert 2048 < ep.ep_layout_workspace_bytes(2, 0, 2, 8, 256) <= 2048 + 256   # one empty chunk per rank
+    assert sync < ep.ep_layout_workspace_bytes(2, 0, 2, 8, 256) <= sync + 256   # one empty chunk per rank
     assert ep.ep_layout_workspace_bytes(3, 4, 2, 8, 256) == 0        # E % R != 0 is invalid
     assert ep.ep_reroute_workspace_bytes(8, 2048, 6, 64) % 16 == 0
 
