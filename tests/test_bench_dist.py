@@ -94,3 +94,19 @@ def test_kernel_time_statistics():
 
     st = bench.stats_ms([3.0, 1.0, 2.0, 10.0, 2.5])
     assert st == {"median": 2.5, "min": 1.0, "max": 10.0}
+
+
+def test_l2_flush_only_for_steps_whose_rows_could_stay_cached():
+    """Prefill's token rows (470 MB) outgrow L2 and go unflushed; decode (15 MB), the sweeps and the
+    replica workload (134 MB) write a buffer larger than L2 before each timed step, and say so."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from combine_get_dispatch_histogram_b200 import inputs
+
+    assert bench.L2_FLUSH_BYTES > bench.L2_BYTES
+    assert not bench.needs_l2_flush(inputs.named("prefill"))
+    assert bench.config_of(inputs.named("prefill"), 1)["l2"].startswith("no flush")
+    for name in ("tiny", "decode", "sweep_T16", "sweep_T512", "sweep_T64_mask5", "replica"):
+        w = inputs.named(name)
+        assert bench.needs_l2_flush(w), name
+        assert bench.config_of(w, 1)["l2"].startswith("flushed"), name
