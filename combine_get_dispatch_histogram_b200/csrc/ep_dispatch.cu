@@ -47,12 +47,14 @@ constexpr int kDispatchMaxStages = 16;
 constexpr uint64_t kPacePeriodNs = 40000;
 constexpr uint64_t kPaceWindowNs = 6000;
 constexpr int64_t kPaceAheadBytes = 300 * 1024;
-// AUTO paces a low-latency dispatch only where it measured faster on B200: rows whose k stores
-// add up to >= 96 KB (so a 14-row ring holds about one read period of stores) and >= 16 rows per
-// SM.  Prefill (k = 8, 14 KB rows): 670 against 770 us; 8 x 512 tokens: 89.6 against 96.2 us.
-// It lost where the stores per row are smaller: the replica workload (k = 6, 8 KB rows) 255
-// against 172 us, normal mode (one row per destination rank) 849 against 455 us.
-constexpr int kPaceMinUnitsPerCta = 16;
+// AUTO paces a low-latency dispatch only where it measured faster on B200 (L2 flushed before each
+// call): rows whose k stores add up to >= 96 KB (so a 14-row ring holds about one read period of
+// stores) and >= 32 rows per SM.  k = 8, 14 KB rows, 8 ranks: T = 4096 672 against 767 us, 2048
+// 345 against 387, 1024 180 against 192, 640 (35 rows per SM) 121 against 129; T = 512 (28 rows
+// per SM) 98 against 94 and T = 256 57 against 51.  It lost where the stores per row are smaller: the replica workload
+// (k = 6, 8 KB rows) 255 against 172 us, normal mode (one row per destination rank) 849 against
+// 455 us.
+constexpr int kPaceMinUnitsPerCta = 32;
 constexpr int64_t kPaceMinStoreBytesPerRow = 96 * 1024;
 
 struct DispatchArgs {

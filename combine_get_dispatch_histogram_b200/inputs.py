@@ -126,6 +126,10 @@ def named(name: str) -> Workload:
         rest = name[len("sweep_T"):]
         masked = rest.endswith("_mask5")
         return sweep(int(rest.replace("_mask5", "")), masked)
+    if name.startswith("prefill_T"):
+        return prefill(int(name[len("prefill_T"):]))
+    if name.startswith("replica_T"):
+        return replica(int(name[len("replica_T"):]))
     raise KeyError(name)
 
 

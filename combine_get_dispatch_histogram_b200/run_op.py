@@ -30,6 +30,8 @@ def main():
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--graph", action="store_true", help="time CUDA-graph replays of the calls")
+    ap.add_argument("--flush", action="store_true",
+                    help="write 256 MB before every call, outside its event pair, and report the median call")
     ap.add_argument("--variant", type=int, default=0, help="ep_cfg_t.variant of dispatch / combine")
     ap.add_argument("--max-ctas", type=int, default=0, help="ep_cfg_t.max_ctas of dispatch / combine")
     ap.add_argument("--threads", type=int, default=0, help="ep_cfg_t.threads of dispatch / combine")
@@ -168,18 +170,33 @@ def main():
         with torch.cuda.graph(graph, stream=stream):
             run_all()
         torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(args.iters):
-            if graph is not None:
-                graph.replay()
-            else:
-                run_all()
-        e1.record(stream)
-    stream.synchronize()
-    us = e0.elapsed_time(e1) * 1e3 / args.iters
+    def one():
+        if graph is not None:
+            graph.replay()
+        else:
+            run_all()
+
+    if args.flush:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.iters)]
+        with torch.cuda.stream(stream):
+            for e0, e1 in evs:
+                flush.zero_()
+                e0.record(stream)
+                one()
+                e1.record(stream)
+        stream.synchronize()
+        us = float(np.median([e0.elapsed_time(e1) for e0, e1 in evs])) * 1e3
+    else:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.iters):
+                one()
+            e1.record(stream)
+        stream.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / args.iters
     live = int(lay.recv_count.sum().item())
     sent = int(lay.is_token_in_rank.view(R * T, R).amax(dim=1).sum().item())
     per_pair = {"dispatch": 2 * H, "combine": 2 * H,
@@ -201,6 +218,7 @@ def main():
     elif args.op == "combine":
         algo = 2 * H * (live + R * T)
     print(json.dumps({"op": args.op, "workload": w.name, "us_per_call": round(us, 2), "graph": args.graph,
+                      "flush": args.flush, "max_ctas": args.max_ctas, "threads": args.threads,
                       "algorithmic_bytes": algo, "gbs": round(algo / us / 1e3, 1) if algo else None,
                       "variant": args.variant, "layout_variant": args.layout_variant, "status": int(status.item())}))
 

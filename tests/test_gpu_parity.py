@@ -580,7 +580,8 @@ def test_cumulative_receive_stats_over_calls():
 def test_dispatch_path_choice():
     """AUTO paces the dispatch only where a row's k stores add up to >= 96 KB with >= 16 rows per SM."""
     assert ep.ep_dispatch_path(8, 4096, 8, 256, 7168) == ep.EP_VARIANT_PACED     # prefill
-    assert ep.ep_dispatch_path(8, 512, 8, 256, 7168) == ep.EP_VARIANT_PACED      # 27 rows per SM
+    assert ep.ep_dispatch_path(8, 1024, 8, 256, 7168) == ep.EP_VARIANT_PACED     # 55 rows per SM
+    assert ep.ep_dispatch_path(8, 512, 8, 256, 7168) == ep.EP_VARIANT_BULK       # 28 rows per SM
     assert ep.ep_dispatch_path(8, 128, 8, 256, 7168) == ep.EP_VARIANT_BULK       # decode: 7 rows per SM
     assert ep.ep_dispatch_path(8, 2048, 6, 80, 4096) == ep.EP_VARIANT_BULK       # replica: 48 KB per row
     assert ep.ep_dispatch_path(8, 128, 8, 256, 7168, cfg=dict(variant=2)) == ep.EP_VARIANT_VECTOR
