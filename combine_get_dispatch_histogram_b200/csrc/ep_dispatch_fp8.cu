@@ -399,30 +399,153 @@ cudaError_t launch_fp8_bulk(const DispatchFp8Args& a, int64_t grid, int consumer
     return launch_pdl(dispatch_fp8_bulk_kernel<FMT>, dim3(unsigned(grid)), dim3(32 * (1 + consumers)), smem, stream, a);
 }
 
-// Column-major scales: block (x, e) covers slab rows [x*256, x*256 + 256) of expert e;
-// a thread owns one valid row, finds its token in src_info and copies that
-// token's scale words, so for each word the block's stores are contiguous.
-__global__ void __launch_bounds__(256) fp8_scale_writer_kernel(DispatchFp8Args a) {
+// Column-major scales: one 256-thread block per chunk of 256 slab rows of an
+// expert; thread t owns the chunk's row t, finds its token in src_info and
+// writes that token's scale words, so for each word the block's stores are
+// contiguous.  With rows of at least kStageMinWords words (fp32 or power-of-two
+// scales) the block first stages the chunk's tokens' scale rows in shared memory
+// -- half-warps read whole rows, 16 bytes a lane where the rows allow it, all of
+// a half-warp's rows in flight at once -- because each thread reading its own
+// 224-byte row from global memory touched 32 rows per load and thrashed L1 (52
+// against 34 us at prefill); shorter rows (UE8M0) are copied by each thread
+// directly, kScaleBatch loads in flight before their stores (staging measured
+// slower there: three barriers per chunk for a 56-byte row).
+// A fixed grid of G blocks walks the non-empty chunks, numbered expert by expert
+// (a prefix of the per-expert chunk counts, scanned in shared memory): block b
+// takes chunks b, b + G, ...  (One block per possible chunk, (R*T/256) x E, was
+// mostly blocks with no rows: 26 us at prefill for 15 MB of UE8M0 words.)
+constexpr int kScaleRows = 256;               // rows per chunk = threads per block
+constexpr int kStageRows = kScaleRows / 16;   // rows each half-warp stages
+constexpr int kStageMinWords = 32;            // rows this long or longer are staged
+constexpr int kScaleBatch = 16;               // words a thread loads before storing them (direct copy)
+
+// Shared-memory words of a staged scale row: odd, so thread t reading word w of row t hits bank
+// (t * stride + w) mod 32, a different bank for every lane.
+__host__ __device__ __forceinline__ int scale_row_stride(int words) { return words | 1; }
+
+size_t scale_writer_smem_bytes(int num_experts, int words, bool staged) {
+    return size_t(num_experts + 1) * 4 + 32 * 4 +
+           (staged ? size_t(kScaleRows) * 8 + size_t(kScaleRows) * scale_row_stride(words) * 4 : 0);
+}
+
+template <bool STAGED>
+__global__ void __launch_bounds__(kScaleRows) fp8_scale_writer_kernel(DispatchFp8Args a) {
     pdl_wait();  // nothing upstream is read before this
     // no early trigger: a streaming grid lets its dependent launch only as it exits
-    const int e = blockIdx.y;
-    const int64_t n = a.recv_count[e] < a.cap ? int64_t(a.recv_count[e]) : a.cap;
-    const int64_t row = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (int64_t(blockIdx.x) * blockDim.x >= n) return;
-    const bool ok = row < n;
-    const uint32_t* ts = nullptr;
-    bool ok_src = false;
-    if (ok) {
-        const int2 src = reinterpret_cast<const int2*>(a.src_info)[int64_t(e) * a.cap + row];
-        const int64_t tok = int64_t(src.x) * a.T + src.y;
-        // a recv_count that does not belong to this dispatch could point at a stale row
-        ok_src = src.y >= 0 && src.y < a.T && tok >= 0 && tok < a.n_tok;
-        if (ok_src) ts = a.tok_scales + tok * a.words;
-        else flag_status(a.status, EP_STATUS_BAD_EXPERT);
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    int64_t* tok_of = reinterpret_cast<int64_t*>(smem_raw);                    // [kScaleRows], -1: no row
+    uint32_t* staged = reinterpret_cast<uint32_t*>(tok_of + kScaleRows);       // [kScaleRows][stride]
+    const int stride = scale_row_stride(a.words);
+    // [E + 1] first chunk number of each expert, then [32] the warps' sums of the scan
+    int32_t* first_chunk = STAGED ? reinterpret_cast<int32_t*>(staged + kScaleRows * stride)
+                                  : reinterpret_cast<int32_t*>(smem_raw);
+    int32_t* warp_sums = first_chunk + a.E + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // chunks per expert, scanned: thread t sums the experts [t*per, (t+1)*per), a scan over the
+    // threads (warp shuffles, then the warps' sums), and each thread writes its experts' prefixes
+    const int per = (a.E + kScaleRows - 1) / kScaleRows;
+    const int e_begin = min(a.E, int(threadIdx.x) * per), e_end = min(a.E, e_begin + per);
+    auto chunks_of = [&](int e) {
+        const int64_t n = a.recv_count[e] < a.cap ? int64_t(a.recv_count[e]) : a.cap;
+        return n > 0 ? int32_t((n + kScaleRows - 1) / kScaleRows) : 0;
+    };
+    int32_t mine = 0;
+    for (int e = e_begin; e < e_end; ++e) mine += chunks_of(e);
+    int32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
     }
-    uint32_t* out = reinterpret_cast<uint32_t*>(a.scales) + int64_t(e) * a.words * a.cap + row;
-    for (int wd = 0; wd < a.words; ++wd)
-        if (ok_src) out[int64_t(wd) * a.cap] = ts[wd];
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int32_t before = 0;
+    for (int w = 0; w < warp; ++w) before += warp_sums[w];
+    int32_t run = before + incl - mine;
+    for (int e = e_begin; e < e_end; ++e) {
+        first_chunk[e] = run;
+        run += chunks_of(e);
+    }
+    if (threadIdx.x == blockDim.x - 1) first_chunk[a.E] = run;
+    __syncthreads();
+    const int32_t total = first_chunk[a.E];
+
+    for (int32_t id = int32_t(blockIdx.x); id < total; id += int32_t(gridDim.x)) {
+        // the expert of chunk id: the last e with first_chunk[e] <= id
+        int lo = 0, hi = a.E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (first_chunk[mid] <= id) lo = mid;
+            else hi = mid - 1;
+        }
+        const int e = lo;
+        const int64_t n = a.recv_count[e] < a.cap ? int64_t(a.recv_count[e]) : a.cap;
+        const int64_t row = int64_t(id - first_chunk[e]) * kScaleRows + threadIdx.x;
+        int64_t tok = -1;
+        if (row < n) {
+            const int2 src = reinterpret_cast<const int2*>(a.src_info)[int64_t(e) * a.cap + row];
+            tok = int64_t(src.x) * a.T + src.y;
+            // a recv_count that does not belong to this dispatch could point at a stale row
+            if (!(src.y >= 0 && src.y < a.T && tok >= 0 && tok < a.n_tok)) {
+                flag_status(a.status, EP_STATUS_BAD_EXPERT);
+                tok = -1;
+            }
+        }
+        if (!STAGED) {
+            if (tok < 0) continue;
+            const uint32_t* ts = a.tok_scales + tok * a.words;
+            uint32_t* out = reinterpret_cast<uint32_t*>(a.scales) + int64_t(e) * a.words * a.cap + row;
+            for (int w0 = 0; w0 < a.words; w0 += kScaleBatch) {
+                uint32_t v[kScaleBatch];
+#pragma unroll
+                for (int jj = 0; jj < kScaleBatch; ++jj) v[jj] = w0 + jj < a.words ? __ldg(ts + w0 + jj) : 0u;
+#pragma unroll
+                for (int jj = 0; jj < kScaleBatch; ++jj)
+                    if (w0 + jj < a.words) out[int64_t(w0 + jj) * a.cap] = v[jj];
+            }
+            continue;
+        }
+        tok_of[threadIdx.x] = tok;
+        __syncthreads();
+        // stage: half-warp h copies the scale rows of the chunk's rows h, h + 16, ..., all of its
+        // kStageRows loads in flight before the shared-memory stores
+        const int half = threadIdx.x >> 4, hl = threadIdx.x & 15;
+        if ((a.words & 3) == 0 && (reinterpret_cast<uintptr_t>(a.tok_scales) & 15u) == 0) {
+            for (int q = hl; q < (a.words >> 2); q += 16) {
+                uint4 v[kStageRows];
+#pragma unroll
+                for (int rr = 0; rr < kStageRows; ++rr) {
+                    const int64_t tr = tok_of[half + 16 * rr];
+                    v[rr] = tr >= 0 ? __ldg(reinterpret_cast<const uint4*>(a.tok_scales + tr * a.words) + q)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int rr = 0; rr < kStageRows; ++rr) {
+                    uint32_t* dst = staged + (half + 16 * rr) * stride + 4 * q;
+                    dst[0] = v[rr].x; dst[1] = v[rr].y; dst[2] = v[rr].z; dst[3] = v[rr].w;
+                }
+            }
+        } else {
+            for (int q = hl; q < a.words; q += 16) {
+                uint32_t v[kStageRows];
+#pragma unroll
+                for (int rr = 0; rr < kStageRows; ++rr) {
+                    const int64_t tr = tok_of[half + 16 * rr];
+                    v[rr] = tr >= 0 ? __ldg(a.tok_scales + tr * a.words + q) : 0u;
+                }
+#pragma unroll
+                for (int rr = 0; rr < kStageRows; ++rr) staged[(half + 16 * rr) * stride + q] = v[rr];
+            }
+        }
+        __syncthreads();
+        if (tok >= 0) {
+            uint32_t* out = reinterpret_cast<uint32_t*>(a.scales) + int64_t(e) * a.words * a.cap + row;
+            const uint32_t* src_row = staged + threadIdx.x * stride;
+            for (int wd = 0; wd < a.words; ++wd) out[int64_t(wd) * a.cap] = src_row[wd];
+        }
+        __syncthreads();  // the staged rows are reused by the next chunk
+    }
 }
 
 }  // namespace
@@ -536,9 +659,19 @@ extern "C" int ep_dispatch_fp8(ep_dims_t d, const uint16_t* x, const int32_t* to
         }
     }
     if (lerr != cudaSuccess) return EP_ERR_CUDA;
-    if (ceil_div(RT, 256) > 65535 * 256LL || d.num_experts > 65535) return EP_ERR_UNSUPPORTED;
-    if (launch_pdl(fp8_scale_writer_kernel, dim3(unsigned(ceil_div(RT, 256)), unsigned(d.num_experts)), dim3(256), 0, st,
-                   a) != cudaSuccess)
+    // the scale writer: a fixed grid (three blocks per SM when staging, eight otherwise); the experts'
+    // row counts, and the staged tokens and rows, in shared memory
+    const bool staged = a.words >= kStageMinWords;
+    const size_t writer_smem = scale_writer_smem_bytes(d.num_experts, a.words, staged);
+    if (writer_smem > size_t(max_smem_optin())) return EP_ERR_UNSUPPORTED;
+    auto writer = staged ? fp8_scale_writer_kernel<true> : fp8_scale_writer_kernel<false>;
+    if (writer_smem > 48 * 1024 &&
+        cudaFuncSetAttribute(writer, cudaFuncAttributeMaxDynamicSharedMemorySize, int(writer_smem)) != cudaSuccess)
+        return EP_ERR_CUDA;
+    const int64_t chunks = ceil_div(RT, kScaleRows) + d.num_experts;  // an upper bound on non-empty chunks
+    const unsigned writer_grid =
+        unsigned(std::max<int64_t>(1, std::min<int64_t>(int64_t(sms) * (staged ? 3 : 8), chunks)));
+    if (launch_pdl(writer, dim3(writer_grid), dim3(kScaleRows), writer_smem, st, a) != cudaSuccess)
         return EP_ERR_CUDA;
     return launch_result();
 }
