@@ -48,14 +48,20 @@ constexpr uint64_t kPacePeriodNs = 40000;
 constexpr uint64_t kPaceWindowNs = 6000;
 constexpr int64_t kPaceAheadBytes = 300 * 1024;
 // AUTO paces a low-latency dispatch only where it measured faster on B200 (L2 flushed before each
-// call): rows whose k stores add up to >= 96 KB (so a 14-row ring holds about one read period of
-// stores) and >= 32 rows per SM.  k = 8, 14 KB rows, 8 ranks: T = 4096 672 against 767 us, 2048
-// 345 against 387, 1024 180 against 192, 640 (35 rows per SM) 121 against 129; T = 512 (28 rows
-// per SM) 98 against 94 and T = 256 57 against 51.  It lost where the stores per row are smaller: the replica workload
-// (k = 6, 8 KB rows) 255 against 172 us, normal mode (one row per destination rank) 849 against
-// 455 us.
+// call): >= 32 rows per SM and rows whose k stores add up to >= 48 KB.  With >= 96 KB per row one
+// CTA per SM runs a 14-row ring (about one read period of stores); k = 8, 14 KB rows, 8 ranks:
+// T = 4096 672 against 767 us, 2048 345 against 387, 1024 180 against 192, 640 (35 rows per SM)
+// 121 against 129; T = 512 (28 rows per SM) 98 against 94 and T = 256 57 against 51.  Between 48
+// and 96 KB per row (the replica workload: k = 6, 8 KB rows) two CTAs per SM share the schedule
+// from 96 rows per SM on: 8 x 2048 tokens 166 against 176 us unpaced (167 against 169 on another
+// box), 8 x 4096 324 against 340, but 8 x 1024 (55 rows per SM) 88 against 84.  One ring per SM
+// took 253 us there (its one issuing warp cannot keep up with 8 KB copies) and three 184 us; the
+// read period and window made no difference.
+// Normal mode (one row per destination rank) is never paced by AUTO: 849 against 455 us.
 constexpr int kPaceMinUnitsPerCta = 32;
-constexpr int64_t kPaceMinStoreBytesPerRow = 96 * 1024;
+constexpr int kPaceTwoRingMinUnitsPerSm = 96;
+constexpr int64_t kPaceMinStoreBytesPerRow = 48 * 1024;
+constexpr int64_t kPaceOneRingStoreBytesPerRow = 96 * 1024;
 
 struct DispatchArgs {
     const uint8_t* x;
@@ -411,8 +417,14 @@ int fill_dispatch_args(DispatchArgs& a, const ep_dims_t& d, const uint16_t* x, c
 
 // AUTO's choice for a low-latency dispatch (see kPaceMinStoreBytesPerRow).
 bool paced_by_default(const DispatchArgs& a, int sms) {
-    return a.n_pieces == 1 && a.n_units >= int64_t(kPaceMinUnitsPerCta) * sms &&
-           int64_t(a.k) * a.row_bytes >= kPaceMinStoreBytesPerRow;
+    const int64_t stores = int64_t(a.k) * a.row_bytes;
+    const int64_t min_units = stores >= kPaceOneRingStoreBytesPerRow ? kPaceMinUnitsPerCta : kPaceTwoRingMinUnitsPerSm;
+    return a.n_pieces == 1 && stores >= kPaceMinStoreBytesPerRow && a.n_units >= min_units * sms;
+}
+
+// CTAs per SM of a paced dispatch: one deep ring where a row's stores add up to >= 96 KB, else two.
+int paced_ctas_per_sm(const DispatchArgs& a) {
+    return int64_t(a.k) * a.row_bytes >= kPaceOneRingStoreBytesPerRow ? 1 : 2;
 }
 
 // Grid, stages and (for the paced path) the read schedule, then the bulk-path launch.  `prefetch`
@@ -420,9 +432,9 @@ bool paced_by_default(const DispatchArgs& a, int sms) {
 template <bool NORMAL, bool NOLOAD = false>
 int run_bulk_dispatch(DispatchArgs& a, const ep_cfg_t& cfg, bool paced, int sms, cudaStream_t stream,
                       int prefetch = -1) {
-    // default grid: 2 CTAs per SM, or 1 with paced reads (one deep ring per SM); cfg.max_ctas
-    // sets the grid (and so the CTAs sharing an SM)
-    int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas) : int64_t(sms) * (paced ? 1 : 2);
+    // default grid: 2 CTAs per SM, or with paced reads 1 (one deep ring per SM) or 2 (shorter rows,
+    // see paced_ctas_per_sm); cfg.max_ctas sets the grid (and so the CTAs sharing an SM)
+    int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas) : int64_t(sms) * (paced ? paced_ctas_per_sm(a) : 2);
     grid = std::max<int64_t>(1, std::min<int64_t>(grid, a.n_units));
     const int ctas_per_sm = int(std::max<int64_t>(1, ceil_div(grid, sms)));
     int budget = std::max(1, max_smem_optin() / ctas_per_sm - 1024);

@@ -583,7 +583,9 @@ def test_dispatch_path_choice():
     assert ep.ep_dispatch_path(8, 1024, 8, 256, 7168) == ep.EP_VARIANT_PACED     # 55 rows per SM
     assert ep.ep_dispatch_path(8, 512, 8, 256, 7168) == ep.EP_VARIANT_BULK       # 28 rows per SM
     assert ep.ep_dispatch_path(8, 128, 8, 256, 7168) == ep.EP_VARIANT_BULK       # decode: 7 rows per SM
-    assert ep.ep_dispatch_path(8, 2048, 6, 80, 4096) == ep.EP_VARIANT_BULK       # replica: 48 KB per row
+    assert ep.ep_dispatch_path(8, 2048, 6, 80, 4096) == ep.EP_VARIANT_PACED      # replica: 48 KB per row, 2 CTAs/SM
+    assert ep.ep_dispatch_path(8, 2048, 4, 80, 4096) == ep.EP_VARIANT_BULK       # 32 KB of stores per row
+    assert ep.ep_dispatch_path(8, 1024, 6, 80, 4096) == ep.EP_VARIANT_BULK       # 48 KB per row, 55 rows per SM
     assert ep.ep_dispatch_path(8, 128, 8, 256, 7168, cfg=dict(variant=2)) == ep.EP_VARIANT_VECTOR
     assert ep.ep_dispatch_path(8, 128, 8, 256, 7168, cfg=dict(variant=3)) == ep.EP_VARIANT_PACED
     with pytest.raises(ep.EPError) as ei:
