@@ -159,13 +159,15 @@ enum {
     EP_VARIANT_BULK = 1,      /* rows staged in shared memory by bulk async copies */
     EP_VARIANT_VECTOR = 2,    /* rows moved through registers as 16-byte vectors */
     EP_VARIANT_PACED = 3      /* ep_dispatch, ep_normal_dispatch, ep_dispatch_fp8: the bulk path
-                                 with paced reads -- one CTA per SM, and the rows about to be staged
-                                 are prefetched into L2 only inside a short window that recurs on
-                                 the GPU-wide clock, so HBM serves reads in bursts and the row stores
-                                 alone in between (the same bits).  AUTO takes it for ep_dispatch
-                                 when a row's k stores add up to >= 96 KB and every SM has >= 16
-                                 rows (e.g. 8 x 4096 tokens, top-8, H = 7168), where it measured
-                                 faster */
+                                 with paced reads -- one CTA per SM (two for ep_dispatch rows whose
+                                 k stores add up to less than 96 KB), and the rows about to be
+                                 staged are prefetched into L2 only inside a short window that
+                                 recurs on the GPU-wide clock, so HBM serves reads in bursts and the
+                                 row stores alone in between (the same bits).  AUTO takes it for
+                                 ep_dispatch where it measured faster: a row's k stores add up to
+                                 >= 96 KB and every SM has >= 32 rows (e.g. 8 x 4096 tokens, top-8,
+                                 H = 7168), or 48-96 KB and >= 96 rows per SM (8 x 2048 tokens,
+                                 top-6, H = 4096) */
 };
 
 /* Human-readable name of an EP_OK / EP_ERR_* code (static storage). */
