@@ -184,3 +184,38 @@ def test_fp8_consumer_warp_counts(threads):
     inp = inputs.make_inputs(w)
     check_fp8(inp, w.num_experts, ep.EP_FP8_SCALE_UE8M0, f"threads {threads}",
               dict(variant=ep.EP_VARIANT_BULK, threads=threads, max_ctas=7))
+
+
+def _fp8_inputs(rng, R, T, k, E, H, idx):
+    x = (rng.standard_normal((R, T, H)) * 10.0 ** rng.uniform(-3, 3, size=(R, T, 1))).astype(np.float32)
+    bits = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    w = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+    return inputs.Inputs(idx.astype(np.int32), w, bits, np.ones(R, np.uint8))
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_fp8_scale_writer_many_experts(fmt):
+    """2048 experts and 256 tokens of top-8: most experts receive no row, so the scale writer's scan
+    of the experts 32 at a time and its chunk numbering skip long runs of empty experts."""
+    rng = np.random.default_rng(8100 + fmt)
+    R, T, k, E, H = 8, 32, 8, 2048, 512
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k)
+    inp = _fp8_inputs(rng, R, T, k, E, H, idx)
+    for variant in VARIANTS:
+        check_fp8(inp, E, fmt, f"E=2048 fmt {fmt} variant {variant}", dict(variant=variant))
+
+
+@pytest.mark.parametrize("H", [4096, 4224, 7168])
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_fp8_scale_writer_hot_experts(fmt, H):
+    """Every token picks its k experts among the first 12 of 64, so a few experts receive thousands
+    of rows: many 256-row chunks per expert, spread over the writer's blocks.  fp32 / power-of-two
+    scales at H = 4096 and 7168 take the staged copy with 16-byte reads, at H = 4224 (33 words a row)
+    the staged copy word by word; UE8M0 rows are copied directly."""
+    if fmt == ep.EP_FP8_SCALE_UE8M0 and H % 512:
+        pytest.skip("UE8M0 needs H % 512 == 0")
+    rng = np.random.default_rng(8200 + fmt + H)
+    R, T, k, E = 8, 300, 6, 64
+    idx = np.stack([rng.permutation(12)[:k] for _ in range(R * T)]).reshape(R, T, k)
+    inp = _fp8_inputs(rng, R, T, k, E, H, idx)
+    check_fp8(inp, E, fmt, f"hot experts H={H} fmt {fmt}", dict(variant=ep.EP_VARIANT_BULK))
