@@ -526,9 +526,15 @@ extern "C" int ep_combine_peer(ep_dims_t d, int32_t rank, const uint64_t* y_slab
     a.rank = rank;
     a.cap = int64_t(d.num_ranks) * d.num_tokens;
     a.row_bytes = int64_t(d.hidden) * 2;
-    const int64_t units = int64_t(d.num_tokens) * ceil_div(a.row_bytes >> 4, 32 * 1);
-    return launch_peer_stream(combine_peer_kernel<1>, a, int(std::min<int64_t>(units, INT32_MAX)), cfg,
-                              static_cast<cudaStream_t>(stream));
+    // cfg.threads = 2: two 16-byte columns per lane and unit (emulated world, prefill: 941-960 against
+    // 962-979 us; at 8 x 512 tokens 166-170 against 158-162 us); otherwise one.  (Four spill registers
+    // under the two-CTAs-per-SM bound and ran 1587 us.)
+    const int U = cfg.threads == 2 ? 2 : 1;
+    const int64_t units = int64_t(d.num_tokens) * ceil_div(a.row_bytes >> 4, 32 * U);
+    const int n = int(std::min<int64_t>(units, INT32_MAX));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return U == 2 ? launch_peer_stream(combine_peer_kernel<2>, a, n, cfg, st)
+                  : launch_peer_stream(combine_peer_kernel<1>, a, n, cfg, st);
 }
 
 extern "C" int ep_ipc_export(const void* ptr, void* handle, uint64_t* offset) {

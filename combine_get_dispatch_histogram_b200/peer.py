@@ -103,10 +103,10 @@ class PeerRank:
                                   status=status, stream=stream)
 
     def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, lay: ep.LocalLayout, counts: torch.Tensor,
-                 active: torch.Tensor, signal: int, *, status=None, stream=None) -> torch.Tensor:
+                 active: torch.Tensor, signal: int, *, status=None, cfg=None, stream=None) -> torch.Tensor:
         return ep.ep_dispatch_peer(x, topk_idx, lay.local_row, counts, active, self.rank, self.slab_table,
                                    self.src_info_table, self.arrival_table, signal, self.bufs.dispatch_ws,
-                                   status=status, stream=stream)
+                                   status=status, cfg=cfg, stream=stream)
 
     def wait_arrivals(self, signal: int, active: torch.Tensor, *, wait_ns=None, status=None,
                       stream=None) -> torch.Tensor:
@@ -123,9 +123,9 @@ class PeerRank:
         return ep.ep_wait_peers(self.bufs.ready, signal, active, status=status, stream=stream)
 
     def combine(self, topk_idx: torch.Tensor, topk_weights: torch.Tensor, lay: ep.LocalLayout, counts: torch.Tensor,
-                active: torch.Tensor, *, out=None, status=None, stream=None):
+                active: torch.Tensor, *, out=None, status=None, cfg=None, stream=None):
         return ep.ep_combine_peer(self.slab_table, topk_idx, topk_weights, lay.local_row, counts, active, self.rank,
-                                  self.H, out=out, status=status, stream=stream)
+                                  self.H, out=out, status=status, cfg=cfg, stream=stream)
 
     def close(self):
         for base in self._mapped:

@@ -150,7 +150,8 @@ def main():
 
         def peer_combine():
             for r in range(R):
-                ranks[r].combine(idxs[r], wts[r], lays[r], counts, act, out=outs[r], status=status, stream=stream)
+                ranks[r].combine(idxs[r], wts[r], lays[r], counts, act, out=outs[r], status=status, cfg=cfg,
+                                 stream=stream)
 
         peer_dispatch()
         calls.append(peer_dispatch if args.op == "peer_dispatch" else peer_combine)

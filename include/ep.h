@@ -654,6 +654,8 @@ EP_API int ep_peer_recv_count(int32_t num_ranks, int32_t num_experts, int32_t ra
  *      topk_idx, topk_weights float [T,k], local_row, counts, active (mask at combine time)
  * out: out bf16 [T,H] = bf16_rne(sum over j = 0..k-1 of w[t,j] * y[row of (t,j)]) in
  *      float32 from +0, over live slots whose destination is active; zeros if active[r] == 0.
+ * cfg.threads = 2 gives each lane two 16-byte columns per unit (default one); cfg.max_ctas caps
+ * the grid.  The bits are the same either way.
  */
 EP_API int ep_combine_peer(ep_dims_t d, int32_t rank, const uint64_t *y_slabs, const int32_t *topk_idx,
                            const float *topk_weights, const int32_t *local_row, const int32_t *counts,

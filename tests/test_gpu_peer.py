@@ -228,3 +228,21 @@ def test_wait_cost_and_receive_stats():
         ep.ep_recv_stats_accumulate(recv[1], stats)
     torch.cuda.synchronize()
     assert np.array_equal(stats.cpu().numpy(), 3 * ref.recv_count[El:2 * El])
+
+
+@pytest.mark.parametrize("cfg", [dict(threads=2), dict(max_ctas=3), dict(threads=2, max_ctas=5)])
+def test_peer_combine_launch_configs_give_the_same_bits(cfg):
+    """Two 16-byte columns per lane, or a grid of a few CTAs (many units per warp), change only the
+    schedule: every output bit equals the default launch's."""
+    w = inputs.named("sweep_T64_mask5")
+    inp = inputs.make_inputs(w)
+    E, H = w.num_physical, w.hidden
+    ranks, lays, counts, recv, status, waits, idx, act_c = _run_world(inp, E, H, signal=1)
+    base, st = _combine_all(ranks, lays, counts, inp, idx, act_c, signal=1)
+    assert st == 0
+    wts = f32_dev(inp.topk_weights)
+    again = torch.stack([ranks[r].combine(idx[r], wts[r], lays[r], counts, act_c, status=status, cfg=cfg)[0]
+                         for r in range(len(ranks))])
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(again.view(torch.int16), base.view(torch.int16)), cfg
