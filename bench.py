@@ -17,7 +17,9 @@ Reported:
                by the step time, summed over ranks and divided by the slowest
                rank's time;
   dispatch/combine/layout microseconds per call, from CUDA events recorded on
-               the launching stream around every call in the timed region;
+               the launching stream around every call in the timed region, and
+               layout + dispatch end to end (the events before the layout and
+               after the dispatch of each step; with --graph, a graph of the two);
   roofline     the dominant kernel's achieved GB/s against the measured copy
                bandwidth of this GPU type (MEASURED_PEAKS.json);
   e2e          the same metric with host buffers: every step copies its inputs
@@ -382,9 +384,9 @@ def run_ours(args, rank, world, local_rank, w, inp):
     t_end = torch.cuda.Event(enable_timing=True)
     graphs = None
     if args.graph:
-        # one graph for the whole step, one per part (for the per-kernel split)
+        # one graph for the whole step, one per part (for the per-kernel split), one of layout + dispatch
         graphs = []
-        for fns in ([step],) + tuple((p,) for p in parts):
+        for fns in ([step],) + tuple((p,) for p in parts) + ((do_layout, do_dispatch),):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 for fn in fns:
@@ -422,6 +424,7 @@ def run_ours(args, rank, world, local_rank, w, inp):
     total_ms = t_start.elapsed_time(t_end) if flush is None else sum(e0.elapsed_time(e1) for e0, e1 in step_ev)
     if graphs is None:
         per_part = [[e[i].elapsed_time(e[i + 1]) for e in events] for i in range(len(parts))]
+        per_part.append([e[0].elapsed_time(e[2]) for e in events])  # layout + dispatch
     else:
         # each part replayed alone as its own graph, one event pair per replay
         per_part = []
@@ -437,8 +440,8 @@ def run_ours(args, rank, world, local_rank, w, inp):
                     e1.record(stream)
             stream.synchronize()
             per_part.append([e0.elapsed_time(e1) for e0, e1 in evs])
-    part_stats = [stats_ms(v) for v in per_part]
-    lay_ms, dis_ms, com_ms = (st["median"] for st in part_stats)
+    part_stats = [stats_ms(v) for v in per_part]  # layout, dispatch, combine, layout + dispatch
+    lay_ms, dis_ms, com_ms = (st["median"] for st in part_stats[:3])
     if int(status.item()) != 0:
         raise SystemExit(f"device status {int(status.item())} after the timed steps")
 
@@ -529,8 +532,8 @@ def run_ours(args, rank, world, local_rank, w, inp):
     flat = [v for st in part_stats for v in (st["median"], st["min"], st["max"])]
     total_ms, e2e_ms, c0_ms, c1_ms, *flat = reduce_over_ranks(
         [total_ms, e2e["ms"] if e2e else 0.0] + ceil_ms + flat, world, dev, "max")
-    part_stats = [dict(median=flat[3 * i], min=flat[3 * i + 1], max=flat[3 * i + 2]) for i in range(len(parts))]
-    lay_ms, dis_ms, com_ms = (st["median"] for st in part_stats)
+    part_stats = [dict(median=flat[3 * i], min=flat[3 * i + 1], max=flat[3 * i + 2]) for i in range(len(flat) // 3)]
+    lay_ms, dis_ms, com_ms = (st["median"] for st in part_stats[:3])
     ms_per_step = total_ms / args.steps
     step_bytes = d_bytes + c_bytes
     (job_bytes,) = reduce_over_ranks([step_bytes], world, dev, "sum")
@@ -562,6 +565,7 @@ def run_ours(args, rank, world, local_rank, w, inp):
         "kernel_us": {name: {k_: round(v * 1e3, 2) for k_, v in st.items()}
                       for name, st in zip(("layout", "dispatch", "combine"), part_stats)},
         "kernel_us_stat": "median over the timed steps (min, max beside it); max over ranks",
+        "layout_dispatch_us": {k_: round(v * 1e3, 2) for k_, v in part_stats[3].items()},
         "dispatch_gbs": round(dis_gbs, 1),
         "combine_gbs": round(com_gbs, 1),
         "dispatch_frac_of_8tbs": round(dis_gbs / NOMINAL_HBM_GBS, 4),
