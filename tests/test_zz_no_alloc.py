@@ -43,10 +43,11 @@ def _empty_layout(R, T, k, E, dev):
 
 @pytest.mark.parametrize("variant", [0, ep.EP_LAYOUT_FUSED])
 def test_noalloc_layout_equals_workspace_layout_on_two_calls_in_a_row(variant):
-    """AUTO takes the chunked / cluster paths; FUSED reads the barrier epoch the array keeps between calls.
+    """AUTO takes the look-back path at prefill and the cluster path at T = 64; the look-back and
+    FUSED paths read the barrier epoch and flags the array keeps between calls.
 
-    The two shapes have different chunk grids (128 and 32 chunks), so the second call
-    starts from the first call's epoch and flags in the shared array.
+    The two shapes have different chunk grids (128 and 32 chunks), so each call starts from the
+    previous call's epoch and flags in the shared array (prefill, T = 64, prefill again).
     """
     fn = _bind()
     dev = torch.device("cuda:0")
