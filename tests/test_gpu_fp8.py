@@ -219,3 +219,30 @@ def test_fp8_scale_writer_hot_experts(fmt, H):
     idx = np.stack([rng.permutation(12)[:k] for _ in range(R * T)]).reshape(R, T, k)
     inp = _fp8_inputs(rng, R, T, k, E, H, idx)
     check_fp8(inp, E, fmt, f"hot experts H={H} fmt {fmt}", dict(variant=ep.EP_VARIANT_BULK))
+
+
+def _host_bytes_available():
+    try:
+        import psutil
+
+        return psutil.virtual_memory().available
+    except Exception:
+        return 0
+
+
+@pytest.mark.parametrize("fmt", [ep.EP_FP8_SCALE_F32, ep.EP_FP8_SCALE_UE8M0])
+def test_fp8_prefill_full_size(fmt):
+    """The prefill shape (8 x 4096 tokens, top-8 of 256 experts with Zipf 1.2 routing, H = 7168) in
+    the default launch configuration: every code row, scale and src_info entry of all 262,144
+    received rows against the oracle -- fp32 scales through the staged scale writer, UE8M0 through
+    the direct one."""
+    w = inputs.prefill()
+    R, T, k, E, H = w.num_ranks, w.num_tokens, w.num_topk, w.num_experts, w.hidden
+    need = E * R * T * (H + (H // 128) * 4 + 8) + R * T * H * 2 + (2 << 30)
+    free, _ = torch.cuda.mem_get_info()
+    if free < need:
+        pytest.skip(f"needs {need / 1e9:.1f} GB of device memory, {free / 1e9:.1f} GB free")
+    if _host_bytes_available() < 3 * R * T * k * H + (8 << 30):
+        pytest.skip("not enough host memory for the oracle's code rows")
+    inp = inputs.make_inputs(w)
+    check_fp8(inp, E, fmt, f"prefill fmt {fmt}")

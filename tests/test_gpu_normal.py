@@ -138,3 +138,25 @@ def test_normal_mode_fuzz(seed):
     for cfg in cfgs:
         check_normal(inputs.Inputs(idx, wts, x, act), E, f"seed {seed} R={R} T={T} k={k} H={H} cfg {cfg}",
                      alignment=alignment, capacity=capacity, active_combine=now, cfg=cfg)
+
+
+def test_normal_mode_prefill_full_size():
+    """Normal mode at the prefill shape (8 x 4096 tokens, top-8 of 256 experts, Zipf 1.2, H = 7168) in
+    the default launch configuration: every receive row, received row and its local top-k, and every
+    unweighted combine output against the oracle."""
+    try:
+        import psutil
+
+        host = psutil.virtual_memory().available
+    except Exception:
+        host = 0
+    w = inputs.prefill()
+    R, T, k, E, H = w.num_ranks, w.num_tokens, w.num_topk, w.num_experts, w.hidden
+    need = 2 * R * (R * T) * H * 2 + 2 * R * T * H * 2 + (2 << 30)
+    free, _ = torch.cuda.mem_get_info()
+    if free < need:
+        pytest.skip(f"needs {need / 1e9:.1f} GB of device memory, {free / 1e9:.1f} GB free")
+    if host < 3 * R * (R * T) * H * 2 + (8 << 30):
+        pytest.skip("not enough host memory for the oracle's receive rows")
+    inp = inputs.make_inputs(w)
+    check_normal(inp, w.num_physical, "prefill")
