@@ -146,7 +146,7 @@ def main():
         def peer_dispatch():
             sig[0] += 1
             for r in range(R):
-                ranks[r].dispatch(x[r], idxs[r], lays[r], counts, act, sig[0], status=status, stream=stream)
+                ranks[r].dispatch(x[r], idxs[r], lays[r], counts, act, sig[0], status=status, cfg=cfg, stream=stream)
 
         def peer_combine():
             for r in range(R):
