@@ -744,7 +744,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill",
                     help="prefill | decode | replica | tiny | sweep_T<n>[_mask5]")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=30,
+                    help="steps of the host-buffer pipeline (its fill and drain are spread over them)")
     ap.add_argument("--graph", action="store_true",
                     help="replay the step as a CUDA graph (per-kernel split from per-kernel graphs)")
     ap.add_argument("--cpu-sample-tokens", type=int, default=None,
