@@ -379,11 +379,12 @@ __device__ __forceinline__ bool walk_part(const LayoutArgs& a, const WarpPart& w
                 r = live ? b + __popc(m & below) : -1;
                 if (!w.one_round && p < w.np) rows[p] = r;
                 if (lanes_per_token) {
-                    uint32_t dst = live ? (1u << rank_of[e]) : 0u;
-                    for (int o = 1; o < a.k; o <<= 1) dst |= __shfl_xor_sync(0xffffffffu, dst, o);
                     const bool head = p < w.np && (lane & (a.k - 1)) == 0;
                     uint8_t* itr = a.is_token_in_rank + ((w.pbase + p) / a.k) * a.R;
                     if (packed) {
+                        // the token's destination ranks (R <= 8: one word)
+                        uint32_t dst = live ? (1u << rank_of[e]) : 0u;
+                        for (int o = 1; o < a.k; o <<= 1) dst |= __shfl_xor_sync(0xffffffffu, dst, o);
                         const uint32_t lo = rank_bytes_lo(dst), hi = rank_bytes_hi(dst);
                         if (head) {
                             if (itr_word == 8) {
@@ -397,6 +398,9 @@ __device__ __forceinline__ bool walk_part(const LayoutArgs& a, const WarpPart& w
                             cnt_hi += hi;
                         }
                     } else {
+                        // the token's destination ranks: 64 bits, since R may reach EP_MAX_RANKS
+                        uint64_t dst = live ? (1ull << rank_of[e]) : 0ull;
+                        for (int o = 1; o < a.k; o <<= 1) dst |= __shfl_xor_sync(0xffffffffu, dst, o);
                         if (head)
                             for (int d = 0; d < a.R; ++d) itr[d] = uint8_t((dst >> d) & 1u);
                         for (int d = 0; d < a.R; ++d) {
