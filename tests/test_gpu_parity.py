@@ -144,6 +144,7 @@ EDGE = {
     "max_ranks": dict(R=64, T=24, k=8, E=512, H=64),        # EP_MAX_RANKS: destination sets past 32 bits
     "max_experts": dict(R=8, T=40, k=8, E=8192, H=64),      # EP_MAX_EXPERTS
     "max_ranks_k32": dict(R=64, T=6, k=32, E=2048, H=128),  # EP_MAX_RANKS with EP_MAX_TOPK
+    "max_ranks_k6": dict(R=64, T=20, k=6, E=640, H=64),     # EP_MAX_RANKS, k not a power of two
 }
 
 
@@ -395,7 +396,7 @@ def test_layout_paths_match_oracle(name, path):
 
 @pytest.mark.parametrize("path", [LAYOUT_CHUNKED, LAYOUT_SINGLE_CTA, LAYOUT_FUSED, LAYOUT_CLUSTER, LAYOUT_LOOKBACK])
 @pytest.mark.parametrize("name", ["k1", "T1", "R1", "E_equals_R", "k32", "many_experts", "max_ranks", "max_experts",
-                                  "max_ranks_k32"])
+                                  "max_ranks_k32", "max_ranks_k6"])
 def test_layout_paths_edge_shapes(name, path):
     c = EDGE[name]
     if path == LAYOUT_SINGLE_CTA and (c["E"] > 1024 or c["R"] > 32 or c["R"] * c["T"] * c["k"] > 32768):
