@@ -246,3 +246,15 @@ def test_fp8_prefill_full_size(fmt):
         pytest.skip("not enough host memory for the oracle's code rows")
     inp = inputs.make_inputs(w)
     check_fp8(inp, E, fmt, f"prefill fmt {fmt}")
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+@pytest.mark.parametrize("R,T,k,E,H", [(8, 24, 8, 8192, 512), (64, 6, 8, 512, 512)])
+def test_fp8_dispatch_maximum_shapes(fmt, R, T, k, E, H):
+    """EP_MAX_EXPERTS (the scale writer scans 8192 experts, almost all of them empty) and
+    EP_MAX_RANKS (64 source ranks, the layout on its look-back path)."""
+    rng = np.random.default_rng(8300 + fmt + E)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k)
+    inp = _fp8_inputs(rng, R, T, k, E, H, idx)
+    for variant in VARIANTS:
+        check_fp8(inp, E, fmt, f"R={R} E={E} fmt {fmt} variant {variant}", dict(variant=variant))
