@@ -246,3 +246,23 @@ def test_peer_combine_launch_configs_give_the_same_bits(cfg):
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     assert torch.equal(again.view(torch.int16), base.view(torch.int16)), cfg
+
+
+def test_sixty_four_rank_world():
+    """EP_MAX_RANKS: 64 emulated ranks, each with its own buffers and a 64-entry address table,
+    three of them masked; every slab row, src_info entry and combined token against the oracle."""
+    R, T, k, E, H = 64, 5, 4, 128, 64
+    rng = np.random.default_rng(9100)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(R * T)]).reshape(R, T, k).astype(np.int32)
+    idx = np.where(rng.random(idx.shape) < 0.1, -1, idx).astype(np.int32)
+    x = (rng.standard_normal((R, T, H))).astype(np.float32)
+    bits = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    act = np.ones(R, np.uint8)
+    act[[3, 40, 63]] = 0
+    inp = inputs.Inputs(idx, inputs.softmax_weights(rng, R * T, k).reshape(R, T, k), bits, act)
+    ranks, lays, counts, recv, status, waits, idx_d, act_c = _run_world(inp, E, H, signal=1)
+    assert int(status.item()) == 0 and all(int(s.item()) == 0 for s in waits)
+    ref, packed = _check_slabs(ranks, recv, inp, E, "R=64")
+    out, st = _combine_all(ranks, lays, counts, inp, idx_d, act_c, signal=1)
+    assert st == 0
+    _check_combine(out, ref, packed, inp, E, inp.active, "R=64")
