@@ -27,7 +27,7 @@ Two ways to build the ranks:
 from __future__ import annotations
 
 import dataclasses
-from typing import List, Optional, Sequence
+from typing import List, Sequence
 
 import torch
 
