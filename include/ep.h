@@ -614,7 +614,8 @@ EP_API size_t ep_dispatch_peer_workspace_bytes(void);
  * out (in the destination ranks' memory): slab rows and src_info (src_rank, src_token)
  *      of every live pair; rows >= CAP are flagged EP_STATUS_OVERFLOW and not written.
  * A masked source (active[r] == 0) sends and signals nothing.  The call launches even
- * with T = 0, so the flags still go out.
+ * with T = 0, so the flags still go out.  cfg.max_ctas caps the grid (default: the CTAs
+ * that fit at once); the other cfg fields are ignored.
  */
 EP_API int ep_dispatch_peer(ep_dims_t d, int32_t rank, ep_peer_table_t peers, const uint16_t *x,
                             const int32_t *topk_idx, const int32_t *local_row, const int32_t *counts,
