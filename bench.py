@@ -699,7 +699,7 @@ def run_reference(args, world):
     for _ in range(args.steps):
         samples.append(oracle_sample(w, args.cpu_sample_tokens, inp))
     secs = sum(s["seconds"] for s in samples) / len(samples)
-    value = statistics.median(s["value"] for s in samples)
+    value = round(statistics.median(s["value"] for s in samples), 4)
     base = dict(samples[0])
     base["value"] = value
     base["seconds"] = round(secs, 3)
