@@ -62,6 +62,15 @@ constexpr int kPaceMinUnitsPerCta = 32;
 constexpr int kPaceTwoRingMinUnitsPerSm = 96;
 constexpr int64_t kPaceMinStoreBytesPerRow = 48 * 1024;
 constexpr int64_t kPaceOneRingStoreBytesPerRow = 96 * 1024;
+// Unpaced normal-mode grid, measured on B200 (L2 flushed before each call, 2 against 4 CTAs per SM).
+// A CTA is one issuing warp that also writes every live rank's slot metadata, so four CTAs per SM
+// issue faster where a 4-way split of shared memory still leaves a ring of >= 6 rows, or where
+// there are few rows: 8 x 2048 tokens of 8 KB (replica) 139 against 195 us, decode (1024 rows of
+// 14 KB) 22.5 against 24.6, T = 512 with rank 5 masked 59 against 63, T = 512 74 against 74.  At
+// prefill (221 rows of 14 KB per SM) four CTAs get 3-row rings: 497 against 466 us.
+constexpr int kNormalWideCtasPerSm = 4;
+constexpr int kNormalWideMinStages = 6;
+constexpr int kNormalWideMaxUnitsPerSm = 32;
 
 struct DispatchArgs {
     const uint8_t* x;
@@ -427,14 +436,25 @@ int paced_ctas_per_sm(const DispatchArgs& a) {
     return int64_t(a.k) * a.row_bytes >= kPaceOneRingStoreBytesPerRow ? 1 : 2;
 }
 
+// CTAs per SM of an unpaced normal-mode dispatch (see kNormalWideCtasPerSm).
+int normal_ctas_per_sm(const DispatchArgs& a, int sms) {
+    const int64_t per_stage = int64_t(a.stage_bytes) + 8 + 2 * 256;
+    const int64_t budget = max_smem_optin() / kNormalWideCtasPerSm - 1024;
+    const bool deep = budget >= kNormalWideMinStages * per_stage;
+    const bool few = a.n_units <= int64_t(kNormalWideMaxUnitsPerSm) * sms;
+    return deep || few ? kNormalWideCtasPerSm : 2;
+}
+
 // Grid, stages and (for the paced path) the read schedule, then the bulk-path launch.  `prefetch`
 // (default: as paced) turns the paced read schedule on; the ceiling diagnostic may turn it off.
+// `unpaced_per_sm` is the default CTAs per SM without paced reads.
 template <bool NORMAL, bool NOLOAD = false>
 int run_bulk_dispatch(DispatchArgs& a, const ep_cfg_t& cfg, bool paced, int sms, cudaStream_t stream,
-                      int prefetch = -1) {
-    // default grid: 2 CTAs per SM, or with paced reads 1 (one deep ring per SM) or 2 (shorter rows,
-    // see paced_ctas_per_sm); cfg.max_ctas sets the grid (and so the CTAs sharing an SM)
-    int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas) : int64_t(sms) * (paced ? paced_ctas_per_sm(a) : 2);
+                      int prefetch = -1, int unpaced_per_sm = 2) {
+    // default grid: `unpaced_per_sm` CTAs per SM, or with paced reads 1 (one deep ring per SM) or 2
+    // (shorter rows, see paced_ctas_per_sm); cfg.max_ctas sets the grid (and so the CTAs sharing an SM)
+    int64_t grid = cfg.max_ctas > 0 ? int64_t(cfg.max_ctas)
+                                    : int64_t(sms) * (paced ? paced_ctas_per_sm(a) : unpaced_per_sm);
     grid = std::max<int64_t>(1, std::min<int64_t>(grid, a.n_units));
     const int ctas_per_sm = int(std::max<int64_t>(1, ceil_div(grid, sms)));
     int budget = std::max(1, max_smem_optin() / ctas_per_sm - 1024);
@@ -539,7 +559,8 @@ extern "C" int ep_normal_dispatch(ep_dims_t d, int32_t recv_capacity, const uint
     // normal mode has only the bulk data path: PACED paces its reads (it measured slower at prefill,
     // so AUTO does not), any other variant runs it unpaced
     const bool paced = cfg.variant == EP_VARIANT_PACED;
-    return run_bulk_dispatch<true>(a, cfg, paced, sms, static_cast<cudaStream_t>(stream));
+    return run_bulk_dispatch<true>(a, cfg, paced, sms, static_cast<cudaStream_t>(stream), -1,
+                                   normal_ctas_per_sm(a, sms));
 }
 
 extern "C" int ep_diag_dispatch_ceiling(ep_dims_t d, const uint16_t* x, const int32_t* topk_idx,

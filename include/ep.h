@@ -127,7 +127,9 @@ typedef struct ep_dims {
  * num_sms on the NeMo page).  A zero field means "choose automatically". */
 typedef struct ep_cfg {
     int32_t max_ctas;     /* CTAs of the row-moving kernels: the grid of dispatch (default 2
-                             per SM, 1 on the paced path) and of the vector combine (default:
+                             per SM, 1 on the paced path; ep_normal_dispatch 4 where a 4-way
+                             split of shared memory leaves >= 6 staged rows or there are at most
+                             32 rows per SM, else 2) and of the vector combine (default:
                              as many as fit at once); a cap for the bulk combine (default 1 per SM) */
     int32_t threads;      /* threads per CTA where the kernel allows a choice */
     int32_t stages;       /* shared-memory pipeline depth of dispatch / combine */
