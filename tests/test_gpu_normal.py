@@ -55,7 +55,9 @@ def check_normal(inp, E, tag, alignment=1, capacity=None, active_combine=None, c
     assert bool(st & ep.EP_STATUS_OVERFLOW) == bool(ref_nl["status"] & oracle.OVERFLOW)
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "sweep_T16_mask5", "sweep_T512", "replica_T256"])
+# "replica" is the full replica shape (8 x 2048 tokens, H = 4096) in the default launch
+# configuration: 4 CTAs per SM with 6-row rings, each ring wrapping many times
+@pytest.mark.parametrize("name", ["tiny", "decode", "sweep_T16_mask5", "sweep_T512", "replica_T256", "replica"])
 def test_normal_mode_matches_oracle(name):
     w = inputs.replica(256) if name == "replica_T256" else inputs.named(name)
     inp = inputs.make_inputs(w)
