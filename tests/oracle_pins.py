@@ -416,6 +416,31 @@ def pin_fp8_dequant_error(lib):
             assert np.array_equal(ue.astype(np.int64) - 127, np.log2(scales).astype(np.int64))
 
 
+def pin_fp8_dispatch_is_cast_of_dispatch(lib):
+    """FP8 dispatch ([P1] low_latency_dispatch with use_fp8) moves the same rows as the bf16
+    dispatch, each cast per 128-channel group: every packed FP8 row (codes, scales and, for
+    power-of-two scales, the UE8M0 bytes) is the row quantiser applied to the bf16 dispatch's row at
+    the same place.  Both the placement (golden files, bijection) and the row quantiser (hand-worked
+    row, e4m3 against torch, dequantisation bound) are pinned on their own."""
+    rng = np.random.default_rng(41)
+    for it in range(30):
+        idx, active, E = _random_case(rng, dup=(it % 5 == 0))
+        R, T, k = idx.shape
+        H = 128 * int(rng.integers(1, 3))
+        x = inputs.bf16_tokens(rng, R * T, H).reshape(R, T, H)
+        lay = oracle.layout(idx, active, E, lib=lib)
+        packed, _ = oracle.dispatch(x, idx, lay, lib=lib)
+        for pow2 in (False, True):
+            codes, scales, ue, st = oracle.dispatch_fp8(x, idx, lay, pow2, lib=lib)
+            assert st == 0 and codes.shape[0] == packed.shape[0]
+            for i in range(packed.shape[0]):
+                c, s_, u = oracle.fp8_quantize_row(packed[i], pow2, lib=lib)
+                assert np.array_equal(codes[i], c), f"case {it} row {i} codes"
+                assert np.array_equal(scales[i], s_), f"case {it} row {i} scales"
+                if pow2:
+                    assert np.array_equal(ue[i], u), f"case {it} row {i} ue8m0"
+
+
 # ----------------------------------------------------------------------------- normal-mode pins
 
 def pin_normal_golden(lib):
@@ -493,6 +518,28 @@ def pin_normal_dispatch_combine(lib):
         assert np.array_equal(out, want)
 
 
+def pin_normal_combine_mask_at_combine(lib):
+    """[P4]'s active-rank mask is read again at combine time: a rank masked after the dispatch
+    contributes nothing, and a source rank masked by then gets zeros.  With identity experts (the
+    received rows returned unchanged) the unweighted combine of token (r, t) is x[r, t] times the
+    number of ranks it reached that are still active, or zero when r itself is masked."""
+    rng = np.random.default_rng(33)
+    for it in range(40):
+        idx, active, E = _random_case(rng, R=int(rng.integers(2, 6)), p_mask=0.0)
+        R, T, k = idx.shape
+        x = inputs.bf16_tokens(rng, R * T, 8).reshape(R, T, 8)
+        w = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+        nl = oracle.normal_layout(idx, active, E, lib=lib)
+        nd = oracle.normal_dispatch(x, idx, w, active, E, nl, lib=lib)
+        now = active.copy()
+        now[rng.permutation(R)[: int(rng.integers(1, R))]] = 0       # 1 .. R-1 ranks masked since
+        out, _ = oracle.normal_combine(nd["recv_x"], nl["token_recv_row"], now, lib=lib)
+        reached = (nl["token_recv_row"] >= 0) & (now[None, None, :] == 1)
+        want = reached.sum(axis=2)[:, :, None] * oracle.bf16_bits_to_f64(x)
+        want[now == 0] = 0
+        assert np.array_equal(out, want), f"case {it}"
+
+
 # ----------------------------------------------------------------------------- replica weights / gradients
 
 def pin_replica_sync_and_reduce(lib):
@@ -517,6 +564,7 @@ def pin_replica_sync_and_reduce(lib):
     assert np.array_equal(r, np.repeat(m, n_rep, axis=0))
 
 
-ALL_PINS = [pin_replica_sync_and_reduce, pin_normal_golden, pin_normal_bruteforce, pin_normal_dispatch_combine, pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
+ALL_PINS = [pin_replica_sync_and_reduce, pin_normal_golden, pin_normal_bruteforce, pin_normal_dispatch_combine,
+            pin_normal_combine_mask_at_combine, pin_fp8_dispatch_is_cast_of_dispatch, pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
             pin_dispatch_golden, pin_dispatch_bijection, pin_combine_golden,
             pin_combine_special_cases, pin_combine_mask, pin_reroute_golden, pin_reroute_invariants]

@@ -49,7 +49,13 @@ MUTANTS = {
     "ue8m0_bias": ("if (ue8m0) *ue8m0 = (uint8_t)(e + 127);", "if (ue8m0) *ue8m0 = (uint8_t)(e + 128);"),
     "pow2_floor": ("e = m == 0.5 ? f - 1 : f;", "e = f - 1;"),
     "fp8_no_saturation": ("if (a >= 448.0) return (uint8_t)(sign | 0x7Eu);", "if (a >= 480.0) return (uint8_t)(sign | 0x7Fu);"),
+    # FP8 dispatch placement (indices stay in bounds: row < L, t * R + r < R * T)
+    "fp8_dispatch_row_base": ("const int64_t at = list_base[e] + row;", "const int64_t at = row;"),
+    "fp8_dispatch_token_transposed": ("oracle_fp8_quantize_row(x + ((int64_t)r * T + t) * H",
+                                      "oracle_fp8_quantize_row(x + ((int64_t)t * R + r) * H"),
+    "fp8_dispatch_scale_stride": ("codes + at * H, scales + at * G,", "codes + at * H, scales + at,"),
     # normal mode
+    "normal_combine_no_dst_mask": ("if (row < 0 || !active_now[d]) continue;", "if (row < 0) continue;"),
     "normal_global_expert_id": ("recv_topk_idx[dst * k + j] = here ? e - d * E_local : -1;",
                                 "recv_topk_idx[dst * k + j] = here ? e : -1;"),
     "normal_weighted_combine": ("for (int h = 0; h < H; h++) o[h] += bf16_to_double(yr[h]);",
