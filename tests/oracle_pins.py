@@ -441,6 +441,74 @@ def pin_fp8_dispatch_is_cast_of_dispatch(lib):
                     assert np.array_equal(ue[i], u), f"case {it} row {i} ue8m0"
 
 
+def _bf16_of(v: float) -> int:
+    b = int(np.array([v], np.float32).view(np.uint32)[0])
+    assert b & 0xFFFF == 0, v
+    return b >> 16
+
+
+def pin_fp8_rounding_readings(lib):
+    """The FP8 cast's arithmetic as the readings fix it (scale = amax/448 in float32, 1 for an
+    all-zero group; code = round-to-nearest-even e4m3 of x/scale with the division in float32;
+    power-of-two scales 2^ceil(log2(amax/448)) clamped to [-127, 127]), checked on values chosen
+    so that a plausible slip (a reciprocal instead of a division, another zero-group scale, the
+    clamp one binade off) changes the result."""
+    import torch
+    from fractions import Fraction
+
+    def e4m3(v):
+        return torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+    # (1) the scale is the float32 nearest to amax/448 (exact rational check against both neighbours)
+    rng = np.random.default_rng(23)
+    bits = inputs.bf16_tokens(rng, 4, 128 * 64)
+    for row in bits:
+        _, scales, _ = oracle.fp8_quantize_row(row, False, lib=lib)
+        amax = np.abs(oracle.bf16_bits_to_f64(row).reshape(-1, 128)).max(axis=1)
+        for a, sc in zip(amax, scales):
+            exact = Fraction(float(a)) / 448
+            err = abs(Fraction(float(sc)) - exact)
+            for nb in (np.nextafter(sc, np.float32(np.inf)), np.nextafter(sc, np.float32(0))):
+                assert err <= abs(Fraction(float(nb)) - exact), f"scale of amax {a} is not amax/448 rounded"
+
+    # (2) codes: element pairs (amax, x) where x/scale and x*(1/scale) round to different codes
+    grid = (np.arange(0x3D80, 0x4280, dtype=np.uint32) << 16).view(np.float32)   # bf16 in [2^-4, 2^6)
+    pairs = []
+    for a in grid:
+        sc = np.float32(a) / np.float32(448)
+        f = grid[grid <= a]
+        q_div = (f / sc).astype(np.float32)
+        q_rcp = (f * (np.float32(1) / sc)).astype(np.float32)
+        for x in f[e4m3(q_div) != e4m3(q_rcp)][:1]:
+            pairs.append((float(a), float(x)))
+    assert len(pairs) >= 48
+    row = np.zeros(128 * len(pairs), np.uint16)
+    for g, (a, x) in enumerate(pairs):
+        row[128 * g] = _bf16_of(a)
+        row[128 * g + 1] = _bf16_of(x)
+    codes, scales, _ = oracle.fp8_quantize_row(row, False, lib=lib)
+    for g, (a, x) in enumerate(pairs):
+        q = np.float32(x) / scales[g]                     # one IEEE float32 division
+        assert codes[128 * g + 1] == e4m3(np.array([q]))[0], f"code of {x} in a group of amax {a}"
+
+    # (3) an all-zero group: scale 1 (and UE8M0 byte 127), codes 0, in both modes
+    row = np.zeros(256, np.uint16)
+    row[128:] = _bf16_of(3.0)
+    for pow2 in (False, True):
+        codes, scales, ue = oracle.fp8_quantize_row(row, pow2, lib=lib)
+        assert scales[0] == 1.0 and not codes[:128].any(), f"zero group, pow2={pow2}"
+        if pow2:
+            assert ue[0] == 127
+
+    # (4) power-of-two clamp: amax 2^-126 -> 2^-134.8 -> clamped to 2^-127 (byte 0);
+    #     amax 2^-118 -> 2^-126.8 -> 2^-126 (byte 1, inside the range)
+    for amax, e in ((2.0 ** -126, -127), (2.0 ** -118, -126)):
+        row = np.zeros(128, np.uint16)
+        row[5] = _bf16_of(amax)
+        _, scales, ue = oracle.fp8_quantize_row(row, True, lib=lib)
+        assert scales[0] == np.float32(2.0 ** e) and ue[0] == e + 127, f"pow2 scale of amax {amax}"
+
+
 # ----------------------------------------------------------------------------- normal-mode pins
 
 def pin_normal_golden(lib):
@@ -540,6 +608,45 @@ def pin_normal_combine_mask_at_combine(lib):
         assert np.array_equal(out, want), f"case {it}"
 
 
+def pin_normal_capacity(lib):
+    """A receive buffer of `capacity` rows (the page's num_worst_tokens): rows are numbered as if
+    the buffer were unbounded; overflow is flagged exactly when some rank receives more than
+    `capacity` tokens, by the layout, the dispatch and the combine alike; rows below the capacity
+    hold what an unbounded buffer holds there; and with identity experts the combine of token
+    (r, t) is x[r, t] times the ranks whose row for it is below the capacity."""
+    rng = np.random.default_rng(34)
+    checked_tight = 0
+    for it in range(60):
+        idx, active, E = _random_case(rng, R=int(rng.integers(2, 5)))
+        R, T, k = idx.shape
+        x = inputs.bf16_tokens(rng, R * T, 8).reshape(R, T, 8)
+        w = inputs.softmax_weights(rng, R * T, k).reshape(R, T, k)
+        full = oracle.normal_layout(idx, active, E, lib=lib)
+        most = int(full["recv_tokens"].max())
+        if most == 0:
+            continue
+        cap = [most, max(1, most - 1), int(rng.integers(1, most + 1))][it % 3]
+        nl = oracle.normal_layout(idx, active, E, capacity=cap, lib=lib)
+        over = most > cap
+        checked_tight += over
+        assert np.array_equal(nl["token_recv_row"], full["token_recv_row"]), f"case {it}"
+        assert np.array_equal(nl["recv_tokens"], full["recv_tokens"]), f"case {it}"
+        assert bool(nl["status"] & oracle.OVERFLOW) == over, f"case {it} layout flag"
+        nd_full = oracle.normal_dispatch(x, idx, w, active, E, full, lib=lib)
+        nd = oracle.normal_dispatch(x, idx, w, active, E, nl, lib=lib)
+        assert bool(nd["status"] & oracle.OVERFLOW) == over, f"case {it} dispatch flag"
+        for key in ("recv_x", "recv_topk_idx", "recv_topk_weights", "src_info"):
+            assert np.array_equal(nd[key], nd_full[key][:, :cap]), f"case {it} {key}"
+        out, st = oracle.normal_combine(nd["recv_x"], nl["token_recv_row"], active, lib=lib)
+        assert bool(st & oracle.OVERFLOW) == over, f"case {it} combine flag"
+        rows = nl["token_recv_row"]
+        kept = ((rows >= 0) & (rows < cap)).sum(axis=2)[:, :, None]
+        want = kept * oracle.bf16_bits_to_f64(x)
+        want[active == 0] = 0
+        assert np.array_equal(out, want), f"case {it} combine"
+    assert checked_tight >= 20
+
+
 # ----------------------------------------------------------------------------- replica weights / gradients
 
 def pin_replica_sync_and_reduce(lib):
@@ -565,6 +672,6 @@ def pin_replica_sync_and_reduce(lib):
 
 
 ALL_PINS = [pin_replica_sync_and_reduce, pin_normal_golden, pin_normal_bruteforce, pin_normal_dispatch_combine,
-            pin_normal_combine_mask_at_combine, pin_fp8_dispatch_is_cast_of_dispatch, pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
+            pin_normal_combine_mask_at_combine, pin_normal_capacity, pin_fp8_dispatch_is_cast_of_dispatch, pin_fp8_rounding_readings, pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
             pin_dispatch_golden, pin_dispatch_bijection, pin_combine_golden,
             pin_combine_special_cases, pin_combine_mask, pin_reroute_golden, pin_reroute_invariants]

@@ -49,6 +49,12 @@ MUTANTS = {
     "ue8m0_bias": ("if (ue8m0) *ue8m0 = (uint8_t)(e + 127);", "if (ue8m0) *ue8m0 = (uint8_t)(e + 128);"),
     "pow2_floor": ("e = m == 0.5 ? f - 1 : f;", "e = f - 1;"),
     "fp8_no_saturation": ("if (a >= 448.0) return (uint8_t)(sign | 0x7Eu);", "if (a >= 480.0) return (uint8_t)(sign | 0x7Fu);"),
+    "fp8_scale_by_reciprocal": ("return amax == 0.0f ? 1.0f : amax / 448.0f;",
+                                "return amax == 0.0f ? 1.0f : amax * (1.0f / 448.0f);"),
+    "fp8_codes_by_reciprocal": ("const float q = f / scale;", "const float q = f * (1.0f / scale);"),
+    "fp8_zero_group_scale": ("return amax == 0.0f ? 1.0f : amax / 448.0f;", "return amax == 0.0f ? 2.0f : amax / 448.0f;"),
+    "pow2_zero_group_scale": ("    int e = 0;\n    if (amax != 0.0f) {", "    int e = -127;\n    if (amax != 0.0f) {"),
+    "pow2_clamp_one_binade_high": ("if (e < -127) e = -127;", "if (e < -126) e = -126;"),
     # FP8 dispatch placement (indices stay in bounds: row < L, t * R + r < R * T)
     "fp8_dispatch_row_base": ("const int64_t at = list_base[e] + row;", "const int64_t at = row;"),
     "fp8_dispatch_token_transposed": ("oracle_fp8_quantize_row(x + ((int64_t)r * T + t) * H",
@@ -56,6 +62,15 @@ MUTANTS = {
     "fp8_dispatch_scale_stride": ("codes + at * H, scales + at * G,", "codes + at * H, scales + at,"),
     # normal mode
     "normal_combine_no_dst_mask": ("if (row < 0 || !active_now[d]) continue;", "if (row < 0) continue;"),
+    "normal_layout_overflow_unflagged": ("if (token_recv_row[at] >= capacity) status |= ORACLE_OVERFLOW;", ""),
+    "normal_layout_overflow_off_by_one": ("if (token_recv_row[at] >= capacity) status |= ORACLE_OVERFLOW;",
+                                          "if (token_recv_row[at] > capacity) status |= ORACLE_OVERFLOW;"),
+    "normal_dispatch_overflow_unflagged": (
+        "if (row >= capacity) { status |= ORACLE_OVERFLOW; continue; }\n                int64_t dst =",
+        "if (row >= capacity) { continue; }\n                int64_t dst ="),
+    "normal_combine_overflow_unflagged": (
+        "if (row >= capacity) { status |= ORACLE_OVERFLOW; continue; }\n                const uint16_t *yr =",
+        "if (row >= capacity) { continue; }\n                const uint16_t *yr ="),
     "normal_global_expert_id": ("recv_topk_idx[dst * k + j] = here ? e - d * E_local : -1;",
                                 "recv_topk_idx[dst * k + j] = here ? e : -1;"),
     "normal_weighted_combine": ("for (int h = 0; h < H; h++) o[h] += bf16_to_double(yr[h]);",
