@@ -163,6 +163,21 @@ def pin_layout_status(lib):
     assert lay.status & oracle.OVERFLOW
     assert lay.recv_count[0] == R * T * k
     assert np.array_equal(np.sort(lay.pair_row.ravel()), np.arange(R * T * k))
+    # combine over that handle: rows R*T.. are past the slab (flagged, contribute nothing); with
+    # row i of expert 0 holding the value i + 1 and unit weights, token (r, t) sums its rows below R*T
+    cap = R * T
+    y = np.zeros((2 * cap, 8), np.uint16)
+    y[:cap] = ((np.arange(1, cap + 1, dtype=np.float32)[:, None] * np.ones(8, np.float32)).view(np.uint32) >> 16)
+    out, st = oracle.combine(y, _slab_row_base(2, cap), idx, np.ones((R, T, k), np.float32), lay.pair_row,
+                             np.ones(R, np.uint8), 2, lib=lib)
+    assert st & oracle.OVERFLOW
+    rows = lay.pair_row
+    want = np.where(rows < cap, rows + 1, 0).sum(axis=2).astype(np.float64)
+    assert np.array_equal(out, np.repeat(want[:, :, None], 8, axis=2))
+    # every token sends slot 0 to expert 0: R*T rows fill it exactly, which is not an overflow
+    idx = np.stack([np.zeros((R, T), np.int32), np.ones((R, T), np.int32)], axis=2)
+    lay = oracle.layout(idx, np.ones(R, np.uint8), 2, lib=lib)
+    assert lay.recv_count.tolist() == [R * T, R * T] and lay.status == 0
 
 
 # ----------------------------------------------------------------------------- dispatch pins
@@ -369,6 +384,32 @@ def pin_reroute_invariants(lib):
             assert np.all((phys[idx == e] >= b[e]) & (phys[idx == e] < b[e + 1]))
 
 
+def pin_reroute_bad_ids_and_exact_ratio(lib):
+    """Ids outside [-1, E) are flagged and map to -1 without counting as load; -1 is a plain empty
+    slot (no flag).  And a near-tie: loads 102 599 and 103 112 with 400 extra replicas, where
+    load/replicas of the two experts agree to float32 precision at 200 / 201 replicas but not
+    exactly; the greedy must still reach a min-max optimal placement (checked over all 401
+    splits with exact rationals)."""
+    idx = np.array([[[0, -1], [3, 1]], [[7, 2], [-5, 0]]], np.int32)     # E = 4: 7 and -5 are bad
+    res = oracle.reroute(idx, 4, 2, lib=lib)
+    assert res["status"] & oracle.BAD_EXPERT
+    assert res["load"].tolist() == [2, 1, 1, 1]
+    phys = res["topk_idx_phys"]
+    assert phys[0, 0, 1] == -1 and phys[1, 0, 0] == -1 and phys[1, 1, 0] == -1
+    assert np.all(phys[idx >= 0][(idx[idx >= 0] < 4)] >= 0)
+    ok = oracle.reroute(np.array([[[0, -1], [1, -1]]], np.int32), 2, 1, lib=lib)
+    assert ok["status"] == 0 and ok["load"].tolist() == [1, 1]
+
+    load = [102599, 103112]
+    extra = 400
+    idx = np.repeat(np.array([0, 1], np.int32), load).reshape(1, -1, 1)
+    n = oracle.reroute(idx, 2, extra, lib=lib)["num_replicas"]
+    assert n.sum() == 2 + extra
+    got = max(Fraction(load[0], int(n[0])), Fraction(load[1], int(n[1])))
+    best = min(max(Fraction(load[0], 1 + a), Fraction(load[1], 1 + extra - a)) for a in range(extra + 1))
+    assert got == best, f"placement {n.tolist()} is not min-max optimal"
+
+
 # ----------------------------------------------------------------------------- fp8 pins
 
 def pin_fp8_golden(lib):
@@ -394,8 +435,11 @@ def pin_e4m3_against_torch(lib):
     want = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.array_equal(oracle.e4m3_codes(v, lib=lib), want), "e4m3 encoder differs from torch"
     # saturating cast: finite overflow and infinities clamp to +-448 (0x7E / 0xFE), NaN stays NaN
-    special = np.array([464.0, 500.0, 1e30, np.inf, -600.0, -np.inf, np.nan], np.float32)
-    assert oracle.e4m3_codes(special, lib=lib).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F]
+    special = np.array([464.0, 500.0, 1e30, np.inf, -600.0, -np.inf, np.nan, -0.0, -np.nan], np.float32)
+    want = [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F, 0x80, 0xFF]
+    # torch's cast (no saturation) agrees on the signed NaNs and the negative zero
+    assert torch.from_numpy(special[-3:]).to(torch.float8_e4m3fn).view(torch.uint8).tolist() == want[-3:]
+    assert oracle.e4m3_codes(special, lib=lib).tolist() == want
 
 
 def pin_fp8_dequant_error(lib):
@@ -658,6 +702,9 @@ def pin_replica_sync_and_reduce(lib):
     # gradients of the replicas: the master gradient is their sum, replica by replica
     g = np.array([[1, 2], [10, 20], [100, 200], [0.5, 0.25], [0.5, 0.75], [7, 8], [-3, -4]], np.float32)
     assert oracle.replica_grad_reduce(g, pb, lib=lib).tolist() == [[111, 222], [1, 1], [7, 8], [-3, -4]]
+    # the sum is float64: 1 + 2^-30 + 2^-30 is exact there (a float32 accumulator would give 1)
+    g = np.array([[1.0], [2.0 ** -30], [2.0 ** -30]], np.float32)
+    assert oracle.replica_grad_reduce(g, np.array([0, 3], np.int32), lib=lib)[0, 0] == 1 + 2.0 ** -29
     # identical replica gradients sum to n_rep times the gradient (exact for these values)
     rng = np.random.default_rng(41)
     n_rep = rng.integers(1, 5, size=9)
@@ -674,4 +721,5 @@ def pin_replica_sync_and_reduce(lib):
 ALL_PINS = [pin_replica_sync_and_reduce, pin_normal_golden, pin_normal_bruteforce, pin_normal_dispatch_combine,
             pin_normal_combine_mask_at_combine, pin_normal_capacity, pin_fp8_dispatch_is_cast_of_dispatch, pin_fp8_rounding_readings, pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
             pin_dispatch_golden, pin_dispatch_bijection, pin_combine_golden,
-            pin_combine_special_cases, pin_combine_mask, pin_reroute_golden, pin_reroute_invariants]
+            pin_combine_special_cases, pin_combine_mask, pin_reroute_golden, pin_reroute_invariants,
+            pin_reroute_bad_ids_and_exact_ratio]

@@ -55,6 +55,8 @@ MUTANTS = {
     "fp8_zero_group_scale": ("return amax == 0.0f ? 1.0f : amax / 448.0f;", "return amax == 0.0f ? 2.0f : amax / 448.0f;"),
     "pow2_zero_group_scale": ("    int e = 0;\n    if (amax != 0.0f) {", "    int e = -127;\n    if (amax != 0.0f) {"),
     "pow2_clamp_one_binade_high": ("if (e < -127) e = -127;", "if (e < -126) e = -126;"),
+    "e4m3_nan_loses_sign": ("if (v != v) return (uint8_t)(sign | 0x7Fu);", "if (v != v) return (uint8_t)0x7Fu;"),
+    "e4m3_negative_zero_unsigned": ("if (a == 0.0) return sign;", "if (a == 0.0) return 0;"),
     # FP8 dispatch placement (indices stay in bounds: row < L, t * R + r < R * T)
     "fp8_dispatch_row_base": ("const int64_t at = list_base[e] + row;", "const int64_t at = row;"),
     "fp8_dispatch_token_transposed": ("oracle_fp8_quantize_row(x + ((int64_t)r * T + t) * H",
@@ -80,11 +82,21 @@ MUTANTS = {
     "normal_sent_any_rank": ("if (pair_is_live(e, r, E, E_local, active) && e / E_local == d) sent = 1;",
                              "if (pair_is_live(e, r, E, E_local, active)) sent = 1;"),
     # replica weights / gradients
+    "grad_reduce_float_accumulator": ("double acc = 0.0;", "float acc = 0.0f;"),
     "grad_reduce_skips_last_replica": ("for (int32_t p = phys_base[e]; p < phys_base[e + 1]; p++) acc +=",
                                        "for (int32_t p = phys_base[e]; p < phys_base[e + 1] - 1; p++) acc +="),
     "weight_sync_shifted": ("replicas[(int64_t)p * param_bytes + b] = master[(int64_t)e * param_bytes + b];",
                             "replicas[(int64_t)p * param_bytes + b] = master[(int64_t)(p - phys_base[e]) * param_bytes + b];"),
     # reroute
+    "reroute_minus_one_flagged": ("else if (e != -1) status |= ORACLE_BAD_EXPERT;", "else status |= ORACLE_BAD_EXPERT;"),
+    "reroute_bad_id_unflagged": ("else if (e != -1) status |= ORACLE_BAD_EXPERT;", ""),
+    "reroute_float_ratio": ("int64_t lhs = (int64_t)load[e] * n_rep[best];\n            int64_t rhs = (int64_t)load[best] * n_rep[e];",
+                            "float lhs = (float)load[e] / n_rep[e];\n            float rhs = (float)load[best] / n_rep[best];"),
+    # layout / combine capacity
+    "layout_full_expert_flagged": ("if (recv_count[e] > capacity) status |= ORACLE_OVERFLOW;",
+                                   "if (recv_count[e] >= capacity) status |= ORACLE_OVERFLOW;"),
+    "combine_overflow_unflagged": ("if (row >= capacity) { status |= ORACLE_OVERFLOW; continue; }\n            double w",
+                                   "if (row >= capacity) { continue; }\n            double w"),
     "reroute_tie_highest": ("if (lhs > rhs) best = e;", "if (lhs >= rhs) best = e;"),
     "reroute_local_token": ("topk_phys[p] = phys_base[e] + (int32_t)(global_token % n_rep[e]);",
                             "topk_phys[p] = phys_base[e] + (int32_t)(t % n_rep[e]);"),
