@@ -447,7 +447,11 @@ def pin_fp8_dequant_error(lib):
 
     rng = np.random.default_rng(22)
     for pow2 in (False, True):
-        bits = inputs.bf16_tokens(rng, 1, 512)[0]
+        # 96 groups, group g scaled by 2^(g - 60) (exact in bf16), so the scales' exponents cover
+        # every binade from about 2^-68 to 2^27 without a gap
+        xf = oracle.bf16_bits_to_f64(inputs.bf16_tokens(rng, 1, 128 * 96)[0]).reshape(-1, 128)
+        xf = xf * np.exp2(np.arange(-60, 36, dtype=np.float64))[:, None]
+        bits = (xf.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16).ravel()
         xv = oracle.bf16_bits_to_f64(bits).reshape(-1, 128)
         codes, scales, ue = oracle.fp8_quantize_row(bits, pow2, lib=lib)
         deq = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy().reshape(-1, 128)
@@ -595,9 +599,21 @@ def pin_normal_bruteforce(lib):
             assert nl["recv_tokens"][d] == len(sent)
         live = brute_layout(idx, active, E)["live"]
         cnt = np.bincount(idx[live], minlength=E)
+        assert nl["status"] == 0
         for a in (1, 2, 5):
             got = oracle.normal_layout(idx, active, E, alignment=a, lib=lib)["num_recv_tokens_per_expert"]
             assert np.array_equal(got, -(-cnt // a) * a)
+
+
+def pin_normal_bad_ids(lib):
+    """Ids outside [-1, E) are flagged by the normal layout and reach no rank; -1 is an empty slot."""
+    idx = np.array([[[0, 9], [-1, 1]], [[-2, 3], [2, -1]]], np.int32)     # E = 4: 9 and -2 are bad
+    nl = oracle.normal_layout(idx, np.ones(2, np.uint8), 4, lib=lib)
+    assert nl["status"] & oracle.BAD_EXPERT
+    assert nl["token_recv_row"][0, 0].tolist() == [0, -1] and nl["token_recv_row"][1, 0].tolist() == [-1, 0]
+    assert nl["num_recv_tokens_per_expert"].tolist() == [1, 1, 1, 1]
+    ok = oracle.normal_layout(np.array([[[0, -1]], [[3, -1]]], np.int32), np.ones(2, np.uint8), 4, lib=lib)
+    assert ok["status"] == 0
 
 
 def pin_normal_dispatch_combine(lib):
@@ -719,7 +735,7 @@ def pin_replica_sync_and_reduce(lib):
 
 
 ALL_PINS = [pin_replica_sync_and_reduce, pin_normal_golden, pin_normal_bruteforce, pin_normal_dispatch_combine,
-            pin_normal_combine_mask_at_combine, pin_normal_capacity, pin_fp8_dispatch_is_cast_of_dispatch, pin_fp8_rounding_readings, pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
+            pin_normal_combine_mask_at_combine, pin_normal_capacity, pin_normal_bad_ids, pin_fp8_dispatch_is_cast_of_dispatch, pin_fp8_rounding_readings, pin_fp8_golden, pin_e4m3_against_torch, pin_fp8_dequant_error, pin_layout_golden, pin_layout_bruteforce, pin_layout_invariants, pin_layout_status,
             pin_dispatch_golden, pin_dispatch_bijection, pin_combine_golden,
             pin_combine_special_cases, pin_combine_mask, pin_reroute_golden, pin_reroute_invariants,
             pin_reroute_bad_ids_and_exact_ratio]

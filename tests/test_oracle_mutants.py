@@ -54,6 +54,8 @@ MUTANTS = {
     "fp8_codes_by_reciprocal": ("const float q = f / scale;", "const float q = f * (1.0f / scale);"),
     "fp8_zero_group_scale": ("return amax == 0.0f ? 1.0f : amax / 448.0f;", "return amax == 0.0f ? 2.0f : amax / 448.0f;"),
     "pow2_zero_group_scale": ("    int e = 0;\n    if (amax != 0.0f) {", "    int e = -127;\n    if (amax != 0.0f) {"),
+    "pow2_one_binade_wrong": ("    if (ue8m0) *ue8m0 = (uint8_t)(e + 127);\n    return (float)ldexp(1.0, e);",
+                              "    if (ue8m0) *ue8m0 = (uint8_t)(e + 127);\n    return (float)ldexp(1.0, e + (e == 3));"),
     "pow2_clamp_one_binade_high": ("if (e < -127) e = -127;", "if (e < -126) e = -126;"),
     "e4m3_nan_loses_sign": ("if (v != v) return (uint8_t)(sign | 0x7Fu);", "if (v != v) return (uint8_t)0x7Fu;"),
     "e4m3_negative_zero_unsigned": ("if (a == 0.0) return sign;", "if (a == 0.0) return 0;"),
@@ -63,6 +65,8 @@ MUTANTS = {
                                       "oracle_fp8_quantize_row(x + ((int64_t)t * R + r) * H"),
     "fp8_dispatch_scale_stride": ("codes + at * H, scales + at * G,", "codes + at * H, scales + at,"),
     # normal mode
+    "normal_bad_id_unflagged": ("if (e < -1 || e >= E) status |= ORACLE_BAD_EXPERT;\n                if (pair_is_live(e, r, E, E_local, active)) num_recv",
+                                "if (pair_is_live(e, r, E, E_local, active)) num_recv"),
     "normal_combine_no_dst_mask": ("if (row < 0 || !active_now[d]) continue;", "if (row < 0) continue;"),
     "normal_layout_overflow_unflagged": ("if (token_recv_row[at] >= capacity) status |= ORACLE_OVERFLOW;", ""),
     "normal_layout_overflow_off_by_one": ("if (token_recv_row[at] >= capacity) status |= ORACLE_OVERFLOW;",
