@@ -150,3 +150,112 @@ def test_fp8_workspace_and_diag_validation(lib):
     assert lib.ep_diag_wait_timeout(None, ctypes.byref(word), None) == ep.EP_ERR_INVALID
     assert lib.ep_diag_wait_timeout(ctypes.c_void_p(4), ctypes.byref(word), None) == ep.EP_ERR_INVALID
     assert lib.ep_diag_wait_timeout(ctypes.c_void_p(8), None, None) == ep.EP_ERR_INVALID
+
+
+def test_host_validation_of_the_other_entry_points(lib):
+    """FP8 dispatch, normal mode, replica sync / reduce, int64 conversion, receive statistics and
+    the multi-GPU transport reject bad sizes, null or misaligned pointers and unknown options on
+    the host with EP_ERR_INVALID (EP_ERR_UNSUPPORTED for shapes the kernels do not take), and
+    return EP_OK for empty problems, all before any device work: every pointer below is a
+    never-dereferenced fake."""
+    from combine_get_dispatch_histogram_b200 import ep
+
+    INV, UNS, OK = ep.EP_ERR_INVALID, ep.EP_ERR_UNSUPPORTED, ep.EP_OK
+    cfg = ep.Cfg(0, 0, 0, 0)
+    P = ctypes.c_void_p
+    a16, a8, a4 = P(0x1000), P(0x1008), P(0x1004)        # 16-, 8- and 4-byte aligned fakes
+    good, bad = ep.Dims(2, 4, 2, 8, 256), ep.Dims(3, 4, 2, 8, 256)   # bad: E % R != 0
+    empty = ep.Dims(2, 0, 2, 8, 256)
+    wide = ep.Dims(40, 4, 2, 80, 256)                     # 40 ranks: more than normal mode's 32 lanes
+
+    # FP8 dispatch: (d, x, topk_idx, pair_row, recv_count, fmt, ws, ws_bytes, recv_x, scales, src_info, status)
+    need = ep.ep_dispatch_fp8_workspace_bytes(2, 4, 2, 8, 256)
+
+    def fp8(d=good, x=a16, fmt=ep.EP_FP8_SCALE_F32, ws=a16, ws_bytes=need, recv_x=a16, src=a16, ptr=a16):
+        return lib.ep_dispatch_fp8(d, x, ptr, ptr, ptr, fmt, ws, ws_bytes, recv_x, ptr, src, None, cfg, None)
+
+    assert fp8(d=bad) == INV
+    assert fp8(fmt=7) == INV
+    assert fp8(d=ep.Dims(2, 4, 2, 8, 200)) == INV                       # H not a multiple of 128
+    assert fp8(fmt=ep.EP_FP8_SCALE_UE8M0) == INV                        # UE8M0 needs H % 512 == 0
+    assert fp8(ptr=None) == INV and fp8(x=None) == INV
+    assert fp8(ws=None) == INV and fp8(ws_bytes=need - 16) == INV and fp8(ws=a8) == INV
+    assert fp8(x=a8) == INV and fp8(recv_x=a4) == INV and fp8(src=a4) == INV
+    assert fp8(d=empty, x=None, ws=None, ptr=None) == OK
+
+    # normal layout: (d, capacity, alignment, itr, per_rank, recv_count, trr, recv_tokens, per_expert, status)
+    def nl(d=good, cap=8, align=1, ptr=a16):
+        return lib.ep_normal_layout(d, cap, align, ptr, ptr, ptr, ptr, ptr, ptr, None, cfg, None)
+
+    assert nl(d=bad) == INV and nl(cap=-1) == INV and nl(align=0) == INV
+    assert nl(d=wide) == UNS and nl(ptr=None) == INV
+
+    # normal dispatch: (d, capacity, x, topk_idx, weights, active, trr, recv_x, rti, rtw, src_info, status)
+    def nd(d=good, cap=8, x=a16, ptr=a16, src=a16):
+        return lib.ep_normal_dispatch(d, cap, x, ptr, ptr, ptr, ptr, ptr, ptr, ptr, src, None, cfg, None)
+
+    assert nd(d=bad) == INV and nd(cap=-1) == INV and nd(d=wide) == UNS
+    assert nd(ptr=None) == INV and nd(x=a8) == INV and nd(src=a4) == INV
+    assert nd(d=empty, x=None, ptr=None, src=None) == OK
+
+    # normal combine: (d, capacity, y, trr, active, out, status, cfg)
+    def nc(d=good, cap=8, y=a16, ptr=a16, out=a16, variant=0):
+        return lib.ep_normal_combine(d, cap, y, ptr, ptr, out, None, ep.Cfg(0, 0, 0, variant), None)
+
+    assert nc(d=bad) == INV and nc(cap=-1) == INV and nc(d=wide) == UNS
+    assert nc(ptr=None) == INV and nc(y=None) == INV and nc(y=a8) == INV and nc(out=a8) == INV
+    assert nc(variant=9) == INV
+    assert nc(d=ep.Dims(16, 4, 2, 16, 256), variant=ep.EP_VARIANT_VECTOR) == UNS   # vector path: R <= 8
+    assert nc(d=empty, y=None, ptr=None, out=None) == OK
+
+    # replica weight sync (bytes) and gradient reduction (floats): (E_log, E_phys, phys_base, n, src, dst, status)
+    for fn, n_ok, n_bad in ((lib.ep_replica_weight_sync, 64, 24), (lib.ep_replica_grad_reduce, 16, 3)):
+        assert fn(0, 4, a16, n_ok, a16, a16, None, cfg, None) == INV             # no logical expert
+        assert fn(4, 3, a16, n_ok, a16, a16, None, cfg, None) == INV             # fewer physical than logical
+        assert fn(4, 6, None, n_ok, a16, a16, None, cfg, None) == INV            # no phys_base
+        assert fn(4, 6, a16, -16, a16, a16, None, cfg, None) == INV              # negative size
+        assert fn(4, 6, a16, n_bad, a16, a16, None, cfg, None) == INV            # rows not 16-byte multiples
+        assert fn(4, 6, a16, n_ok, a8, a16, None, cfg, None) == INV              # misaligned source
+        assert fn(4, 6, a16, n_ok, a16, None, None, cfg, None) == INV            # no destination
+        assert fn(70000, 70000, a16, n_ok, a16, a16, None, cfg, None) == UNS     # more experts than grid rows
+        assert fn(4, 6, a16, 0, None, None, None, cfg, None) == OK               # nothing to move
+
+    # int64 -> int32 routing and receive statistics
+    assert lib.ep_topk_idx_to_int32(a16, a16, -1, None) == INV
+    assert lib.ep_topk_idx_to_int32(None, None, 0, None) == OK
+    assert lib.ep_topk_idx_to_int32(None, a16, 8, None) == INV
+    assert lib.ep_topk_idx_to_int32(a4, a16, 8, None) == INV                    # int64 source misaligned
+    assert lib.ep_recv_stats_accumulate(-1, a16, a16, None) == INV
+    assert lib.ep_recv_stats_accumulate(0, None, None, None) == OK
+    assert lib.ep_recv_stats_accumulate(4, None, a16, None) == INV
+
+    # multi-GPU transport
+    ws = lib.ep_layout_local_workspace_bytes(good)
+    for rank in (-1, 2):
+        assert lib.ep_layout_local(good, rank, a16, a16, a16, ws, a16, a16, a16, a16, None, cfg, None) == INV
+    assert lib.ep_layout_local(good, 0, a16, None, a16, ws, a16, a16, a16, a16, None, cfg, None) == INV
+    assert lib.ep_layout_local(good, 0, None, a16, a16, ws, a16, a16, a16, a16, None, cfg, None) == INV
+    table = ep.PeerTable(0x1000, 0x1000, 0x1000)
+    peer_ws = lib.ep_dispatch_peer_workspace_bytes()
+
+    def dp(d=good, rank=0, tab=table, x=a16, ws_=a16, ptr=a16):
+        return lib.ep_dispatch_peer(d, rank, tab, x, ptr, ptr, ptr, ptr, 1, ws_, peer_ws, None, cfg, None)
+
+    assert dp(d=bad) == INV and dp(rank=2) == INV and dp(tab=ep.PeerTable(0, 0x1000, 0x1000)) == INV
+    assert dp(ws_=None) == INV and dp(ws_=a4) == INV and dp(x=a8) == INV and dp(ptr=None) == INV
+
+    def cp(d=good, rank=0, ptr=a16, out=a16):
+        return lib.ep_combine_peer(d, rank, ptr, ptr, ptr, ptr, ptr, ptr, out, None, cfg, None)
+
+    assert cp(rank=-1) == INV and cp(ptr=None) == INV and cp(out=a8) == INV
+    assert cp(d=empty, ptr=None, out=None) == OK
+    assert lib.ep_wait_peers(0, a16, 1, a16, None, a16, None) == INV
+    assert lib.ep_wait_peers(65, a16, 1, a16, None, a16, None) == INV          # more than 64 ranks
+    assert lib.ep_wait_peers(2, a4, 1, a16, None, a16, None) == INV            # flags not 8-byte aligned
+    assert lib.ep_wait_peers(2, a16, 1, a16, a4, a16, None) == INV             # wait_ns not 8-byte aligned
+    assert lib.ep_wait_peers(2, a16, 1, a16, None, None, None) == INV          # no status word
+    assert lib.ep_signal_peers(2, 2, a16, a16, 1, None) == INV
+    assert lib.ep_signal_peers(2, 0, None, a16, 1, None) == INV
+    assert lib.ep_peer_recv_count(3, 8, 0, a16, a16, None) == INV              # E % R != 0
+    assert lib.ep_peer_recv_count(2, 8, 2, a16, a16, None) == INV              # rank out of range
+    assert lib.ep_peer_recv_count(2, 8, 0, None, a16, None) == INV
