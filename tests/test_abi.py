@@ -24,7 +24,8 @@ def declared_symbols():
     names = []
     for fn in os.listdir(os.path.join(ROOT, "include")):
         if fn.endswith(".h"):
-            text = open(os.path.join(ROOT, "include", fn)).read()
+            with open(os.path.join(ROOT, "include", fn)) as f:
+                text = f.read()
             names += re.findall(r"^EP_API\s+[\w\s\*]+?\**\b(ep_\w+)\s*\(", text, flags=re.M)
     return names
 

@@ -36,7 +36,7 @@ def _worker(rank, world, port, out):
 
 def test_reduce_over_ranks_gloo_world2():
     port = _free_port()
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()   # no fork of this (threaded) process
     out = manager.dict()
     mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
     for rank in (0, 1):

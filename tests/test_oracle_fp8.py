@@ -47,7 +47,8 @@ def test_e4m3_encoder_signs_specials_and_tiny_values(oracle_lib):
 
 
 def test_fp8_cast_golden_row(oracle_lib):
-    g = json.load(open(os.path.join(GOLDEN, "fp8_tiny.json")))
+    with open(os.path.join(GOLDEN, "fp8_tiny.json")) as f:
+        g = json.load(f)
     x = np.zeros(g["H"], np.float32)
     for i, v in g["nonzero"]:
         x[i] = v

@@ -114,7 +114,8 @@ MUTANTS = {
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_mutant_is_caught(name, tmp_path):
     find, repl = MUTANTS[name]
-    src = open(SRC).read()
+    with open(SRC) as f:
+        src = f.read()
     assert src.count(find) >= 1, f"mutation site for {name} not found"
     mutated = src.replace(find, repl, 1)
     path = tmp_path / "ep_oracle_mutant.c"

@@ -67,7 +67,7 @@ def _worker(rank, world, port, seed, out):
 @pytest.mark.parametrize("world", [2, 4])
 def test_count_exchange_and_offsets_match_the_oracle(world):
     port = _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()   # no fork of this (threaded) process
     mp.spawn(_worker, args=(world, port, 5 + world, out), nprocs=world, join=True)
     for rank in range(world):
         res = out[rank]
