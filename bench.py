@@ -746,7 +746,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill",
-                    help="prefill | decode | replica | tiny | sweep_T<n>[_mask5]")
+                    help="prefill | decode | replica | tiny | sweep_T<n>[_mask5] | prefill_T<n> | replica_T<n> | "
+                         "small_slab | paced_slab")
     ap.add_argument("--e2e-steps", type=int, default=30,
                     help="steps of the host-buffer pipeline (its fill and drain are spread over them)")
     ap.add_argument("--graph", action="store_true",
