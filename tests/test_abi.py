@@ -260,3 +260,36 @@ def test_host_validation_of_the_other_entry_points(lib):
     assert lib.ep_peer_recv_count(3, 8, 0, a16, a16, None) == INV              # E % R != 0
     assert lib.ep_peer_recv_count(2, 8, 2, a16, a16, None) == INV              # rank out of range
     assert lib.ep_peer_recv_count(2, 8, 0, None, a16, None) == INV
+
+
+def test_size_queries_at_the_edges_of_the_valid_range(lib):
+    """The host's size and path arithmetic at the largest valid shapes (R*T*k just under 2^31,
+    E = 8192, k = 32, a hidden size of 2^30) gives exact, positive answers and no wrap-around.
+    Under the sanitizer build of this file, a signed overflow anywhere on these paths aborts."""
+    from combine_get_dispatch_histogram_b200 import ep
+
+    shapes = [
+        (64, (2 ** 31 - 1) // (64 * 32), 32, 8192, 65536),   # every limit at once
+        (1, 2 ** 31 - 1, 1, 1, 8),                           # one rank, 2^31 - 1 tokens
+        (8, (2 ** 31 - 1) // 8, 1, 2048, 2 ** 30),           # a 2 GB token row
+        (64, 1, 32, 8192, 8),
+    ]
+    for R, T, k, E, H in shapes:
+        assert R * T * k < 2 ** 31
+        sync = ep.ep_layout_workspace_bytes(1, 0, 1, 1, 8)
+        lw = ep.ep_layout_workspace_bytes(R, T, k, E, H)
+        assert lw >= sync and lw % 16 == 0, (R, T, k, E, H, lw)
+        llw = ep.ep_layout_local_workspace_bytes(R, T, k, E, H)
+        assert llw > 0 and llw % 16 == 0
+        for fmt, per in ((ep.EP_FP8_SCALE_F32, 128), (ep.EP_FP8_SCALE_UE8M0, 512)):
+            want = -(-(R * T * (H // per) * 4) // 16) * 16 if H % per == 0 else 0
+            assert ep.ep_dispatch_fp8_workspace_bytes(R, T, k, E, H, fmt) == want, (R, T, H, fmt)
+        rw = ep.ep_reroute_workspace_bytes(R, T, k, E)
+        assert rw > 0 and rw % 16 == 0
+        assert ep.ep_layout_path(R, T, k, E, H) in (ep.EP_LAYOUT_SINGLE_CTA, ep.EP_LAYOUT_CLUSTER,
+                                                    ep.EP_LAYOUT_LOOKBACK, ep.EP_LAYOUT_CHUNKED)
+    # one past the pair limit is refused, not wrapped
+    with pytest.raises(ep.EPError) as ei:
+        ep.ep_layout_path(1, 2 ** 31 - 1, 2, 2, 8)
+    assert ei.value.code == ep.EP_ERR_UNSUPPORTED
+    assert ep.ep_layout_workspace_bytes(1, 2 ** 31 - 1, 2, 2, 8) == 0
