@@ -252,7 +252,11 @@ EP_API int ep_topk_idx_to_int32(const int64_t *topk_idx64, int32_t *topk_idx32, 
  *                         only: its first 64 KiB carry barrier state from call to
  *                         call (cf. Buffer.clean_low_latency_buffer on the NeMo
  *                         page); the rest is scratch.  Calls sharing a workspace
- *                         must be ordered on the GPU.
+ *                         must be ordered on the GPU.  After a call whose status
+ *                         has EP_STATUS_TIMEOUT, zero-fill those 64 KiB again
+ *                         before the next call: a chunk that started after the
+ *                         wait limit can leave a flag that the next call would
+ *                         take for its own.
  * out (every element written):
  *   num_tokens_per_expert int32 [R,E]     live pairs of source rank r on expert e
  *   num_tokens_per_rank   int32 [R,R]     tokens of r with >= 1 live pair on rank d
@@ -302,6 +306,10 @@ enum { EP_LAYOUT_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024 };
  *     barrier state requires, and every call leaves that state ready for the
  *     next, so nothing is cleared per call.  Calls whose kernels may overlap
  *     on the same GPU race on it: order them (one stream, or events).
+ *   - After a call whose status has EP_STATUS_TIMEOUT the array's barrier
+ *     state may be left for the next call to misread, and it cannot be
+ *     cleared from outside: use ep_layout with a workspace on that device
+ *     from then on.
  */
 EP_API int ep_layout_noalloc(ep_dims_t d, const int32_t *topk_idx, const uint8_t *active,
               int32_t *num_tokens_per_expert, int32_t *num_tokens_per_rank,
